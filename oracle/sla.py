@@ -1,0 +1,377 @@
+"""Plain fp64 CPU oracle of the Sparse-Linear Attention forward pass (SLA and SLA2).
+
+TEST INFRASTRUCTURE ONLY.  This module is the independent checker of the CUDA
+path: it shares no code, constants or helpers with the package
+``block_sparse_linear_pool_b200`` and must never be imported by it.  Only the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may
+import it.  It is slow on purpose: every step is written out in the order the
+pages give it, in float64, with numpy primitives (matmul, sort, exp) only.
+
+Sources, cited by page title and section:
+  [SLA]  "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable
+         Sparse-Linear Attention" (detail page, arXiv 2509.24006): §2 Q2 (the
+         algorithm, steps 1-4), §3 Fig. 4 (the forward flowchart), §4 (notation
+         table, Eq. 1, Eq. 3-4, Eq. 6, the six checks), §5 Table 2 (phi ablation),
+         §7 (code cross-reference: Proj init, linear-over-all-tokens variant,
+         smooth-K, exp2 online softmax, LUT-driven loop).
+  [SLA2] "SLA2: Sparse-Linear Attention with Learnable Routing and QAT"
+         (summary page, arXiv 2602.12675): §3 SLA2 Design (alpha combine),
+         §4 Learnable Router (pooling, proj_q/proj_k, row-wise Top-k),
+         §5 Quantization-aware Training (low-bit Q/K with scales).
+
+Readings taken where the pages are silent (each also listed in the design doc):
+  * the last block may be partial (N not a multiple of b): its pooled mean is
+    over its real tokens only and no padding token enters any sum;
+  * block counts: n_h = max(1, floor(k_h*T + 1e-9)),
+    n_l = min(floor(k_l*T + 1e-9), T - n_h), per row;
+  * Top-k / Bottom-k is row-wise ([SLA2] §4), ranking by compressed attention
+    weight, descending, ties broken by the lower key-block index first; the
+    bottom n_l of that same order are negligible;
+  * the 1e-5 epsilon ([SLA] §4 check 5) is added to the linear denominator;
+  * Proj follows the nn.Linear convention Proj(x) = x W^T + b and is shared by
+    all heads; router projections are bias-free d x d maps shared by all heads;
+  * alpha is one scalar per head.
+
+Parity unpinned: the FP8 path's exact values (only the tolerance bound is
+checked against this oracle's unquantised result).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+
+EPS_DEFAULT = 1e-5
+
+
+# --------------------------------------------------------------------------
+# Parameters
+# --------------------------------------------------------------------------
+@dataclass
+class OracleParams:
+    """Hyper-parameters of one SLA / SLA2 forward ([SLA] §4 notation table)."""
+
+    b_q: int = 64
+    b_kv: int = 64
+    k_h: float = 0.05           # critical fraction per row
+    k_l: float = 0.10           # negligible fraction per row
+    combine: str = "proj"       # "proj" (SLA, [SLA] Eq. 6) or "alpha" (SLA2, [SLA2] §3)
+    eps: float = EPS_DEFAULT    # [SLA] §4 check 5
+    smooth_k: bool = False      # [SLA] §7 item 3 (code only)
+    linear_over_all: bool = False  # [SLA] §7 item 2 (code variant)
+    phi: str = "softmax"        # "softmax" ([SLA] Fig. 4) or "elu1" ([SLA] Table 2)
+
+
+def block_counts(T_kv: int, k_h: float, k_l: float) -> tuple[int, int]:
+    """Number of critical (n_h) and negligible (n_l) key blocks per query row.
+
+    [SLA] §2 Q2 step 2 gives "top k_h%" and "bottom k_l%"; [SLA2] §4 / §6 make
+    the count per row (k% x N/b_k).  Reading: floor, with at least one critical
+    block so that the sparse softmax is defined.
+    """
+    n_h = max(1, int(np.floor(k_h * T_kv + 1e-9)))
+    n_l = min(int(np.floor(k_l * T_kv + 1e-9)), T_kv - n_h)
+    n_l = max(n_l, 0)
+    return n_h, n_l
+
+
+def num_blocks(N: int, b: int) -> int:
+    return -(-N // b)
+
+
+def block_range(i: int, b: int, N: int) -> tuple[int, int]:
+    """Token range [start, stop) of block i; the last block may be partial."""
+    return i * b, min((i + 1) * b, N)
+
+
+# --------------------------------------------------------------------------
+# Step 1: compressed attention prediction ([SLA] §2 Q2 step 1, Fig. 4)
+# --------------------------------------------------------------------------
+def smooth_keys(K: np.ndarray) -> np.ndarray:
+    """K minus its mean over tokens ([SLA] §7 item 3: zero-mean K before the mask)."""
+    K = np.asarray(K, dtype=np.float64)
+    return K - K.mean(axis=-2, keepdims=True)
+
+
+def mean_pool(X: np.ndarray, b: int) -> np.ndarray:
+    """Mean of X over consecutive blocks of b tokens: [..., N, d] -> [..., T, d].
+
+    [SLA] §2 Q2 step 1 and Fig. 4 (mean_pool); [SLA2] §4 (pooling adjacent
+    tokens before routing).  A partial last block is averaged over its real
+    tokens.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    N = X.shape[-2]
+    T = num_blocks(N, b)
+    out = np.empty(X.shape[:-2] + (T, X.shape[-1]), dtype=np.float64)
+    for i in range(T):
+        s, e = block_range(i, b, N)
+        out[..., i, :] = X[..., s:e, :].sum(axis=-2) / (e - s)
+    return out
+
+
+def compressed_logits(Q, K, p: OracleParams, Wq=None, Wk=None) -> np.ndarray:
+    """pool(Q) . pool(K)^T / sqrt(d), with SLA2's router projections if given.
+
+    [SLA] §2 Q2 step 1 / Fig. 4: P_c = Softmax(pool(Q) pool(K)^T / sqrt(d)).
+    [SLA2] §4: proj_q, proj_k (d -> d) transform the pooled Q and K first.
+    Returns the pre-softmax logits [..., T_q, T_kv].
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    d = Q.shape[-1]
+    if p.smooth_k:
+        K = smooth_keys(K)
+    Qc = mean_pool(Q, p.b_q)
+    Kc = mean_pool(K, p.b_kv)
+    if Wq is not None:
+        Qc = Qc @ np.asarray(Wq, dtype=np.float64).T
+    if Wk is not None:
+        Kc = Kc @ np.asarray(Wk, dtype=np.float64).T
+    return (Qc @ np.swapaxes(Kc, -1, -2)) / np.sqrt(d)
+
+
+def compressed_attention(logits: np.ndarray) -> np.ndarray:
+    """Row softmax of the compressed logits: P_c ([SLA] Fig. 4)."""
+    m = logits.max(axis=-1, keepdims=True)
+    e = np.exp(logits - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def classify(Pc: np.ndarray, n_h: int, n_l: int) -> np.ndarray:
+    """Three-way block classification M_c in {1, 0, -1} ([SLA] §2 Q2 step 2).
+
+    Per row ([SLA2] §4: "highest-scoring k% positions in each row"): order the
+    key blocks by P_c descending, ties by lower index first; the first n_h are
+    critical (1), the last n_l negligible (-1), the rest marginal (0).
+    """
+    Pc = np.asarray(Pc, dtype=np.float64)
+    T = Pc.shape[-1]
+    flat = Pc.reshape(-1, T)
+    Mc = np.zeros(flat.shape, dtype=np.int8)
+    idx = np.arange(T)
+    for r in range(flat.shape[0]):
+        order = np.lexsort((idx, -flat[r]))  # primary: -P ascending; secondary: index
+        rank = np.empty(T, dtype=np.int64)
+        rank[order] = idx
+        Mc[r, rank < n_h] = 1
+        if n_l > 0:
+            Mc[r, rank >= T - n_l] = -1
+    return Mc.reshape(Pc.shape)
+
+
+def predict_mask(Q, K, p: OracleParams, Wq=None, Wk=None):
+    """Compressed mask prediction, Fig. 4 left: returns (M_c, logits, P_c)."""
+    logits = compressed_logits(Q, K, p, Wq, Wk)
+    Pc = compressed_attention(logits)
+    T_kv = logits.shape[-1]
+    n_h, n_l = block_counts(T_kv, p.k_h, p.k_l)
+    return classify(Pc, n_h, n_l), logits, Pc
+
+
+def critical_lut(Mc: np.ndarray) -> np.ndarray:
+    """Per query block, the critical key-block indices in ascending order
+    ([SLA] §7 item 5: the kernel walks a per-row list of critical blocks)."""
+    n_h = int((Mc[(0,) * (Mc.ndim - 1)] == 1).sum())
+    out = np.zeros(Mc.shape[:-1] + (n_h,), dtype=np.int32)
+    flat_m = Mc.reshape(-1, Mc.shape[-1])
+    flat_o = out.reshape(-1, n_h)
+    for r in range(flat_m.shape[0]):
+        flat_o[r] = np.nonzero(flat_m[r] == 1)[0]
+    return out
+
+
+# --------------------------------------------------------------------------
+# Step 3 ingredients: feature map and per-block linear statistics
+# --------------------------------------------------------------------------
+def feature_map(X: np.ndarray, kind: str = "softmax") -> np.ndarray:
+    """phi applied per token over the head dimension.
+
+    "softmax" is the map of [SLA] Fig. 4 ("feature map (softmax)"); "elu1" is
+    elu(x) + 1, the ablation of [SLA] Table 2.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    if kind == "softmax":
+        m = X.max(axis=-1, keepdims=True)
+        e = np.exp(X - m)
+        return e / e.sum(axis=-1, keepdims=True)
+    if kind == "elu1":
+        return np.where(X > 0, X + 1.0, np.exp(np.minimum(X, 0.0)))
+    raise ValueError(kind)
+
+
+def linear_block_stats(K, V, b_kv: int, phi: str = "softmax"):
+    """h_j = phi(K_j)^T V_j  (d x d) and z_j = rowsum(phi(K_j)^T) (d).
+
+    [SLA] §2 Q2 step 3 and Fig. 4 ("h_j = phi(K_j)^T V_j, z_j =
+    rowsum(phi(K_j)^T)").  Only the real tokens of a partial block count.
+    Returns h [..., T, d, d] (index [j, a, b]) and z [..., T, d].
+    """
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    N, d = K.shape[-2], K.shape[-1]
+    T = num_blocks(N, b_kv)
+    fK = feature_map(K, phi)
+    h = np.empty(K.shape[:-2] + (T, d, V.shape[-1]), dtype=np.float64)
+    z = np.empty(K.shape[:-2] + (T, d), dtype=np.float64)
+    for j in range(T):
+        s, e = block_range(j, b_kv, N)
+        h[..., j, :, :] = np.swapaxes(fK[..., s:e, :], -1, -2) @ V[..., s:e, :]
+        z[..., j, :] = fK[..., s:e, :].sum(axis=-2)
+    return h, z
+
+
+# --------------------------------------------------------------------------
+# Steps 3-4: the per-query-block computation and the combination
+# --------------------------------------------------------------------------
+def quantize_e4m3(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest FP8 E4M3 value (ties to even), saturating at 448.
+
+    Written from the OCP 8-bit floating point specification: 1 sign bit,
+    4 exponent bits (bias 7), 3 mantissa bits; normal numbers 2^-6 .. 448,
+    subnormals m * 2^-9.  Used by the low-bit path of [SLA2] §5.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    a = np.minimum(np.abs(x), 448.0)
+    # exponent of the quantisation step: 2^(e-3) for a in [2^e, 2^(e+1)), e >= -6
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, -6.0)
+    step = np.exp2(e - 3.0)
+    q = np.round(a / step) * step  # np.round is round-half-to-even
+    q = np.minimum(q, 448.0)
+    return np.sign(x) * q
+
+
+def _fp8_dequant_tile(X: np.ndarray) -> np.ndarray:
+    """Quantise one 64-row tile with scale max|X|/448 and return the
+    dequantised values ([SLA2] §5: tensors mapped to FP8 with scales)."""
+    amax = np.abs(X).max()
+    if amax == 0:
+        return np.zeros_like(X)
+    s = amax / 448.0
+    return quantize_e4m3(X / s) * s
+
+
+def forward_given_mask(Q, K, V, Mc, p: OracleParams, proj_w=None, proj_b=None, alpha=None,
+                       qblocks: Optional[Sequence[int]] = None, heads: Optional[Sequence] = None,
+                       qk_fp8: bool = False, return_branches: bool = False):
+    """SLA / SLA2 output for a given compressed mask M_c.
+
+    Q, K, V: [B, H, N, d] (any float dtype; upcast to float64).
+    Mc: int8 [B, H, T_q, T_kv].
+    For each query block i ([SLA] §2 Q2 step 3, Fig. 4 "Fused kernel"):
+      * critical blocks (M_c = 1): exact softmax attention over their tokens,
+        O^s = diag(l)^-1 O^s_acc  (two-pass softmax: max, then exp / sum);
+      * marginal blocks (M_c = 0): H_i = sum h_j, Z_i = sum z_j and
+        O^l = phi(Q_i) H_i / (phi(Q_i) Z_i + eps)  ([SLA] Eq. 3-4, §4 check 5);
+      * negligible blocks (M_c = -1) contribute nothing.
+    Combination ([SLA] Eq. 6 / [SLA2] §3):
+      "proj":  O = O^s + O^l W^T + b
+      "alpha": O = alpha_h O^s + (1 - alpha_h) O^l
+    `qblocks` / `heads` restrict the work to a sample (rows of other blocks are
+    left as NaN).  `qk_fp8` quantises Q and K per 64-row tile to E4M3 before
+    Q K^T ([SLA2] §5); diagnosis only.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    B, H, N, d = Q.shape
+    dv = V.shape[-1]
+    T_q = num_blocks(N, p.b_q)
+    T_kv = num_blocks(N, p.b_kv)
+    assert Mc.shape == (B, H, T_q, T_kv), Mc.shape
+    scale = 1.0 / np.sqrt(d)
+    O = np.full((B, H, N, dv), np.nan)
+    Os = np.full((B, H, N, dv), np.nan)
+    Ol = np.full((B, H, N, dv), np.nan)
+    if heads is None:
+        heads = [(b, h) for b in range(B) for h in range(H)]
+    qsel = range(T_q) if qblocks is None else qblocks
+    W = None if proj_w is None else np.asarray(proj_w, dtype=np.float64)
+    bias = None if proj_b is None else np.asarray(proj_b, dtype=np.float64)
+
+    for (bb, hh) in heads:
+        h_stats, z_stats = linear_block_stats(K[bb, hh], V[bb, hh], p.b_kv, p.phi)
+        fQ = feature_map(Q[bb, hh], p.phi)
+        for i in qsel:
+            qs, qe = block_range(i, p.b_q, N)
+            q = Q[bb, hh, qs:qe]
+            row = Mc[bb, hh, i]
+            # --- sparse branch over critical blocks
+            crit = np.nonzero(row == 1)[0]
+            if qk_fp8:
+                q = _fp8_dequant_tile(q)
+            keys, vals = [], []
+            for j in crit:
+                ks, ke = block_range(int(j), p.b_kv, N)
+                kj = K[bb, hh, ks:ke]
+                if qk_fp8:
+                    kj = _fp8_dequant_tile(kj)
+                keys.append(kj)
+                vals.append(V[bb, hh, ks:ke])
+            if keys:
+                kk = np.concatenate(keys, axis=0)
+                vv = np.concatenate(vals, axis=0)
+                s = (q @ kk.T) * scale
+                m = s.max(axis=1, keepdims=True)
+                e = np.exp(s - m)
+                o_s = (e @ vv) / e.sum(axis=1, keepdims=True)
+            else:
+                o_s = np.zeros((qe - qs, dv))
+            # --- linear branch over marginal blocks
+            marg = np.arange(T_kv) if p.linear_over_all else np.nonzero(row == 0)[0]
+            Hi = h_stats[marg].sum(axis=0) if len(marg) else np.zeros((d, dv))
+            Zi = z_stats[marg].sum(axis=0) if len(marg) else np.zeros(d)
+            fq = fQ[qs:qe]
+            o_l = (fq @ Hi) / ((fq @ Zi) + p.eps)[:, None]
+            # --- combine
+            if p.combine == "proj":
+                proj = o_l @ W.T if W is not None else np.zeros_like(o_l)
+                if bias is not None:
+                    proj = proj + bias
+                o = o_s + proj
+            elif p.combine == "alpha":
+                a = float(np.asarray(alpha, dtype=np.float64).reshape(B, H)[bb, hh]) \
+                    if np.ndim(alpha) else float(alpha)
+                o = a * o_s + (1.0 - a) * o_l
+            else:
+                raise ValueError(p.combine)
+            O[bb, hh, qs:qe] = o
+            Os[bb, hh, qs:qe] = o_s
+            Ol[bb, hh, qs:qe] = o_l
+    if return_branches:
+        return O, Os, Ol
+    return O
+
+
+def forward(Q, K, V, p: OracleParams, proj_w=None, proj_b=None, alpha=None, Wq=None, Wk=None,
+            **kw):
+    """Full SLA / SLA2 forward: predict M_c, then the fused computation.
+
+    Returns (O, M_c)."""
+    Mc, _, _ = predict_mask(Q, K, p, Wq, Wk)
+    return forward_given_mask(Q, K, V, Mc, p, proj_w, proj_b, alpha, **kw), Mc
+
+
+def mask_grading(logits: np.ndarray, n_h: int, n_l: int, gap: float = 1e-4) -> np.ndarray:
+    """Which mask entries are decided by more than `gap` on the logit scale.
+
+    An entry is graded when its logit lies farther than `gap` from both the
+    top-k threshold (midpoint of the n_h-th and (n_h+1)-th largest) and the
+    bottom-k threshold (midpoint of the n_l-th and (n_l+1)-th smallest).
+    Returns a boolean array shaped like `logits`.
+    """
+    L = np.asarray(logits, dtype=np.float64)
+    T = L.shape[-1]
+    srt = -np.sort(-L, axis=-1)  # descending
+    big = np.inf
+    t_hi = 0.5 * (srt[..., n_h - 1] + srt[..., n_h]) if n_h < T else np.full(L.shape[:-1], -big)
+    if n_l > 0:
+        t_lo = 0.5 * (srt[..., T - n_l - 1] + srt[..., T - n_l])
+    else:
+        t_lo = np.full(L.shape[:-1], big)
+    dh = np.abs(L - t_hi[..., None])
+    dl = np.abs(L - t_lo[..., None])
+    return (dh > gap) & (dl > gap)
