@@ -1,0 +1,226 @@
+"""Thin ctypes binding of libsla.so (include/sla.h) for torch tensors.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of the library.  torch provides device memory and the current stream.
+The functions carry the C names; outputs and workspaces are allocated here
+with torch (the library itself allocates nothing).  If libsla.so is missing,
+every call raises: there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libsla.so")
+
+SLA_COMBINE_PROJ, SLA_COMBINE_ALPHA = 0, 1
+SLA_QK_BF16, SLA_QK_FP8_E4M3 = 0, 1
+
+STATUS = {
+    0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "SLA_ERR_WORKSPACE",
+    4: "SLA_ERR_CUDA", 5: "SLA_ERR_DEVICE_TIMEOUT", 6: "SLA_ERR_DEVICE_BAD_INDEX",
+}
+
+# Every symbol include/sla.h declares (checked by the CPU tests).
+EXPORTS = (
+    "sla_params_default", "sla_block_counts", "sla_workspace_size", "sla_hz_size",
+    "sla_predict_mask", "sla_precompute_linear", "sla_forward", "sla_attention_workspace_size",
+    "sla_attention", "sla_backward", "sla_get_device_status", "sla_status_string",
+    "sla_abi_version",
+)
+
+
+class SlaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class sla_params_t(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("d", ctypes.c_int),
+        ("b_q", ctypes.c_int), ("b_kv", ctypes.c_int),
+        ("k_h", ctypes.c_float), ("k_l", ctypes.c_float),
+        ("combine", ctypes.c_int), ("qk_prec", ctypes.c_int), ("smooth_k", ctypes.c_int),
+        ("eps", ctypes.c_float),
+        ("stride_q", ctypes.c_int64 * 3), ("stride_k", ctypes.c_int64 * 3),
+        ("stride_v", ctypes.c_int64 * 3), ("stride_o", ctypes.c_int64 * 3),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run `python -m block_sparse_linear_pool_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P = ctypes.POINTER(sla_params_t)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        L.sla_params_default.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_float, ctypes.c_float, ctypes.c_int]
+        L.sla_params_default.restype = None
+        ip = ctypes.POINTER(ctypes.c_int)
+        L.sla_block_counts.argtypes = [P, ip, ip, ip, ip]
+        for f in ("sla_workspace_size", "sla_hz_size", "sla_attention_workspace_size"):
+            getattr(L, f).argtypes = [P, ctypes.POINTER(sz)]
+        L.sla_predict_mask.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_precompute_linear.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_attention.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_get_device_status.argtypes = [vp, vp, ip]
+        L.sla_status_string.argtypes = [ctypes.c_int]
+        L.sla_status_string.restype = ctypes.c_char_p
+        for f in EXPORTS:
+            if f not in ("sla_params_default", "sla_status_string"):
+                getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise SlaError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _strides(t: torch.Tensor):
+    s = t.stride()
+    if s[3] != 1:
+        raise ValueError("the head dimension must be contiguous")
+    return (ctypes.c_int64 * 3)(s[0], s[1], s[2])
+
+
+@dataclass
+class SlaConfig:
+    """Settings of one forward ([SLA] §4 notation table; [SLA2] §3-5)."""
+    k_h: float
+    k_l: float
+    combine: str = "proj"     # "proj" (SLA) or "alpha" (SLA2)
+    qk: str = "bf16"          # "bf16" or "fp8_e4m3"
+    smooth_k: bool = False
+    eps: float = 1e-5
+
+
+def make_params(Q: torch.Tensor, cfg: SlaConfig, K=None, V=None, O=None) -> sla_params_t:
+    B, H, N, d = Q.shape
+    p = sla_params_t()
+    lib().sla_params_default(ctypes.byref(p), B, H, N, d, cfg.k_h, cfg.k_l,
+                             SLA_COMBINE_PROJ if cfg.combine == "proj" else SLA_COMBINE_ALPHA)
+    p.qk_prec = SLA_QK_BF16 if cfg.qk == "bf16" else SLA_QK_FP8_E4M3
+    p.smooth_k = int(cfg.smooth_k)
+    p.eps = cfg.eps
+    p.stride_q = _strides(Q)
+    p.stride_k = _strides(K if K is not None else Q)
+    p.stride_v = _strides(V if V is not None else Q)
+    if O is not None:
+        p.stride_o = _strides(O)
+    return p
+
+
+def sla_block_counts(p: sla_params_t):
+    out = [ctypes.c_int() for _ in range(4)]
+    _check(lib().sla_block_counts(ctypes.byref(p), *[ctypes.byref(x) for x in out]), "sla_block_counts")
+    return tuple(x.value for x in out)  # T_q, T_kv, n_h, n_l
+
+
+def _size(fn: str, p: sla_params_t) -> int:
+    n = ctypes.c_size_t()
+    _check(getattr(lib(), fn)(ctypes.byref(p), ctypes.byref(n)), fn)
+    return n.value
+
+
+def sla_workspace_size(p: sla_params_t) -> int:
+    return _size("sla_workspace_size", p)
+
+
+def sla_hz_size(p: sla_params_t) -> int:
+    return _size("sla_hz_size", p)
+
+
+def sla_attention_workspace_size(p: sla_params_t) -> int:
+    return _size("sla_attention_workspace_size", p)
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """Zero-initialised workspace (the first word is the device error word)."""
+    return torch.zeros(nbytes, dtype=torch.uint8, device=device)
+
+
+def _f32(t: Optional[torch.Tensor], device):
+    return None if t is None else t.to(device=device, dtype=torch.float32).contiguous()
+
+
+def sla_predict_mask(Q, K, cfg: SlaConfig, Wq=None, Wk=None, workspace=None):
+    """Returns (mc int8 [B*H, T_q, T_kv], lut int32 [B*H, T_q, n_h])."""
+    p = make_params(Q, cfg, K=K)
+    Tq, Tkv, nh, _ = sla_block_counts(p)
+    BH = Q.shape[0] * Q.shape[1]
+    mc = torch.empty((BH, Tq, Tkv), dtype=torch.int8, device=Q.device)
+    lut = torch.empty((BH, Tq, nh), dtype=torch.int32, device=Q.device)
+    ws = workspace if workspace is not None else new_workspace(sla_workspace_size(p), Q.device)
+    Wq, Wk = _f32(Wq, Q.device), _f32(Wk, Q.device)
+    _check(lib().sla_predict_mask(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(Wq), _ptr(Wk), _ptr(mc),
+                                  _ptr(lut), _ptr(ws), ws.numel(), _stream()), "sla_predict_mask")
+    return mc, lut
+
+
+def sla_precompute_linear(K, V, cfg: SlaConfig, proj_w=None, workspace=None):
+    """Returns hz bf16 [B*H, T_kv, d*d + d] (see include/sla.h for the layout)."""
+    p = make_params(K, cfg, K=K, V=V)
+    _, Tkv, _, _ = sla_block_counts(p)
+    BH, d = K.shape[0] * K.shape[1], K.shape[3]
+    hz = torch.empty((BH, Tkv, d * d + d), dtype=torch.bfloat16, device=K.device)
+    ws = workspace if workspace is not None else new_workspace(sla_workspace_size(p), K.device)
+    proj_w = _f32(proj_w, K.device)
+    _check(lib().sla_precompute_linear(ctypes.byref(p), _ptr(K), _ptr(V), _ptr(proj_w), _ptr(hz),
+                                       _ptr(ws), ws.numel(), _stream()), "sla_precompute_linear")
+    return hz
+
+
+def sla_forward(Q, K, V, mc, lut, hz, cfg: SlaConfig, proj_b=None, alpha=None, out=None,
+                workspace=None):
+    """O bf16 [B, H, N, d]."""
+    O = out if out is not None else torch.empty_like(Q)
+    p = make_params(Q, cfg, K=K, V=V, O=O)
+    ws = workspace if workspace is not None else new_workspace(sla_workspace_size(p), Q.device)
+    proj_b, alpha = _f32(proj_b, Q.device), _f32(alpha, Q.device)
+    _check(lib().sla_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(mc), _ptr(lut), _ptr(hz),
+                             _ptr(proj_b), _ptr(alpha), _ptr(O), _ptr(ws), ws.numel(), _stream()),
+           "sla_forward")
+    return O
+
+
+def sla_attention(Q, K, V, cfg: SlaConfig, proj_w=None, proj_b=None, alpha=None, Wq=None, Wk=None,
+                  out=None, workspace=None):
+    """The whole forward in one library call.  O bf16 [B, H, N, d]."""
+    O = out if out is not None else torch.empty_like(Q)
+    p = make_params(Q, cfg, K=K, V=V, O=O)
+    ws = workspace if workspace is not None else new_workspace(sla_attention_workspace_size(p), Q.device)
+    dev = Q.device
+    args = [_f32(x, dev) for x in (proj_w, proj_b, alpha, Wq, Wk)]
+    _check(lib().sla_attention(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), *[_ptr(x) for x in args],
+                               _ptr(O), _ptr(ws), ws.numel(), _stream()), "sla_attention")
+    return O
+
+
+def sla_get_device_status(workspace) -> int:
+    detail = ctypes.c_int()
+    code = lib().sla_get_device_status(_ptr(workspace), _stream(), ctypes.byref(detail))
+    return code, detail.value

@@ -1,0 +1,442 @@
+// Host side of the C ABI declared in include/sla.h: argument validation,
+// workspace layout, TMA descriptor encoding and kernel launches.  Nothing here
+// allocates device memory or synchronises a stream (except
+// sla_get_device_status).
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "sla.h"
+#include "kernels.cuh"
+
+using namespace sla;
+
+namespace {
+
+constexpr int kMaxN = 262144;
+constexpr size_t kAlign = 256;
+
+struct Plan {
+  int B, H, N, d, BH, Tq, Tkv, nh, nl, NN, Tkvp;
+};
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+struct Layout {
+  size_t err, qc, kc, qr, kr, kmean, mm, hagg, end;       // sla_workspace_size
+  size_t mc, lut, hz, end_attn;                           // + sla_attention extras
+};
+
+Layout layout_of(const Plan& p) {
+  Layout L;
+  size_t o = 0;
+  L.err = o;   o = align_up(o + 256);
+  L.qc = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.d * 4);
+  L.kc = o;    o = align_up(o + (size_t)p.BH * p.Tkv * p.d * 4);
+  L.qr = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.d * 4);
+  L.kr = o;    o = align_up(o + (size_t)p.BH * p.Tkv * p.d * 4);
+  L.kmean = o; o = align_up(o + (size_t)p.BH * p.d * 4);
+  L.mm = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkvp * 2);
+  L.hagg = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.NN * 2);
+  L.end = o;
+  L.mc = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkv);
+  L.lut = o;   o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
+  L.hz = o;    o = align_up(o + (size_t)p.BH * p.Tkv * p.NN * 2);
+  L.end_attn = o;
+  return L;
+}
+
+void counts(int T, double kh, double kl, int* nh, int* nl) {
+  int h = (int)std::floor(kh * T + 1e-9);
+  if (h < 1) h = 1;
+  if (h > T) h = T;
+  int l = (int)std::floor(kl * T + 1e-9);
+  if (l > T - h) l = T - h;
+  if (l < 0) l = 0;
+  *nh = h;
+  *nl = l;
+}
+
+bool stride_ok(const int64_t* s, int d) {
+  for (int i = 0; i < 3; ++i)
+    if (s[i] <= 0 || (s[i] % 8) != 0) return false;
+  return s[2] >= d;
+}
+
+sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
+  if (!p) return SLA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->H < 1 || p->N < 1) return SLA_ERR_INVALID_ARG;
+  if (!(p->k_h >= 0.f && p->k_h <= 1.f && p->k_l >= 0.f && p->k_l <= 1.f)) return SLA_ERR_INVALID_ARG;
+  if (!(p->eps >= 0.f) || !std::isfinite(p->eps)) return SLA_ERR_INVALID_ARG;
+  if (p->combine != SLA_COMBINE_PROJ && p->combine != SLA_COMBINE_ALPHA) return SLA_ERR_INVALID_ARG;
+  if (p->qk_prec != SLA_QK_BF16 && p->qk_prec != SLA_QK_FP8_E4M3) return SLA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
+  if (p->b_q != 64 || p->b_kv != 64) return SLA_ERR_UNSUPPORTED;
+  if (p->N > kMaxN || (int64_t)p->B * p->H > 65535) return SLA_ERR_UNSUPPORTED;
+  if (!stride_ok(p->stride_q, p->d) || !stride_ok(p->stride_k, p->d) ||
+      !stride_ok(p->stride_v, p->d) || !stride_ok(p->stride_o, p->d))
+    return SLA_ERR_INVALID_ARG;
+  pl->B = p->B;
+  pl->H = p->H;
+  pl->N = p->N;
+  pl->d = p->d;
+  pl->BH = p->B * p->H;
+  pl->Tq = (p->N + p->b_q - 1) / p->b_q;
+  pl->Tkv = (p->N + p->b_kv - 1) / p->b_kv;
+  counts(pl->Tkv, p->k_h, p->k_l, &pl->nh, &pl->nl);
+  pl->NN = p->d * p->d + p->d;
+  pl->Tkvp = (pl->Tkv + 7) & ~7;
+  return SLA_OK;
+}
+
+bool aligned16(const void* x) { return (reinterpret_cast<uintptr_t>(x) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// rank-r bf16 tiled map, 128-byte swizzle; dims/strides innermost first,
+// strides in bytes for dims 1..r-1.
+bool encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+            const uint64_t* strides, const uint32_t* box) {
+  auto fn = encoder();
+  if (!fn) return false;
+  cuuint64_t gd[5], gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Q/K/V/O [B,H,N,d] with element strides s (B, H, N), box of `rows` tokens x 64 columns.
+bool map_bhnd(CUtensorMap* m, const void* base, const Plan& p, const int64_t* s, int rows) {
+  const uint64_t dims[4] = {(uint64_t)p.d, (uint64_t)p.N, (uint64_t)p.H, (uint64_t)p.B};
+  const uint64_t strides[3] = {(uint64_t)s[2] * 2, (uint64_t)s[1] * 2, (uint64_t)s[0] * 2};
+  const uint32_t box[4] = {64, (uint32_t)rows, 1, 1};
+  return encode(m, base, 4, dims, strides, box);
+}
+
+sla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SLA_OK : SLA_ERR_CUDA; }
+
+#define SLA_TRY(x)                      \
+  do {                                  \
+    sla_status_t st_ = (x);             \
+    if (st_ != SLA_OK) return st_;      \
+  } while (0)
+
+sla_status_t check_ws(const Plan& p, void* ws, size_t bytes, bool attn) {
+  const Layout L = layout_of(p);
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return SLA_ERR_WORKSPACE;
+  if (bytes < (attn ? L.end_attn : L.end)) return SLA_ERR_WORKSPACE;
+  return SLA_OK;
+}
+
+template <class T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+sla_status_t predict_mask_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
+                               const float* Wq, const float* Wk, int8_t* mc, int32_t* lut,
+                               void* ws, cudaStream_t s) {
+  const Layout L = layout_of(pl);
+  PoolArgs pa;
+  pa.Q = static_cast<const __nv_bfloat16*>(Q);
+  pa.K = static_cast<const __nv_bfloat16*>(K);
+  for (int i = 0; i < 3; ++i) {
+    pa.sq[i] = p->stride_q[i];
+    pa.sk[i] = p->stride_k[i];
+  }
+  pa.Qc = at<float>(ws, L.qc);
+  pa.Kc = at<float>(ws, L.kc);
+  pa.H = pl.H;
+  pa.N = pl.N;
+  pa.T = pl.Tq;  // b_q == b_kv: T_q == T_kv
+  pa.bs = 64;
+  SLA_TRY(cuda_status(launch_pool(pa, pl.d, pl.BH, s)));
+  const float* qsrc = pa.Qc;
+  const float* ksrc = pa.Kc;
+  if (Wq || Wk || p->smooth_k) {
+    SLA_TRY(cuda_status(launch_router(pa.Qc, pa.Kc, at<float>(ws, L.qr), at<float>(ws, L.kr),
+                                      at<float>(ws, L.kmean), Wq, Wk, p->smooth_k != 0, pl.BH,
+                                      pl.Tq, pl.Tkv, pl.N, 64, pl.d, s)));
+    qsrc = at<float>(ws, L.qr);
+    ksrc = at<float>(ws, L.kr);
+  }
+  SelectArgs sa;
+  sa.Qc = qsrc;
+  sa.Kc = ksrc;
+  sa.mc = mc;
+  sa.lut = lut;
+  sa.d = pl.d;
+  sa.Tq = pl.Tq;
+  sa.Tkv = pl.Tkv;
+  sa.nh = pl.nh;
+  sa.nl = pl.nl;
+  return cuda_status(launch_select(sa, pl.BH, s));
+}
+
+sla_status_t precompute_impl(const Plan& pl, const sla_params_t* p, const void* K, const void* V,
+                             const float* proj_w, void* hz, void* ws, cudaStream_t s) {
+  CUtensorMap mk, mv;
+  if (!map_bhnd(&mk, K, pl, p->stride_k, 64) || !map_bhnd(&mv, V, pl, p->stride_v, 64))
+    return SLA_ERR_CUDA;
+  KvPrepArgs a;
+  a.proj_w = (p->combine == SLA_COMBINE_PROJ) ? proj_w : nullptr;
+  a.hz = static_cast<__nv_bfloat16*>(hz);
+  a.err = at<int>(ws, layout_of(pl).err);
+  a.H = pl.H;
+  a.N = pl.N;
+  a.Tkv = pl.Tkv;
+  a.nitems = pl.BH * pl.Tkv;
+  return cuda_status(launch_kv_prep(mk, mv, a, pl.d, s));
+}
+
+sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
+                          const void* V, const int8_t* mc, const int32_t* lut, const void* hz,
+                          const float* proj_b, const float* alpha, void* O, void* ws,
+                          cudaStream_t s) {
+  const Layout L = layout_of(pl);
+  __nv_bfloat16* mm = at<__nv_bfloat16>(ws, L.mm);
+  __nv_bfloat16* hagg = at<__nv_bfloat16>(ws, L.hagg);
+  int* err = at<int>(ws, L.err);
+  SLA_TRY(cuda_status(launch_marg_matrix(mc, mm, pl.BH, pl.Tq, pl.Tkv, pl.Tkvp, s)));
+  {
+    CUtensorMap ma, mb;
+    const uint64_t da[3] = {(uint64_t)pl.Tkvp, (uint64_t)pl.Tq, (uint64_t)pl.BH};
+    const uint64_t sa[2] = {(uint64_t)pl.Tkvp * 2, (uint64_t)pl.Tq * pl.Tkvp * 2};
+    const uint32_t ba[3] = {64, 128, 1};
+    const uint64_t db[3] = {(uint64_t)pl.NN, (uint64_t)pl.Tkv, (uint64_t)pl.BH};
+    const uint64_t sb[2] = {(uint64_t)pl.NN * 2, (uint64_t)pl.Tkv * pl.NN * 2};
+    const uint32_t bb[3] = {64, 64, 1};
+    if (!encode(&ma, mm, 3, da, sa, ba) || !encode(&mb, hz, 3, db, sb, bb)) return SLA_ERR_CUDA;
+    MargArgs a;
+    a.Hout = hagg;
+    a.err = err;
+    a.Tq = pl.Tq;
+    a.Tkv = pl.Tkv;
+    a.NN = pl.NN;
+    a.ktiles = (pl.Tkv + 63) / 64;
+    SLA_TRY(cuda_status(launch_marg_gemm(ma, mb, a, pl.BH, s)));
+  }
+  CUtensorMap mq, mk, mv, mh;
+  if (!map_bhnd(&mq, Q, pl, p->stride_q, 128) || !map_bhnd(&mk, K, pl, p->stride_k, 64) ||
+      !map_bhnd(&mv, V, pl, p->stride_v, 64))
+    return SLA_ERR_CUDA;
+  {
+    const uint64_t dh[4] = {(uint64_t)pl.d, (uint64_t)pl.d, (uint64_t)pl.Tq, (uint64_t)pl.BH};
+    const uint64_t sh[3] = {(uint64_t)pl.d * 2, (uint64_t)pl.NN * 2,
+                            (uint64_t)pl.Tq * pl.NN * 2};
+    const uint32_t bxh[4] = {64, (uint32_t)pl.d, 1, 1};
+    if (!encode(&mh, hagg, 4, dh, sh, bxh)) return SLA_ERR_CUDA;
+  }
+  FusedArgs a;
+  a.lut = lut;
+  a.Hz = hagg;
+  a.proj_b = (p->combine == SLA_COMBINE_PROJ) ? proj_b : nullptr;
+  a.alpha = alpha;
+  a.O = static_cast<__nv_bfloat16*>(O);
+  a.err = err;
+  a.so0 = p->stride_o[0];
+  a.so1 = p->stride_o[1];
+  a.so2 = p->stride_o[2];
+  a.H = pl.H;
+  a.N = pl.N;
+  a.Tq = pl.Tq;
+  a.Tkv = pl.Tkv;
+  a.nh = pl.nh;
+  a.NN = pl.NN;
+  a.combine = p->combine;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)pl.d));
+  a.eps = p->eps;
+  return cuda_status(launch_fused(mq, mk, mv, mh, a, pl.d, pl.BH, s));
+}
+
+}  // namespace
+
+extern "C" {
+
+void sla_params_default(sla_params_t* p, int B, int H, int N, int d, float k_h, float k_l,
+                        int combine) {
+  if (!p) return;
+  std::memset(p, 0, sizeof(*p));
+  p->B = B;
+  p->H = H;
+  p->N = N;
+  p->d = d;
+  p->b_q = 64;
+  p->b_kv = 64;
+  p->k_h = k_h;
+  p->k_l = k_l;
+  p->combine = combine;
+  p->qk_prec = SLA_QK_BF16;
+  p->smooth_k = 0;
+  p->eps = 1e-5f;
+  const int64_t s[3] = {(int64_t)H * N * d, (int64_t)N * d, (int64_t)d};
+  for (int i = 0; i < 3; ++i) {
+    p->stride_q[i] = s[i];
+    p->stride_k[i] = s[i];
+    p->stride_v[i] = s[i];
+    p->stride_o[i] = s[i];
+  }
+}
+
+sla_status_t sla_block_counts(const sla_params_t* p, int* T_q, int* T_kv, int* n_h, int* n_l) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (T_q) *T_q = pl.Tq;
+  if (T_kv) *T_kv = pl.Tkv;
+  if (n_h) *n_h = pl.nh;
+  if (n_l) *n_l = pl.nl;
+  return SLA_OK;
+}
+
+sla_status_t sla_workspace_size(const sla_params_t* p, size_t* bytes) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!bytes) return SLA_ERR_INVALID_ARG;
+  *bytes = layout_of(pl).end;
+  return SLA_OK;
+}
+
+sla_status_t sla_hz_size(const sla_params_t* p, size_t* bytes) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!bytes) return SLA_ERR_INVALID_ARG;
+  *bytes = (size_t)pl.BH * pl.Tkv * pl.NN * 2;
+  return SLA_OK;
+}
+
+sla_status_t sla_attention_workspace_size(const sla_params_t* p, size_t* bytes) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!bytes) return SLA_ERR_INVALID_ARG;
+  *bytes = layout_of(pl).end_attn;
+  return SLA_OK;
+}
+
+sla_status_t sla_predict_mask(const sla_params_t* p, const void* Q, const void* K, const float* Wq,
+                              const float* Wk, int8_t* mc, int32_t* lut, void* workspace,
+                              size_t workspace_bytes, sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !mc || !lut || !aligned16(Q) || !aligned16(K)) return SLA_ERR_INVALID_ARG;
+  if ((Wq && !aligned16(Wq)) || (Wk && !aligned16(Wk))) return SLA_ERR_INVALID_ARG;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, false));
+  return predict_mask_impl(pl, p, Q, K, Wq, Wk, mc, lut, workspace,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+sla_status_t sla_precompute_linear(const sla_params_t* p, const void* K, const void* V,
+                                   const float* proj_w, void* hz, void* workspace,
+                                   size_t workspace_bytes, sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!K || !V || !hz || !aligned16(K) || !aligned16(V) || !aligned16(hz)) return SLA_ERR_INVALID_ARG;
+  if (proj_w && !aligned16(proj_w)) return SLA_ERR_INVALID_ARG;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, false));
+  return precompute_impl(pl, p, K, V, proj_w, hz, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                         const int8_t* mc, const int32_t* lut, const void* hz,
+                         const float* proj_b, const float* alpha, void* O, void* workspace,
+                         size_t workspace_bytes, sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !V || !mc || !lut || !hz || !O) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(hz))
+    return SLA_ERR_INVALID_ARG;
+  if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
+  if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, false));
+  return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, workspace,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+sla_status_t sla_attention(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                           const float* proj_w, const float* proj_b, const float* alpha,
+                           const float* Wq, const float* Wk, void* O, void* workspace,
+                           size_t workspace_bytes, sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !V || !O) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SLA_ERR_INVALID_ARG;
+  if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
+  if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, true));
+  const Layout L = layout_of(pl);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int8_t* mc = at<int8_t>(workspace, L.mc);
+  int32_t* lut = at<int32_t>(workspace, L.lut);
+  void* hz = at<void>(workspace, L.hz);
+  const bool alpha_mode = p->combine == SLA_COMBINE_ALPHA;
+  SLA_TRY(predict_mask_impl(pl, p, Q, K, alpha_mode ? Wq : nullptr, alpha_mode ? Wk : nullptr, mc,
+                            lut, workspace, s));
+  SLA_TRY(precompute_impl(pl, p, K, V, alpha_mode ? nullptr : proj_w, hz, workspace, s));
+  return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, workspace, s);
+}
+
+sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                          const void* O, const void* dO, void* dQ, void* dK, void* dV,
+                          void* workspace, size_t workspace_bytes, sla_stream_t stream) {
+  (void)stream;
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !V || !O || !dO || !dQ || !dK || !dV) return SLA_ERR_INVALID_ARG;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, false));
+  return SLA_ERR_UNSUPPORTED;
+}
+
+sla_status_t sla_get_device_status(void* workspace, sla_stream_t stream, int* detail) {
+  if (!workspace) return SLA_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int code = 0;
+  if (cudaMemcpyAsync(&code, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SLA_ERR_CUDA;
+  if (code != 0) {
+    if (cudaMemsetAsync(workspace, 0, sizeof(int), s) != cudaSuccess) return SLA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SLA_ERR_CUDA;
+  }
+  if (detail) *detail = code;
+  if (code == DEV_OK) return SLA_OK;
+  if (code == DEV_BAD_INDEX) return SLA_ERR_DEVICE_BAD_INDEX;
+  return SLA_ERR_DEVICE_TIMEOUT;
+}
+
+const char* sla_status_string(sla_status_t s) {
+  switch (s) {
+    case SLA_OK: return "SLA_OK";
+    case SLA_ERR_INVALID_ARG: return "SLA_ERR_INVALID_ARG";
+    case SLA_ERR_UNSUPPORTED: return "SLA_ERR_UNSUPPORTED";
+    case SLA_ERR_WORKSPACE: return "SLA_ERR_WORKSPACE";
+    case SLA_ERR_CUDA: return "SLA_ERR_CUDA";
+    case SLA_ERR_DEVICE_TIMEOUT: return "SLA_ERR_DEVICE_TIMEOUT";
+    case SLA_ERR_DEVICE_BAD_INDEX: return "SLA_ERR_DEVICE_BAD_INDEX";
+  }
+  return "SLA_ERR_UNKNOWN";
+}
+
+int sla_abi_version(void) { return 100; }
+
+}  // extern "C"

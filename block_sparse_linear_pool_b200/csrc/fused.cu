@@ -1,0 +1,441 @@
+// Fused SLA / SLA2 forward for one pair of query blocks ("SLA: Beyond
+// Sparsity in Diffusion Transformers via Fine-Tunable Sparse-Linear
+// Attention", §2 Q2 step 3-4 and Fig. 4 "Fused kernel"; "SLA2: Sparse-Linear
+// Attention with Learnable Routing and QAT", §3).
+//
+// A CTA owns 128 query rows = query blocks 2p and 2p+1 of one head, so every
+// tcgen05.mma runs at M = 128.  It walks the union of the two blocks' critical
+// lists (ascending); a key block that is critical for only one of the two
+// query blocks is masked out of the other half (its probabilities are 0).
+//
+//   warp 0      TMA producer: Q tile, then K_j/V_j per union entry, then the
+//               two aggregated [H_i^T | Z_i] tiles, through an NST-stage ring
+//   warp 1      MMA issuer:  S_k = Q K_j^T into TMEM (double-buffered),
+//               O += P_k V_j with P_k read from TMEM, and at the end
+//               phi(Q) H_i for both query blocks
+//   warps 2-5   one query row per thread: phi(Q) and phi(Q).Z at the start;
+//               online softmax with exp2 (lazy rescale of O in TMEM only when
+//               the running max grows by more than 2^8); epilogue
+//               O = O^s + O^l (+ bias)  or  alpha O^s + (1 - alpha) O^l.
+//
+// TMEM columns (512 allocated): S0 [0,64) S1 [64,128) P0 [128,160)
+// P1 [160,192) O [256,256+d) L_a [384,384+d) L_b [0,d) (L_b reuses S after
+// the last score tile has been consumed).
+#include "kernels.cuh"
+
+namespace sla {
+
+template <int D>
+struct FusedSmem {
+  static constexpr int CH = D / 64;
+  static constexpr int NST = (D == 128) ? 4 : 6;
+  static constexpr int Q_BYTES = 128 * D * 2;
+  static constexpr int KT_BYTES = 64 * D * 2;          // one K or V tile
+  static constexpr int STAGE = 2 * KT_BYTES;           // K tile then V tile (or one H tile)
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_PHI = OFF_Q + Q_BYTES;
+  static constexpr int OFF_KV = OFF_PHI + Q_BYTES;
+  static constexpr int OFF_BAR = OFF_KV + NST * STAGE;
+  static constexpr int OFF_U = OFF_BAR + 256;
+  static size_t bytes(int Tkv) { return (size_t)OFF_U + 5 * (size_t)((Tkv + 15) & ~15) + 1024; }
+};
+static_assert(2 * 64 * 128 * 2 >= 128 * 128 * 2, "an H tile must fit one ring stage");
+
+namespace {
+constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 256, COL_LA = 384, COL_LB = 0;
+constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+}  // namespace
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    sla_fused_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
+                     const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH,
+                     FusedArgs a) {
+  using L = FusedSmem<D>;
+  constexpr int NST = L::NST;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint8_t* sQ = sm + L::OFF_Q;
+  uint8_t* sPhi = sm + L::OFF_PHI;
+  uint8_t* sKV = sm + L::OFF_KV;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  uint64_t* q_full = bars + 0;
+  uint64_t* phiq_ready = bars + 1;
+  uint64_t* l_full = bars + 2;
+  uint64_t* s_full = bars + 3;     // [2]
+  uint64_t* p_ready = bars + 5;    // [2]
+  uint64_t* pv_done = bars + 7;    // [2]
+  uint64_t* kv_full = bars + 9;    // [NST]
+  uint64_t* kv_empty = kv_full + NST;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(kv_empty + NST);
+  int* s_count = reinterpret_cast<int*>(tslot + 1);
+  const int Tkvr = (a.Tkv + 15) & ~15;
+  uint8_t* fa = sm + L::OFF_U;
+  uint8_t* fb = fa + Tkvr;
+  uint8_t* uflag = fb + Tkvr;
+  uint16_t* uidx = reinterpret_cast<uint16_t*>(uflag + Tkvr);
+
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  const int p = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int ia = 2 * p, ib = 2 * p + 1;
+  const bool has_b = ib < a.Tq;
+
+  // ---------------- set-up: TMEM, barriers, union of the two critical lists
+  if (w == 1) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(phiq_ready, 128);
+    mbar_init(l_full, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_ready[x], 128);
+      mbar_init(&pv_done[x], 1);
+    }
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    fence_barrier_init();
+  }
+  for (int j = tid; j < 2 * Tkvr; j += blockDim.x) fa[j] = 0;  // fa and fb
+  __syncthreads();
+  {
+    const int32_t* la = a.lut + ((int64_t)bh * a.Tq + ia) * a.nh;
+    const int32_t* lb = a.lut + ((int64_t)bh * a.Tq + (has_b ? ib : ia)) * a.nh;
+    const int tot = has_b ? 2 * a.nh : a.nh;
+    for (int e = tid; e < tot; e += blockDim.x) {
+      const bool second = e >= a.nh;
+      const int j = second ? lb[e - a.nh] : la[e];
+      if (j < 0 || j >= a.Tkv) {
+        atomicCAS(a.err, 0, DEV_BAD_INDEX);
+        continue;
+      }
+      (second ? fb : fa)[j] = 1;
+    }
+  }
+  __syncthreads();
+  if (w == 0) {
+    int base = 0;
+    const uint32_t lt = (1u << ln) - 1u;
+    for (int j0 = 0; j0 < a.Tkv; j0 += 32) {
+      const int j = j0 + ln;
+      const uint32_t f = (j < a.Tkv) ? (uint32_t)(fa[j] | (fb[j] << 1)) : 0u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, f != 0);
+      if (f) {
+        const int pos = base + __popc(bal & lt);
+        uidx[pos] = (uint16_t)j;
+        uflag[pos] = (uint8_t)f;
+      }
+      base += __popc(bal);
+    }
+    if (ln == 0) *s_count = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int U = *s_count;
+  const uint32_t tbase = *tslot;
+
+  if (w == 0) {
+    // ---------------- TMA producer
+    if (ln == 0) {
+      tma_prefetch_desc(&mapQ);
+      tma_prefetch_desc(&mapK);
+      tma_prefetch_desc(&mapV);
+      tma_prefetch_desc(&mapH);
+      mbar_arrive_expect_tx(q_full, L::Q_BYTES);
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c) tma_load_4d(sQ + c * 16384, &mapQ, q_full, c * 64, 128 * p, h, b);
+      for (int k = 0; k < U + 2; ++k) {
+        const int s = k % NST;
+        if (k >= NST && !mbar_wait(&kv_empty[s], ((k / NST) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) break;
+        uint8_t* st = sKV + s * L::STAGE;
+        if (k < U) {
+          const int j = uidx[k];
+          mbar_arrive_expect_tx(&kv_full[s], L::STAGE);
+#pragma unroll
+          for (int c = 0; c < L::CH; ++c) {
+            tma_load_4d(st + c * 8192, &mapK, &kv_full[s], c * 64, 64 * j, h, b);
+            tma_load_4d(st + L::KT_BYTES + c * 8192, &mapV, &kv_full[s], c * 64, 64 * j, h, b);
+          }
+        } else {
+          const int i = (k == U) ? ia : (has_b ? ib : ia);
+          mbar_arrive_expect_tx(&kv_full[s], D * D * 2);
+#pragma unroll
+          for (int c = 0; c < L::CH; ++c) tma_load_4d(st + c * (D * 128), &mapH, &kv_full[s], c * 64, 0, i, bh);
+        }
+      }
+    }
+  } else if (w == 1) {
+    // ---------------- MMA issuer
+    if (ln == 0) {
+      const uint32_t id_s = idesc_bf16(128, 64, false, false);
+      const uint32_t id_pv = idesc_bf16(128, D, false, true);
+      const uint32_t id_l = idesc_bf16(128, D, false, false);
+      const uint32_t q0 = smem_u32(sQ);
+      bool ok = mbar_wait(q_full, 0, a.err, DEV_TIMEOUT_TMA);
+      auto issue_pv = [&](int kp) -> bool {
+        if (!mbar_wait(&p_ready[kp & 1], (kp >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
+        tc_fence_after();
+        const uint32_t vt = smem_u32(sKV + (kp % NST) * L::STAGE + L::KT_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t bd = sdesc_sw128(vt + kk * 2048, 8192, 1024);
+          umma_ts(tbase + COL_O, tbase + COL_P + 32 * (kp & 1) + 8 * kk, bd, id_pv,
+                  (kp > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&pv_done[kp & 1]);
+        umma_commit(&kv_empty[kp % NST]);
+        return true;
+      };
+      for (int k = 0; k < U && ok; ++k) {
+        const int s = k % NST;
+        if (!mbar_wait(&kv_full[s], (k / NST) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t kt = smem_u32(sKV + s * L::STAGE);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(q0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(kt + (kk / 4) * 8192 + (kk % 4) * 32, 16, 1024);
+          umma_ss(tbase + COL_S + 64 * (k & 1), ad, bd, id_s, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[k & 1]);
+        if (k >= 1 && !issue_pv(k - 1)) { ok = false; break; }
+      }
+      if (ok && U >= 1) ok = issue_pv(U - 1);
+      // phi(Q) H_i for both query blocks
+      if (ok) ok = mbar_wait(phiq_ready, 0, a.err, DEV_TIMEOUT_SYNC);
+      for (int t = 0; t < 2 && ok; ++t) {
+        const int k = U + t, s = k % NST;
+        if (!mbar_wait(&kv_full[s], (k / NST) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ht = smem_u32(sKV + s * L::STAGE);
+        const uint32_t ph = smem_u32(sPhi);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(ph + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(ht + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024);
+          umma_ss(tbase + (t == 0 ? COL_LA : COL_LB), ad, bd, id_l, kk > 0 ? 1u : 0u);
+        }
+      }
+      if (ok) umma_commit(l_full);
+    }
+  } else {
+    // ---------------- softmax / epilogue warps: one query row per thread
+    const int q4 = w & 3;
+    const int r = 32 * q4 + ln;
+    const int half = r >> 6;
+    const uint32_t bit = 1u << half;
+    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
+    const int i_me = (half == 0) ? ia : (has_b ? ib : ia);
+    bool ok = mbar_wait(q_full, 0, a.err, DEV_TIMEOUT_TMA);
+    // phi(q_r) -> sPhi (bf16, same swizzled layout as Q) and den = phi(q_r).Z_i
+    float den = 0.f;
+    {
+      const __nv_bfloat16* Z = a.Hz + ((int64_t)bh * a.Tq + i_me) * a.NN + D * D;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mx = fmaxf(mx, fmaxf(__low2float(p2[u]), __high2float(p2[u])));
+      }
+      constexpr float LOG2E = 1.4426950408889634f;
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          sum += exp2f((__low2float(p2[u]) - mx) * LOG2E) + exp2f((__high2float(p2[u]) - mx) * LOG2E);
+      }
+      const float inv = 1.f / sum;
+#pragma unroll 1
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+        const uint4 zv = __ldg(reinterpret_cast<const uint4*>(Z + c * 8));
+        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv);
+        uint32_t o[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float f0 = exp2f((__low2float(p2[u]) - mx) * LOG2E) * inv;
+          const float f1 = exp2f((__high2float(p2[u]) - mx) * LOG2E) * inv;
+          o[u] = pack_bf16x2(f0, f1);
+          const __nv_bfloat162 fb2 = *reinterpret_cast<__nv_bfloat162*>(&o[u]);
+          den = fmaf(__low2float(fb2), __low2float(z2[u]), den);
+          den = fmaf(__high2float(fb2), __high2float(z2[u]), den);
+        }
+        *reinterpret_cast<uint4*>(sPhi + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16)) =
+            make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(phiq_ready);
+    }
+    // online softmax over the union list
+    float m = -INFINITY, l = 0.f;
+    const float sl2 = a.scale_log2;
+    for (int k = 0; k < U && ok; ++k) {
+      const int sb = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (k >> 1) & 1, a.err, DEV_TIMEOUT_MMA))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t s0[32], s1[32];
+      tmem_ld32(tbase + lane_off + COL_S + 64 * sb, s0);
+      tmem_ld32(tbase + lane_off + COL_S + 64 * sb + 32, s1);
+      tmem_ld_wait();
+      const bool crit = (uflag[k] & bit) != 0;  // uniform over the warp
+      const int j = uidx[k];
+      const int nvalid = min(64, a.N - 64 * j);
+      float mx = -INFINITY;
+      if (crit) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          if (c < nvalid) mx = fmaxf(mx, __uint_as_float(s0[c]));
+          if (c + 32 < nvalid) mx = fmaxf(mx, __uint_as_float(s1[c]));
+        }
+        mx *= sl2;
+      }
+      // lazy rescale: keep the running max unless it grows by more than 2^8
+      const float m_new = fmaxf(m, mx);
+      const bool grow = crit && (m == -INFINITY ? false : (m_new - m > RESCALE_THRESHOLD));
+      if (crit && m == -INFINITY) m = m_new;  // O and l of this row are still exactly 0
+      if (__any_sync(0xffffffffu, grow)) {
+        // O must hold P_{k-1} V_{k-1} before it is rescaled
+        if (!__all_sync(0xffffffffu,
+                        mbar_wait(&pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, a.err, DEV_TIMEOUT_MMA))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const float f = grow ? exp2f(m - m_new) : 1.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tbase + lane_off + COL_O + c0, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+          tmem_st32(tbase + lane_off + COL_O + c0, o);
+        }
+        tmem_st_wait();
+        if (grow) {
+          l *= f;
+          m = m_new;
+        }
+      }
+      uint32_t pk[32];
+      float ls = 0.f;
+      // P row: columns 0..63 packed as bf16 pairs (column 2c in the low half)
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        const int c0 = 2 * c, c1 = 2 * c + 1;
+        const float p0 = (crit && c0 < nvalid) ? exp2f(fmaf(__uint_as_float(s0[c0]), sl2, -m)) : 0.f;
+        const float p1 = (crit && c1 < nvalid) ? exp2f(fmaf(__uint_as_float(s0[c1]), sl2, -m)) : 0.f;
+        const float p2 = (crit && c0 + 32 < nvalid) ? exp2f(fmaf(__uint_as_float(s1[c0]), sl2, -m)) : 0.f;
+        const float p3 = (crit && c1 + 32 < nvalid) ? exp2f(fmaf(__uint_as_float(s1[c1]), sl2, -m)) : 0.f;
+        ls += (p0 + p1) + (p2 + p3);
+        pk[c] = pack_bf16x2(p0, p1);
+        pk[16 + c] = pack_bf16x2(p2, p3);
+      }
+      l += ls;
+      // P_k overwrites the buffer P_{k-2} was read from
+      if (k >= 2 && !__all_sync(0xffffffffu, mbar_wait(&pv_done[sb], ((k - 2) >> 1) & 1, a.err,
+                                                          DEV_TIMEOUT_MMA))) {
+        ok = false;
+        break;
+      }
+      tmem_st32(tbase + lane_off + COL_P + 32 * sb, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_ready[sb]);
+    }
+    // ---------------- epilogue
+    if (ok && U >= 1)
+      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, DEV_TIMEOUT_MMA));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(l_full, 0, a.err, DEV_TIMEOUT_MMA));
+    if (ok) {
+      tc_fence_after();
+      const int n = 128 * p + r;
+      const bool store = (n < a.N) && (half == 0 || has_b);
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float inv_den = 1.f / (den + a.eps);
+      float wa, wl;
+      if (a.combine == 1) {
+        const float al = a.alpha[bh];
+        wa = al * inv_l;
+        wl = (1.f - al) * inv_den;
+      } else {
+        wa = inv_l;
+        wl = inv_den;
+      }
+      const uint32_t col_l = (half == 0) ? COL_LA : COL_LB;
+      __nv_bfloat16* orow = a.O + (int64_t)b * a.so0 + (int64_t)h * a.so1 + (int64_t)n * a.so2;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t os[32], ol[32];
+        tmem_ld32(tbase + lane_off + COL_O + c0, os);
+        tmem_ld32(tbase + lane_off + col_l + c0, ol);
+        tmem_ld_wait();
+        if (store) {
+          float bias[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) bias[c] = (a.combine == 0 && a.proj_b) ? __ldg(a.proj_b + c0 + c) : 0.f;
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int c = 8 * v + e;
+              y[e] = __uint_as_float(os[c]) * wa + __uint_as_float(ol[c]) * wl + bias[c];
+            }
+            dst[v] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                                pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+template <int D>
+static cudaError_t launch_fused_t(const CUtensorMap& mapQ, const CUtensorMap& mapK,
+                                  const CUtensorMap& mapV, const CUtensorMap& mapH,
+                                  const FusedArgs& a, int BH, cudaStream_t s) {
+  const size_t smem = FusedSmem<D>::bytes(a.Tkv);
+  cudaError_t e = cudaFuncSetAttribute(sla_fused_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.Tq + 1) / 2, BH);
+  sla_fused_kernel<D><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, a);
+  return cudaGetLastError();
+}
+
+size_t fused_smem_bytes(int D, int Tkv) {
+  return D == 128 ? FusedSmem<128>::bytes(Tkv) : FusedSmem<64>::bytes(Tkv);
+}
+
+cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                         const CUtensorMap& mapH, const FusedArgs& a, int D, int BH,
+                         cudaStream_t s) {
+  return D == 128 ? launch_fused_t<128>(mapQ, mapK, mapV, mapH, a, BH, s)
+                  : launch_fused_t<64>(mapQ, mapK, mapV, mapH, a, BH, s);
+}
+
+}  // namespace sla

@@ -1,0 +1,163 @@
+// Marginal aggregation ("SLA: Beyond Sparsity in Diffusion Transformers via
+// Fine-Tunable Sparse-Linear Attention", §2 Q2 step 3 and Fig. 4: for every
+// marginal block, H_i += h_j and Z_i += z_j).
+//
+// Summing the marginal h_j row by row would read n_m * d^2 values per query
+// block.  Instead all rows are formed at once as one dense product per head,
+//     [H_i^T | Z_i] = sum_j Mmarg[i][j] [h_j^T | z_j],   Mmarg = (M_c == 0),
+// a (T_q x T_kv) x (T_kv x (d^2 + d)) GEMM on the tensor cores (0/1 weights
+// are exact in bf16, accumulation in fp32).
+//
+//   marg_matrix_kernel  M_c (int8) -> Mmarg (bf16 0/1, rows padded to T_kvp)
+//   marg_gemm_kernel    128 x 256 output tile per CTA, K step 64, 4-stage
+//                       TMA ring; warp 0 loads, warp 1 issues tcgen05.mma,
+//                       warps 2-5 drain TMEM and store bf16.
+#include "kernels.cuh"
+
+namespace sla {
+
+__global__ void marg_matrix_kernel(const int8_t* __restrict__ mc, __nv_bfloat16* __restrict__ mm,
+                                   int BH, int Tq, int Tkv, int Tkvp) {
+  const int64_t total = (int64_t)BH * Tq * Tkvp;
+  const __nv_bfloat16 one = __float2bfloat16(1.f), zero = __float2bfloat16(0.f);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int j = (int)(e % Tkvp);
+    const int64_t row = e / Tkvp;  // bh * Tq + i
+    mm[e] = (j < Tkv && mc[row * Tkv + j] == 0) ? one : zero;
+  }
+}
+
+namespace {
+constexpr int BM = 128, BN = 256, BK = 64, NST = 4;
+constexpr int A_BYTES = BM * BK * 2;   // 16 KB
+constexpr int B_BYTES = BK * BN * 2;   // 32 KB
+constexpr int STAGE = A_BYTES + B_BYTES;
+constexpr int OFF_BAR = NST * STAGE;
+constexpr int SMEM = OFF_BAR + 256 + 1024;
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
+                                                           const __grid_constant__ CUtensorMap mapB,
+                                                           MargArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* empty = full + NST;
+  uint64_t* acc_bar = empty + NST;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM, bh = blockIdx.z;
+  const int nvalid_chunks = min(4, (a.NN - n0 + 63) / 64);
+
+  if (w == 1) {
+    tmem_alloc(tslot, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_bar, 1);
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tacc = *tslot;
+
+  if (w == 0) {
+    if (ln == 0) {
+      tma_prefetch_desc(&mapA);
+      tma_prefetch_desc(&mapB);
+      for (int kt = 0; kt < a.ktiles; ++kt) {
+        const int s = kt % NST;
+        if (kt >= NST && !mbar_wait(&empty[s], ((kt / NST) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) break;
+        uint8_t* sA = sm + s * STAGE;
+        uint8_t* sB = sA + A_BYTES;
+        mbar_arrive_expect_tx(&full[s], A_BYTES + nvalid_chunks * 8192);
+        tma_load_3d(sA, &mapA, &full[s], kt * BK, m0, bh);
+        for (int c = 0; c < nvalid_chunks; ++c)
+          tma_load_3d(sB + c * 8192, &mapB, &full[s], n0 + c * 64, kt * BK, bh);
+      }
+    }
+  } else if (w == 1) {
+    if (ln == 0) {
+      const uint32_t id = idesc_bf16(BM, BN, false, true);
+      bool ok = true;
+      for (int kt = 0; kt < a.ktiles; ++kt) {
+        const int s = kt % NST;
+        if (!mbar_wait(&full[s], (kt / NST) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t sA = smem_u32(sm + s * STAGE);
+        const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+        for (int k = 0; k < BK / 16; ++k) {
+          const uint64_t ad = sdesc_sw128(sA + k * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sB + k * 2048, 8192, 1024);
+          umma_ss(tacc, ad, bd, id, (kt > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      if (ok) umma_commit(acc_bar);
+    }
+  } else {
+    const int q4 = w & 3;
+    const int row = 32 * q4 + ln;
+    const int i = m0 + row;
+    const bool ok = mbar_wait(acc_bar, 0, a.err, DEV_TIMEOUT_MMA);
+    if (__all_sync(0xffffffffu, ok)) {
+      tc_fence_after();
+      const uint32_t taddr = tacc + ((uint32_t)(32 * q4) << 16);
+      __nv_bfloat16* out = a.Hout + ((int64_t)bh * a.Tq + i) * a.NN;
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c0, r);
+        tmem_ld_wait();
+        if (i < a.Tq) {
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const int n = n0 + c0 + v * 8;
+            if (n < a.NN) {
+              uint4 q;
+              q.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              q.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              q.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              q.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              *reinterpret_cast<uint4*>(out + n) = q;
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 1) {
+    tc_fence_after();
+    tmem_dealloc(tacc, 256);
+  }
+}
+
+cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int Tq, int Tkv,
+                               int Tkvp, cudaStream_t s) {
+  const int64_t total = (int64_t)BH * Tq * Tkvp;
+  const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
+  marg_matrix_kernel<<<blocks, 256, 0, s>>>(mc, mm, BH, Tq, Tkv, Tkvp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const MargArgs& a,
+                             int BH, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(marg_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.NN + BN - 1) / BN, (a.Tq + BM - 1) / BM, BH);
+  marg_gemm_kernel<<<grid, 192, SMEM, s>>>(mapA, mapB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -1,0 +1,187 @@
+/*
+ * sla.h - C ABI of the Sparse-Linear Attention (SLA / SLA2) forward on B200.
+ *
+ * Sources (cited by page title and section):
+ *   [SLA]  "SLA: Beyond Sparsity in Diffusion Transformers via Fine-Tunable
+ *          Sparse-Linear Attention": §2 Q2 (algorithm steps 1-4), §3 Fig. 4
+ *          (forward flowchart), §4 (notation table, Eq. 3-4, Eq. 6, check 5),
+ *          §7 (code cross-reference).
+ *   [SLA2] "SLA2: Sparse-Linear Attention with Learnable Routing and QAT":
+ *          §3 SLA2 Design, §4 Learnable Router, §5 Quantization-aware Training.
+ *
+ * Conventions shared by every call
+ *   - Tensors Q, K, V, O are bf16 [B, H, N, d] with the head dimension
+ *     contiguous; strides of the B, H and N dimensions are given in elements
+ *     in sla_params_t (they must be multiples of 8 elements; base pointers
+ *     16-byte aligned).
+ *   - The caller owns and allocates every device buffer, including the
+ *     workspace (size from sla_workspace_size).  The library allocates nothing
+ *     on the device and never synchronises the stream, except
+ *     sla_get_device_status which reads back the device error word.
+ *   - All compute calls are asynchronous on `stream`.  Arguments are validated
+ *     on the host before any launch; a rejected call launches nothing.
+ *   - Kernels never trap.  A wait that cannot complete within one second, or
+ *     a LUT entry out of range, is recorded in the workspace's device error
+ *     word and the kernel returns; sla_get_device_status reports it.
+ *   - T_q = ceil(N / b_q), T_kv = ceil(N / b_kv).  The last block may be
+ *     partial; its pooled mean is over its real tokens.
+ *   - Supported: d in {64, 128}, b_q = b_kv = 64, N <= 262144, B*H <= 65535.
+ */
+#ifndef SLA_H_
+#define SLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* sla_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  SLA_OK = 0,
+  SLA_ERR_INVALID_ARG = 1,   /* NULL pointer, bad size, bad stride or alignment */
+  SLA_ERR_UNSUPPORTED = 2,   /* d, block size or precision this build does not implement */
+  SLA_ERR_WORKSPACE = 3,     /* workspace NULL, too small or misaligned */
+  SLA_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (launch, encode) */
+  SLA_ERR_DEVICE_TIMEOUT = 5,/* a kernel gave up waiting (device error word) */
+  SLA_ERR_DEVICE_BAD_INDEX = 6 /* a kernel met a LUT index out of range */
+} sla_status_t;
+
+typedef enum {
+  SLA_COMBINE_PROJ = 0,  /* [SLA] Eq. 6:  O = O^s + Proj(O^l), Proj(x) = x W^T + b */
+  SLA_COMBINE_ALPHA = 1  /* [SLA2] §3:    O = alpha_h O^s + (1 - alpha_h) O^l       */
+} sla_combine_t;
+
+typedef enum {
+  SLA_QK_BF16 = 0,      /* Q K^T of critical blocks in bf16, fp32 accumulate */
+  SLA_QK_FP8_E4M3 = 1   /* [SLA2] §5: Q, K quantised to E4M3 with one scale per
+                           64-row block (max|x|/448) before Q K^T */
+} sla_qk_prec_t;
+
+typedef struct {
+  int B, H, N, d;      /* batch, heads, tokens, head dimension */
+  int b_q, b_kv;       /* query / key-value block sizes ([SLA] §4 notation: 64) */
+  float k_h;           /* critical fraction per row (top k_h%, [SLA] §2 Q2 step 2) */
+  float k_l;           /* negligible fraction per row (bottom k_l%) */
+  int combine;         /* sla_combine_t */
+  int qk_prec;         /* sla_qk_prec_t */
+  int smooth_k;        /* 1: subtract the token mean of K before mask prediction
+                          ([SLA] §7 item 3); it cannot change a row-wise ranking */
+  float eps;           /* added to the linear-branch denominator ([SLA] §4 check 5) */
+  int64_t stride_q[3]; /* element strides of Q for the B, H, N dimensions */
+  int64_t stride_k[3];
+  int64_t stride_v[3];
+  int64_t stride_o[3];
+} sla_params_t;
+
+/* Fills a params struct for contiguous [B,H,N,d] tensors, b = 64, eps = 1e-5. */
+void sla_params_default(sla_params_t* p, int B, int H, int N, int d, float k_h, float k_l,
+                        int combine);
+
+/* Block counts per row: n_h = max(1, floor(k_h*T_kv + 1e-9)),
+ * n_l = min(floor(k_l*T_kv + 1e-9), T_kv - n_h).  The pages give "top k_h%"
+ * and "bottom k_l%" per row without a rounding rule; flooring keeps at least
+ * the stated sparsity and one critical block keeps the sparse softmax defined.
+ * Any output pointer may be NULL. */
+sla_status_t sla_block_counts(const sla_params_t* p, int* T_q, int* T_kv, int* n_h, int* n_l);
+
+/* Bytes of device workspace the calls below need (the same size serves all
+ * of them, including sla_attention). */
+sla_status_t sla_workspace_size(const sla_params_t* p, size_t* bytes);
+
+/* Bytes of the caller-owned linear statistics buffer `hz`:
+ * bf16 [B*H][T_kv][d*d + d]. */
+sla_status_t sla_hz_size(const sla_params_t* p, size_t* bytes);
+
+/*
+ * Compressed mask prediction ([SLA] §2 Q2 steps 1-2, Fig. 4 left; [SLA2] §4).
+ *   Q_c = mean_pool(Q), K_c = mean_pool(K) over blocks of b_q / b_kv tokens;
+ *   SLA2 router: Q_c <- Q_c Wq^T, K_c <- K_c Wk^T (Wq, Wk fp32 [d][d],
+ *   shared by all heads, no bias; NULL = identity, which is SLA);
+ *   logits = Q_c K_c^T / sqrt(d); P_c = row softmax (monotone, so the
+ *   selection ranks logits directly).  Per row: the n_h highest blocks are
+ *   critical (1), the n_l lowest negligible (-1), the rest marginal (0); ties
+ *   rank the lower block index first.
+ * Outputs (device, caller-allocated):
+ *   mc  int8  [B*H][T_q][T_kv]   values in {1, 0, -1}
+ *   lut int32 [B*H][T_q][n_h]    critical block indices in ascending order
+ */
+sla_status_t sla_predict_mask(const sla_params_t* p, const void* Q, const void* K,
+                              const float* Wq, const float* Wk, int8_t* mc, int32_t* lut,
+                              void* workspace, size_t workspace_bytes, sla_stream_t stream);
+
+/*
+ * Per-key-block linear-attention statistics ([SLA] §2 Q2 step 3, Fig. 4
+ * "Linear Attention Precomputation"):
+ *   h_j = phi(K_j)^T V_j  (d x d),   z_j = rowsum(phi(K_j)^T)  (d),
+ * phi = softmax over the head dimension, only real tokens of a partial block.
+ * For the SLA combine, Proj's weight (fp32 [d][d], nn.Linear convention) is
+ * folded in: h_j W^T is stored, which is exact by linearity because
+ * Proj(O^l) = (phi(Q) H / den) W^T + b = phi(Q) (H W^T) / den + b.  Pass
+ * proj_w = NULL for SLA2 (or Proj = identity).
+ * Output hz (device, caller-allocated, sla_hz_size bytes): bf16
+ *   [B*H][T_kv][d*d + d]: element (b*d + a) holds (h_j W^T)[a][b] (the
+ *   transpose, row b contiguous in a), element d*d + a holds z_j[a].
+ */
+sla_status_t sla_precompute_linear(const sla_params_t* p, const void* K, const void* V,
+                                   const float* proj_w, void* hz, void* workspace,
+                                   size_t workspace_bytes, sla_stream_t stream);
+
+/*
+ * The fused forward given a mask ([SLA] §2 Q2 steps 3-4, Fig. 4 right):
+ * for every query block i
+ *   O^s_i = softmax attention over the tokens of its critical blocks (lut),
+ *           computed block by block with an online softmax;
+ *   H_i = sum of h_j, Z_i = sum of z_j over its marginal blocks (mc == 0);
+ *   O^l_i = phi(Q_i) H_i / (phi(Q_i) Z_i + eps)        ([SLA] Eq. 3-4);
+ *   negligible blocks (mc == -1) are never read;
+ *   SLA:  O = O^s + O^l W^T + proj_b  (W folded into hz; proj_b fp32 [d] or NULL)
+ *   SLA2: O = alpha[b*H+h] O^s + (1 - alpha[b*H+h]) O^l  (alpha fp32 [B*H])
+ * mc and lut must come from sla_predict_mask with the same params (or obey
+ * its contract: n_h ascending in-range indices per row, consistent with mc).
+ * O is bf16 [B,H,N,d] (strides from params).
+ */
+sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                         const int8_t* mc, const int32_t* lut, const void* hz,
+                         const float* proj_b, const float* alpha, void* O, void* workspace,
+                         size_t workspace_bytes, sla_stream_t stream);
+
+/*
+ * The whole forward in one call: sla_predict_mask, sla_precompute_linear and
+ * sla_forward, with mc, lut and hz kept in the workspace
+ * (sla_attention_workspace_size bytes).  proj_w / proj_b are used by the SLA
+ * combine, Wq / Wk / alpha by SLA2 (Wq, Wk may be NULL).
+ */
+sla_status_t sla_attention_workspace_size(const sla_params_t* p, size_t* bytes);
+sla_status_t sla_attention(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                           const float* proj_w, const float* proj_b, const float* alpha,
+                           const float* Wq, const float* Wk, void* O, void* workspace,
+                           size_t workspace_bytes, sla_stream_t stream);
+
+/*
+ * Backward of the forward above ([SLA2] App. A; [SLA] §4 check 6).  Not
+ * implemented in this build: returns SLA_ERR_UNSUPPORTED after validating
+ * its arguments.
+ */
+sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                          const void* O, const void* dO, void* dQ, void* dK, void* dV,
+                          void* workspace, size_t workspace_bytes, sla_stream_t stream);
+
+/* Reads the device error word of `workspace` (synchronises `stream`) and
+ * clears it.  Returns SLA_OK, SLA_ERR_DEVICE_TIMEOUT or
+ * SLA_ERR_DEVICE_BAD_INDEX; *detail (may be NULL) receives the raw code. */
+sla_status_t sla_get_device_status(void* workspace, sla_stream_t stream, int* detail);
+
+/* Human-readable name of a status code (static storage). */
+const char* sla_status_string(sla_status_t s);
+
+/* Version of this ABI (major * 100 + minor). */
+int sla_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SLA_H_ */

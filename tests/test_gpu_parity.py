@@ -1,0 +1,173 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Tolerances (fixed by the benchmark spec of the method's accuracy):
+  * M_c bit-exact wherever the logit gap to the top-k / bottom-k threshold
+    exceeds 1e-4 (the remaining entries must still form a valid mask);
+  * bf16 outputs within max-abs 2e-2 and mean-abs 2e-3, relative to max|O_ref|.
+The output comparison feeds the GPU's own M_c to the oracle, so a sub-1e-4
+near-tie flip cannot fail it spuriously.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from block_sparse_linear_pool_b200 import binding as bnd
+from block_sparse_linear_pool_b200 import inputs as I
+from block_sparse_linear_pool_b200.build import build
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS, MEAN_ABS, GAP = 2e-2, 2e-3, 1e-4
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    build()
+    bnd.lib()
+
+
+def _np(t):
+    return None if t is None else t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _oparams(cfg: bnd.SlaConfig):
+    return O.OracleParams(k_h=cfg.k_h, k_l=cfg.k_l, combine=cfg.combine, eps=cfg.eps,
+                          smooth_k=cfg.smooth_k)
+
+
+def _check_mask(Q, K, cfg, mc, lut, Wq=None, Wk=None):
+    """Graded entries bit-exact; every row a valid mask; LUT = critical indices ascending."""
+    p = _oparams(cfg)
+    M_ref, logits, _ = O.predict_mask(_np(Q), _np(K), p, _np(Wq), _np(Wk))
+    B, H = Q.shape[:2]
+    T = M_ref.shape[-1]
+    n_h, n_l = O.block_counts(T, cfg.k_h, cfg.k_l)
+    g = O.mask_grading(logits, n_h, n_l, GAP).reshape(B * H, T, T)
+    M_ref = M_ref.reshape(B * H, T, T)
+    m = mc.cpu().numpy()
+    assert (m == M_ref)[g].all(), f"{(m != M_ref)[g].sum()} graded mask entries differ"
+    assert ((m == 1).sum(-1) == n_h).all() and ((m == -1).sum(-1) == n_l).all()
+    l = lut.cpu().numpy()
+    crit = np.stack([np.nonzero(r == 1)[0] for r in m.reshape(-1, T)]).reshape(l.shape)
+    np.testing.assert_array_equal(l, crit)
+    return g.mean()
+
+
+def _check_out(out, ref, what=""):
+    o = _np(out)
+    mask = ~np.isnan(ref)
+    scale = np.abs(ref[mask]).max()
+    err = np.abs(o[mask] - ref[mask])
+    assert err.max() <= MAX_ABS * scale, f"{what} max-abs {err.max():.3e} > {MAX_ABS}*{scale:.3e}"
+    assert err.mean() <= MEAN_ABS * scale, f"{what} mean-abs {err.mean():.3e} > {MEAN_ABS}*{scale:.3e}"
+    return err.max() / scale, err.mean() / scale
+
+
+def _run(data, cfg, qblocks=None, heads=None):
+    dev = "cuda"
+    Q, K, V = (data[k].to(dev) for k in ("Q", "K", "V"))
+    proj_w, proj_b = data.get("proj_w"), data.get("proj_b")
+    alpha, Wq, Wk = data.get("alpha"), data.get("Wq"), data.get("Wk")
+    ws = bnd.new_workspace(bnd.sla_workspace_size(bnd.make_params(Q, cfg, K, V)), dev)
+    mc, lut = bnd.sla_predict_mask(Q, K, cfg, Wq, Wk, workspace=ws)
+    hz = bnd.sla_precompute_linear(K, V, cfg, proj_w if cfg.combine == "proj" else None, workspace=ws)
+    out = bnd.sla_forward(Q, K, V, mc, lut, hz, cfg, proj_b=proj_b, alpha=alpha, workspace=ws)
+    torch.cuda.synchronize()
+    code, detail = bnd.sla_get_device_status(ws)
+    assert code == 0, (code, detail)
+    graded = _check_mask(Q, K, cfg, mc, lut, Wq, Wk)
+    B, H, N, d = Q.shape
+    T = mc.shape[-1]
+    Mc = mc.cpu().numpy().reshape(B, H, T, T)
+    ref = O.forward_given_mask(_np(Q), _np(K), _np(V), Mc, _oparams(cfg), proj_w=_np(proj_w),
+                               proj_b=_np(proj_b), alpha=_np(alpha), qblocks=qblocks, heads=heads)
+    rel = _check_out(out, ref, "forward")
+    # the one-call entry point must give the same output bits
+    out2 = bnd.sla_attention(Q, K, V, cfg, proj_w=proj_w, proj_b=proj_b, alpha=alpha, Wq=Wq, Wk=Wk)
+    torch.cuda.synchronize()
+    assert torch.equal(out, out2)
+    return graded, rel, hz, mc
+
+
+def _small(B, H, N, d, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    T = -(-N // 64)
+    x = {}
+    for name in ("Q", "K", "V"):
+        base = torch.randn(B, H, N, d, generator=g)
+        mean = torch.randn(B, H, T, d, generator=g).repeat_interleave(64, dim=2)[:, :, :N]
+        x[name] = (base + mean * 0.7).to(torch.bfloat16)
+    x["proj_w"] = torch.randn(d, d, generator=g) * 0.05
+    x["proj_b"] = torch.randn(d, generator=g) * 0.1
+    x["alpha"] = torch.rand(B, H, generator=g) * 0.35 + 0.6
+    x["Wq"] = (torch.rand(d, d, generator=g) * 2 - 1) / d ** 0.5
+    x["Wk"] = (torch.rand(d, d, generator=g) * 2 - 1) / d ** 0.5
+    return x
+
+
+def test_tiny_sla_workload():
+    data, w = I.make_workload("tiny_sla")
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine="proj")
+    graded, rel, hz, _ = _run(data, cfg)
+    assert graded > 0.95
+    # the linear statistics themselves: (h_j W^T)^T and z_j
+    h, z = O.linear_block_stats(_np(data["K"]), _np(data["V"]), 64)
+    W = _np(data["proj_w"])
+    d = 64
+    got = hz.float().cpu().numpy().reshape(2, 16, d * d + d)
+    ref_h = np.einsum("hjab,ob->hjoa", h[0], W)
+    np.testing.assert_allclose(got[:, :, :d * d].reshape(2, 16, d, d), ref_h,
+                               atol=1e-2 * np.abs(ref_h).max())
+    np.testing.assert_allclose(got[:, :, d * d:], z[0], atol=1e-2 * np.abs(z).max())
+
+
+@pytest.mark.parametrize("B,H,N,d,kh,kl,combine", [
+    (1, 2, 1024, 64, 0.10, 0.60, "alpha"),
+    (1, 1, 1000, 64, 0.10, 0.50, "proj"),     # ragged tail (40 tokens)
+    (2, 1, 130, 128, 0.34, 0.33, "proj"),     # 3 blocks, tail of 2 tokens, B > 1
+    (1, 3, 2049, 128, 0.05, 0.70, "alpha"),   # tail of 1 token, odd T_q (33)
+    (1, 1, 640, 128, 1.0, 0.0, "proj"),       # k_h = 100%: dense attention
+    (1, 2, 768, 64, 0.25, 0.75, "alpha"),     # no marginal blocks: block-sparse attention
+    (1, 1, 4096, 128, 0.0, 0.0, "proj"),      # n_h = 1, everything else marginal
+    (1, 2, 3000, 128, 0.10, 0.40, "proj"),
+])
+def test_small_shapes(B, H, N, d, kh, kl, combine):
+    data = _small(B, H, N, d, seed=N + d)
+    cfg = bnd.SlaConfig(k_h=kh, k_l=kl, combine=combine)
+    if combine == "proj":
+        data["Wq"] = data["Wk"] = None
+    _run(data, cfg)
+
+
+def test_smooth_k_changes_nothing_graded():
+    data = _small(1, 2, 2048, 128, seed=3)
+    data["K"] = (data["K"].float() + 2.0).to(torch.bfloat16)
+    cfg = bnd.SlaConfig(k_h=0.1, k_l=0.5, combine="proj", smooth_k=True)
+    data["Wq"] = data["Wk"] = None
+    _run(data, cfg)
+
+
+@pytest.fixture(scope="module")
+def wan13():
+    return I.make_workload("wan1.3b_sla")
+
+
+def test_wan13b_sla_full_size_sampled(wan13):
+    data, w = wan13
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine="proj")
+    # every mask row is checked; outputs on sampled query blocks incl. the partial last one
+    qb = [0, 1, 100, 255, 256, 300, 510, 511]
+    _run(data, cfg, qblocks=qb, heads=[(0, 0), (0, 7), (0, 11)])
+
+
+def test_wan13b_sla2_full_size_sampled():
+    data, w = I.make_workload("wan1.3b_sla2")
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine="alpha")
+    _run(data, cfg, qblocks=[0, 37, 200, 511], heads=[(0, 0), (0, 5)])
+
+
+def test_wan14b_720p_sla2_full_size_sampled():
+    data, w = I.make_workload("wan14b_720p_sla2")
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine="alpha")
+    _run(data, cfg, qblocks=[0, 590, 1181], heads=[(0, 0), (0, 39)])
