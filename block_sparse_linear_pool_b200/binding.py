@@ -30,8 +30,9 @@ STATUS = {
 EXPORTS = (
     "sla_params_default", "sla_block_counts", "sla_workspace_size", "sla_hz_size",
     "sla_predict_mask", "sla_precompute_linear", "sla_forward", "sla_attention_workspace_size",
-    "sla_attention", "sla_backward", "sla_get_device_status", "sla_status_string",
-    "sla_abi_version",
+    "sla_attention", "sla_aggregate_marginal", "sla_fused_forward",
+    "sla_attention_host_workspace_size", "sla_attention_host", "sla_backward",
+    "sla_get_device_status", "sla_status_string", "sla_abi_version",
 )
 
 
@@ -70,12 +71,16 @@ def lib() -> ctypes.CDLL:
         L.sla_params_default.restype = None
         ip = ctypes.POINTER(ctypes.c_int)
         L.sla_block_counts.argtypes = [P, ip, ip, ip, ip]
-        for f in ("sla_workspace_size", "sla_hz_size", "sla_attention_workspace_size"):
+        for f in ("sla_workspace_size", "sla_hz_size", "sla_attention_workspace_size",
+                  "sla_attention_host_workspace_size"):
             getattr(L, f).argtypes = [P, ctypes.POINTER(sz)]
         L.sla_predict_mask.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_precompute_linear.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
         L.sla_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_attention.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_aggregate_marginal.argtypes = [P, vp, vp, vp, sz, vp]
+        L.sla_fused_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_attention_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_get_device_status.argtypes = [vp, vp, ip]
         L.sla_status_string.argtypes = [ctypes.c_int]
@@ -218,6 +223,34 @@ def sla_attention(Q, K, V, cfg: SlaConfig, proj_w=None, proj_b=None, alpha=None,
     _check(lib().sla_attention(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), *[_ptr(x) for x in args],
                                _ptr(O), _ptr(ws), ws.numel(), _stream()), "sla_attention")
     return O
+
+
+def sla_attention_host_workspace_size(p: sla_params_t) -> int:
+    return _size("sla_attention_host_workspace_size", p)
+
+
+def sla_aggregate_marginal(p: sla_params_t, mc, hz, workspace):
+    """[H_i^T | Z_i] of every query block into `workspace` (first half of sla_forward)."""
+    _check(lib().sla_aggregate_marginal(ctypes.byref(p), _ptr(mc), _ptr(hz), _ptr(workspace),
+                                        workspace.numel(), _stream()), "sla_aggregate_marginal")
+
+
+def sla_fused_forward(p: sla_params_t, Q, K, V, lut, O, workspace, proj_b=None, alpha=None):
+    """The fused kernel (second half of sla_forward); proj_b / alpha fp32 on the device."""
+    _check(lib().sla_fused_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(lut), _ptr(proj_b),
+                                   _ptr(alpha), _ptr(O), _ptr(workspace), workspace.numel(), _stream()),
+           "sla_fused_forward")
+
+
+def sla_attention_host(p: sla_params_t, Qh, Kh, Vh, Oh, workspace, proj_w=None, proj_b=None,
+                       alpha=None, Wq=None, Wk=None):
+    """Host-memory activations (pinned CPU tensors); parameters are device tensors."""
+    for t in (Qh, Kh, Vh, Oh):
+        if t.is_cuda or not t.is_contiguous():
+            raise ValueError("host variant takes contiguous CPU tensors")
+    _check(lib().sla_attention_host(ctypes.byref(p), _ptr(Qh), _ptr(Kh), _ptr(Vh), _ptr(proj_w),
+                                    _ptr(proj_b), _ptr(alpha), _ptr(Wq), _ptr(Wk), _ptr(Oh),
+                                    _ptr(workspace), workspace.numel(), _stream()), "sla_attention_host")
 
 
 def sla_get_device_status(workspace) -> int:

@@ -27,6 +27,7 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 struct Layout {
   size_t err, qc, kc, qr, kr, kmean, mm, hagg, end;       // sla_workspace_size
   size_t mc, lut, hz, end_attn;                           // + sla_attention extras
+  size_t hq, hk, hv, ho, end_host;                        // + sla_attention_host staging
 };
 
 Layout layout_of(const Plan& p) {
@@ -45,6 +46,12 @@ Layout layout_of(const Plan& p) {
   L.lut = o;   o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
   L.hz = o;    o = align_up(o + (size_t)p.BH * p.Tkv * p.NN * 2);
   L.end_attn = o;
+  const size_t act = (size_t)p.BH * p.N * p.d * 2;
+  L.hq = o;    o = align_up(o + act);
+  L.hk = o;    o = align_up(o + act);
+  L.hv = o;    o = align_up(o + act);
+  L.ho = o;    o = align_up(o + act);
+  L.end_host = o;
   return L;
 }
 
@@ -143,10 +150,13 @@ sla_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SLA_OK : SLA
     if (st_ != SLA_OK) return st_;      \
   } while (0)
 
-sla_status_t check_ws(const Plan& p, void* ws, size_t bytes, bool attn) {
+enum WsKind { WS_BASE, WS_ATTN, WS_HOST };
+
+sla_status_t check_ws(const Plan& p, void* ws, size_t bytes, WsKind kind) {
   const Layout L = layout_of(p);
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return SLA_ERR_WORKSPACE;
-  if (bytes < (attn ? L.end_attn : L.end)) return SLA_ERR_WORKSPACE;
+  const size_t need = kind == WS_BASE ? L.end : (kind == WS_ATTN ? L.end_attn : L.end_host);
+  if (bytes < need) return SLA_ERR_WORKSPACE;
   return SLA_OK;
 }
 
@@ -211,33 +221,34 @@ sla_status_t precompute_impl(const Plan& pl, const sla_params_t* p, const void* 
   return cuda_status(launch_kv_prep(mk, mv, a, pl.d, s));
 }
 
-sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
-                          const void* V, const int8_t* mc, const int32_t* lut, const void* hz,
-                          const float* proj_b, const float* alpha, void* O, void* ws,
-                          cudaStream_t s) {
+sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, void* ws,
+                            cudaStream_t s) {
   const Layout L = layout_of(pl);
   __nv_bfloat16* mm = at<__nv_bfloat16>(ws, L.mm);
-  __nv_bfloat16* hagg = at<__nv_bfloat16>(ws, L.hagg);
-  int* err = at<int>(ws, L.err);
   SLA_TRY(cuda_status(launch_marg_matrix(mc, mm, pl.BH, pl.Tq, pl.Tkv, pl.Tkvp, s)));
-  {
-    CUtensorMap ma, mb;
-    const uint64_t da[3] = {(uint64_t)pl.Tkvp, (uint64_t)pl.Tq, (uint64_t)pl.BH};
-    const uint64_t sa[2] = {(uint64_t)pl.Tkvp * 2, (uint64_t)pl.Tq * pl.Tkvp * 2};
-    const uint32_t ba[3] = {64, 128, 1};
-    const uint64_t db[3] = {(uint64_t)pl.NN, (uint64_t)pl.Tkv, (uint64_t)pl.BH};
-    const uint64_t sb[2] = {(uint64_t)pl.NN * 2, (uint64_t)pl.Tkv * pl.NN * 2};
-    const uint32_t bb[3] = {64, 64, 1};
-    if (!encode(&ma, mm, 3, da, sa, ba) || !encode(&mb, hz, 3, db, sb, bb)) return SLA_ERR_CUDA;
-    MargArgs a;
-    a.Hout = hagg;
-    a.err = err;
-    a.Tq = pl.Tq;
-    a.Tkv = pl.Tkv;
-    a.NN = pl.NN;
-    a.ktiles = (pl.Tkv + 63) / 64;
-    SLA_TRY(cuda_status(launch_marg_gemm(ma, mb, a, pl.BH, s)));
-  }
+  CUtensorMap ma, mb;
+  const uint64_t da[3] = {(uint64_t)pl.Tkvp, (uint64_t)pl.Tq, (uint64_t)pl.BH};
+  const uint64_t sa[2] = {(uint64_t)pl.Tkvp * 2, (uint64_t)pl.Tq * pl.Tkvp * 2};
+  const uint32_t ba[3] = {64, 128, 1};
+  const uint64_t db[3] = {(uint64_t)pl.NN, (uint64_t)pl.Tkv, (uint64_t)pl.BH};
+  const uint64_t sb[2] = {(uint64_t)pl.NN * 2, (uint64_t)pl.Tkv * pl.NN * 2};
+  const uint32_t bb[3] = {64, 64, 1};
+  if (!encode(&ma, mm, 3, da, sa, ba) || !encode(&mb, hz, 3, db, sb, bb)) return SLA_ERR_CUDA;
+  MargArgs a;
+  a.Hout = at<__nv_bfloat16>(ws, L.hagg);
+  a.err = at<int>(ws, L.err);
+  a.Tq = pl.Tq;
+  a.Tkv = pl.Tkv;
+  a.NN = pl.NN;
+  a.ktiles = (pl.Tkv + 63) / 64;
+  return cuda_status(launch_marg_gemm(ma, mb, a, pl.BH, s));
+}
+
+sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
+                        const void* V, const int32_t* lut, const float* proj_b, const float* alpha,
+                        void* O, void* ws, cudaStream_t s) {
+  const Layout L = layout_of(pl);
+  __nv_bfloat16* hagg = at<__nv_bfloat16>(ws, L.hagg);
   CUtensorMap mq, mk, mv, mh;
   if (!map_bhnd(&mq, Q, pl, p->stride_q, 128) || !map_bhnd(&mk, K, pl, p->stride_k, 64) ||
       !map_bhnd(&mv, V, pl, p->stride_v, 64))
@@ -255,7 +266,7 @@ sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, 
   a.proj_b = (p->combine == SLA_COMBINE_PROJ) ? proj_b : nullptr;
   a.alpha = alpha;
   a.O = static_cast<__nv_bfloat16*>(O);
-  a.err = err;
+  a.err = at<int>(ws, L.err);
   a.so0 = p->stride_o[0];
   a.so1 = p->stride_o[1];
   a.so2 = p->stride_o[2];
@@ -269,6 +280,38 @@ sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, 
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)pl.d));
   a.eps = p->eps;
   return cuda_status(launch_fused(mq, mk, mv, mh, a, pl.d, pl.BH, s));
+}
+
+sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
+                          const void* V, const int8_t* mc, const int32_t* lut, const void* hz,
+                          const float* proj_b, const float* alpha, void* O, void* ws,
+                          cudaStream_t s) {
+  SLA_TRY(aggregate_impl(pl, mc, hz, ws, s));
+  return fused_impl(pl, p, Q, K, V, lut, proj_b, alpha, O, ws, s);
+}
+
+bool contiguous(const sla_params_t* p) {
+  const int64_t s[3] = {(int64_t)p->H * p->N * p->d, (int64_t)p->N * p->d, (int64_t)p->d};
+  for (int i = 0; i < 3; ++i)
+    if (p->stride_q[i] != s[i] || p->stride_k[i] != s[i] || p->stride_v[i] != s[i] ||
+        p->stride_o[i] != s[i])
+      return false;
+  return true;
+}
+
+sla_status_t attention_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
+                            const void* V, const float* proj_w, const float* proj_b,
+                            const float* alpha, const float* Wq, const float* Wk, void* O,
+                            void* ws, cudaStream_t s) {
+  const Layout L = layout_of(pl);
+  int8_t* mc = at<int8_t>(ws, L.mc);
+  int32_t* lut = at<int32_t>(ws, L.lut);
+  void* hz = at<void>(ws, L.hz);
+  const bool alpha_mode = p->combine == SLA_COMBINE_ALPHA;
+  SLA_TRY(predict_mask_impl(pl, p, Q, K, alpha_mode ? Wq : nullptr, alpha_mode ? Wk : nullptr, mc,
+                            lut, ws, s));
+  SLA_TRY(precompute_impl(pl, p, K, V, alpha_mode ? nullptr : proj_w, hz, ws, s));
+  return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, ws, s);
 }
 
 }  // namespace
@@ -341,7 +384,7 @@ sla_status_t sla_predict_mask(const sla_params_t* p, const void* Q, const void* 
   SLA_TRY(make_plan(p, &pl));
   if (!Q || !K || !mc || !lut || !aligned16(Q) || !aligned16(K)) return SLA_ERR_INVALID_ARG;
   if ((Wq && !aligned16(Wq)) || (Wk && !aligned16(Wk))) return SLA_ERR_INVALID_ARG;
-  SLA_TRY(check_ws(pl, workspace, workspace_bytes, false));
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
   return predict_mask_impl(pl, p, Q, K, Wq, Wk, mc, lut, workspace,
                            reinterpret_cast<cudaStream_t>(stream));
 }
@@ -353,7 +396,7 @@ sla_status_t sla_precompute_linear(const sla_params_t* p, const void* K, const v
   SLA_TRY(make_plan(p, &pl));
   if (!K || !V || !hz || !aligned16(K) || !aligned16(V) || !aligned16(hz)) return SLA_ERR_INVALID_ARG;
   if (proj_w && !aligned16(proj_w)) return SLA_ERR_INVALID_ARG;
-  SLA_TRY(check_ws(pl, workspace, workspace_bytes, false));
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
   return precompute_impl(pl, p, K, V, proj_w, hz, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -368,7 +411,7 @@ sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, co
     return SLA_ERR_INVALID_ARG;
   if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
   if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
-  SLA_TRY(check_ws(pl, workspace, workspace_bytes, false));
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
   return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, workspace,
                       reinterpret_cast<cudaStream_t>(stream));
 }
@@ -383,17 +426,67 @@ sla_status_t sla_attention(const sla_params_t* p, const void* Q, const void* K, 
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SLA_ERR_INVALID_ARG;
   if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
   if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
-  SLA_TRY(check_ws(pl, workspace, workspace_bytes, true));
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_ATTN));
+  return attention_impl(pl, p, Q, K, V, proj_w, proj_b, alpha, Wq, Wk, O, workspace,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+sla_status_t sla_attention_host_workspace_size(const sla_params_t* p, size_t* bytes) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!bytes) return SLA_ERR_INVALID_ARG;
+  *bytes = layout_of(pl).end_host;
+  return SLA_OK;
+}
+
+sla_status_t sla_attention_host(const sla_params_t* p, const void* Q_host, const void* K_host,
+                                const void* V_host, const float* proj_w, const float* proj_b,
+                                const float* alpha, const float* Wq, const float* Wk,
+                                void* O_host, void* workspace, size_t workspace_bytes,
+                                sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q_host || !K_host || !V_host || !O_host) return SLA_ERR_INVALID_ARG;
+  if (!contiguous(p)) return SLA_ERR_INVALID_ARG;
+  if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
+  if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_HOST));
   const Layout L = layout_of(pl);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int8_t* mc = at<int8_t>(workspace, L.mc);
-  int32_t* lut = at<int32_t>(workspace, L.lut);
-  void* hz = at<void>(workspace, L.hz);
-  const bool alpha_mode = p->combine == SLA_COMBINE_ALPHA;
-  SLA_TRY(predict_mask_impl(pl, p, Q, K, alpha_mode ? Wq : nullptr, alpha_mode ? Wk : nullptr, mc,
-                            lut, workspace, s));
-  SLA_TRY(precompute_impl(pl, p, K, V, alpha_mode ? nullptr : proj_w, hz, workspace, s));
-  return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, workspace, s);
+  const size_t act = (size_t)pl.BH * pl.N * pl.d * 2;
+  void* dq = at<void>(workspace, L.hq);
+  void* dk = at<void>(workspace, L.hk);
+  void* dv = at<void>(workspace, L.hv);
+  void* dout = at<void>(workspace, L.ho);
+  SLA_TRY(cuda_status(cudaMemcpyAsync(dq, Q_host, act, cudaMemcpyHostToDevice, s)));
+  SLA_TRY(cuda_status(cudaMemcpyAsync(dk, K_host, act, cudaMemcpyHostToDevice, s)));
+  SLA_TRY(cuda_status(cudaMemcpyAsync(dv, V_host, act, cudaMemcpyHostToDevice, s)));
+  SLA_TRY(attention_impl(pl, p, dq, dk, dv, proj_w, proj_b, alpha, Wq, Wk, dout, workspace, s));
+  return cuda_status(cudaMemcpyAsync(O_host, dout, act, cudaMemcpyDeviceToHost, s));
+}
+
+sla_status_t sla_aggregate_marginal(const sla_params_t* p, const int8_t* mc, const void* hz,
+                                    void* workspace, size_t workspace_bytes, sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!mc || !hz || !aligned16(hz)) return SLA_ERR_INVALID_ARG;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
+  return aggregate_impl(pl, mc, hz, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sla_status_t sla_fused_forward(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                               const int32_t* lut, const float* proj_b, const float* alpha,
+                               void* O, void* workspace, size_t workspace_bytes,
+                               sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !V || !lut || !O) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SLA_ERR_INVALID_ARG;
+  if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
+  if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
+  return fused_impl(pl, p, Q, K, V, lut, proj_b, alpha, O, workspace,
+                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, const void* V,
@@ -403,7 +496,7 @@ sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, c
   Plan pl;
   SLA_TRY(make_plan(p, &pl));
   if (!Q || !K || !V || !O || !dO || !dQ || !dK || !dV) return SLA_ERR_INVALID_ARG;
-  SLA_TRY(check_ws(pl, workspace, workspace_bytes, false));
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
   return SLA_ERR_UNSUPPORTED;
 }
 

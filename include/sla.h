@@ -149,6 +149,28 @@ sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, co
                          size_t workspace_bytes, sla_stream_t stream);
 
 /*
+ * The two halves of sla_forward, for callers that schedule or time them
+ * separately (sla_forward is exactly sla_aggregate_marginal followed by
+ * sla_fused_forward on the same stream and workspace).
+ *
+ * sla_aggregate_marginal: for every query block i, [H_i^T | Z_i] = sum over
+ * its marginal blocks (mc == 0) of [h_j^T | z_j] ([SLA] §2 Q2 step 3,
+ * "H_i += h_j, Z_i += z_j"), computed as one 0/1-matrix product per head on
+ * the tensor cores; the result stays in the workspace.
+ *
+ * sla_fused_forward: the per-query-block kernel (sparse branch over the
+ * critical blocks of lut, linear branch from the workspace's [H_i^T | Z_i],
+ * combine), writing O.  Requires a preceding sla_aggregate_marginal on the
+ * same workspace.
+ */
+sla_status_t sla_aggregate_marginal(const sla_params_t* p, const int8_t* mc, const void* hz,
+                                    void* workspace, size_t workspace_bytes, sla_stream_t stream);
+sla_status_t sla_fused_forward(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                               const int32_t* lut, const float* proj_b, const float* alpha,
+                               void* O, void* workspace, size_t workspace_bytes,
+                               sla_stream_t stream);
+
+/*
  * The whole forward in one call: sla_predict_mask, sla_precompute_linear and
  * sla_forward, with mc, lut and hz kept in the workspace
  * (sla_attention_workspace_size bytes).  proj_w / proj_b are used by the SLA
@@ -159,6 +181,22 @@ sla_status_t sla_attention(const sla_params_t* p, const void* Q, const void* K, 
                            const float* proj_w, const float* proj_b, const float* alpha,
                            const float* Wq, const float* Wk, void* O, void* workspace,
                            size_t workspace_bytes, sla_stream_t stream);
+
+/*
+ * sla_attention with the activations in host memory: copies Q, K, V (host,
+ * contiguous [B,H,N,d] bf16; page-locked memory makes the copies
+ * asynchronous) into device staging buffers inside the workspace, runs
+ * sla_attention and copies O back to O_host, all enqueued on `stream`.  The
+ * parameters proj_w, proj_b, alpha, Wq, Wk stay device pointers.  The call
+ * returns after enqueueing; O_host is valid once the stream has been
+ * synchronised.  The params' strides must describe contiguous tensors.
+ */
+sla_status_t sla_attention_host_workspace_size(const sla_params_t* p, size_t* bytes);
+sla_status_t sla_attention_host(const sla_params_t* p, const void* Q_host, const void* K_host,
+                                const void* V_host, const float* proj_w, const float* proj_b,
+                                const float* alpha, const float* Wq, const float* Wk,
+                                void* O_host, void* workspace, size_t workspace_bytes,
+                                sla_stream_t stream);
 
 /*
  * Backward of the forward above ([SLA2] App. A; [SLA] §4 check 6).  Not

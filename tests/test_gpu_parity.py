@@ -171,3 +171,43 @@ def test_wan14b_720p_sla2_full_size_sampled():
     data, w = I.make_workload("wan14b_720p_sla2")
     cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine="alpha")
     _run(data, cfg, qblocks=[0, 590, 1181], heads=[(0, 0), (0, 39)])
+
+
+def test_split_entry_points_and_host_buffers_match_forward():
+    data = _small(1, 2, 2000, 128, seed=11)
+    cfg = bnd.SlaConfig(k_h=0.1, k_l=0.5, combine="proj")
+    dev = "cuda"
+    Q, K, V = (data[k].to(dev) for k in ("Q", "K", "V"))
+    pw, pb = data["proj_w"].to(dev), data["proj_b"].to(dev)
+    ref = bnd.sla_attention(Q, K, V, cfg, proj_w=pw, proj_b=pb)
+    # predict / precompute / aggregate / fused, one call each
+    p = bnd.make_params(Q, cfg, K, V, Q)
+    ws = bnd.new_workspace(bnd.sla_workspace_size(p), dev)
+    mc, lut = bnd.sla_predict_mask(Q, K, cfg, workspace=ws)
+    hz = bnd.sla_precompute_linear(K, V, cfg, pw, workspace=ws)
+    bnd.sla_aggregate_marginal(p, mc, hz, ws)
+    O2 = torch.empty_like(Q)
+    bnd.sla_fused_forward(p, Q, K, V, lut, O2, ws, proj_b=pb.float())
+    # host-buffer variant
+    Qh, Kh, Vh = (t.cpu().pin_memory() for t in (Q, K, V))
+    Oh = torch.empty_like(Qh).pin_memory()
+    ph = bnd.make_params(Qh, cfg, Kh, Vh, Oh)
+    wsh = bnd.new_workspace(bnd.sla_attention_host_workspace_size(ph), dev)
+    bnd.sla_attention_host(ph, Qh, Kh, Vh, Oh, wsh, pw.float(), pb.float())
+    torch.cuda.synchronize()
+    assert torch.equal(O2, ref)
+    assert torch.equal(Oh, ref.cpu())
+    assert bnd.sla_get_device_status(ws)[0] == 0 and bnd.sla_get_device_status(wsh)[0] == 0
+
+
+def test_strided_views_are_honoured():
+    # Q, K, V as views of one [B, N, 3, H, d] buffer (strides != contiguous)
+    B, H, N, d = 1, 2, 1500, 128
+    g = torch.Generator().manual_seed(5)
+    qkv = torch.randn(B, N, 3, H, d, generator=g).to(torch.bfloat16).cuda()
+    Q, K, V = (qkv[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    cfg = bnd.SlaConfig(k_h=0.1, k_l=0.5, combine="proj")
+    out = bnd.sla_attention(Q, K, V, cfg)
+    ref = bnd.sla_attention(Q.contiguous(), K.contiguous(), V.contiguous(), cfg)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
