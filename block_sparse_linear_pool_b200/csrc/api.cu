@@ -114,10 +114,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return fn;
 }
 
-// rank-r bf16 tiled map, 128-byte swizzle; dims/strides innermost first,
+// rank-r bf16 tiled map, 128-byte swizzle (or none); dims/strides innermost first,
 // strides in bytes for dims 1..r-1.
 bool encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-            const uint64_t* strides, const uint32_t* box) {
+            const uint64_t* strides, const uint32_t* box, bool swizzle = true) {
   auto fn = encoder();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -129,7 +129,8 @@ bool encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -249,16 +250,21 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
                         void* O, void* ws, cudaStream_t s) {
   const Layout L = layout_of(pl);
   __nv_bfloat16* hagg = at<__nv_bfloat16>(ws, L.hagg);
-  CUtensorMap mq, mk, mv, mh;
+  CUtensorMap mq, mk, mv, mh, mz;
   if (!map_bhnd(&mq, Q, pl, p->stride_q, 128) || !map_bhnd(&mk, K, pl, p->stride_k, 64) ||
       !map_bhnd(&mv, V, pl, p->stride_v, 64))
     return SLA_ERR_CUDA;
   {
+    // H_i^T as (a, b, i, bh) tiles of d x d; Z_i as one unswizzled row of d
     const uint64_t dh[4] = {(uint64_t)pl.d, (uint64_t)pl.d, (uint64_t)pl.Tq, (uint64_t)pl.BH};
     const uint64_t sh[3] = {(uint64_t)pl.d * 2, (uint64_t)pl.NN * 2,
                             (uint64_t)pl.Tq * pl.NN * 2};
     const uint32_t bxh[4] = {64, (uint32_t)pl.d, 1, 1};
     if (!encode(&mh, hagg, 4, dh, sh, bxh)) return SLA_ERR_CUDA;
+    const uint64_t dz[3] = {(uint64_t)pl.NN, (uint64_t)pl.Tq, (uint64_t)pl.BH};
+    const uint64_t sz[2] = {(uint64_t)pl.NN * 2, (uint64_t)pl.Tq * pl.NN * 2};
+    const uint32_t bxz[3] = {64, 1, 1};
+    if (!encode(&mz, hagg, 3, dz, sz, bxz, false)) return SLA_ERR_CUDA;
   }
   FusedArgs a;
   a.lut = lut;
@@ -279,7 +285,7 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.combine = p->combine;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)pl.d));
   a.eps = p->eps;
-  return cuda_status(launch_fused(mq, mk, mv, mh, a, pl.d, pl.BH, s));
+  return cuda_status(launch_fused(mq, mk, mv, mh, mz, a, pl.d, pl.BH, s));
 }
 
 sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,

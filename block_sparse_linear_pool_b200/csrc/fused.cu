@@ -1,6 +1,6 @@
 // Fused SLA / SLA2 forward for one pair of query blocks ("SLA: Beyond
 // Sparsity in Diffusion Transformers via Fine-Tunable Sparse-Linear
-// Attention", §2 Q2 step 3-4 and Fig. 4 "Fused kernel"; "SLA2: Sparse-Linear
+// Attention", §2 Q2 steps 3-4 and Fig. 4 "Fused kernel"; "SLA2: Sparse-Linear
 // Attention with Learnable Routing and QAT", §3).
 //
 // A CTA owns 128 query rows = query blocks 2p and 2p+1 of one head, so every
@@ -8,19 +8,28 @@
 // lists (ascending); a key block that is critical for only one of the two
 // query blocks is masked out of the other half (its probabilities are 0).
 //
-//   warp 0      TMA producer: Q tile, then K_j/V_j per union entry, then the
-//               two aggregated [H_i^T | Z_i] tiles, through an NST-stage ring
-//   warp 1      MMA issuer:  S_k = Q K_j^T into TMEM (double-buffered),
-//               O += P_k V_j with P_k read from TMEM, and at the end
-//               phi(Q) H_i for both query blocks
-//   warps 2-5   one query row per thread: phi(Q) and phi(Q).Z at the start;
-//               online softmax with exp2 (lazy rescale of O in TMEM only when
-//               the running max grows by more than 2^8); epilogue
-//               O = O^s + O^l (+ bias)  or  alpha O^s + (1 - alpha) O^l.
+//   warp 0      TMA producer: Q tile, K_j/V_j per union entry, then the two
+//               aggregated H_i^T tiles and Z_i rows, through an NST-stage ring
+//   warp 1      MMA issuer: S_k = Q K_j^T into TMEM (two buffers), O += P_k V_j
+//               with P_k read back from TMEM, and at the end
+//               L = phi~(Q) H_i^T for both query blocks
+//   warps 2-5   one query row per thread: online softmax with exp2 (lazy
+//               rescale of O in TMEM only when the running max grows by more
+//               than 2^8), P_k written over S_k; after the loop phi~(Q)
+//               (unnormalised softmax of q over d) in place of Q, then the
+//               combine  O = O^s + O^l (+ bias)  or  a O^s + (1 - a) O^l.
 //
-// TMEM columns (512 allocated): S0 [0,64) S1 [64,128) P0 [128,160)
-// P1 [160,192) O [256,256+d) L_a [384,384+d) L_b [0,d) (L_b reuses S after
-// the last score tile has been consumed).
+// Resources are sized for two co-resident CTAs per SM (256 TMEM columns,
+// about 100 KB of shared memory), so one CTA's softmax, prologue and epilogue
+// overlap the other CTA's tensor-core work.
+//
+// TMEM columns: S0 [0,64) (P0 over its first 32 columns), S1 [64,128) (P1),
+// O [128,128+d).  After the last P V the S/P region [0,d) holds L_a; once the
+// rows of query block 2p have been written out it holds L_b.
+//
+// Linear branch with unnormalised feature map: for e_a = 2^((q_a - max q) log2 e)
+// and s = sum_a e_a, phi(q) = e / s, so
+//     phi(q) H / (phi(q) Z + eps) = (e H) / (e Z + s eps)      exactly.
 #include "kernels.cuh"
 
 namespace sla {
@@ -28,45 +37,54 @@ namespace sla {
 template <int D>
 struct FusedSmem {
   static constexpr int CH = D / 64;
-  static constexpr int NST = (D == 128) ? 4 : 6;
+  static constexpr int NST = (D == 128) ? 2 : 4;
   static constexpr int Q_BYTES = 128 * D * 2;
   static constexpr int KT_BYTES = 64 * D * 2;          // one K or V tile
   static constexpr int STAGE = 2 * KT_BYTES;           // K tile then V tile (or one H tile)
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_PHI = OFF_Q + Q_BYTES;
-  static constexpr int OFF_KV = OFF_PHI + Q_BYTES;
-  static constexpr int OFF_BAR = OFF_KV + NST * STAGE;
+  static constexpr int OFF_KV = OFF_Q + Q_BYTES;
+  static constexpr int OFF_Z = OFF_KV + NST * STAGE;   // Z_a, Z_b: 2 x D bf16 (unswizzled rows)
+  static constexpr int OFF_BAR = OFF_Z + 2 * CH * 128;
   static constexpr int OFF_U = OFF_BAR + 256;
   static size_t bytes(int Tkv) { return (size_t)OFF_U + 5 * (size_t)((Tkv + 15) & ~15) + 1024; }
 };
 static_assert(2 * 64 * 128 * 2 >= 128 * 128 * 2, "an H tile must fit one ring stage");
 
 namespace {
-constexpr uint32_t COL_S = 0, COL_P = 128, COL_O = 256, COL_LA = 384, COL_LB = 0;
+constexpr uint32_t COL_S = 0, COL_O = 128, COL_L = 0;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+constexpr float LOG2E = 1.4426950408889634f;
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     sla_fused_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                      const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH,
-                     FusedArgs a) {
+                     const __grid_constant__ CUtensorMap mapZ, FusedArgs a) {
   using L = FusedSmem<D>;
   constexpr int NST = L::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   uint8_t* sQ = sm + L::OFF_Q;
-  uint8_t* sPhi = sm + L::OFF_PHI;
   uint8_t* sKV = sm + L::OFF_KV;
+  uint8_t* sZ = sm + L::OFF_Z;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
   uint64_t* q_full = bars + 0;
   uint64_t* phiq_ready = bars + 1;
-  uint64_t* l_full = bars + 2;
-  uint64_t* s_full = bars + 3;     // [2]
-  uint64_t* p_ready = bars + 5;    // [2]
-  uint64_t* pv_done = bars + 7;    // [2]
-  uint64_t* kv_full = bars + 9;    // [NST]
+  uint64_t* la_full = bars + 2;
+  uint64_t* lb_full = bars + 3;
+  uint64_t* la_free = bars + 4;
+  uint64_t* s_full = bars + 5;     // [2]
+  uint64_t* p_ready = bars + 7;    // [2]
+  uint64_t* pv_done = bars + 9;    // [2]
+  uint64_t* kv_full = bars + 11;   // [NST]
   uint64_t* kv_empty = kv_full + NST;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(kv_empty + NST);
   int* s_count = reinterpret_cast<int*>(tslot + 1);
@@ -84,13 +102,15 @@ __global__ void __launch_bounds__(192, 1)
 
   // ---------------- set-up: TMEM, barriers, union of the two critical lists
   if (w == 1) {
-    tmem_alloc(tslot, 512);
+    tmem_alloc(tslot, 256);
     tmem_relinquish();
   }
   if (tid == 0) {
     mbar_init(q_full, 1);
     mbar_init(phiq_ready, 128);
-    mbar_init(l_full, 1);
+    mbar_init(la_full, 1);
+    mbar_init(lb_full, 1);
+    mbar_init(la_free, 64);
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
       mbar_init(&p_ready[x], 128);
@@ -148,6 +168,7 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch_desc(&mapK);
       tma_prefetch_desc(&mapV);
       tma_prefetch_desc(&mapH);
+      tma_prefetch_desc(&mapZ);
       mbar_arrive_expect_tx(q_full, L::Q_BYTES);
 #pragma unroll
       for (int c = 0; c < L::CH; ++c) tma_load_4d(sQ + c * 16384, &mapQ, q_full, c * 64, 128 * p, h, b);
@@ -164,10 +185,14 @@ __global__ void __launch_bounds__(192, 1)
             tma_load_4d(st + L::KT_BYTES + c * 8192, &mapV, &kv_full[s], c * 64, 64 * j, h, b);
           }
         } else {
-          const int i = (k == U) ? ia : (has_b ? ib : ia);
-          mbar_arrive_expect_tx(&kv_full[s], D * D * 2);
+          const int t = k - U;
+          const int i = (t == 0) ? ia : (has_b ? ib : ia);
+          mbar_arrive_expect_tx(&kv_full[s], D * D * 2 + D * 2);
 #pragma unroll
-          for (int c = 0; c < L::CH; ++c) tma_load_4d(st + c * (D * 128), &mapH, &kv_full[s], c * 64, 0, i, bh);
+          for (int c = 0; c < L::CH; ++c) {
+            tma_load_4d(st + c * (D * 128), &mapH, &kv_full[s], c * 64, 0, i, bh);
+            tma_load_3d(sZ + (t * L::CH + c) * 128, &mapZ, &kv_full[s], D * D + c * 64, i, bh);
+          }
         }
       }
     }
@@ -186,7 +211,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = sdesc_sw128(vt + kk * 2048, 8192, 1024);
-          umma_ts(tbase + COL_O, tbase + COL_P + 32 * (kp & 1) + 8 * kk, bd, id_pv,
+          umma_ts(tbase + COL_O, tbase + COL_S + 64 * (kp & 1) + 8 * kk, bd, id_pv,
                   (kp > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[kp & 1]);
@@ -196,6 +221,11 @@ __global__ void __launch_bounds__(192, 1)
       for (int k = 0; k < U && ok; ++k) {
         const int s = k % NST;
         if (!mbar_wait(&kv_full[s], (k / NST) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        // S buffer k&1 still holds P_{k-2}: wait until that P V has completed
+        if (k >= 2 && !mbar_wait(&pv_done[k & 1], ((k - 2) >> 1) & 1, a.err, DEV_TIMEOUT_MMA)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t kt = smem_u32(sKV + s * L::STAGE);
 #pragma unroll
@@ -208,22 +238,25 @@ __global__ void __launch_bounds__(192, 1)
         if (k >= 1 && !issue_pv(k - 1)) { ok = false; break; }
       }
       if (ok && U >= 1) ok = issue_pv(U - 1);
-      // phi(Q) H_i for both query blocks
+      // linear branch: L = phi~(Q) H_i^T into the S/P region, first for query
+      // block 2p, then (after its rows are written out) for 2p+1
+      if (ok && U >= 1)
+        ok = mbar_wait(&pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, DEV_TIMEOUT_MMA);
       if (ok) ok = mbar_wait(phiq_ready, 0, a.err, DEV_TIMEOUT_SYNC);
       for (int t = 0; t < 2 && ok; ++t) {
         const int k = U + t, s = k % NST;
         if (!mbar_wait(&kv_full[s], (k / NST) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        if (t == 1 && !mbar_wait(la_free, 0, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
         tc_fence_after();
         const uint32_t ht = smem_u32(sKV + s * L::STAGE);
-        const uint32_t ph = smem_u32(sPhi);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(ph + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+          const uint64_t ad = sdesc_sw128(q0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(ht + (kk / 4) * (D * 128) + (kk % 4) * 32, 16, 1024);
-          umma_ss(tbase + (t == 0 ? COL_LA : COL_LB), ad, bd, id_l, kk > 0 ? 1u : 0u);
+          umma_ss(tbase + COL_L, ad, bd, id_l, kk > 0 ? 1u : 0u);
         }
+        umma_commit(t == 0 ? la_full : lb_full);
       }
-      if (ok) umma_commit(l_full);
     }
   } else {
     // ---------------- softmax / epilogue warps: one query row per thread
@@ -231,144 +264,152 @@ __global__ void __launch_bounds__(192, 1)
     const int r = 32 * q4 + ln;
     const int half = r >> 6;
     const uint32_t bit = 1u << half;
-    const uint32_t lane_off = (uint32_t)(32 * q4) << 16;
-    const int i_me = (half == 0) ? ia : (has_b ? ib : ia);
-    bool ok = mbar_wait(q_full, 0, a.err, DEV_TIMEOUT_TMA);
-    // phi(q_r) -> sPhi (bf16, same swizzled layout as Q) and den = phi(q_r).Z_i
-    float den = 0.f;
-    {
-      const __nv_bfloat16* Z = a.Hz + ((int64_t)bh * a.Tq + i_me) * a.NN + D * D;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16));
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-        for (int u = 0; u < 4; ++u) mx = fmaxf(mx, fmaxf(__low2float(p2[u]), __high2float(p2[u])));
-      }
-      constexpr float LOG2E = 1.4426950408889634f;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16));
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          sum += exp2f((__low2float(p2[u]) - mx) * LOG2E) + exp2f((__high2float(p2[u]) - mx) * LOG2E);
-      }
-      const float inv = 1.f / sum;
-#pragma unroll 1
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16));
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-        const uint4 zv = __ldg(reinterpret_cast<const uint4*>(Z + c * 8));
-        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv);
-        uint32_t o[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float f0 = exp2f((__low2float(p2[u]) - mx) * LOG2E) * inv;
-          const float f1 = exp2f((__high2float(p2[u]) - mx) * LOG2E) * inv;
-          o[u] = pack_bf16x2(f0, f1);
-          const __nv_bfloat162 fb2 = *reinterpret_cast<__nv_bfloat162*>(&o[u]);
-          den = fmaf(__low2float(fb2), __low2float(z2[u]), den);
-          den = fmaf(__high2float(fb2), __high2float(z2[u]), den);
-        }
-        *reinterpret_cast<uint4*>(sPhi + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16)) =
-            make_uint4(o[0], o[1], o[2], o[3]);
-      }
-      fence_proxy_async_smem();
-      mbar_arrive(phiq_ready);
-    }
-    // online softmax over the union list
-    float m = -INFINITY, l = 0.f;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
     const float sl2 = a.scale_log2;
-    for (int k = 0; k < U && ok; ++k) {
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int k = 0; k < U; ++k) {
       const int sb = k & 1;
+      const uint32_t ts = tl + COL_S + 64 * sb;
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (k >> 1) & 1, a.err, DEV_TIMEOUT_MMA))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t s0[32], s1[32];
-      tmem_ld32(tbase + lane_off + COL_S + 64 * sb, s0);
-      tmem_ld32(tbase + lane_off + COL_S + 64 * sb + 32, s1);
-      tmem_ld_wait();
       const bool crit = (uflag[k] & bit) != 0;  // uniform over the warp
-      const int j = uidx[k];
-      const int nvalid = min(64, a.N - 64 * j);
-      float mx = -INFINITY;
-      if (crit) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          if (c < nvalid) mx = fmaxf(mx, __uint_as_float(s0[c]));
-          if (c + 32 < nvalid) mx = fmaxf(mx, __uint_as_float(s1[c]));
-        }
-        mx *= sl2;
-      }
-      // lazy rescale: keep the running max unless it grows by more than 2^8
-      const float m_new = fmaxf(m, mx);
-      const bool grow = crit && (m == -INFINITY ? false : (m_new - m > RESCALE_THRESHOLD));
-      if (crit && m == -INFINITY) m = m_new;  // O and l of this row are still exactly 0
-      if (__any_sync(0xffffffffu, grow)) {
-        // O must hold P_{k-1} V_{k-1} before it is rescaled
-        if (!__all_sync(0xffffffffu,
-                        mbar_wait(&pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, a.err, DEV_TIMEOUT_MMA))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const float f = grow ? exp2f(m - m_new) : 1.f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tbase + lane_off + COL_O + c0, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
-          tmem_st32(tbase + lane_off + COL_O + c0, o);
-        }
-        tmem_st_wait();
-        if (grow) {
-          l *= f;
-          m = m_new;
-        }
-      }
       uint32_t pk[32];
-      float ls = 0.f;
-      // P row: columns 0..63 packed as bf16 pairs (column 2c in the low half)
+      if (crit) {
+        uint32_t s0[32], s1[32];
+        tmem_ld32(ts, s0);
+        tmem_ld32(ts + 32, s1);
+        tmem_ld_wait();
+        const int nvalid = a.N - 64 * (int)uidx[k];
+        if (nvalid < 64) {  // partial last key block: padding columns get -inf
 #pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        const int c0 = 2 * c, c1 = 2 * c + 1;
-        const float p0 = (crit && c0 < nvalid) ? exp2f(fmaf(__uint_as_float(s0[c0]), sl2, -m)) : 0.f;
-        const float p1 = (crit && c1 < nvalid) ? exp2f(fmaf(__uint_as_float(s0[c1]), sl2, -m)) : 0.f;
-        const float p2 = (crit && c0 + 32 < nvalid) ? exp2f(fmaf(__uint_as_float(s1[c0]), sl2, -m)) : 0.f;
-        const float p3 = (crit && c1 + 32 < nvalid) ? exp2f(fmaf(__uint_as_float(s1[c1]), sl2, -m)) : 0.f;
-        ls += (p0 + p1) + (p2 + p3);
-        pk[c] = pack_bf16x2(p0, p1);
-        pk[16 + c] = pack_bf16x2(p2, p3);
+          for (int c = 0; c < 32; ++c) {
+            if (c >= nvalid) s0[c] = __float_as_uint(-INFINITY);
+            if (c + 32 >= nvalid) s1[c] = __float_as_uint(-INFINITY);
+          }
+        }
+        float t[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) t[c] = fmaxf(__uint_as_float(s0[c]), __uint_as_float(s1[c]));
+#pragma unroll
+        for (int st = 16; st >= 1; st >>= 1)
+#pragma unroll
+          for (int c = 0; c < st; ++c) t[c] = fmaxf(t[c], t[c + st]);
+        const float mx = t[0] * sl2;
+        // lazy rescale: keep the running max unless it grows by more than 2^8
+        const bool first = (m == -INFINITY);
+        const bool grow = !first && (mx - m > RESCALE_THRESHOLD);
+        if (first) m = mx;  // O and l of this row are still exactly 0
+        if (__any_sync(0xffffffffu, grow)) {
+          // O must hold P_{k-1} V_{k-1} before it is rescaled
+          if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, a.err,
+                                                  DEV_TIMEOUT_MMA))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = grow ? ex2(m - mx) : 1.f;
+#pragma unroll 1
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tl + COL_O + c0, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * f);
+            tmem_st32(tl + COL_O + c0, o);
+          }
+          tmem_st_wait();
+          if (grow) {
+            l *= f;
+            m = mx;
+          }
+        }
+        const float nm = -m;
+        float u[32];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const float p0 = ex2(fmaf(__uint_as_float(s0[2 * c]), sl2, nm));
+          const float p1 = ex2(fmaf(__uint_as_float(s0[2 * c + 1]), sl2, nm));
+          const float p2 = ex2(fmaf(__uint_as_float(s1[2 * c]), sl2, nm));
+          const float p3 = ex2(fmaf(__uint_as_float(s1[2 * c + 1]), sl2, nm));
+          u[c] = p0 + p1;
+          u[16 + c] = p2 + p3;
+          pk[c] = pack_bf16x2(p0, p1);
+          pk[16 + c] = pack_bf16x2(p2, p3);
+        }
+#pragma unroll
+        for (int st = 16; st >= 1; st >>= 1)
+#pragma unroll
+          for (int c = 0; c < st; ++c) u[c] += u[c + st];
+        l += u[0];
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      l += ls;
-      // P_k overwrites the buffer P_{k-2} was read from
-      if (k >= 2 && !__all_sync(0xffffffffu, mbar_wait(&pv_done[sb], ((k - 2) >> 1) & 1, a.err,
-                                                          DEV_TIMEOUT_MMA))) {
-        ok = false;
-        break;
-      }
-      tmem_st32(tbase + lane_off + COL_P + 32 * sb, pk);
+      tmem_st32(ts, pk);  // P_k over the first 32 columns of S_k
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[sb]);
     }
+    // ---------------- linear branch operand: phi~(q_r) in place of q_r
+    float esum = 0.f, edotz = 0.f;
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, a.err, DEV_TIMEOUT_TMA));
+    if (ok && U >= 1)  // every S MMA has read Q once the last score tile is done
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err,
+                                             DEV_TIMEOUT_MMA));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[U % NST], (U / NST) & 1, a.err,
+                                                   DEV_TIMEOUT_TMA));  // Z_a
+    if (ok && has_b)
+      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[(U + 1) % NST], ((U + 1) / NST) & 1, a.err,
+                                             DEV_TIMEOUT_TMA));  // Z_b
+    if (ok) {
+      const uint8_t* zrow = sZ + (half == 1 && has_b ? L::CH * 128 : 0);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fmaxf(__low2float(p2[e]), __high2float(p2[e])));
+      }
+      const float nmx = -mx * LOG2E;
+#pragma unroll 4
+      for (int c = 0; c < D / 8; ++c) {
+        uint8_t* qp = sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16);
+        const uint4 v = *reinterpret_cast<const uint4*>(qp);
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+        const uint4 zv = *reinterpret_cast<const uint4*>(zrow + (c / 8) * 128 + (c % 8) * 16);
+        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv);
+        uint32_t o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          o[e] = pack_bf16x2(ex2(fmaf(__low2float(p2[e]), LOG2E, nmx)),
+                             ex2(fmaf(__high2float(p2[e]), LOG2E, nmx)));
+          const __nv_bfloat162 eb = *reinterpret_cast<const __nv_bfloat162*>(&o[e]);
+          const float e0 = __low2float(eb), e1 = __high2float(eb);
+          esum += e0 + e1;
+          edotz = fmaf(e0, __low2float(z2[e]), fmaf(e1, __high2float(z2[e]), edotz));
+        }
+        *reinterpret_cast<uint4*>(qp) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(phiq_ready);
+    }
     // ---------------- epilogue
     if (ok && U >= 1)
-      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, DEV_TIMEOUT_MMA));
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(l_full, 0, a.err, DEV_TIMEOUT_MMA));
+      ok = __all_sync(0xffffffffu, mbar_wait(&pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err,
+                                             DEV_TIMEOUT_MMA));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(half == 0 ? la_full : lb_full, 0, a.err,
+                                                   DEV_TIMEOUT_MMA));
     if (ok) {
       tc_fence_after();
       const int n = 128 * p + r;
       const bool store = (n < a.N) && (half == 0 || has_b);
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const float inv_den = 1.f / (den + a.eps);
+      const float inv_den = 1.f / (edotz + esum * a.eps);
       float wa, wl;
       if (a.combine == 1) {
         const float al = a.alpha[bh];
@@ -378,18 +419,14 @@ __global__ void __launch_bounds__(192, 1)
         wa = inv_l;
         wl = inv_den;
       }
-      const uint32_t col_l = (half == 0) ? COL_LA : COL_LB;
       __nv_bfloat16* orow = a.O + (int64_t)b * a.so0 + (int64_t)h * a.so1 + (int64_t)n * a.so2;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t os[32], ol[32];
-        tmem_ld32(tbase + lane_off + COL_O + c0, os);
-        tmem_ld32(tbase + lane_off + col_l + c0, ol);
+        uint32_t ov[32], lv[32];
+        tmem_ld32(tl + COL_O + c0, ov);
+        tmem_ld32(tl + COL_L + c0, lv);
         tmem_ld_wait();
         if (store) {
-          float bias[32];
-#pragma unroll
-          for (int c = 0; c < 32; ++c) bias[c] = (a.combine == 0 && a.proj_b) ? __ldg(a.proj_b + c0 + c) : 0.f;
           uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -397,12 +434,17 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int c = 8 * v + e;
-              y[e] = __uint_as_float(os[c]) * wa + __uint_as_float(ol[c]) * wl + bias[c];
+              const float bias = (a.combine == 0 && a.proj_b) ? __ldg(a.proj_b + c0 + c) : 0.f;
+              y[e] = __uint_as_float(ov[c]) * wa + __uint_as_float(lv[c]) * wl + bias;
             }
             dst[v] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
                                 pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
           }
         }
+      }
+      if (half == 0) {  // L_a has been read: the S/P region can take L_b
+        tc_fence_before();
+        mbar_arrive(la_free);
       }
     }
   }
@@ -410,32 +452,29 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (w == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, 512);
+    tmem_dealloc(tbase, 256);
   }
 }
 
 template <int D>
 static cudaError_t launch_fused_t(const CUtensorMap& mapQ, const CUtensorMap& mapK,
                                   const CUtensorMap& mapV, const CUtensorMap& mapH,
-                                  const FusedArgs& a, int BH, cudaStream_t s) {
+                                  const CUtensorMap& mapZ, const FusedArgs& a, int BH,
+                                  cudaStream_t s) {
   const size_t smem = FusedSmem<D>::bytes(a.Tkv);
   cudaError_t e = cudaFuncSetAttribute(sla_fused_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.Tq + 1) / 2, BH);
-  sla_fused_kernel<D><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, a);
+  sla_fused_kernel<D><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, mapZ, a);
   return cudaGetLastError();
 }
 
-size_t fused_smem_bytes(int D, int Tkv) {
-  return D == 128 ? FusedSmem<128>::bytes(Tkv) : FusedSmem<64>::bytes(Tkv);
-}
-
 cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                         const CUtensorMap& mapH, const FusedArgs& a, int D, int BH,
-                         cudaStream_t s) {
-  return D == 128 ? launch_fused_t<128>(mapQ, mapK, mapV, mapH, a, BH, s)
-                  : launch_fused_t<64>(mapQ, mapK, mapV, mapH, a, BH, s);
+                         const CUtensorMap& mapH, const CUtensorMap& mapZ, const FusedArgs& a,
+                         int D, int BH, cudaStream_t s) {
+  return D == 128 ? launch_fused_t<128>(mapQ, mapK, mapV, mapH, mapZ, a, BH, s)
+                  : launch_fused_t<64>(mapQ, mapK, mapV, mapH, mapZ, a, BH, s);
 }
 
 }  // namespace sla

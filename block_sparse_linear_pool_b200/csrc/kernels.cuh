@@ -65,7 +65,7 @@ cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, c
                              int BH, cudaStream_t s);
 
 cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                         const CUtensorMap& mapH, const FusedArgs& a, int D, int BH,
-                         cudaStream_t s);
+                         const CUtensorMap& mapH, const CUtensorMap& mapZ, const FusedArgs& a,
+                         int D, int BH, cudaStream_t s);
 
 }  // namespace sla
