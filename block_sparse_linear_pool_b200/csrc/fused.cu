@@ -8,8 +8,11 @@
 // lists (ascending); a key block that is critical for only one of the two
 // query blocks is masked out of the other half (its probabilities are 0).
 //
-//   warp 0      TMA producer: Q tile, K_j/V_j per union entry, then the two
-//               aggregated H_i^T tiles and Z_i rows, through an NST-stage ring
+//   warp 0      TMA producer: Q tile, then K_j and V_j per union entry through
+//               two separate rings (a K slot frees when its S MMA completes, a
+//               V slot when its P V completes, so K tiles run ahead), then the
+//               aggregated H_i^T tiles and Z_i rows (H_a into the K ring, H_b
+//               into the V ring)
 //   warp 1      MMA issuer: S_k = Q K_j^T into TMEM (two buffers), O += P_k V_j
 //               with P_k read back from TMEM, and at the end
 //               L = phi~(Q) H_i^T for both query blocks
@@ -37,18 +40,20 @@ namespace sla {
 template <int D>
 struct FusedSmem {
   static constexpr int CH = D / 64;
-  static constexpr int NST = (D == 128) ? 2 : 4;
+  static constexpr int NR = (D == 128) ? 2 : 4;        // slots per ring (K ring and V ring)
   static constexpr int Q_BYTES = 128 * D * 2;
   static constexpr int KT_BYTES = 64 * D * 2;          // one K or V tile
-  static constexpr int STAGE = 2 * KT_BYTES;           // K tile then V tile (or one H tile)
+  static constexpr int RING = NR * KT_BYTES;           // holds one d x d H tile as well
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + Q_BYTES;
-  static constexpr int OFF_Z = OFF_KV + NST * STAGE;   // Z_a, Z_b: 2 x D bf16 (unswizzled rows)
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + RING;
+  static constexpr int OFF_Z = OFF_V + RING;           // Z_a, Z_b: 2 x D bf16 (unswizzled rows)
   static constexpr int OFF_BAR = OFF_Z + 2 * CH * 128;
   static constexpr int OFF_U = OFF_BAR + 256;
   static size_t bytes(int Tkv) { return (size_t)OFF_U + 5 * (size_t)((Tkv + 15) & ~15) + 1024; }
 };
-static_assert(2 * 64 * 128 * 2 >= 128 * 128 * 2, "an H tile must fit one ring stage");
+static_assert(FusedSmem<128>::RING >= 128 * 128 * 2 && FusedSmem<64>::RING >= 64 * 64 * 2,
+              "an H tile must fit one ring");
 
 namespace {
 constexpr uint32_t COL_S = 0, COL_O = 128, COL_L = 0;
@@ -68,12 +73,13 @@ __global__ void __launch_bounds__(192, 2)
                      const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH,
                      const __grid_constant__ CUtensorMap mapZ, FusedArgs a) {
   using L = FusedSmem<D>;
-  constexpr int NST = L::NST;
+  constexpr int NR = L::NR;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   uint8_t* sQ = sm + L::OFF_Q;
-  uint8_t* sKV = sm + L::OFF_KV;
+  uint8_t* sK = sm + L::OFF_K;
+  uint8_t* sV = sm + L::OFF_V;
   uint8_t* sZ = sm + L::OFF_Z;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
   uint64_t* q_full = bars + 0;
@@ -84,9 +90,13 @@ __global__ void __launch_bounds__(192, 2)
   uint64_t* s_full = bars + 5;     // [2]
   uint64_t* p_ready = bars + 7;    // [2]
   uint64_t* pv_done = bars + 9;    // [2]
-  uint64_t* kv_full = bars + 11;   // [NST]
-  uint64_t* kv_empty = kv_full + NST;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(kv_empty + NST);
+  uint64_t* ha_full = bars + 11;
+  uint64_t* hb_full = bars + 12;
+  uint64_t* k_full = bars + 13;    // [NR]
+  uint64_t* k_empty = k_full + NR;
+  uint64_t* v_full = k_empty + NR;
+  uint64_t* v_empty = v_full + NR;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(v_empty + NR);
   int* s_count = reinterpret_cast<int*>(tslot + 1);
   const int Tkvr = (a.Tkv + 15) & ~15;
   uint8_t* fa = sm + L::OFF_U;
@@ -116,9 +126,13 @@ __global__ void __launch_bounds__(192, 2)
       mbar_init(&p_ready[x], 128);
       mbar_init(&pv_done[x], 1);
     }
-    for (int s = 0; s < NST; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    mbar_init(ha_full, 1);
+    mbar_init(hb_full, 1);
+    for (int s = 0; s < NR; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     fence_barrier_init();
   }
@@ -172,27 +186,53 @@ __global__ void __launch_bounds__(192, 2)
       mbar_arrive_expect_tx(q_full, L::Q_BYTES);
 #pragma unroll
       for (int c = 0; c < L::CH; ++c) tma_load_4d(sQ + c * 16384, &mapQ, q_full, c * 64, 128 * p, h, b);
-      for (int k = 0; k < U + 2; ++k) {
-        const int s = k % NST;
-        if (k >= NST && !mbar_wait(&kv_empty[s], ((k / NST) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) break;
-        uint8_t* st = sKV + s * L::STAGE;
+      bool ok = true;
+      // K_k is issued one step ahead of V_{k-1}
+      for (int k = 0; k <= U && ok; ++k) {
         if (k < U) {
+          const int s = k % NR;
+          if (k >= NR && !mbar_wait(&k_empty[s], ((k / NR) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
+            ok = false;
+            break;
+          }
           const int j = uidx[k];
-          mbar_arrive_expect_tx(&kv_full[s], L::STAGE);
+          mbar_arrive_expect_tx(&k_full[s], L::KT_BYTES);
 #pragma unroll
-          for (int c = 0; c < L::CH; ++c) {
-            tma_load_4d(st + c * 8192, &mapK, &kv_full[s], c * 64, 64 * j, h, b);
-            tma_load_4d(st + L::KT_BYTES + c * 8192, &mapV, &kv_full[s], c * 64, 64 * j, h, b);
+          for (int c = 0; c < L::CH; ++c)
+            tma_load_4d(sK + s * L::KT_BYTES + c * 8192, &mapK, &k_full[s], c * 64, 64 * j, h, b);
+        }
+        if (k >= 1) {
+          const int kv = k - 1, s = kv % NR;
+          if (kv >= NR && !mbar_wait(&v_empty[s], ((kv / NR) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
+            ok = false;
+            break;
           }
-        } else {
-          const int t = k - U;
-          const int i = (t == 0) ? ia : (has_b ? ib : ia);
-          mbar_arrive_expect_tx(&kv_full[s], D * D * 2 + D * 2);
+          const int j = uidx[kv];
+          mbar_arrive_expect_tx(&v_full[s], L::KT_BYTES);
 #pragma unroll
-          for (int c = 0; c < L::CH; ++c) {
-            tma_load_4d(st + c * (D * 128), &mapH, &kv_full[s], c * 64, 0, i, bh);
-            tma_load_3d(sZ + (t * L::CH + c) * 128, &mapZ, &kv_full[s], D * D + c * 64, i, bh);
+          for (int c = 0; c < L::CH; ++c)
+            tma_load_4d(sV + s * L::KT_BYTES + c * 8192, &mapV, &v_full[s], c * 64, 64 * j, h, b);
+        }
+      }
+      // H_a (+ Z_a) into the K ring once its last S MMAs completed, H_b (+ Z_b)
+      // into the V ring once its last P V completed
+      for (int t = 0; t < 2 && ok; ++t) {
+        uint64_t* empty = (t == 0) ? k_empty : v_empty;
+        for (int s = 0; s < NR && ok; ++s) {
+          if (U > s) {
+            const int last = s + NR * ((U - 1 - s) / NR);
+            ok = mbar_wait(&empty[s], (last / NR) & 1, a.err, DEV_TIMEOUT_SYNC);
           }
+        }
+        if (!ok) break;
+        const int i = (t == 0) ? ia : (has_b ? ib : ia);
+        uint64_t* full = (t == 0) ? ha_full : hb_full;
+        uint8_t* dst = (t == 0) ? sK : sV;
+        mbar_arrive_expect_tx(full, D * D * 2 + D * 2);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c) {
+          tma_load_4d(dst + c * (D * 128), &mapH, full, c * 64, 0, i, bh);
+          tma_load_3d(sZ + (t * L::CH + c) * 128, &mapZ, full, D * D + c * 64, i, bh);
         }
       }
     }
@@ -206,8 +246,10 @@ __global__ void __launch_bounds__(192, 2)
       bool ok = mbar_wait(q_full, 0, a.err, DEV_TIMEOUT_TMA);
       auto issue_pv = [&](int kp) -> bool {
         if (!mbar_wait(&p_ready[kp & 1], (kp >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
+        const int sv = kp % NR;
+        if (!mbar_wait(&v_full[sv], (kp / NR) & 1, a.err, DEV_TIMEOUT_TMA)) return false;
         tc_fence_after();
-        const uint32_t vt = smem_u32(sKV + (kp % NST) * L::STAGE + L::KT_BYTES);
+        const uint32_t vt = smem_u32(sV + sv * L::KT_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = sdesc_sw128(vt + kk * 2048, 8192, 1024);
@@ -215,19 +257,17 @@ __global__ void __launch_bounds__(192, 2)
                   (kp > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&pv_done[kp & 1]);
-        umma_commit(&kv_empty[kp % NST]);
+        umma_commit(&v_empty[sv]);
         return true;
       };
       for (int k = 0; k < U && ok; ++k) {
-        const int s = k % NST;
-        if (!mbar_wait(&kv_full[s], (k / NST) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
-        // S buffer k&1 still holds P_{k-2}: wait until that P V has completed
-        if (k >= 2 && !mbar_wait(&pv_done[k & 1], ((k - 2) >> 1) & 1, a.err, DEV_TIMEOUT_MMA)) {
-          ok = false;
-          break;
-        }
+        const int s = k % NR;
+        if (!mbar_wait(&k_full[s], (k / NR) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        // S buffer k&1 still holds P_{k-2}.  No wait is needed before
+        // overwriting it: P_{k-2} V was issued earlier by this thread, and
+        // tcgen05.mma operations issued by one thread execute in issue order.
         tc_fence_after();
-        const uint32_t kt = smem_u32(sKV + s * L::STAGE);
+        const uint32_t kt = smem_u32(sK + s * L::KT_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(q0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
@@ -235,6 +275,7 @@ __global__ void __launch_bounds__(192, 2)
           umma_ss(tbase + COL_S + 64 * (k & 1), ad, bd, id_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[k & 1]);
+        umma_commit(&k_empty[s]);
         if (k >= 1 && !issue_pv(k - 1)) { ok = false; break; }
       }
       if (ok && U >= 1) ok = issue_pv(U - 1);
@@ -244,11 +285,10 @@ __global__ void __launch_bounds__(192, 2)
         ok = mbar_wait(&pv_done[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err, DEV_TIMEOUT_MMA);
       if (ok) ok = mbar_wait(phiq_ready, 0, a.err, DEV_TIMEOUT_SYNC);
       for (int t = 0; t < 2 && ok; ++t) {
-        const int k = U + t, s = k % NST;
-        if (!mbar_wait(&kv_full[s], (k / NST) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        if (!mbar_wait(t == 0 ? ha_full : hb_full, 0, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
         if (t == 1 && !mbar_wait(la_free, 0, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ht = smem_u32(sKV + s * L::STAGE);
+        const uint32_t ht = smem_u32(t == 0 ? sK : sV);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(q0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
@@ -360,13 +400,7 @@ __global__ void __launch_bounds__(192, 2)
     if (ok && U >= 1)  // every S MMA has read Q once the last score tile is done
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[(U - 1) & 1], ((U - 1) >> 1) & 1, a.err,
                                              DEV_TIMEOUT_MMA));
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[U % NST], (U / NST) & 1, a.err,
-                                                   DEV_TIMEOUT_TMA));  // Z_a
-    if (ok && has_b)
-      ok = __all_sync(0xffffffffu, mbar_wait(&kv_full[(U + 1) % NST], ((U + 1) / NST) & 1, a.err,
-                                             DEV_TIMEOUT_TMA));  // Z_b
     if (ok) {
-      const uint8_t* zrow = sZ + (half == 1 && has_b ? L::CH * 128 : 0);
       float mx = -INFINITY;
 #pragma unroll
       for (int c = 0; c < D / 8; ++c) {
@@ -381,22 +415,35 @@ __global__ void __launch_bounds__(192, 2)
         uint8_t* qp = sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16);
         const uint4 v = *reinterpret_cast<const uint4*>(qp);
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&v);
-        const uint4 zv = *reinterpret_cast<const uint4*>(zrow + (c / 8) * 128 + (c % 8) * 16);
-        const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv);
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           o[e] = pack_bf16x2(ex2(fmaf(__low2float(p2[e]), LOG2E, nmx)),
                              ex2(fmaf(__high2float(p2[e]), LOG2E, nmx)));
           const __nv_bfloat162 eb = *reinterpret_cast<const __nv_bfloat162*>(&o[e]);
-          const float e0 = __low2float(eb), e1 = __high2float(eb);
-          esum += e0 + e1;
-          edotz = fmaf(e0, __low2float(z2[e]), fmaf(e1, __high2float(z2[e]), edotz));
+          esum += __low2float(eb) + __high2float(eb);
         }
         *reinterpret_cast<uint4*>(qp) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       fence_proxy_async_smem();
       mbar_arrive(phiq_ready);
+      // phi~(q_r) . Z_i (Z arrives with this half's H tile)
+      ok = __all_sync(0xffffffffu, mbar_wait(half == 1 && has_b ? hb_full : ha_full, 0, a.err,
+                                             DEV_TIMEOUT_TMA));
+      if (ok) {
+        const uint8_t* zrow = sZ + (half == 1 && has_b ? L::CH * 128 : 0);
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16));
+          const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+          const uint4 zv = *reinterpret_cast<const uint4*>(zrow + (c / 8) * 128 + (c % 8) * 16);
+          const __nv_bfloat162* z2 = reinterpret_cast<const __nv_bfloat162*>(&zv);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            edotz = fmaf(__low2float(e2[e]), __low2float(z2[e]),
+                         fmaf(__high2float(e2[e]), __high2float(z2[e]), edotz));
+        }
+      }
     }
     // ---------------- epilogue
     if (ok && U >= 1)
