@@ -136,7 +136,11 @@ def fused_traffic_per_launch(d: int):
 
 # --------------------------------------------------------------------------- FLOP accounting
 def flop_model(cfg, dims, lut_np):
-    """Executed and algorithmic FLOPs of one step (Measurement)."""
+    """Executed and algorithmic FLOPs of one step.
+
+    Executed = every tensor-core MMA the kernels issue (union entries of the fused
+    kernel, padded GEMM tiles) plus the fp32 logits; algorithmic (fused) = QK^T and
+    PV over the critical pairs plus phi(Q)H per query row."""
     BH, N, d, Tq, Tkv, nh, nl = (dims[k] for k in ("BH", "N", "d", "Tq", "Tkv", "nh", "nl"))
     NN = d * d + d
     # fused kernel: per CTA (pair of query blocks) U union entries x (S + PV), + 2 phi(Q)H tiles

@@ -155,7 +155,7 @@ sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, co
  *
  * sla_aggregate_marginal: for every query block i, [H_i^T | Z_i] = sum over
  * its marginal blocks (mc == 0) of [h_j^T | z_j] ([SLA] §2 Q2 step 3,
- * "H_i += h_j, Z_i += z_j"), computed as one 0/1-matrix product per head on
+ * marginal blocks accumulate h_j and z_j), computed as one 0/1-matrix product per head on
  * the tensor cores; the result stays in the workspace.
  *
  * sla_fused_forward: the per-query-block kernel (sparse branch over the

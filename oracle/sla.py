@@ -19,7 +19,7 @@ Sources, cited by page title and section:
          §4 Learnable Router (pooling, proj_q/proj_k, row-wise Top-k),
          §5 Quantization-aware Training (low-bit Q/K with scales).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * the last block may be partial (N not a multiple of b): its pooled mean is
     over its real tokens only and no padding token enters any sum;
   * block counts: n_h = max(1, floor(k_h*T + 1e-9)),
@@ -66,9 +66,10 @@ class OracleParams:
 def block_counts(T_kv: int, k_h: float, k_l: float) -> tuple[int, int]:
     """Number of critical (n_h) and negligible (n_l) key blocks per query row.
 
-    [SLA] §2 Q2 step 2 gives "top k_h%" and "bottom k_l%"; [SLA2] §4 / §6 make
-    the count per row (k% x N/b_k).  Reading: floor, with at least one critical
-    block so that the sparse softmax is defined.
+    [SLA] §2 Q2 step 2 gives the critical and negligible shares as
+    percentages; [SLA2] §4 / §6 make the count per row (k% of the N/b_k
+    blocks).  Reading: floor, with at least one critical block so that the
+    sparse softmax is defined.
     """
     n_h = max(1, int(np.floor(k_h * T_kv + 1e-9)))
     n_l = min(int(np.floor(k_l * T_kv + 1e-9)), T_kv - n_h)
@@ -142,7 +143,7 @@ def compressed_attention(logits: np.ndarray) -> np.ndarray:
 def classify(Pc: np.ndarray, n_h: int, n_l: int) -> np.ndarray:
     """Three-way block classification M_c in {1, 0, -1} ([SLA] §2 Q2 step 2).
 
-    Per row ([SLA2] §4: "highest-scoring k% positions in each row"): order the
+    Per row ([SLA2] §4: Top-k is taken within each row): order the
     key blocks by P_c descending, ties by lower index first; the first n_h are
     critical (1), the last n_l negligible (-1), the rest marginal (0).
     """
@@ -188,7 +189,7 @@ def critical_lut(Mc: np.ndarray) -> np.ndarray:
 def feature_map(X: np.ndarray, kind: str = "softmax") -> np.ndarray:
     """phi applied per token over the head dimension.
 
-    "softmax" is the map of [SLA] Fig. 4 ("feature map (softmax)"); "elu1" is
+    "softmax" is the map of [SLA] Fig. 4 (a softmax feature map); "elu1" is
     elu(x) + 1, the ablation of [SLA] Table 2.
     """
     X = np.asarray(X, dtype=np.float64)
