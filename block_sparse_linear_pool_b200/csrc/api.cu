@@ -20,12 +20,14 @@ constexpr size_t kAlign = 256;
 
 struct Plan {
   int B, H, N, d, BH, Tq, Tkv, nh, nl, NN, Tkvp;
+  bool fp8;  // Q K^T on E4M3 with per-block scales
 };
 
 inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
-  size_t err, qc, kc, qr, kr, kmean, mm, hagg, end;       // sla_workspace_size
+  size_t err, qc, kc, qr, kr, kmean, mm, hagg;            // sla_workspace_size ...
+  size_t q8, k8, scq, sck, end;                           // ... (+ FP8 operands)
   size_t mc, lut, hz, end_attn;                           // + sla_attention extras
   size_t hq, hk, hv, ho, end_host;                        // + sla_attention_host staging
 };
@@ -41,6 +43,12 @@ Layout layout_of(const Plan& p) {
   L.kmean = o; o = align_up(o + (size_t)p.BH * p.d * 4);
   L.mm = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkvp * 2);
   L.hagg = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.NN * 2);
+  const size_t q8 = p.fp8 ? (size_t)p.BH * p.Tq * 64 * p.d : 0;
+  const size_t k8 = p.fp8 ? (size_t)p.BH * p.Tkv * 64 * p.d : 0;
+  L.q8 = o;    o = align_up(o + q8);
+  L.k8 = o;    o = align_up(o + k8);
+  L.scq = o;   o = align_up(o + (p.fp8 ? (size_t)p.BH * p.Tq * 4 : 0));
+  L.sck = o;   o = align_up(o + (p.fp8 ? (size_t)p.BH * p.Tkv * 4 : 0));
   L.end = o;
   L.mc = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkv);
   L.lut = o;   o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
@@ -80,6 +88,7 @@ sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
   if (p->combine != SLA_COMBINE_PROJ && p->combine != SLA_COMBINE_ALPHA) return SLA_ERR_INVALID_ARG;
   if (p->qk_prec != SLA_QK_BF16 && p->qk_prec != SLA_QK_FP8_E4M3) return SLA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
+  if (p->qk_prec == SLA_QK_FP8_E4M3 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if (p->b_q != 64 || p->b_kv != 64) return SLA_ERR_UNSUPPORTED;
   if (p->N > kMaxN || (int64_t)p->B * p->H > 65535) return SLA_ERR_UNSUPPORTED;
   if (!stride_ok(p->stride_q, p->d) || !stride_ok(p->stride_k, p->d) ||
@@ -95,6 +104,7 @@ sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
   counts(pl->Tkv, p->k_h, p->k_l, &pl->nh, &pl->nl);
   pl->NN = p->d * p->d + p->d;
   pl->Tkvp = (pl->Tkv + 7) & ~7;
+  pl->fp8 = p->qk_prec == SLA_QK_FP8_E4M3;
   return SLA_OK;
 }
 
@@ -114,10 +124,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return fn;
 }
 
-// rank-r bf16 tiled map, 128-byte swizzle (or none); dims/strides innermost first,
+// rank-r tiled map (bf16 unless dt says otherwise), 128-byte swizzle (or none);
+// dims/strides innermost first,
 // strides in bytes for dims 1..r-1.
 bool encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-            const uint64_t* strides, const uint32_t* box, bool swizzle = true) {
+            const uint64_t* strides, const uint32_t* box, bool swizzle = true,
+            CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto fn = encoder();
   if (!fn) return false;
   cuuint64_t gd[5], gs[4];
@@ -128,7 +140,7 @@ bool encode(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
     es[i] = 1;
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides[i];
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, bx, es,
+  CUresult r = fn(m, dt, rank, const_cast<void*>(base), gd, gs, bx, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
                   swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -266,6 +278,38 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
     const uint32_t bxz[3] = {64, 1, 1};
     if (!encode(&mz, hagg, 3, dz, sz, bxz, false)) return SLA_ERR_CUDA;
   }
+  CUtensorMap mq8 = mq, mk8 = mk;  // placeholders unless the FP8 path runs
+  const float* scq = nullptr;
+  const float* sck = nullptr;
+  if (pl.fp8) {
+    QuantArgs qa;
+    qa.Q = static_cast<const __nv_bfloat16*>(Q);
+    qa.K = static_cast<const __nv_bfloat16*>(K);
+    for (int i = 0; i < 3; ++i) {
+      qa.sq[i] = p->stride_q[i];
+      qa.sk[i] = p->stride_k[i];
+    }
+    qa.Q8 = at<uint8_t>(ws, L.q8);
+    qa.K8 = at<uint8_t>(ws, L.k8);
+    qa.scale_q = at<float>(ws, L.scq);
+    qa.scale_k = at<float>(ws, L.sck);
+    qa.H = pl.H;
+    qa.N = pl.N;
+    qa.Tq = pl.Tq;
+    qa.Tkv = pl.Tkv;
+    SLA_TRY(cuda_status(launch_quant_fp8(qa, pl.BH, s)));
+    const uint64_t dq[3] = {(uint64_t)pl.d, (uint64_t)pl.Tq * 64, (uint64_t)pl.BH};
+    const uint64_t sq[2] = {(uint64_t)pl.d, (uint64_t)pl.Tq * 64 * pl.d};
+    const uint32_t bq[3] = {(uint32_t)pl.d, 128, 1};
+    const uint64_t dk[3] = {(uint64_t)pl.d, (uint64_t)pl.Tkv * 64, (uint64_t)pl.BH};
+    const uint64_t sk[2] = {(uint64_t)pl.d, (uint64_t)pl.Tkv * 64 * pl.d};
+    const uint32_t bk[3] = {(uint32_t)pl.d, 64, 1};
+    if (!encode(&mq8, qa.Q8, 3, dq, sq, bq, true, CU_TENSOR_MAP_DATA_TYPE_UINT8) ||
+        !encode(&mk8, qa.K8, 3, dk, sk, bk, true, CU_TENSOR_MAP_DATA_TYPE_UINT8))
+      return SLA_ERR_CUDA;
+    scq = qa.scale_q;
+    sck = qa.scale_k;
+  }
   FusedArgs a;
   a.lut = lut;
   a.Hz = hagg;
@@ -285,7 +329,9 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.combine = p->combine;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)pl.d));
   a.eps = p->eps;
-  return cuda_status(launch_fused(mq, mk, mv, mh, mz, a, pl.d, pl.BH, s));
+  a.scale_q = scq;
+  a.scale_k = sck;
+  return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, pl.fp8, pl.BH, s));
 }
 
 sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
@@ -416,7 +462,6 @@ sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, co
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(hz))
     return SLA_ERR_INVALID_ARG;
   if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
-  if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
   SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
   return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, workspace,
                       reinterpret_cast<cudaStream_t>(stream));
@@ -431,7 +476,6 @@ sla_status_t sla_attention(const sla_params_t* p, const void* Q, const void* K, 
   if (!Q || !K || !V || !O) return SLA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SLA_ERR_INVALID_ARG;
   if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
-  if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
   SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_ATTN));
   return attention_impl(pl, p, Q, K, V, proj_w, proj_b, alpha, Wq, Wk, O, workspace,
                         reinterpret_cast<cudaStream_t>(stream));
@@ -455,7 +499,6 @@ sla_status_t sla_attention_host(const sla_params_t* p, const void* Q_host, const
   if (!Q_host || !K_host || !V_host || !O_host) return SLA_ERR_INVALID_ARG;
   if (!contiguous(p)) return SLA_ERR_INVALID_ARG;
   if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
-  if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
   SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_HOST));
   const Layout L = layout_of(pl);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -489,7 +532,6 @@ sla_status_t sla_fused_forward(const sla_params_t* p, const void* Q, const void*
   if (!Q || !K || !V || !lut || !O) return SLA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SLA_ERR_INVALID_ARG;
   if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
-  if (p->qk_prec != SLA_QK_BF16) return SLA_ERR_UNSUPPORTED;
   SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
   return fused_impl(pl, p, Q, K, V, lut, proj_b, alpha, O, workspace,
                     reinterpret_cast<cudaStream_t>(stream));

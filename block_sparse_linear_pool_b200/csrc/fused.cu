@@ -30,6 +30,12 @@
 // O [128,128+d).  After the last P V the S/P region [0,d) holds L_a; once the
 // rows of query block 2p have been written out it holds L_b.
 //
+// Low-bit variant ([SLA2] §5): Q and K arrive as E4M3 with one scale per
+// (head, 64-row block) and S = Q^ K^^T runs as tcgen05.mma kind::f8f6f4; the
+// softmax multiplies the scores by s_Q s_K.  P V stays in bf16.  The FP8 Q tile
+// and K ring are half the size, so the bf16 Q tile (needed for phi(Q)) fits
+// beside them and H_a loads over the FP8 Q tile and K ring.
+//
 // Linear branch with unnormalised feature map: for e_a = 2^((q_a - max q) log2 e)
 // and s = sum_a e_a, phi(q) = e / s, so
 //     phi(q) H / (phi(q) Z + eps) = (e H) / (e Z + s eps)      exactly.
@@ -37,23 +43,30 @@
 
 namespace sla {
 
-template <int D>
+template <int D, bool FP8>
 struct FusedSmem {
   static constexpr int CH = D / 64;
   static constexpr int NR = (D == 128) ? 2 : 4;        // slots per ring (K ring and V ring)
-  static constexpr int Q_BYTES = 128 * D * 2;
-  static constexpr int KT_BYTES = 64 * D * 2;          // one K or V tile
-  static constexpr int RING = NR * KT_BYTES;           // holds one d x d H tile as well
+  static constexpr int Q_BYTES = 128 * D * 2;          // bf16 Q tile
+  static constexpr int Q8_BYTES = FP8 ? 128 * D : 0;   // e4m3 Q tile
+  static constexpr int KT_BYTES = 64 * D * 2;          // one bf16 K or V tile
+  static constexpr int KSLOT = FP8 ? 64 * D : KT_BYTES;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + RING;
-  static constexpr int OFF_Z = OFF_V + RING;           // Z_a, Z_b: 2 x D bf16 (unswizzled rows)
+  static constexpr int OFF_Q8 = OFF_Q + Q_BYTES;
+  static constexpr int OFF_K = OFF_Q8 + Q8_BYTES;
+  static constexpr int OFF_V = OFF_K + NR * KSLOT;
+  static constexpr int OFF_HA = FP8 ? OFF_Q8 : OFF_K;  // H_a goes where Q8 / K were
+  static constexpr int OFF_Z = OFF_V + NR * KT_BYTES;  // Z_a, Z_b: 2 x D bf16 (unswizzled rows)
   static constexpr int OFF_BAR = OFF_Z + 2 * CH * 128;
   static constexpr int OFF_U = OFF_BAR + 256;
-  static size_t bytes(int Tkv) { return (size_t)OFF_U + 5 * (size_t)((Tkv + 15) & ~15) + 1024; }
+  static size_t bytes(int Tkv) { return (size_t)OFF_U + 9 * (size_t)((Tkv + 15) & ~15) + 1024; }
 };
-static_assert(FusedSmem<128>::RING >= 128 * 128 * 2 && FusedSmem<64>::RING >= 64 * 64 * 2,
-              "an H tile must fit one ring");
+static_assert(FusedSmem<128, false>::OFF_V - FusedSmem<128, false>::OFF_HA >= 128 * 128 * 2 &&
+                  FusedSmem<128, true>::OFF_V - FusedSmem<128, true>::OFF_HA >= 128 * 128 * 2 &&
+                  FusedSmem<64, false>::OFF_V - FusedSmem<64, false>::OFF_HA >= 64 * 64 * 2,
+              "an H tile must fit where it is loaded");
+static_assert(FusedSmem<128, false>::NR * FusedSmem<128, false>::KT_BYTES >= 128 * 128 * 2,
+              "H_b must fit the V ring");
 
 namespace {
 constexpr uint32_t COL_S = 0, COL_O = 128, COL_L = 0;
@@ -67,19 +80,23 @@ __device__ __forceinline__ float ex2(float x) {
 }
 }  // namespace
 
-template <int D>
+template <int D, bool FP8>
 __global__ void __launch_bounds__(192, 2)
     sla_fused_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                      const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH,
-                     const __grid_constant__ CUtensorMap mapZ, FusedArgs a) {
-  using L = FusedSmem<D>;
+                     const __grid_constant__ CUtensorMap mapZ, const __grid_constant__ CUtensorMap mapQ8,
+                     const __grid_constant__ CUtensorMap mapK8, FusedArgs a) {
+  static_assert(!FP8 || D == 128, "the FP8 path is built for d = 128");
+  using L = FusedSmem<D, FP8>;
   constexpr int NR = L::NR;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   uint8_t* sQ = sm + L::OFF_Q;
+  uint8_t* sQ8 = sm + L::OFF_Q8;
   uint8_t* sK = sm + L::OFF_K;
   uint8_t* sV = sm + L::OFF_V;
+  uint8_t* sHa = sm + L::OFF_HA;
   uint8_t* sZ = sm + L::OFF_Z;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
   uint64_t* q_full = bars + 0;
@@ -103,6 +120,7 @@ __global__ void __launch_bounds__(192, 2)
   uint8_t* fb = fa + Tkvr;
   uint8_t* uflag = fb + Tkvr;
   uint16_t* uidx = reinterpret_cast<uint16_t*>(uflag + Tkvr);
+  float* usk = reinterpret_cast<float*>(uidx + Tkvr);  // FP8: K scale per union entry
 
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const int p = blockIdx.x, bh = blockIdx.y;
@@ -164,6 +182,7 @@ __global__ void __launch_bounds__(192, 2)
         const int pos = base + __popc(bal & lt);
         uidx[pos] = (uint16_t)j;
         uflag[pos] = (uint8_t)f;
+        if (FP8) usk[pos] = a.scale_k[(int64_t)bh * a.Tkv + j];
       }
       base += __popc(bal);
     }
@@ -183,9 +202,11 @@ __global__ void __launch_bounds__(192, 2)
       tma_prefetch_desc(&mapV);
       tma_prefetch_desc(&mapH);
       tma_prefetch_desc(&mapZ);
-      mbar_arrive_expect_tx(q_full, L::Q_BYTES);
+      if (FP8) tma_prefetch_desc(&mapQ8), tma_prefetch_desc(&mapK8);
+      mbar_arrive_expect_tx(q_full, L::Q_BYTES + L::Q8_BYTES);
 #pragma unroll
       for (int c = 0; c < L::CH; ++c) tma_load_4d(sQ + c * 16384, &mapQ, q_full, c * 64, 128 * p, h, b);
+      if (FP8) tma_load_3d(sQ8, &mapQ8, q_full, 0, 128 * p, bh);
       bool ok = true;
       // K_k is issued one step ahead of V_{k-1}
       for (int k = 0; k <= U && ok; ++k) {
@@ -196,10 +217,14 @@ __global__ void __launch_bounds__(192, 2)
             break;
           }
           const int j = uidx[k];
-          mbar_arrive_expect_tx(&k_full[s], L::KT_BYTES);
+          mbar_arrive_expect_tx(&k_full[s], L::KSLOT);
+          if (FP8) {
+            tma_load_3d(sK + s * L::KSLOT, &mapK8, &k_full[s], 0, 64 * j, bh);
+          } else {
 #pragma unroll
-          for (int c = 0; c < L::CH; ++c)
-            tma_load_4d(sK + s * L::KT_BYTES + c * 8192, &mapK, &k_full[s], c * 64, 64 * j, h, b);
+            for (int c = 0; c < L::CH; ++c)
+              tma_load_4d(sK + s * L::KSLOT + c * 8192, &mapK, &k_full[s], c * 64, 64 * j, h, b);
+          }
         }
         if (k >= 1) {
           const int kv = k - 1, s = kv % NR;
@@ -227,7 +252,7 @@ __global__ void __launch_bounds__(192, 2)
         if (!ok) break;
         const int i = (t == 0) ? ia : (has_b ? ib : ia);
         uint64_t* full = (t == 0) ? ha_full : hb_full;
-        uint8_t* dst = (t == 0) ? sK : sV;
+        uint8_t* dst = (t == 0) ? sHa : sV;
         mbar_arrive_expect_tx(full, D * D * 2 + D * 2);
 #pragma unroll
         for (int c = 0; c < L::CH; ++c) {
@@ -240,6 +265,7 @@ __global__ void __launch_bounds__(192, 2)
     // ---------------- MMA issuer
     if (ln == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
+      const uint32_t id_s8 = idesc_e4m3(128, 64);
       const uint32_t id_pv = idesc_bf16(128, D, false, true);
       const uint32_t id_l = idesc_bf16(128, D, false, false);
       const uint32_t q0 = smem_u32(sQ);
@@ -267,12 +293,23 @@ __global__ void __launch_bounds__(192, 2)
         // overwriting it: P_{k-2} V was issued earlier by this thread, and
         // tcgen05.mma operations issued by one thread execute in issue order.
         tc_fence_after();
-        const uint32_t kt = smem_u32(sK + s * L::KT_BYTES);
+        const uint32_t kt = smem_u32(sK + s * L::KSLOT);
+        if (FP8) {
+          // e4m3: 128-byte rows hold all d = 128 values; K = 32 per instruction
+          const uint32_t q8 = smem_u32(sQ8);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(q0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(kt + (kk / 4) * 8192 + (kk % 4) * 32, 16, 1024);
-          umma_ss(tbase + COL_S + 64 * (k & 1), ad, bd, id_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 32; ++kk) {
+            const uint64_t ad = sdesc_sw128(q8 + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(kt + kk * 32, 16, 1024);
+            umma_ss_f8(tbase + COL_S + 64 * (k & 1), ad, bd, id_s8, kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(q0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(kt + (kk / 4) * 8192 + (kk % 4) * 32, 16, 1024);
+            umma_ss(tbase + COL_S + 64 * (k & 1), ad, bd, id_s, kk > 0 ? 1u : 0u);
+          }
         }
         umma_commit(&s_full[k & 1]);
         umma_commit(&k_empty[s]);
@@ -288,7 +325,7 @@ __global__ void __launch_bounds__(192, 2)
         if (!mbar_wait(t == 0 ? ha_full : hb_full, 0, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
         if (t == 1 && !mbar_wait(la_free, 0, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ht = smem_u32(t == 0 ? sK : sV);
+        const uint32_t ht = smem_u32(t == 0 ? sHa : sV);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = sdesc_sw128(q0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
@@ -306,6 +343,7 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t bit = 1u << half;
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
     const float sl2 = a.scale_log2;
+    const float sq_half = FP8 ? a.scale_q[(int64_t)bh * a.Tq + ((half == 1 && has_b) ? ib : ia)] : 1.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int k = 0; k < U; ++k) {
@@ -338,7 +376,9 @@ __global__ void __launch_bounds__(192, 2)
         for (int st = 16; st >= 1; st >>= 1)
 #pragma unroll
           for (int c = 0; c < st; ++c) t[c] = fmaxf(t[c], t[c + st]);
-        const float mx = t[0] * sl2;
+        // FP8 scores carry the two block scales: s = (q^ . k^) s_Q s_K
+        const float sc = FP8 ? sl2 * sq_half * usk[k] : sl2;
+        const float mx = t[0] * sc;
         // lazy rescale: keep the running max unless it grows by more than 2^8
         const bool first = (m == -INFINITY);
         const bool grow = !first && (mx - m > RESCALE_THRESHOLD);
@@ -371,10 +411,10 @@ __global__ void __launch_bounds__(192, 2)
         float u[32];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2(fmaf(__uint_as_float(s0[2 * c]), sl2, nm));
-          const float p1 = ex2(fmaf(__uint_as_float(s0[2 * c + 1]), sl2, nm));
-          const float p2 = ex2(fmaf(__uint_as_float(s1[2 * c]), sl2, nm));
-          const float p3 = ex2(fmaf(__uint_as_float(s1[2 * c + 1]), sl2, nm));
+          const float p0 = ex2(fmaf(__uint_as_float(s0[2 * c]), sc, nm));
+          const float p1 = ex2(fmaf(__uint_as_float(s0[2 * c + 1]), sc, nm));
+          const float p2 = ex2(fmaf(__uint_as_float(s1[2 * c]), sc, nm));
+          const float p3 = ex2(fmaf(__uint_as_float(s1[2 * c + 1]), sc, nm));
           u[c] = p0 + p1;
           u[16 + c] = p2 + p3;
           pk[c] = pack_bf16x2(p0, p1);
@@ -503,25 +543,28 @@ __global__ void __launch_bounds__(192, 2)
   }
 }
 
-template <int D>
+template <int D, bool FP8>
 static cudaError_t launch_fused_t(const CUtensorMap& mapQ, const CUtensorMap& mapK,
                                   const CUtensorMap& mapV, const CUtensorMap& mapH,
-                                  const CUtensorMap& mapZ, const FusedArgs& a, int BH,
+                                  const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
+                                  const CUtensorMap& mapK8, const FusedArgs& a, int BH,
                                   cudaStream_t s) {
-  const size_t smem = FusedSmem<D>::bytes(a.Tkv);
-  cudaError_t e = cudaFuncSetAttribute(sla_fused_kernel<D>,
+  const size_t smem = FusedSmem<D, FP8>::bytes(a.Tkv);
+  cudaError_t e = cudaFuncSetAttribute(sla_fused_kernel<D, FP8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.Tq + 1) / 2, BH);
-  sla_fused_kernel<D><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, mapZ, a);
+  sla_fused_kernel<D, FP8><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                         const CUtensorMap& mapH, const CUtensorMap& mapZ, const FusedArgs& a,
-                         int D, int BH, cudaStream_t s) {
-  return D == 128 ? launch_fused_t<128>(mapQ, mapK, mapV, mapH, mapZ, a, BH, s)
-                  : launch_fused_t<64>(mapQ, mapK, mapV, mapH, mapZ, a, BH, s);
+                         const CUtensorMap& mapH, const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
+                         const CUtensorMap& mapK8, const FusedArgs& a, int D, bool fp8, int BH,
+                         cudaStream_t s) {
+  if (fp8) return launch_fused_t<128, true>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
+  return D == 128 ? launch_fused_t<128, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s)
+                  : launch_fused_t<64, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
 }
 
 }  // namespace sla

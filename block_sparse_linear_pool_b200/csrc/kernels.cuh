@@ -35,6 +35,18 @@ struct MargArgs {
   int Tq, Tkv, NN, ktiles;
 };
 
+struct QuantArgs {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  int64_t sq[3];       // element strides of Q for B, H, N
+  int64_t sk[3];
+  uint8_t* Q8;         // [BH][T_q*64][d] e4m3
+  uint8_t* K8;         // [BH][T_kv*64][d] e4m3
+  float* scale_q;      // [BH][T_q]
+  float* scale_k;      // [BH][T_kv]
+  int H, N, Tq, Tkv;
+};
+
 struct FusedArgs {
   const int32_t* lut;     // [BH][Tq][nh]
   const __nv_bfloat16* Hz;  // [BH][Tq][NN] aggregated H_i^T and Z_i
@@ -47,6 +59,8 @@ struct FusedArgs {
   int combine;            // 0 proj, 1 alpha
   float scale_log2;       // log2(e) / sqrt(d)
   float eps;
+  const float* scale_q;   // FP8 path: per (head, query block) scale of Q, else nullptr
+  const float* scale_k;   // FP8 path: per (head, key block) scale of K, else nullptr
 };
 
 cudaError_t launch_pool(const PoolArgs& a, int D, int BH, cudaStream_t s);
@@ -64,8 +78,12 @@ cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int 
 cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const MargArgs& a,
                              int BH, cudaStream_t s);
 
+cudaError_t launch_quant_fp8(const QuantArgs& a, int BH, cudaStream_t s);
+
+// mapQ8 / mapK8 are used only when fp8 is set (d = 128 only).
 cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
-                         const CUtensorMap& mapH, const CUtensorMap& mapZ, const FusedArgs& a,
-                         int D, int BH, cudaStream_t s);
+                         const CUtensorMap& mapH, const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
+                         const CUtensorMap& mapK8, const FusedArgs& a, int D, bool fp8, int BH,
+                         cudaStream_t s);
 
 }  // namespace sla

@@ -1,0 +1,74 @@
+// Low-bit Q and K for the sparse branch ("SLA2: Sparse-Linear Attention with
+// Learnable Routing and QAT", §5: Q and K are mapped to FP8 with scales before
+// Q K^T, and the product is rescaled).
+//
+// One scale per (head, 64-row block): s = max|x| / 448 (448 = largest finite
+// E4M3 value), x_q = round-to-nearest-even(x / s) with saturation.  Rows past N
+// in the last block are written as zeros, so every block occupies 64 rows.
+#include <cuda_fp8.h>
+
+#include "kernels.cuh"
+
+namespace sla {
+
+// grid (T, B*H, 2): z = 0 quantises Q, z = 1 quantises K.  128 threads; thread
+// t owns row t/2 and the 64 columns starting at 64*(t%2) (d = 128).
+__global__ void __launch_bounds__(128) quant_fp8_kernel(QuantArgs a) {
+  __shared__ float red[4];
+  const int blk = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const int T = which == 0 ? a.Tq : a.Tkv;
+  if (blk >= T) return;
+  const int b = bh / a.H, h = bh % a.H;
+  const __nv_bfloat16* src = which == 0 ? a.Q : a.K;
+  const int64_t* st = which == 0 ? a.sq : a.sk;
+  uint8_t* dst = which == 0 ? a.Q8 : a.K8;
+  float* scale = which == 0 ? a.scale_q : a.scale_k;
+  const int t = threadIdx.x, row = t >> 1, c0 = 64 * (t & 1);
+  const int n = 64 * blk + row;
+  const bool valid = n < a.N;
+  float x[64];
+  float amax = 0.f;
+  const __nv_bfloat16* p = src + (int64_t)b * st[0] + (int64_t)h * st[1] + (int64_t)n * st[2] + c0;
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    uint4 q = valid ? __ldg(reinterpret_cast<const uint4*>(p) + v) : make_uint4(0, 0, 0, 0);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      x[8 * v + 2 * u] = __low2float(p2[u]);
+      x[8 * v + 2 * u + 1] = __high2float(p2[u]);
+      amax = fmaxf(amax, fmaxf(fabsf(x[8 * v + 2 * u]), fabsf(x[8 * v + 2 * u + 1])));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((t & 31) == 0) red[t >> 5] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const float s = amax > 0.f ? amax / 448.f : 1.f;
+  const float inv = amax > 0.f ? 448.f / amax : 0.f;
+  uint8_t* out = dst + ((int64_t)bh * T * 64 + 64 * blk + row) * 128 + c0;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    uint32_t w[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = 16 * v + 4 * u;
+      const __nv_fp8x2_storage_t lo =
+          __nv_cvt_float2_to_fp8x2(make_float2(x[e] * inv, x[e + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+      const __nv_fp8x2_storage_t hi =
+          __nv_cvt_float2_to_fp8x2(make_float2(x[e + 2] * inv, x[e + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+      w[u] = (uint32_t)lo | ((uint32_t)hi << 16);
+    }
+    reinterpret_cast<uint4*>(out)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+  if (t == 0) scale[(int64_t)bh * T + blk] = s;
+}
+
+cudaError_t launch_quant_fp8(const QuantArgs& a, int BH, cudaStream_t s) {
+  const int T = a.Tq > a.Tkv ? a.Tq : a.Tkv;
+  quant_fp8_kernel<<<dim3(T, BH, 2), 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace sla
