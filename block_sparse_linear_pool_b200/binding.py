@@ -33,6 +33,7 @@ EXPORTS = (
     "sla_attention", "sla_aggregate_marginal", "sla_fused_forward",
     "sla_attention_host_workspace_size", "sla_attention_host", "sla_backward",
     "sla_get_device_status", "sla_status_string", "sla_abi_version",
+    "sla_predict_mask_noalloc",
 )
 
 
@@ -81,6 +82,7 @@ def lib() -> ctypes.CDLL:
         L.sla_aggregate_marginal.argtypes = [P, vp, vp, vp, sz, vp]
         L.sla_fused_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_attention_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_predict_mask_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.sla_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_get_device_status.argtypes = [vp, vp, ip]
         L.sla_status_string.argtypes = [ctypes.c_int]
@@ -257,3 +259,16 @@ def sla_get_device_status(workspace) -> int:
     detail = ctypes.c_int()
     code = lib().sla_get_device_status(_ptr(workspace), _stream(), ctypes.byref(detail))
     return code, detail.value
+
+
+def sla_predict_mask_noalloc(Q, K, cfg: SlaConfig, Wq=None, Wk=None):
+    """sla_predict_mask with the library's static scratch instead of a workspace."""
+    p = make_params(Q, cfg, K=K)
+    Tq, Tkv, nh, _ = sla_block_counts(p)
+    BH = Q.shape[0] * Q.shape[1]
+    mc = torch.empty((BH, Tq, Tkv), dtype=torch.int8, device=Q.device)
+    lut = torch.empty((BH, Tq, nh), dtype=torch.int32, device=Q.device)
+    Wq, Wk = _f32(Wq, Q.device), _f32(Wk, Q.device)
+    _check(lib().sla_predict_mask_noalloc(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(Wq), _ptr(Wk),
+                                          _ptr(mc), _ptr(lut), _stream()), "sla_predict_mask_noalloc")
+    return mc, lut

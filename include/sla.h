@@ -199,6 +199,28 @@ sla_status_t sla_attention_host(const sla_params_t* p, const void* Q_host, const
                                 sla_stream_t stream);
 
 /*
+ * sla_predict_mask without a workspace argument.  The pages describe no such
+ * call: it exists for callers that cannot allocate device memory when they
+ * predict the mask (allocation-free hot loops, host callbacks, memory planned
+ * up front by an arena the caller does not own).  Its scratch (error word and
+ * pooled / routed Q and K blocks) lives in one static device array of
+ * SLA_NOALLOC_SCRATCH_BYTES that every GPU using the library holds until the
+ * process exits.  Inputs, outputs and results are those of sla_predict_mask.
+ *   - Problems whose scratch exceeds the array (B*H*(T_q + T_kv)*d*4 bytes,
+ *     twice that plus B*H*d*4 with a router or smooth-K, plus 256) return
+ *     SLA_ERR_WORKSPACE before any launch.
+ *   - The first call on a device looks up the array's address on that device
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls on a device share the array: calls that overlap on the GPU
+ *     race and must be serialised by the caller.
+ *   - Nothing is allocated; the error word is cleared with cudaMemsetAsync.
+ */
+#define SLA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+sla_status_t sla_predict_mask_noalloc(const sla_params_t* p, const void* Q, const void* K,
+                                      const float* Wq, const float* Wk, int8_t* mc,
+                                      int32_t* lut, sla_stream_t stream);
+
+/*
  * Backward of the forward above ([SLA2] App. A; [SLA] §4 check 6).  Not
  * implemented in this build: returns SLA_ERR_UNSUPPORTED after validating
  * its arguments.
