@@ -220,9 +220,15 @@ sla_status_t predict_mask_impl(const Plan& pl, const sla_params_t* p, const void
 
 sla_status_t precompute_impl(const Plan& pl, const sla_params_t* p, const void* K, const void* V,
                              const float* proj_w, void* hz, void* ws, cudaStream_t s) {
-  CUtensorMap mk, mv;
+  CUtensorMap mk, mv, mo;
   if (!map_bhnd(&mk, K, pl, p->stride_k, 64) || !map_bhnd(&mv, V, pl, p->stride_v, 64))
     return SLA_ERR_CUDA;
+  {
+    const uint64_t dims[4] = {(uint64_t)pl.d, (uint64_t)pl.d, (uint64_t)pl.Tkv, (uint64_t)pl.BH};
+    const uint64_t str[3] = {(uint64_t)pl.d * 2, (uint64_t)pl.NN * 2, (uint64_t)pl.Tkv * pl.NN * 2};
+    const uint32_t box[4] = {64, (uint32_t)pl.d, 1, 1};
+    if (!encode(&mo, hz, 4, dims, str, box)) return SLA_ERR_CUDA;
+  }
   KvPrepArgs a;
   a.proj_w = (p->combine == SLA_COMBINE_PROJ) ? proj_w : nullptr;
   a.hz = static_cast<__nv_bfloat16*>(hz);
@@ -231,7 +237,7 @@ sla_status_t precompute_impl(const Plan& pl, const sla_params_t* p, const void* 
   a.N = pl.N;
   a.Tkv = pl.Tkv;
   a.nitems = pl.BH * pl.Tkv;
-  return cuda_status(launch_kv_prep(mk, mv, a, pl.d, s));
+  return cuda_status(launch_kv_prep(mk, mv, mo, a, pl.d, s));
 }
 
 sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, void* ws,

@@ -32,7 +32,7 @@ struct KvPrepArgs {
 struct MargArgs {
   __nv_bfloat16* Hout;   // [BH][Tq][NN]
   int* err;
-  int Tq, Tkv, NN, ktiles;
+  int Tq, Tkv, NN, ktiles, BH;
 };
 
 struct QuantArgs {
@@ -70,8 +70,9 @@ cudaError_t launch_router(const float* Qc, const float* Kc, float* Qr, float* Kr
 size_t select_smem_bytes(int D, int Tk);
 cudaError_t launch_select(const SelectArgs& a, int BH, cudaStream_t s);
 
-cudaError_t launch_kv_prep(const CUtensorMap& mapK, const CUtensorMap& mapV, const KvPrepArgs& a,
-                           int D, cudaStream_t s);
+// mapO: hz viewed as (a: d, b: d, j: T_kv, bh) tiles of 64 x d for TMA stores.
+cudaError_t launch_kv_prep(const CUtensorMap& mapK, const CUtensorMap& mapV, const CUtensorMap& mapO,
+                           const KvPrepArgs& a, int D, cudaStream_t s);
 
 cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int Tq, int Tkv,
                                int Tkvp, cudaStream_t s);

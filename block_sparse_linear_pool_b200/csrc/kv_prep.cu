@@ -5,12 +5,15 @@
 // With the SLA combine, Proj's weight W is folded in (h_j W^T is stored):
 // Proj(O^l) = phi(Q) (H W^T) / den + b because den is a per-row scalar.
 //
-// One CTA (4 warps) walks key blocks of 64 tokens persistently:
-//   TMA      K_j, V_j  -> smem (128B-swizzled, d contiguous)
+// One CTA (4 warps) walks key blocks of 64 tokens persistently through two
+// shared-memory stages, the next block's K_j, V_j loading while the current one
+// is processed:
+//   TMA      K_j, V_j  -> stage (128B-swizzled, d contiguous)
 //   tcgen05  D1 = W V_j^T          (M = d, N = 64, K = d)   [SLA only]
-//   threads  phi(K_j) -> smem (bf16), V'^T = D1 -> smem (bf16)
+//   threads  phi(K_j) in place of K_j; V'^T = D1 in place of V_j (bf16)
 //   tcgen05  D2 = V'^T phi(K_j)    (M = d, N = d, K = 64)  = (h_j W^T)^T
-//   threads  z_j = column sums of phi(K_j); D2 and z_j -> hz (bf16)
+//   threads  z_j = column sums of phi(K_j); D2 -> the stage as a swizzled
+//            d x d tile, then one TMA store writes it to hz (coalesced)
 #include "kernels.cuh"
 
 namespace sla {
@@ -20,32 +23,29 @@ struct KvSmem {
   static constexpr int CH = D / 64;                 // 64-column chunks of d
   static constexpr int W_BYTES = D * D * 2;         // W, K-major [CH][D rows][128B]
   static constexpr int T_BYTES = 64 * D * 2;        // one 64-token tile
+  static constexpr int STAGE = 2 * T_BYTES;         // K (then phi) | V (then V'^T); then the h tile
   static constexpr int OFF_W = 0;
-  static constexpr int OFF_K = OFF_W + W_BYTES;
-  static constexpr int OFF_V = OFF_K + T_BYTES;
-  static constexpr int OFF_PHI = OFF_V + T_BYTES;   // MN-major [CH][64 t][128B]
-  static constexpr int OFF_VT = OFF_PHI + T_BYTES;  // K-major [D rows][128B]
-  static constexpr int OFF_BAR = OFF_VT + D * 128;
+  static constexpr int OFF_ST = OFF_W + W_BYTES;
+  static constexpr int OFF_BAR = OFF_ST + 2 * STAGE;
   static constexpr int BYTES = OFF_BAR + 64;
   static constexpr int ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
 };
+static_assert(KvSmem<128>::STAGE >= 128 * 128 * 2 && KvSmem<64>::STAGE >= 64 * 64 * 2,
+              "the h tile must fit one stage");
 
 template <int D>
 __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CUtensorMap mapK,
                                                       const __grid_constant__ CUtensorMap mapV,
+                                                      const __grid_constant__ CUtensorMap mapO,
                                                       KvPrepArgs a) {
   using L = KvSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   uint8_t* sW = sm + L::OFF_W;
-  uint8_t* sK = sm + L::OFF_K;
-  uint8_t* sV = sm + L::OFF_V;
-  uint8_t* sPhi = sm + L::OFF_PHI;
-  uint8_t* sVt = sm + L::OFF_VT;
-  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
-  uint64_t* mma_bar = tma_bar + 1;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(tma_bar + 2);
+  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);  // [2]
+  uint64_t* mma_bar = tma_bar + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(tma_bar + 3);
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const bool proj = a.proj_w != nullptr;
 
@@ -54,11 +54,13 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(tma_bar, 1);
+    mbar_init(&tma_bar[0], 1);
+    mbar_init(&tma_bar[1], 1);
     mbar_init(mma_bar, 1);
     fence_barrier_init();
     tma_prefetch_desc(&mapK);
     tma_prefetch_desc(&mapV);
+    tma_prefetch_desc(&mapO);
   }
   if (proj) {  // W (fp32 [o][b]) -> bf16, K-major over b
     for (int g = tid; g < D * D / 8; g += 128) {
@@ -85,23 +87,36 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
   // 16 per 32-lane quarter).
   const int my_row = (D == 128) ? tid : ((ln < 16) ? 16 * w + ln : -1);
 
+  auto issue_load = [&](int item, int s) {
+    const int bh = item / a.Tkv, j = item % a.Tkv;
+    const int b = bh / a.H, h = bh % a.H;
+    uint8_t* st = sm + L::OFF_ST + s * L::STAGE;
+    mbar_arrive_expect_tx(&tma_bar[s], 2 * L::T_BYTES);
+#pragma unroll
+    for (int c = 0; c < L::CH; ++c) {
+      tma_load_4d(st + c * 8192, &mapK, &tma_bar[s], c * 64, j * 64, h, b);
+      tma_load_4d(st + L::T_BYTES + c * 8192, &mapV, &tma_bar[s], c * 64, j * 64, h, b);
+    }
+  };
+  if (tid == 0 && (int)blockIdx.x < a.nitems) issue_load(blockIdx.x, 0);
+
   uint32_t mma_phase = 0;
   int n = 0;
   // Every wait result is agreed on by the whole CTA (__syncthreads_and), so a
   // timeout makes all threads leave the loop at the same point.
   for (int item = blockIdx.x; item < a.nitems; item += gridDim.x, ++n) {
+    const int s = n & 1;
+    uint8_t* sK = sm + L::OFF_ST + s * L::STAGE;
+    uint8_t* sV = sK + L::T_BYTES;
     const int bh = item / a.Tkv, j = item % a.Tkv;
-    const int b = bh / a.H, h = bh % a.H;
     const int cnt = min(64, a.N - j * 64);
-    if (tid == 0) {
-      mbar_arrive_expect_tx(tma_bar, 2 * L::T_BYTES);
-#pragma unroll
-      for (int c = 0; c < L::CH; ++c) {
-        tma_load_4d(sK + c * 8192, &mapK, tma_bar, c * 64, j * 64, h, b);
-        tma_load_4d(sV + c * 8192, &mapV, tma_bar, c * 64, j * 64, h, b);
-      }
+    // next block into the other stage, once the store that last used it has
+    // finished reading shared memory
+    if (tid == 0 && item + (int)gridDim.x < a.nitems) {
+      bulk_wait_read_all();
+      issue_load(item + gridDim.x, s ^ 1);
     }
-    if (!__syncthreads_and(mbar_wait(tma_bar, n & 1, a.err, DEV_TIMEOUT_TMA))) break;
+    if (!__syncthreads_and(mbar_wait(&tma_bar[s], (n >> 1) & 1, a.err, DEV_TIMEOUT_TMA))) break;
     if (proj && tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(D, 64, false, false);
@@ -114,7 +129,7 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       }
       umma_commit(mma_bar);
     }
-    {  // phi(K_j): two threads per token row, each owning D/2 columns.
+    {  // phi(K_j) in place: two threads per token row, each owning D/2 columns.
       constexpr int NE = D / 2;
       const int t = tid >> 1, half = tid & 1;
       const int chunk = (D == 128) ? half : 0;
@@ -136,14 +151,14 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       for (int e = 1; e < NE; ++e) m = fmaxf(m, x[e]);
       m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
       constexpr float LOG2E = 1.4426950408889634f;
-      float s = 0.f;
+      float sum = 0.f;
 #pragma unroll
       for (int e = 0; e < NE; ++e) {
         x[e] = exp2f((x[e] - m) * LOG2E);
-        s += x[e];
+        sum += x[e];
       }
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      const float inv = (t < cnt) ? 1.f / s : 0.f;  // padding tokens of a partial block: phi = 0
+      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+      const float inv = (t < cnt) ? 1.f / sum : 0.f;  // padding tokens of a partial block: phi = 0
 #pragma unroll
       for (int v = 0; v < NE / 8; ++v) {
         uint4 q;
@@ -151,10 +166,10 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
         q.y = pack_bf16x2(x[v * 8 + 2] * inv, x[v * 8 + 3] * inv);
         q.z = pack_bf16x2(x[v * 8 + 4] * inv, x[v * 8 + 5] * inv);
         q.w = pack_bf16x2(x[v * 8 + 6] * inv, x[v * 8 + 7] * inv);
-        *reinterpret_cast<uint4*>(sPhi + chunk * 8192 + sw128_offset(t, byte0 + v * 16)) = q;
+        *reinterpret_cast<uint4*>(sK + chunk * 8192 + sw128_offset(t, byte0 + v * 16)) = q;
       }
     }
-    if (proj) {  // V'^T = D1 (row o = output feature, 64 token columns) -> bf16
+    if (proj) {  // V'^T = D1 (row o = output feature, 64 token columns) in place of V
       const bool ok = mbar_wait(mma_bar, mma_phase & 1, a.err, DEV_TIMEOUT_MMA);
       ++mma_phase;
       if (!__syncthreads_and(ok)) break;
@@ -171,12 +186,12 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
           q.y = pack_bf16x2(__uint_as_float(r0[8 * v + 2]), __uint_as_float(r0[8 * v + 3]));
           q.z = pack_bf16x2(__uint_as_float(r0[8 * v + 4]), __uint_as_float(r0[8 * v + 5]));
           q.w = pack_bf16x2(__uint_as_float(r0[8 * v + 6]), __uint_as_float(r0[8 * v + 7]));
-          *reinterpret_cast<uint4*>(sVt + sw128_offset(my_row, v * 16)) = q;
+          *reinterpret_cast<uint4*>(sV + sw128_offset(my_row, v * 16)) = q;
           q.x = pack_bf16x2(__uint_as_float(r1[8 * v + 0]), __uint_as_float(r1[8 * v + 1]));
           q.y = pack_bf16x2(__uint_as_float(r1[8 * v + 2]), __uint_as_float(r1[8 * v + 3]));
           q.z = pack_bf16x2(__uint_as_float(r1[8 * v + 4]), __uint_as_float(r1[8 * v + 5]));
           q.w = pack_bf16x2(__uint_as_float(r1[8 * v + 6]), __uint_as_float(r1[8 * v + 7]));
-          *reinterpret_cast<uint4*>(sVt + sw128_offset(my_row, 64 + v * 16)) = q;
+          *reinterpret_cast<uint4*>(sV + sw128_offset(my_row, 64 + v * 16)) = q;
         }
       }
     }
@@ -188,9 +203,9 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       const uint32_t id = idesc_bf16(D, D, !proj, true);
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint64_t ad = proj ? sdesc_sw128(smem_u32(sVt) + k * 32, 16, 1024)
+        const uint64_t ad = proj ? sdesc_sw128(smem_u32(sV) + k * 32, 16, 1024)
                                  : sdesc_sw128(smem_u32(sV) + k * 2048, 8192, 1024);
-        const uint64_t bd = sdesc_sw128(smem_u32(sPhi) + k * 2048, 8192, 1024);
+        const uint64_t bd = sdesc_sw128(smem_u32(sK) + k * 2048, 8192, 1024);
         umma_ss(tD2, ad, bd, id, k > 0);
       }
       umma_commit(mma_bar);
@@ -201,7 +216,7 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       const int chunk = tid / 64, byte = (tid % 64) * 2;
       for (int t = 0; t < 64; ++t) {
         const __nv_bfloat16 v =
-            *reinterpret_cast<const __nv_bfloat16*>(sPhi + chunk * 8192 + sw128_offset(t, byte));
+            *reinterpret_cast<const __nv_bfloat16*>(sK + chunk * 8192 + sw128_offset(t, byte));
         z += __bfloat162float(v);
       }
     }
@@ -211,14 +226,13 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       if (!__syncthreads_and(ok)) break;
     }
     tc_fence_after();
-    __nv_bfloat16* out = a.hz + ((int64_t)bh * a.Tkv + j) * (int64_t)(D * D + D);
+    // (h_j W^T)^T rows -> the stage as [chunk of a][row b][128 B] (swizzled)
 #pragma unroll
     for (int c0 = 0; c0 < D; c0 += 32) {
       uint32_t r[32];
       tmem_ld32(tD2 + lane_off + c0, r);
       tmem_ld_wait();
       if (my_row >= 0) {
-        uint4* dst = reinterpret_cast<uint4*>(out + (int64_t)my_row * D + c0);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           uint4 q;
@@ -226,14 +240,24 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
           q.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
           q.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
           q.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-          dst[v] = q;
+          const int col = c0 + 8 * v;  // a index of this 16-byte group
+          *reinterpret_cast<uint4*>(sK + (col / 64) * (D * 128) +
+                                    sw128_offset(my_row, (col % 64) * 2)) = q;
         }
       }
     }
-    if (tid < D) out[D * D + tid] = __float2bfloat16(z);
+    __nv_bfloat16* zout = a.hz + ((int64_t)bh * a.Tkv + j) * (int64_t)(D * D + D) + D * D;
+    if (tid < D) zout[tid] = __float2bfloat16(z);
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) {
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c) tma_store_4d(&mapO, sK + c * (D * 128), c * 64, 0, j, bh);
+      bulk_commit_group();
+    }
   }
+  if (tid == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (w == 0) {
@@ -244,7 +268,7 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
 
 template <int D>
 static cudaError_t launch_kv_prep_t(const CUtensorMap& mapK, const CUtensorMap& mapV,
-                                    const KvPrepArgs& a, cudaStream_t s) {
+                                    const CUtensorMap& mapO, const KvPrepArgs& a, cudaStream_t s) {
   using L = KvSmem<D>;
   cudaError_t e = cudaFuncSetAttribute(kv_prep_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
@@ -253,13 +277,14 @@ static cudaError_t launch_kv_prep_t(const CUtensorMap& mapK, const CUtensorMap& 
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = min(a.nitems, 2 * sms);
-  kv_prep_kernel<D><<<grid, 128, L::ALLOC, s>>>(mapK, mapV, a);
+  kv_prep_kernel<D><<<grid, 128, L::ALLOC, s>>>(mapK, mapV, mapO, a);
   return cudaGetLastError();
 }
 
-cudaError_t launch_kv_prep(const CUtensorMap& mapK, const CUtensorMap& mapV, const KvPrepArgs& a,
-                           int D, cudaStream_t s) {
-  return D == 128 ? launch_kv_prep_t<128>(mapK, mapV, a, s) : launch_kv_prep_t<64>(mapK, mapV, a, s);
+cudaError_t launch_kv_prep(const CUtensorMap& mapK, const CUtensorMap& mapV, const CUtensorMap& mapO,
+                           const KvPrepArgs& a, int D, cudaStream_t s) {
+  return D == 128 ? launch_kv_prep_t<128>(mapK, mapV, mapO, a, s)
+                  : launch_kv_prep_t<64>(mapK, mapV, mapO, a, s);
 }
 
 }  // namespace sla

@@ -9,9 +9,10 @@
 // are exact in bf16, accumulation in fp32).
 //
 //   marg_matrix_kernel  M_c (int8) -> Mmarg (bf16 0/1, rows padded to T_kvp)
-//   marg_gemm_kernel    128 x 256 output tile per CTA, K step 64, 4-stage
-//                       TMA ring; warp 0 loads, warp 1 issues tcgen05.mma,
-//                       warps 2-5 drain TMEM and store bf16.
+//   marg_gemm_kernel    persistent, 128 x 256 output tiles, K step 64,
+//                       4-stage TMA ring, two TMEM accumulators; warp 0 loads,
+//                       warp 1 issues tcgen05.mma, warps 2-5 drain TMEM and
+//                       store bf16 while the next tile accumulates.
 #include "kernels.cuh"
 
 namespace sla {
@@ -37,6 +38,10 @@ constexpr int OFF_BAR = NST * STAGE;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
 }  // namespace
 
+// Persistent: CTA c takes tiles c, c + G, c + 2G, ... with the M tile index
+// fastest, so CTAs running at the same time share their B (h) tiles in L2.
+// Two TMEM accumulators (2 x 256 columns): the epilogue of one tile overlaps
+// the main loop of the next.
 __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
                                                            const __grid_constant__ CUtensorMap mapB,
                                                            MargArgs a) {
@@ -45,14 +50,15 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
                                            ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint64_t* empty = full + NST;
-  uint64_t* acc_bar = empty + NST;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+  uint64_t* acc_full = empty + NST;   // [2]
+  uint64_t* acc_empty = acc_full + 2; // [2]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * BM, bh = blockIdx.z;
-  const int nvalid_chunks = min(4, (a.NN - n0 + 63) / 64);
+  const int Mt = (a.Tq + BM - 1) / BM, Nt = (a.NN + BN - 1) / BN;
+  const int ntiles = Mt * Nt * a.BH;
 
   if (w == 1) {
-    tmem_alloc(tslot, 256);
+    tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
@@ -60,7 +66,10 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(acc_bar, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&acc_full[x], 1);
+      mbar_init(&acc_empty[x], 128);
+    }
     fence_barrier_init();
   }
   tc_fence_before();
@@ -72,45 +81,71 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
     if (ln == 0) {
       tma_prefetch_desc(&mapA);
       tma_prefetch_desc(&mapB);
-      for (int kt = 0; kt < a.ktiles; ++kt) {
-        const int s = kt % NST;
-        if (kt >= NST && !mbar_wait(&empty[s], ((kt / NST) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) break;
-        uint8_t* sA = sm + s * STAGE;
-        uint8_t* sB = sA + A_BYTES;
-        mbar_arrive_expect_tx(&full[s], A_BYTES + nvalid_chunks * 8192);
-        tma_load_3d(sA, &mapA, &full[s], kt * BK, m0, bh);
-        for (int c = 0; c < nvalid_chunks; ++c)
-          tma_load_3d(sB + c * 8192, &mapB, &full[s], n0 + c * 64, kt * BK, bh);
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+        const int m0 = (t % Mt) * BM, n0 = ((t / Mt) % Nt) * BN, bh = t / (Mt * Nt);
+        const int nvalid_chunks = min(4, (a.NN - n0 + 63) / 64);
+        for (int kt = 0; kt < a.ktiles; ++kt, ++it) {
+          const int s = it % NST;
+          if (it >= NST && !mbar_wait(&empty[s], ((it / NST) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sA = sm + s * STAGE;
+          uint8_t* sB = sA + A_BYTES;
+          mbar_arrive_expect_tx(&full[s], A_BYTES + nvalid_chunks * 8192);
+          tma_load_3d(sA, &mapA, &full[s], kt * BK, m0, bh);
+          for (int c = 0; c < nvalid_chunks; ++c)
+            tma_load_3d(sB + c * 8192, &mapB, &full[s], n0 + c * 64, kt * BK, bh);
+        }
       }
     }
   } else if (w == 1) {
     if (ln == 0) {
       const uint32_t id = idesc_bf16(BM, BN, false, true);
+      int it = 0, lt = 0;
       bool ok = true;
-      for (int kt = 0; kt < a.ktiles; ++kt) {
-        const int s = kt % NST;
-        if (!mbar_wait(&full[s], (kt / NST) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t sA = smem_u32(sm + s * STAGE);
-        const uint32_t sB = sA + A_BYTES;
-#pragma unroll
-        for (int k = 0; k < BK / 16; ++k) {
-          const uint64_t ad = sdesc_sw128(sA + k * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(sB + k * 2048, 8192, 1024);
-          umma_ss(tacc, ad, bd, id, (kt > 0 || k > 0) ? 1u : 0u);
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++lt) {
+        const int ab = lt & 1;
+        if (lt >= 2 && !mbar_wait(&acc_empty[ab], ((lt >> 1) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
+          ok = false;
+          break;
         }
-        umma_commit(&empty[s]);
+        tc_fence_after();
+        const uint32_t d = tacc + 256 * ab;
+        for (int kt = 0; kt < a.ktiles; ++kt, ++it) {
+          const int s = it % NST;
+          if (!mbar_wait(&full[s], (it / NST) & 1, a.err, DEV_TIMEOUT_TMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sA = smem_u32(sm + s * STAGE);
+          const uint32_t sB = sA + A_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t ad = sdesc_sw128(sA + k * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sB + k * 2048, 8192, 1024);
+            umma_ss(d, ad, bd, id, (kt > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&acc_full[ab]);
       }
-      if (ok) umma_commit(acc_bar);
     }
   } else {
     const int q4 = w & 3;
     const int row = 32 * q4 + ln;
-    const int i = m0 + row;
-    const bool ok = mbar_wait(acc_bar, 0, a.err, DEV_TIMEOUT_MMA);
-    if (__all_sync(0xffffffffu, ok)) {
+    int lt = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
+      const int m0 = (t % Mt) * BM, n0 = ((t / Mt) % Nt) * BN, bh = t / (Mt * Nt);
+      const int ab = lt & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (lt >> 1) & 1, a.err, DEV_TIMEOUT_MMA)))
+        break;
       tc_fence_after();
-      const uint32_t taddr = tacc + ((uint32_t)(32 * q4) << 16);
+      const int i = m0 + row;
+      const uint32_t taddr = tacc + 256 * ab + ((uint32_t)(32 * q4) << 16);
       __nv_bfloat16* out = a.Hout + ((int64_t)bh * a.Tq + i) * a.NN;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
@@ -132,13 +167,15 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
           }
         }
       }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[ab]);
     }
   }
   tc_fence_before();
   __syncthreads();
   if (w == 1) {
     tc_fence_after();
-    tmem_dealloc(tacc, 256);
+    tmem_dealloc(tacc, 512);
   }
 }
 
@@ -155,8 +192,13 @@ cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, c
   cudaError_t e = cudaFuncSetAttribute(marg_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.NN + BN - 1) / BN, (a.Tq + BM - 1) / BM, BH);
-  marg_gemm_kernel<<<grid, 192, SMEM, s>>>(mapA, mapB, a);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ntiles = ((a.NN + BN - 1) / BN) * ((a.Tq + BM - 1) / BM) * BH;
+  MargArgs b = a;
+  b.BH = BH;
+  marg_gemm_kernel<<<ntiles < sms ? ntiles : sms, 192, SMEM, s>>>(mapA, mapB, b);
   return cudaGetLastError();
 }
 
