@@ -26,7 +26,7 @@ struct Plan {
 inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
-  size_t err, qc, kc, qr, kr, kmean, mm, hagg;            // sla_workspace_size ...
+  size_t err, qc, kc, qr, kr, kmean, keys, mm, hagg;      // sla_workspace_size ...
   size_t q8, k8, scq, sck, end;                           // ... (+ FP8 operands)
   size_t mc, lut, hz, end_attn;                           // + sla_attention extras
   size_t hq, hk, hv, ho, end_host;                        // + sla_attention_host staging
@@ -41,6 +41,7 @@ Layout layout_of(const Plan& p) {
   L.qr = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.d * 4);
   L.kr = o;    o = align_up(o + (size_t)p.BH * p.Tkv * p.d * 4);
   L.kmean = o; o = align_up(o + (size_t)p.BH * p.d * 4);
+  L.keys = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.Tkv * 4);
   L.mm = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkvp * 2);
   L.hagg = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.NN * 2);
   const size_t q8 = p.fp8 ? (size_t)p.BH * p.Tq * 64 * p.d : 0;
@@ -208,6 +209,7 @@ sla_status_t predict_mask_impl(const Plan& pl, const sla_params_t* p, const void
   SelectArgs sa;
   sa.Qc = qsrc;
   sa.Kc = ksrc;
+  sa.keys = at<uint32_t>(ws, L.keys);
   sa.mc = mc;
   sa.lut = lut;
   sa.d = pl.d;

@@ -17,9 +17,17 @@ struct PoolArgs {
 struct SelectArgs {
   const float* Qc;  // [BH][Tq][d] pooled (and routed) queries
   const float* Kc;  // [BH][Tkv][d]
+  uint32_t* keys;   // [BH][Tq][Tkv] scratch: order-preserving logit keys
   int8_t* mc;       // [BH][Tq][Tkv]
   int32_t* lut;     // [BH][Tq][nh]
-  int d, Tq, Tkv, nh, nl;
+  int d, Tq, Tkv, nh, nl, BH;
+};
+
+struct LogitArgs {
+  const float* Qc;
+  const float* Kc;
+  uint32_t* keys;
+  int d, Tq, Tkv;
 };
 
 struct KvPrepArgs {
@@ -67,7 +75,7 @@ cudaError_t launch_pool(const PoolArgs& a, int D, int BH, cudaStream_t s);
 cudaError_t launch_router(const float* Qc, const float* Kc, float* Qr, float* Kr, float* kmean,
                           const float* Wq, const float* Wk, bool smooth, int BH, int Tq, int Tk,
                           int N, int bs, int D, cudaStream_t s);
-size_t select_smem_bytes(int D, int Tk);
+size_t select_smem_bytes(int Tk);
 cudaError_t launch_select(const SelectArgs& a, int BH, cudaStream_t s);
 
 // mapO: hz viewed as (a: d, b: d, j: T_kv, bh) tiles of 64 x d for TMA stores.

@@ -5,8 +5,9 @@
 // allocation-free hot loop, embedders whose memory is fully pre-planned by an
 // arena they do not control, or runtimes that forbid allocation after start-up.
 // For them this file keeps the scratch that mask prediction needs (the error
-// word and the pooled / routed Q and K blocks) in one statically sized device
-// array, so sla_predict_mask_noalloc needs only the caller's inputs and outputs.
+// word, the pooled / routed Q and K blocks and the logit keys) in one
+// statically sized device array, so sla_predict_mask_noalloc needs only the
+// caller's inputs and outputs.
 //
 // The array lives for as long as the library is loaded, on every GPU the
 // library is used on.  Its device address is looked up once per device (on the
@@ -65,8 +66,9 @@ extern "C" sla_status_t sla_predict_mask_noalloc(const sla_params_t* p, const vo
     return SLA_ERR_INVALID_ARG;
   const int BH = p->B * p->H, d = p->d;
   const bool route = Wq || Wk || p->smooth_k;
-  // scratch: error word | Q_c | K_c | (routed Q_c | routed K_c | token mean of K)
-  const size_t off_qc = 256;
+  // scratch: error word | logit keys | Q_c | K_c | (routed Q_c | routed K_c | token mean of K)
+  const size_t off_keys = 256;
+  const size_t off_qc = off_keys + up256((size_t)BH * Tq * Tkv * 4);
   const size_t off_kc = off_qc + up256((size_t)BH * Tq * d * 4);
   const size_t off_qr = off_kc + up256((size_t)BH * Tkv * d * 4);
   const size_t off_kr = off_qr + (route ? up256((size_t)BH * Tq * d * 4) : 0);
@@ -110,6 +112,7 @@ extern "C" sla_status_t sla_predict_mask_noalloc(const sla_params_t* p, const vo
   sla::SelectArgs sa;
   sa.Qc = qsrc;
   sa.Kc = ksrc;
+  sa.keys = reinterpret_cast<uint32_t*>(s + off_keys);
   sa.mc = mc;
   sa.lut = lut;
   sa.d = d;

@@ -202,13 +202,14 @@ sla_status_t sla_attention_host(const sla_params_t* p, const void* Q_host, const
  * sla_predict_mask without a workspace argument.  The pages describe no such
  * call: it exists for callers that cannot allocate device memory when they
  * predict the mask (allocation-free hot loops, host callbacks, memory planned
- * up front by an arena the caller does not own).  Its scratch (error word and
- * pooled / routed Q and K blocks) lives in one static device array of
+ * up front by an arena the caller does not own).  Its scratch (error word,
+ * pooled / routed Q and K blocks, logit keys) lives in one static device array of
  * SLA_NOALLOC_SCRATCH_BYTES that every GPU using the library holds until the
  * process exits.  Inputs, outputs and results are those of sla_predict_mask.
- *   - Problems whose scratch exceeds the array (B*H*(T_q + T_kv)*d*4 bytes,
- *     twice that plus B*H*d*4 with a router or smooth-K, plus 256) return
- *     SLA_ERR_WORKSPACE before any launch.
+ *   - Problems whose scratch exceeds the array (B*H*T_q*T_kv*4 bytes of
+ *     logit keys plus B*H*(T_q + T_kv)*d*4, twice the latter plus B*H*d*4
+ *     with a router or smooth-K, plus 256) return SLA_ERR_WORKSPACE before
+ *     any launch.
  *   - The first call on a device looks up the array's address on that device
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
  *   - All calls on a device share the array: calls that overlap on the GPU
