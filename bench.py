@@ -113,10 +113,11 @@ def bus_id_of(dev):
         return None
 
 
-def fused_traffic_per_launch(d: int):
+def fused_traffic_per_launch(workload: str, heads: int, qk: str):
     """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    or None if the kernel source changed since those counters were taken."""
-    path = os.path.join(ROOT, "profiles", "fused_wan1.3b_sla_traffic.txt")
+    or None if the summary is for another workload or the kernel source changed
+    since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"fused_{workload}_traffic.txt")
     src = os.path.join(ROOT, "block_sparse_linear_pool_b200", "csrc", "fused.cu")
     if not os.path.exists(path):
         return None
@@ -127,6 +128,8 @@ def fused_traffic_per_launch(d: int):
             k, v = line.split("=", 1)
             vals[k.strip()] = v.strip()
     if vals.get("fused_cu_sha256_16") != sha:
+        return None
+    if vals.get("heads") != str(heads) or vals.get("qk", "bf16") != qk:
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
@@ -169,10 +172,21 @@ def flop_model(cfg, dims, lut_np):
 
 
 # --------------------------------------------------------------------------- our arm
+def reduce_over_ranks(ms_total: float, flops_per_step: float, device):
+    """Whole-job figures of a data-parallel run: the slowest rank's timed-region
+    duration (max over ranks) and the executed FLOPs of one step summed over the
+    ranks' independent problems.  Every rank must call this, in the same order."""
+    t_ms = torch.tensor([ms_total], dtype=torch.float64, device=device)
+    t_fl = torch.tensor([flops_per_step], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t_ms, op=torch.distributed.ReduceOp.MAX)
+    torch.distributed.all_reduce(t_fl, op=torch.distributed.ReduceOp.SUM)
+    return float(t_ms.item()), float(t_fl.item())
+
+
 def run_ours(args, rank, world, dev):
     torch.cuda.set_device(dev)
     over = {} if args.heads is None else {"H": args.heads}
-    data, w = I.make_workload(args.workload, device=f"cuda:{dev}", **over)
+    data, w = I.make_workload(args.workload, device=f"cuda:{dev}", problem=rank, **over)
     cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"], qk=args.qk)
     Q, K, V = (data[k].to(dev) for k in ("Q", "K", "V"))
     O = torch.empty_like(Q)
@@ -252,10 +266,9 @@ def run_ours(args, rank, world, dev):
     ms_total = start.elapsed_time(end)
     stage_ms = [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)) / args.steps
                 for i in range(4)]
+    job_flops = fl["step_exec"]
     if world > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_total = float(t.item())
+        ms_total, job_flops = reduce_over_ranks(ms_total, fl["step_exec"], torch.device(f"cuda:{dev}"))
     code, detail = bnd.sla_get_device_status(ws)
     if code != 0:
         raise RuntimeError(f"device status {code} ({detail}) after timing")
@@ -267,9 +280,9 @@ def run_ours(args, rank, world, dev):
         fused_ms = stage_ms[3]
         ach = fl["fused_alg"] / (fused_ms * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])
-        traffic = fused_traffic_per_launch(d)
+        traffic = fused_traffic_per_launch(args.workload, H, args.qk)
         result = {
-            "metric": METRIC, "value": round(fl["step_exec"] * world / (ms_total * 1e-3 / args.steps) / 1e12, 3),
+            "metric": METRIC, "value": round(job_flops / (ms_total * 1e-3 / args.steps) / 1e12, 3),
             "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if args.qk == "bf16" else "bf16+e4m3",

@@ -131,14 +131,19 @@ WORKLOADS = {
 }
 
 
-def make_workload(name: str, device: Optional[str] = None, **overrides):
-    """Inputs of a named workload (see WORKLOADS) as a dict, plus its settings."""
+def make_workload(name: str, device: Optional[str] = None, problem: int = 0, **overrides):
+    """Inputs of a named workload (see WORKLOADS) as a dict, plus its settings.
+
+    `problem` selects one of many independent problems of the same shape (seeds
+    4p .. 4p+3); problem 0 is the default instance.  Data-parallel runs give each
+    rank its own problem."""
     cfg = dict(WORKLOADS[name])
     cfg.update(overrides)
     if cfg["kind"] == "block_mean":
-        data = block_mean_inputs(B=cfg["B"], H=cfg["H"], N=cfg["N"], d=cfg["d"])
+        data = block_mean_inputs(B=cfg["B"], H=cfg["H"], N=cfg["N"], d=cfg["d"], seed=problem)
     else:
+        seeds = tuple(4 * problem + i for i in range(4))
         data = grid_field_inputs(B=cfg["B"], H=cfg["H"], d=cfg["d"], grid=cfg["grid"],
-                                 combine=cfg["combine"], device=device)
+                                 combine=cfg["combine"], seeds=seeds, device=device)
         cfg["N"] = int(np.prod(cfg["grid"]))
     return data, cfg
