@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libsla.so")
 
 SLA_COMBINE_PROJ, SLA_COMBINE_ALPHA = 0, 1
 SLA_QK_BF16, SLA_QK_FP8_E4M3 = 0, 1
+SLA_PHI_SOFTMAX, SLA_PHI_ELU1 = 0, 1
 
 STATUS = {
     0: "SLA_OK", 1: "SLA_ERR_INVALID_ARG", 2: "SLA_ERR_UNSUPPORTED", 3: "SLA_ERR_WORKSPACE",
@@ -52,6 +53,7 @@ class sla_params_t(ctypes.Structure):
         ("eps", ctypes.c_float),
         ("stride_q", ctypes.c_int64 * 3), ("stride_k", ctypes.c_int64 * 3),
         ("stride_v", ctypes.c_int64 * 3), ("stride_o", ctypes.c_int64 * 3),
+        ("phi", ctypes.c_int), ("linear_over_all", ctypes.c_int),
     ]
 
 
@@ -123,6 +125,8 @@ class SlaConfig:
     qk: str = "bf16"          # "bf16" or "fp8_e4m3"
     smooth_k: bool = False
     eps: float = 1e-5
+    phi: str = "softmax"      # "softmax" ([SLA] Fig. 4) or "elu1" ([SLA] Table 2 ablation)
+    linear_over_all: bool = False  # linear branch over every key block ([SLA] §7 item 2)
 
 
 def make_params(Q: torch.Tensor, cfg: SlaConfig, K=None, V=None, O=None) -> sla_params_t:
@@ -133,6 +137,10 @@ def make_params(Q: torch.Tensor, cfg: SlaConfig, K=None, V=None, O=None) -> sla_
     p.qk_prec = SLA_QK_BF16 if cfg.qk == "bf16" else SLA_QK_FP8_E4M3
     p.smooth_k = int(cfg.smooth_k)
     p.eps = cfg.eps
+    if cfg.phi not in ("softmax", "elu1"):
+        raise ValueError(f"phi must be 'softmax' or 'elu1', not {cfg.phi!r}")
+    p.phi = SLA_PHI_SOFTMAX if cfg.phi == "softmax" else SLA_PHI_ELU1
+    p.linear_over_all = int(cfg.linear_over_all)
     p.stride_q = _strides(Q)
     p.stride_k = _strides(K if K is not None else Q)
     p.stride_v = _strides(V if V is not None else Q)

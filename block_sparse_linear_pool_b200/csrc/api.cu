@@ -21,6 +21,8 @@ constexpr size_t kAlign = 256;
 struct Plan {
   int B, H, N, d, BH, Tq, Tkv, nh, nl, NN, Tkvp;
   bool fp8;  // Q K^T on E4M3 with per-block scales
+  int phi;   // sla_phi_t
+  bool all;  // linear branch over every key block
 };
 
 inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
@@ -88,6 +90,8 @@ sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
   if (!(p->eps >= 0.f) || !std::isfinite(p->eps)) return SLA_ERR_INVALID_ARG;
   if (p->combine != SLA_COMBINE_PROJ && p->combine != SLA_COMBINE_ALPHA) return SLA_ERR_INVALID_ARG;
   if (p->qk_prec != SLA_QK_BF16 && p->qk_prec != SLA_QK_FP8_E4M3) return SLA_ERR_INVALID_ARG;
+  if (p->phi != SLA_PHI_SOFTMAX && p->phi != SLA_PHI_ELU1) return SLA_ERR_INVALID_ARG;
+  if (p->linear_over_all != 0 && p->linear_over_all != 1) return SLA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if (p->qk_prec == SLA_QK_FP8_E4M3 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if (p->b_q != 64 || p->b_kv != 64) return SLA_ERR_UNSUPPORTED;
@@ -106,6 +110,8 @@ sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
   pl->NN = p->d * p->d + p->d;
   pl->Tkvp = (pl->Tkv + 7) & ~7;
   pl->fp8 = p->qk_prec == SLA_QK_FP8_E4M3;
+  pl->phi = p->phi;
+  pl->all = p->linear_over_all != 0;
   return SLA_OK;
 }
 
@@ -239,6 +245,7 @@ sla_status_t precompute_impl(const Plan& pl, const sla_params_t* p, const void* 
   a.N = pl.N;
   a.Tkv = pl.Tkv;
   a.nitems = pl.BH * pl.Tkv;
+  a.phi = pl.phi;
   return cuda_status(launch_kv_prep(mk, mv, mo, a, pl.d, s));
 }
 
@@ -246,7 +253,7 @@ sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, vo
                             cudaStream_t s) {
   const Layout L = layout_of(pl);
   __nv_bfloat16* mm = at<__nv_bfloat16>(ws, L.mm);
-  SLA_TRY(cuda_status(launch_marg_matrix(mc, mm, pl.BH, pl.Tq, pl.Tkv, pl.Tkvp, s)));
+  SLA_TRY(cuda_status(launch_marg_matrix(mc, mm, pl.BH, pl.Tq, pl.Tkv, pl.Tkvp, pl.all, s)));
   CUtensorMap ma, mb;
   const uint64_t da[3] = {(uint64_t)pl.Tkvp, (uint64_t)pl.Tq, (uint64_t)pl.BH};
   const uint64_t sa[2] = {(uint64_t)pl.Tkvp * 2, (uint64_t)pl.Tq * pl.Tkvp * 2};
@@ -339,6 +346,7 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.eps = p->eps;
   a.scale_q = scq;
   a.scale_k = sck;
+  a.phi = pl.phi;
   return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, pl.fp8, pl.BH, s));
 }
 
@@ -394,6 +402,8 @@ void sla_params_default(sla_params_t* p, int B, int H, int N, int d, float k_h, 
   p->qk_prec = SLA_QK_BF16;
   p->smooth_k = 0;
   p->eps = 1e-5f;
+  p->phi = SLA_PHI_SOFTMAX;
+  p->linear_over_all = 0;
   const int64_t s[3] = {(int64_t)H * N * d, (int64_t)N * d, (int64_t)d};
   for (int i = 0; i < 3; ++i) {
     p->stride_q[i] = s[i];
@@ -586,6 +596,6 @@ const char* sla_status_string(sla_status_t s) {
   return "SLA_ERR_UNKNOWN";
 }
 
-int sla_abi_version(void) { return 100; }
+int sla_abi_version(void) { return 101; }
 
 }  // extern "C"

@@ -39,6 +39,7 @@
 // Linear branch with unnormalised feature map: for e_a = 2^((q_a - max q) log2 e)
 // and s = sum_a e_a, phi(q) = e / s, so
 //     phi(q) H / (phi(q) Z + eps) = (e H) / (e Z + s eps)      exactly.
+// With the elu + 1 feature map ([SLA] Table 2 ablation) e = phi(q) and s = 1.
 #include "kernels.cuh"
 
 namespace sla {
@@ -450,6 +451,10 @@ __global__ void __launch_bounds__(192, 2)
         for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fmaxf(__low2float(p2[e]), __high2float(p2[e])));
       }
       const float nmx = -mx * LOG2E;
+      // softmax over d: e = 2^((q - max q) log2 e), phi = e / sum(e);
+      // elu + 1: e = phi itself, and the denominator's sum is 1
+      const bool elu = a.phi == 1;
+      auto feat = [&](float x) { return elu ? (x > 0.f ? x + 1.f : ex2(x * LOG2E)) : ex2(fmaf(x, LOG2E, nmx)); };
 #pragma unroll 4
       for (int c = 0; c < D / 8; ++c) {
         uint8_t* qp = sQ + (c / 8) * 16384 + sw128_offset(r, (c % 8) * 16);
@@ -458,13 +463,13 @@ __global__ void __launch_bounds__(192, 2)
         uint32_t o[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          o[e] = pack_bf16x2(ex2(fmaf(__low2float(p2[e]), LOG2E, nmx)),
-                             ex2(fmaf(__high2float(p2[e]), LOG2E, nmx)));
+          o[e] = pack_bf16x2(feat(__low2float(p2[e])), feat(__high2float(p2[e])));
           const __nv_bfloat162 eb = *reinterpret_cast<const __nv_bfloat162*>(&o[e]);
           esum += __low2float(eb) + __high2float(eb);
         }
         *reinterpret_cast<uint4*>(qp) = make_uint4(o[0], o[1], o[2], o[3]);
       }
+      if (elu) esum = 1.f;
       fence_proxy_async_smem();
       mbar_arrive(phiq_ready);
       // phi~(q_r) . Z_i (Z arrives with this half's H tile)

@@ -35,6 +35,7 @@ struct KvPrepArgs {
   __nv_bfloat16* hz;     // [BH][Tkv][d*d + d]
   int* err;
   int H, N, Tkv, nitems;
+  int phi;               // 0 softmax over d, 1 elu + 1
 };
 
 struct MargArgs {
@@ -69,6 +70,7 @@ struct FusedArgs {
   float eps;
   const float* scale_q;   // FP8 path: per (head, query block) scale of Q, else nullptr
   const float* scale_k;   // FP8 path: per (head, key block) scale of K, else nullptr
+  int phi;                // 0 softmax over d, 1 elu + 1
 };
 
 cudaError_t launch_pool(const PoolArgs& a, int D, int BH, cudaStream_t s);
@@ -83,7 +85,7 @@ cudaError_t launch_kv_prep(const CUtensorMap& mapK, const CUtensorMap& mapV, con
                            const KvPrepArgs& a, int D, cudaStream_t s);
 
 cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int Tq, int Tkv,
-                               int Tkvp, cudaStream_t s);
+                               int Tkvp, bool all, cudaStream_t s);
 cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const MargArgs& a,
                              int BH, cudaStream_t s);
 

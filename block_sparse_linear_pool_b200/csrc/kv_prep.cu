@@ -1,7 +1,8 @@
 // Per-key-block linear-attention statistics ("SLA: Beyond Sparsity in
 // Diffusion Transformers via Fine-Tunable Sparse-Linear Attention", §2 Q2
 // step 3 and Fig. 4 "Linear Attention Precomputation"):
-//     h_j = phi(K_j)^T V_j,   z_j = rowsum(phi(K_j)^T),   phi = softmax over d.
+//     h_j = phi(K_j)^T V_j,   z_j = rowsum(phi(K_j)^T),   phi = softmax over d
+// (or elu + 1, the feature-map ablation of the same page's Table 2).
 // With the SLA combine, Proj's weight W is folded in (h_j W^T is stored):
 // Proj(O^l) = phi(Q) (H W^T) / den + b because den is a per-row scalar.
 //
@@ -146,19 +147,27 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
           x[v * 8 + 2 * u + 1] = __high2float(p2[u]);
         }
       }
-      float m = x[0];
-#pragma unroll
-      for (int e = 1; e < NE; ++e) m = fmaxf(m, x[e]);
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
       constexpr float LOG2E = 1.4426950408889634f;
-      float sum = 0.f;
+      float inv;
+      if (a.phi == 1) {  // elu(x) + 1
 #pragma unroll
-      for (int e = 0; e < NE; ++e) {
-        x[e] = exp2f((x[e] - m) * LOG2E);
-        sum += x[e];
+        for (int e = 0; e < NE; ++e) x[e] = x[e] > 0.f ? x[e] + 1.f : exp2f(x[e] * LOG2E);
+        inv = (t < cnt) ? 1.f : 0.f;
+      } else {           // softmax over d
+        float m = x[0];
+#pragma unroll
+        for (int e = 1; e < NE; ++e) m = fmaxf(m, x[e]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < NE; ++e) {
+          x[e] = exp2f((x[e] - m) * LOG2E);
+          sum += x[e];
+        }
+        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+        inv = (t < cnt) ? 1.f / sum : 0.f;
       }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      const float inv = (t < cnt) ? 1.f / sum : 0.f;  // padding tokens of a partial block: phi = 0
+      // padding tokens of a partial block get phi = 0 (inv = 0)
 #pragma unroll
       for (int v = 0; v < NE / 8; ++v) {
         uint4 q;

@@ -8,7 +8,8 @@
 // a (T_q x T_kv) x (T_kv x (d^2 + d)) GEMM on the tensor cores (0/1 weights
 // are exact in bf16, accumulation in fp32).
 //
-//   marg_matrix_kernel  M_c (int8) -> Mmarg (bf16 0/1, rows padded to T_kvp)
+//   marg_matrix_kernel  M_c (int8) -> Mmarg (bf16 0/1, rows padded to T_kvp); all
+//                       ones for the variant whose linear branch covers every block
 //   marg_gemm_kernel    persistent, 128 x 256 output tiles, K step 64,
 //                       4-stage TMA ring, two TMEM accumulators; warp 0 loads,
 //                       warp 1 issues tcgen05.mma, warps 2-5 drain TMEM and
@@ -18,14 +19,14 @@
 namespace sla {
 
 __global__ void marg_matrix_kernel(const int8_t* __restrict__ mc, __nv_bfloat16* __restrict__ mm,
-                                   int BH, int Tq, int Tkv, int Tkvp) {
+                                   int BH, int Tq, int Tkv, int Tkvp, bool all) {
   const int64_t total = (int64_t)BH * Tq * Tkvp;
   const __nv_bfloat16 one = __float2bfloat16(1.f), zero = __float2bfloat16(0.f);
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
     const int j = (int)(e % Tkvp);
     const int64_t row = e / Tkvp;  // bh * Tq + i
-    mm[e] = (j < Tkv && mc[row * Tkv + j] == 0) ? one : zero;
+    mm[e] = (j < Tkv && (all || mc[row * Tkv + j] == 0)) ? one : zero;
   }
 }
 
@@ -180,10 +181,10 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
 }
 
 cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int Tq, int Tkv,
-                               int Tkvp, cudaStream_t s) {
+                               int Tkvp, bool all, cudaStream_t s) {
   const int64_t total = (int64_t)BH * Tq * Tkvp;
   const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
-  marg_matrix_kernel<<<blocks, 256, 0, s>>>(mc, mm, BH, Tq, Tkv, Tkvp);
+  marg_matrix_kernel<<<blocks, 256, 0, s>>>(mc, mm, BH, Tq, Tkv, Tkvp, all);
   return cudaGetLastError();
 }
 

@@ -60,6 +60,11 @@ typedef enum {
                            64-row block (max|x|/448) before Q K^T */
 } sla_qk_prec_t;
 
+typedef enum {
+  SLA_PHI_SOFTMAX = 0,  /* phi(x) = softmax of x over the head dimension ([SLA] Fig. 4) */
+  SLA_PHI_ELU1 = 1      /* phi(x) = elu(x) + 1, the ablation of [SLA] Table 2 */
+} sla_phi_t;
+
 typedef struct {
   int B, H, N, d;      /* batch, heads, tokens, head dimension */
   int b_q, b_kv;       /* query / key-value block sizes ([SLA] §4 notation: 64) */
@@ -74,9 +79,13 @@ typedef struct {
   int64_t stride_k[3];
   int64_t stride_v[3];
   int64_t stride_o[3];
+  int phi;             /* sla_phi_t: the linear branch's feature map, for K and Q */
+  int linear_over_all; /* 1: H_i, Z_i sum h_j, z_j over every key block instead of the
+                          marginal ones (the released code's variant, [SLA] §7 item 2) */
 } sla_params_t;
 
-/* Fills a params struct for contiguous [B,H,N,d] tensors, b = 64, eps = 1e-5. */
+/* Fills a params struct for contiguous [B,H,N,d] tensors, b = 64, eps = 1e-5,
+ * bf16 Q K^T, softmax feature map, linear branch over the marginal blocks. */
 void sla_params_default(sla_params_t* p, int B, int H, int N, int d, float k_h, float k_l,
                         int combine);
 
@@ -116,7 +125,8 @@ sla_status_t sla_predict_mask(const sla_params_t* p, const void* Q, const void* 
  * Per-key-block linear-attention statistics ([SLA] §2 Q2 step 3, Fig. 4
  * "Linear Attention Precomputation"):
  *   h_j = phi(K_j)^T V_j  (d x d),   z_j = rowsum(phi(K_j)^T)  (d),
- * phi = softmax over the head dimension, only real tokens of a partial block.
+ * phi = softmax over the head dimension (elu + 1 with phi = SLA_PHI_ELU1),
+ * only real tokens of a partial block.
  * For the SLA combine, Proj's weight (fp32 [d][d], nn.Linear convention) is
  * folded in: h_j W^T is stored, which is exact by linearity because
  * Proj(O^l) = (phi(Q) H / den) W^T + b = phi(Q) (H W^T) / den + b.  Pass
@@ -134,7 +144,8 @@ sla_status_t sla_precompute_linear(const sla_params_t* p, const void* K, const v
  * for every query block i
  *   O^s_i = softmax attention over the tokens of its critical blocks (lut),
  *           computed block by block with an online softmax;
- *   H_i = sum of h_j, Z_i = sum of z_j over its marginal blocks (mc == 0);
+ *   H_i = sum of h_j, Z_i = sum of z_j over its marginal blocks (mc == 0;
+ *         every block with linear_over_all);
  *   O^l_i = phi(Q_i) H_i / (phi(Q_i) Z_i + eps)        ([SLA] Eq. 3-4);
  *   negligible blocks (mc == -1) are never read;
  *   SLA:  O = O^s + O^l W^T + proj_b  (W folded into hz; proj_b fp32 [d] or NULL)
@@ -154,7 +165,8 @@ sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, co
  * sla_fused_forward on the same stream and workspace).
  *
  * sla_aggregate_marginal: for every query block i, [H_i^T | Z_i] = sum over
- * its marginal blocks (mc == 0) of [h_j^T | z_j] ([SLA] §2 Q2 step 3,
+ * its marginal blocks (mc == 0; every block with linear_over_all) of
+ * [h_j^T | z_j] ([SLA] §2 Q2 step 3,
  * marginal blocks accumulate h_j and z_j), computed as one 0/1-matrix product per head on
  * the tensor cores; the result stays in the workspace.
  *

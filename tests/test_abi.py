@@ -65,6 +65,12 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
     p.stride_q[2] = 60  # not a multiple of 8 / smaller than d
     assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == 1
     p = _params()
+    p.phi = 2  # no such feature map
+    assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == 1
+    p = _params()
+    p.linear_over_all = 7
+    assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == 1
+    p = _params()
     ws = (ctypes.c_uint8 * 1024)()
     # NULL tensors
     assert L.sla_predict_mask(ctypes.byref(p), None, None, None, None, None, None, ws, 1024, None) == 1
@@ -84,6 +90,12 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
                           ctypes.c_void_p(1 << 20), need, None) == 2
 
 
+def test_defaults_are_the_pages_main_method(L):
+    p = _params()
+    assert (p.phi, p.linear_over_all, p.qk_prec, p.smooth_k) == (0, 0, 0, 0)
+    assert abs(p.eps - 1e-5) < 1e-12
+
+
 def test_workspace_sizes_grow_with_the_problem(L):
     small, big = _params(N=1024), _params(N=32760, H=12, d=128)
     assert bnd.sla_workspace_size(small) < bnd.sla_workspace_size(big)
@@ -95,4 +107,4 @@ def test_workspace_sizes_grow_with_the_problem(L):
 def test_status_strings(L):
     for code, name in bnd.STATUS.items():
         assert L.sla_status_string(code).decode() == name
-    assert L.sla_abi_version() == 100
+    assert L.sla_abi_version() == 101

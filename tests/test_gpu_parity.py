@@ -34,7 +34,7 @@ def _np(t):
 
 def _oparams(cfg: bnd.SlaConfig):
     return O.OracleParams(k_h=cfg.k_h, k_l=cfg.k_l, combine=cfg.combine, eps=cfg.eps,
-                          smooth_k=cfg.smooth_k)
+                          smooth_k=cfg.smooth_k, phi=cfg.phi, linear_over_all=cfg.linear_over_all)
 
 
 def _check_mask(Q, K, cfg, mc, lut, Wq=None, Wk=None):
@@ -152,6 +152,21 @@ def test_tiny_sla_workload():
 def test_small_shapes(B, H, N, d, kh, kl, combine):
     data = _small(B, H, N, d, seed=N + d)
     cfg = bnd.SlaConfig(k_h=kh, k_l=kl, combine=combine)
+    if combine == "proj":
+        data["Wq"] = data["Wk"] = None
+    _run(data, cfg)
+
+
+@pytest.mark.parametrize("B,H,N,d,kh,kl,combine,phi,over_all", [
+    (1, 2, 1000, 64, 0.10, 0.50, "proj", "elu1", False),    # elu + 1 feature map
+    (1, 2, 2049, 128, 0.05, 0.70, "alpha", "elu1", False),
+    (1, 2, 1000, 64, 0.10, 0.50, "alpha", "softmax", True),  # linear branch over every block
+    (1, 1, 3000, 128, 0.10, 0.40, "proj", "softmax", True),
+    (1, 1, 1500, 128, 0.10, 0.40, "proj", "elu1", True),
+])
+def test_code_variants(B, H, N, d, kh, kl, combine, phi, over_all):
+    data = _small(B, H, N, d, seed=N + d + 7)
+    cfg = bnd.SlaConfig(k_h=kh, k_l=kl, combine=combine, phi=phi, linear_over_all=over_all)
     if combine == "proj":
         data["Wq"] = data["Wk"] = None
     _run(data, cfg)
