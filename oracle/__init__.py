@@ -1,4 +1,4 @@
-"""fp64 CPU oracle of the SLA / SLA2 forward pass.
+"""fp64 CPU oracle of the SLA / SLA2 forward and backward passes.
 
 TEST INFRASTRUCTURE ONLY: imported by tests/, __graft_entry__.smoke() and the
 CPU-baseline leg of bench.py, never by the package block_sparse_linear_pool_b200.
@@ -23,4 +23,6 @@ from .sla import (  # noqa: F401
     forward_given_mask,
     forward,
     mask_grading,
+    feature_map_backward,
+    backward_given_mask,
 )

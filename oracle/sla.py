@@ -1,4 +1,5 @@
-"""Plain fp64 CPU oracle of the Sparse-Linear Attention forward pass (SLA and SLA2).
+"""Plain fp64 CPU oracle of the Sparse-Linear Attention forward and backward passes
+(SLA and SLA2).
 
 TEST INFRASTRUCTURE ONLY.  This module is the independent checker of the CUDA
 path: it shares no code, constants or helpers with the package
@@ -17,7 +18,8 @@ Sources, cited by page title and section:
   [SLA2] "SLA2: Sparse-Linear Attention with Learnable Routing and QAT"
          (summary page, arXiv 2602.12675): §3 SLA2 Design (alpha combine),
          §4 Learnable Router (pooling, proj_q/proj_k, row-wise Top-k),
-         §5 Quantization-aware Training (low-bit Q/K with scales).
+         §5 Quantization-aware Training (low-bit Q/K with scales), App. A
+         (backward pass: dH_i, dZ_i accumulated into the marginal blocks).
 
 Readings taken where the pages are silent:
   * the last block may be partial (N not a multiple of b): its pooled mean is
@@ -30,7 +32,9 @@ Readings taken where the pages are silent:
   * the 1e-5 epsilon ([SLA] §4 check 5) is added to the linear denominator;
   * Proj follows the nn.Linear convention Proj(x) = x W^T + b and is shared by
     all heads; router projections are bias-free d x d maps shared by all heads;
-  * alpha is one scalar per head.
+  * alpha is one scalar per head;
+  * the backward treats M_c as a constant (hard Top-k has no gradient) and
+    returns gradients for Q, K, V and the combine's parameters only.
 
 Parity unpinned: the FP8 path's exact values (only the tolerance bound is
 checked against this oracle's unquantised result).
@@ -376,3 +380,128 @@ def mask_grading(logits: np.ndarray, n_h: int, n_l: int, gap: float = 1e-4) -> n
     dh = np.abs(L - t_hi[..., None])
     dl = np.abs(L - t_lo[..., None])
     return (dh > gap) & (dl > gap)
+
+
+# --------------------------------------------------------------------------
+# Backward pass given the mask ([SLA] §4 check 6; [SLA2] App. A)
+# --------------------------------------------------------------------------
+def feature_map_backward(X: np.ndarray, fX: np.ndarray, dF: np.ndarray, kind: str = "softmax"):
+    """Gradient through phi, per token over the head dimension.
+
+    softmax: d x = phi * (d phi - <phi, d phi>);  elu + 1: d x = d phi * (1 if x > 0 else e^x).
+    """
+    X = np.asarray(X, dtype=np.float64)
+    if kind == "softmax":
+        return fX * (dF - (fX * dF).sum(axis=-1, keepdims=True))
+    if kind == "elu1":
+        return dF * np.where(X > 0, 1.0, np.exp(np.minimum(X, 0.0)))
+    raise ValueError(kind)
+
+
+def backward_given_mask(Q, K, V, Mc, dO, p: OracleParams, proj_w=None, proj_b=None, alpha=None):
+    """Gradients of L = sum(O * dO) for the forward of ``forward_given_mask``.
+
+    The mask M_c is a constant of the backward (hard Top-k / Bottom-k has no
+    gradient; SLA2 trains its router through a soft Top-k that is not part of
+    this path).  Both pages describe the same split ([SLA] §4 check 6,
+    [SLA2] App. A): the sparse branch takes the FlashAttention backward over
+    the critical blocks, and the linear branch forms dH_i, dZ_i per query block,
+    accumulates them into every marginal key block's dh_j, dz_j (the mirror of
+    the forward's H_i = sum h_j), and goes back through h_j = phi(K_j)^T V_j,
+    z_j = colsum phi(K_j) and through phi.
+
+    With o_s = P V (P the row softmax over critical keys), o_l = num / den,
+    num = phi(q) H_i, den = phi(q) . Z_i + eps, and the combine's
+      proj:  O = o_s + o_l W^T + b    ->  do_s = dO, do_l = dO W, dW = dO^T o_l, db = sum dO
+      alpha: O = a o_s + (1 - a) o_l  ->  do_s = a dO, do_l = (1 - a) dO,
+                                          da = sum (o_s - o_l) . dO
+    sparse:  dP = do_s V^T, D = rowsum(do_s * o_s), dS = P (dP - D),
+             dq = dS K / sqrt(d), dk = dS^T q / sqrt(d), dv = P^T do_s
+    linear:  g = do_l / den, gden = -(do_l . o_l) / den,
+             d phi(q) = g H_i^T + gden Z_i,  dH_i = phi(q)^T g,  dZ_i = gden^T phi(q),
+             dh_j = sum over query blocks with j marginal of dH_i (dz_j likewise),
+             d phi(k_t) = dh_j v_t + dz_j,  dv_t += dh_j^T phi(k_t)   (t in block j)
+    Returns a dict with dQ, dK, dV [B,H,N,d], dproj_w [d,d], dproj_b [d] and
+    dalpha [B,H] (zeros for the combine that does not use them).
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    dO = np.asarray(dO, dtype=np.float64)
+    B, H, N, d = Q.shape
+    dv_dim = V.shape[-1]
+    T_q = num_blocks(N, p.b_q)
+    T_kv = num_blocks(N, p.b_kv)
+    assert Mc.shape == (B, H, T_q, T_kv), Mc.shape
+    scale = 1.0 / np.sqrt(d)
+    W = None if proj_w is None else np.asarray(proj_w, dtype=np.float64)
+    dQ = np.zeros_like(Q)
+    dK = np.zeros_like(K)
+    dV = np.zeros_like(V)
+    dW = np.zeros((dv_dim, dv_dim))
+    db = np.zeros(dv_dim)
+    dalpha = np.zeros((B, H))
+    for bb in range(B):
+        for hh in range(H):
+            q, k, v, do = Q[bb, hh], K[bb, hh], V[bb, hh], dO[bb, hh]
+            h_stats, z_stats = linear_block_stats(k, v, p.b_kv, p.phi)
+            fQ = feature_map(q, p.phi)
+            fK = feature_map(k, p.phi)
+            dfQ = np.zeros_like(q)
+            dfK = np.zeros_like(k)
+            dh = np.zeros_like(h_stats)
+            dz = np.zeros_like(z_stats)
+            for i in range(T_q):
+                qs, qe = block_range(i, p.b_q, N)
+                qi, doi = q[qs:qe], do[qs:qe]
+                row = Mc[bb, hh, i]
+                # forward quantities of this block
+                crit = np.nonzero(row == 1)[0]
+                idx = np.concatenate([np.arange(*block_range(int(j), p.b_kv, N)) for j in crit])
+                s = (qi @ k[idx].T) * scale
+                e = np.exp(s - s.max(axis=1, keepdims=True))
+                P = e / e.sum(axis=1, keepdims=True)
+                o_s = P @ v[idx]
+                marg = np.arange(T_kv) if p.linear_over_all else np.nonzero(row == 0)[0]
+                Hi = h_stats[marg].sum(axis=0) if len(marg) else np.zeros((d, dv_dim))
+                Zi = z_stats[marg].sum(axis=0) if len(marg) else np.zeros(d)
+                fq = fQ[qs:qe]
+                den = fq @ Zi + p.eps
+                o_l = (fq @ Hi) / den[:, None]
+                # the combine
+                if p.combine == "proj":
+                    do_s = doi
+                    do_l = doi @ W if W is not None else np.zeros_like(doi)
+                    dW += doi.T @ o_l
+                    db += doi.sum(axis=0)
+                elif p.combine == "alpha":
+                    a = float(np.asarray(alpha, dtype=np.float64).reshape(B, H)[bb, hh]) \
+                        if np.ndim(alpha) else float(alpha)
+                    do_s = a * doi
+                    do_l = (1.0 - a) * doi
+                    dalpha[bb, hh] += ((o_s - o_l) * doi).sum()
+                else:
+                    raise ValueError(p.combine)
+                # sparse branch: FlashAttention backward over the critical tokens
+                dP = do_s @ v[idx].T
+                Drow = (do_s * o_s).sum(axis=1, keepdims=True)
+                dS = P * (dP - Drow)
+                dQ[bb, hh, qs:qe] += (dS @ k[idx]) * scale
+                dK[bb, hh, idx] += (dS.T @ qi) * scale
+                dV[bb, hh, idx] += P.T @ do_s
+                # linear branch
+                g = do_l / den[:, None]
+                gden = -(do_l * o_l).sum(axis=1) / den
+                dfQ[qs:qe] += g @ Hi.T + gden[:, None] * Zi[None, :]
+                dHi = fq.T @ g
+                dZi = (gden[:, None] * fq).sum(axis=0)
+                for j in marg:
+                    dh[j] += dHi
+                    dz[j] += dZi
+            for j in range(T_kv):
+                ks, ke = block_range(j, p.b_kv, N)
+                dfK[ks:ke] += v[ks:ke] @ dh[j].T + dz[j][None, :]
+                dV[bb, hh, ks:ke] += fK[ks:ke] @ dh[j]
+            dQ[bb, hh] += feature_map_backward(q, fQ, dfQ, p.phi)
+            dK[bb, hh] += feature_map_backward(k, fK, dfK, p.phi)
+    return {"dQ": dQ, "dK": dK, "dV": dV, "dproj_w": dW, "dproj_b": db, "dalpha": dalpha}
