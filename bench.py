@@ -219,7 +219,7 @@ def run_ours(args, rank, world, dev):
                                    P(O), P(ws), wsz, st())
 
     names = ["predict_mask", "precompute_linear", "aggregate_marginal", "fused_forward"]
-    launches_per_step = {"predict_mask": 2 + (2 if Wq is not None or Wk is not None else 0),
+    launches_per_step = {"predict_mask": 3 + (2 if Wq is not None or Wk is not None else 0),
                          "precompute_linear": 1, "aggregate_marginal": 2,
                          "fused_forward": 1 + (1 if args.qk != "bf16" else 0)}
 
@@ -340,6 +340,96 @@ def run_e2e(ctx, steps):
     return {"value": round(ctx["fl"]["step_exec"] / (ms * 1e-3) / 1e12, 3), "unit": UNIT,
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": 3 * act, "d2h_bytes_per_step": act,
             "api": "sla_attention_host (pinned host Q, K, V, O)"}
+
+
+def run_train(ctx, steps=10):
+    """Forward + backward of the same workload (the fine-tuning step): the four
+    forward stages with the LSE output, then sla_backward with dO ~ N(0, 1) bf16.
+    Also times dense attention's forward + backward (torch SDPA) on the same inputs."""
+    Q, K, V, cfg, dev = ctx["Q"], ctx["K"], ctx["V"], ctx["cfg"], ctx["dev"]
+    proj_w, proj_b, alpha, Wq, Wk = ctx["params"]
+    L, P = bnd.lib(), bnd._ptr
+    B, H, N, d = Q.shape
+    O = torch.empty_like(Q)
+    p = bnd.make_params(Q, cfg, K, V, O)
+    Tq, Tkv, nh, nl = bnd.sla_block_counts(p)
+    BH = B * H
+    ws = bnd.new_workspace(bnd.sla_workspace_size(p), dev)
+    bws = bnd.new_workspace(bnd.sla_backward_workspace_size(p), dev)
+    mc = torch.empty((BH, Tq, Tkv), dtype=torch.int8, device=dev)
+    lut = torch.empty((BH, Tq, nh), dtype=torch.int32, device=dev)
+    hz = torch.empty((BH, Tkv, d * d + d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((BH, N), dtype=torch.float32, device=dev)
+    osp = torch.empty((BH, N, d), dtype=torch.float32, device=dev)
+    g = torch.Generator(device=dev).manual_seed(7)
+    dO = torch.randn(Q.shape, generator=g, device=dev).to(torch.bfloat16)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    proj = cfg.combine == "proj"
+    dW = torch.empty((d, d), dtype=torch.float32, device=dev) if proj else None
+    db = torch.empty(d, dtype=torch.float32, device=dev) if proj else None
+    da = None if proj else torch.empty(BH, dtype=torch.float32, device=dev)
+    pw = proj_w if proj else None
+    st = bnd._stream
+    names = ["predict_mask", "precompute_linear", "forward_train", "backward"]
+
+    def stage(i):
+        if i == 0:
+            return L.sla_predict_mask(bnd.ctypes.byref(p), P(Q), P(K), P(Wq), P(Wk), P(mc), P(lut),
+                                      P(ws), ws.numel(), st())
+        if i == 1:
+            return L.sla_precompute_linear(bnd.ctypes.byref(p), P(K), P(V), P(pw), P(hz), P(ws),
+                                           ws.numel(), st())
+        if i == 2:
+            return L.sla_forward_train(bnd.ctypes.byref(p), P(Q), P(K), P(V), P(mc), P(lut), P(hz),
+                                       P(proj_b), P(alpha), P(O), P(lse), P(osp), P(ws), ws.numel(), st())
+        return L.sla_backward(bnd.ctypes.byref(p), P(Q), P(K), P(V), P(mc), P(lut), P(hz), P(pw),
+                              P(proj_b), P(alpha), P(osp), P(lse), P(dO), P(dQ), P(dK), P(dV), P(dW),
+                              P(db), P(da), P(bws), bws.numel(), st())
+
+    def step(ev=None):
+        for i in range(4):
+            if ev is not None:
+                ev[i].record()
+            code = stage(i)
+            if code != 0:
+                raise bnd.SlaError(code, names[i])
+        if ev is not None:
+            ev[4].record()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
+    for k in range(steps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    for w_ in (ws, bws):
+        code, detail = bnd.sla_get_device_status(w_)
+        if code != 0:
+            raise RuntimeError(f"device status {code} ({detail}) in the training step")
+    stage_ms = [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps)) / steps for i in range(4)]
+    res = {"workload": "forward + backward of the bench workload, dO ~ N(0, 1) bf16",
+           "ms_per_step": round(sum(stage_ms), 4),
+           "stage_ms": {n: round(x, 4) for n, x in zip(names, stage_ms)}}
+    # dense attention forward + backward on the same inputs
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        q, k_, v = (t.detach().clone().requires_grad_(True) for t in (Q, K, V))
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION]):
+            for _ in range(2):
+                torch.nn.functional.scaled_dot_product_attention(q, k_, v).backward(dO)
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(5):
+                torch.nn.functional.scaled_dot_product_attention(q, k_, v).backward(dO)
+            b.record()
+            torch.cuda.synchronize()
+        res["dense_fwd_bwd_ms"] = round(a.elapsed_time(b) / 5, 3)
+        res["speedup_vs_dense"] = round(res["dense_fwd_bwd_ms"] / res["ms_per_step"], 2)
+    except Exception as e:  # backend not available for this shape
+        res["dense_fwd_bwd_ms"] = f"unavailable: {type(e).__name__}"
+    return res
 
 
 def run_dense(ctx, iters=10):
@@ -480,6 +570,7 @@ def main():
         if not args.no_extras:
             res["e2e"] = run_e2e(ctx, steps=min(args.steps, 10))
             res["dense_baseline"] = run_dense(ctx)
+            res["train_step"] = run_train(ctx)
             best = min((v["ms"] for v in res["dense_baseline"].values() if "ms" in v), default=None)
             res["speedup_vs_dense"] = None if best is None else round(best / res["ms_per_step"], 2)
             if world == 1:

@@ -34,7 +34,7 @@ EXPORTS = (
     "sla_attention", "sla_aggregate_marginal", "sla_fused_forward",
     "sla_attention_host_workspace_size", "sla_attention_host", "sla_backward",
     "sla_get_device_status", "sla_status_string", "sla_abi_version",
-    "sla_predict_mask_noalloc",
+    "sla_predict_mask_noalloc", "sla_forward_train", "sla_backward_workspace_size",
 )
 
 
@@ -75,7 +75,7 @@ def lib() -> ctypes.CDLL:
         ip = ctypes.POINTER(ctypes.c_int)
         L.sla_block_counts.argtypes = [P, ip, ip, ip, ip]
         for f in ("sla_workspace_size", "sla_hz_size", "sla_attention_workspace_size",
-                  "sla_attention_host_workspace_size"):
+                  "sla_attention_host_workspace_size", "sla_backward_workspace_size"):
             getattr(L, f).argtypes = [P, ctypes.POINTER(sz)]
         L.sla_predict_mask.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_precompute_linear.argtypes = [P, vp, vp, vp, vp, vp, sz, vp]
@@ -85,7 +85,8 @@ def lib() -> ctypes.CDLL:
         L.sla_fused_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_attention_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_predict_mask_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
-        L.sla_backward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_forward_train.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_backward.argtypes = [P] + [vp] * 18 + [vp, sz, vp]
         L.sla_get_device_status.argtypes = [vp, vp, ip]
         L.sla_status_string.argtypes = [ctypes.c_int]
         L.sla_status_string.restype = ctypes.c_char_p
@@ -220,6 +221,52 @@ def sla_forward(Q, K, V, mc, lut, hz, cfg: SlaConfig, proj_b=None, alpha=None, o
                              _ptr(proj_b), _ptr(alpha), _ptr(O), _ptr(ws), ws.numel(), _stream()),
            "sla_forward")
     return O
+
+
+def sla_forward_train(Q, K, V, mc, lut, hz, cfg: SlaConfig, proj_b=None, alpha=None, workspace=None):
+    """sla_forward plus what the backward needs: (O, lse fp32 [B*H, N], o_sparse fp32 [B*H, N, d])."""
+    O = torch.empty_like(Q)
+    p = make_params(Q, cfg, K=K, V=V, O=O)
+    B, H, N, d = Q.shape
+    lse = torch.empty((B * H, N), dtype=torch.float32, device=Q.device)
+    os_ = torch.empty((B * H, N, d), dtype=torch.float32, device=Q.device)
+    ws = workspace if workspace is not None else new_workspace(sla_workspace_size(p), Q.device)
+    proj_b, alpha = _f32(proj_b, Q.device), _f32(alpha, Q.device)
+    _check(lib().sla_forward_train(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(mc), _ptr(lut),
+                                   _ptr(hz), _ptr(proj_b), _ptr(alpha), _ptr(O), _ptr(lse), _ptr(os_),
+                                   _ptr(ws), ws.numel(), _stream()), "sla_forward_train")
+    return O, lse, os_
+
+
+def sla_backward_workspace_size(p: sla_params_t) -> int:
+    return _size("sla_backward_workspace_size", p)
+
+
+def sla_backward(Q, K, V, mc, lut, hz, o_sparse, lse, dO, cfg: SlaConfig, proj_w=None, proj_b=None,
+                 alpha=None, workspace=None):
+    """Gradients of sum(O * dO): dict with dQ, dK, dV (bf16 like Q, K, V) and
+    dproj_w, dproj_b (SLA) or dalpha (SLA2), fp32."""
+    dev = Q.device
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    p = make_params(Q, cfg, K=K, V=V, O=dO)
+    d = Q.shape[-1]
+    B, H = Q.shape[:2]
+    proj = cfg.combine == "proj"
+    dW = torch.empty((d, d), dtype=torch.float32, device=dev) if proj else None
+    db = torch.empty(d, dtype=torch.float32, device=dev) if proj else None
+    da = None if proj else torch.empty(B * H, dtype=torch.float32, device=dev)
+    ws = workspace if workspace is not None else new_workspace(sla_backward_workspace_size(p), dev)
+    args = [_f32(x, dev) for x in (proj_w, proj_b, alpha)]
+    _check(lib().sla_backward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(mc), _ptr(lut), _ptr(hz),
+                              *[_ptr(x) for x in args], _ptr(o_sparse), _ptr(lse), _ptr(dO), _ptr(dQ), _ptr(dK),
+                              _ptr(dV), _ptr(dW), _ptr(db), _ptr(da), _ptr(ws), ws.numel(), _stream()),
+           "sla_backward")
+    out = {"dQ": dQ, "dK": dK, "dV": dV}
+    if proj:
+        out.update(dproj_w=dW, dproj_b=db)
+    else:
+        out["dalpha"] = da.view(B, H)
+    return out, ws
 
 
 def sla_attention(Q, K, V, cfg: SlaConfig, proj_w=None, proj_b=None, alpha=None, Wq=None, Wk=None,

@@ -272,9 +272,32 @@ sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, vo
   return cuda_status(launch_marg_gemm(ma, mb, a, pl.BH, s));
 }
 
+// out[bh][m][:] = sum_k A[bh][m][k] B[bh][k][:] for the 0/1 matrix A (bf16
+// [BH][M][Kp], Kp = K rounded up to 8) and rows B (bf16 [BH][K][NN]).
+sla_status_t zero_one_product(const Plan& pl, const __nv_bfloat16* A, int M, int Kdim, int Kp,
+                              const void* B, __nv_bfloat16* out, int* err, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  const uint64_t da[3] = {(uint64_t)Kp, (uint64_t)M, (uint64_t)pl.BH};
+  const uint64_t sa[2] = {(uint64_t)Kp * 2, (uint64_t)M * Kp * 2};
+  const uint32_t ba[3] = {64, 128, 1};
+  const uint64_t db[3] = {(uint64_t)pl.NN, (uint64_t)Kdim, (uint64_t)pl.BH};
+  const uint64_t sb[2] = {(uint64_t)pl.NN * 2, (uint64_t)Kdim * pl.NN * 2};
+  const uint32_t bb[3] = {64, 64, 1};
+  if (!encode(&ma, A, 3, da, sa, ba) || !encode(&mb, B, 3, db, sb, bb)) return SLA_ERR_CUDA;
+  MargArgs a;
+  a.Hout = out;
+  a.err = err;
+  a.Tq = M;
+  a.Tkv = Kdim;
+  a.NN = pl.NN;
+  a.ktiles = (Kdim + 63) / 64;
+  return cuda_status(launch_marg_gemm(ma, mb, a, pl.BH, s));
+}
+
 sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
                         const void* V, const int32_t* lut, const float* proj_b, const float* alpha,
-                        void* O, void* ws, cudaStream_t s) {
+                        void* O, void* ws, cudaStream_t s, float* lse = nullptr,
+                        float* o_sparse = nullptr) {
   const Layout L = layout_of(pl);
   __nv_bfloat16* hagg = at<__nv_bfloat16>(ws, L.hagg);
   CUtensorMap mq, mk, mv, mh, mz;
@@ -347,15 +370,17 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.scale_q = scq;
   a.scale_k = sck;
   a.phi = pl.phi;
+  a.lse = lse;
+  a.os = o_sparse;
   return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, pl.fp8, pl.BH, s));
 }
 
 sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
                           const void* V, const int8_t* mc, const int32_t* lut, const void* hz,
                           const float* proj_b, const float* alpha, void* O, void* ws,
-                          cudaStream_t s) {
+                          cudaStream_t s, float* lse = nullptr, float* o_sparse = nullptr) {
   SLA_TRY(aggregate_impl(pl, mc, hz, ws, s));
-  return fused_impl(pl, p, Q, K, V, lut, proj_b, alpha, O, ws, s);
+  return fused_impl(pl, p, Q, K, V, lut, proj_b, alpha, O, ws, s, lse, o_sparse);
 }
 
 bool contiguous(const sla_params_t* p) {
@@ -380,6 +405,159 @@ sla_status_t attention_impl(const Plan& pl, const sla_params_t* p, const void* Q
                             lut, ws, s));
   SLA_TRY(precompute_impl(pl, p, K, V, alpha_mode ? nullptr : proj_w, hz, ws, s));
   return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, ws, s);
+}
+
+// ---------------------------------------------------------------------------
+// Backward
+// ---------------------------------------------------------------------------
+struct BwdLayout {
+  size_t err, mm, hagg, drow, dqlin, dhzq, mmt, dhzk, dklin, dvlin, rcnt, rptr, rows, end;
+};
+
+BwdLayout bwd_layout_of(const Plan& p) {
+  BwdLayout L;
+  const size_t Tqp = (size_t)((p.Tq + 7) & ~7);
+  const size_t act32 = (size_t)p.BH * p.N * p.d * 4;
+  size_t o = 0;
+  L.err = o;   o = align_up(o + 256);
+  L.mm = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkvp * 2);
+  L.hagg = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.NN * 2);
+  L.drow = o;  o = align_up(o + (size_t)p.BH * p.N * 4);
+  L.dqlin = o; o = align_up(o + act32);
+  L.dhzq = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.NN * 2);
+  L.mmt = o;   o = align_up(o + (size_t)p.BH * p.Tkv * Tqp * 2);
+  L.dhzk = o;  o = align_up(o + (size_t)p.BH * p.Tkv * p.NN * 2);
+  L.dklin = o; o = align_up(o + act32);
+  L.dvlin = o; o = align_up(o + act32);
+  L.rcnt = o;  o = align_up(o + (size_t)p.BH * p.Tkv * 4);
+  L.rptr = o;  o = align_up(o + (size_t)p.BH * (p.Tkv + 1) * 4);
+  L.rows = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
+  L.end = o;
+  return L;
+}
+
+sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
+                           const void* V, const int8_t* mc, const int32_t* lut, const void* hz,
+                           const float* proj_w, const float* proj_b, const float* alpha,
+                           const float* o_sparse, const float* lse, const void* dO, void* dQ,
+                           void* dK, void* dV, float* dproj_w, float* dproj_b, float* dalpha,
+                           void* ws, cudaStream_t s) {
+  const BwdLayout L = bwd_layout_of(pl);
+  const bool alpha_mode = p->combine == SLA_COMBINE_ALPHA;
+  const int Tqp = (pl.Tq + 7) & ~7;
+  int* err = at<int>(ws, L.err);
+  // the forward's [H'_i^T | Z_i] (recomputed: the same 0/1 product as the forward)
+  __nv_bfloat16* mm = at<__nv_bfloat16>(ws, L.mm);
+  __nv_bfloat16* hagg = at<__nv_bfloat16>(ws, L.hagg);
+  SLA_TRY(cuda_status(launch_marg_matrix(mc, mm, pl.BH, pl.Tq, pl.Tkv, pl.Tkvp, pl.all, s)));
+  SLA_TRY(zero_one_product(pl, mm, pl.Tq, pl.Tkv, pl.Tkvp, hz, hagg, err, s));
+  // outputs accumulated with atomics start at zero
+  if (dproj_w && !alpha_mode &&
+      cudaMemsetAsync(dproj_w, 0, (size_t)pl.d * pl.d * 4, s) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  if (dproj_b && !alpha_mode && cudaMemsetAsync(dproj_b, 0, (size_t)pl.d * 4, s) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  if (dalpha && alpha_mode && cudaMemsetAsync(dalpha, 0, (size_t)pl.BH * 4, s) != cudaSuccess)
+    return SLA_ERR_CUDA;
+  // query side of the linear branch and of the combine
+  BwdRowsArgs ra;
+  ra.Q = static_cast<const __nv_bfloat16*>(Q);
+  ra.os = o_sparse;
+  ra.dO = static_cast<const __nv_bfloat16*>(dO);
+  for (int i = 0; i < 3; ++i) {
+    ra.sq[i] = p->stride_q[i];
+    ra.so[i] = p->stride_o[i];
+  }
+  ra.hagg = hagg;
+  ra.alpha = alpha_mode ? alpha : nullptr;
+  ra.Drow = at<float>(ws, L.drow);
+  ra.dq_lin = at<float>(ws, L.dqlin);
+  ra.dhz = at<__nv_bfloat16>(ws, L.dhzq);
+  ra.dalpha = alpha_mode ? dalpha : nullptr;
+  ra.dproj_b = alpha_mode ? nullptr : dproj_b;
+  ra.H = pl.H;
+  ra.N = pl.N;
+  ra.Tq = pl.Tq;
+  ra.NN = pl.NN;
+  ra.combine = p->combine;
+  ra.phi = pl.phi;
+  ra.eps = p->eps;
+  SLA_TRY(cuda_status(launch_bwd_rows(ra, pl.d, pl.BH, s)));
+  // dh'_j = sum of dH'_i over the query blocks that have j marginal
+  __nv_bfloat16* mmt = at<__nv_bfloat16>(ws, L.mmt);
+  SLA_TRY(cuda_status(launch_marg_matrix_t(mc, mmt, pl.BH, pl.Tq, pl.Tkv, Tqp, pl.all, s)));
+  SLA_TRY(zero_one_product(pl, mmt, pl.Tkv, pl.Tq, Tqp, ra.dhz, at<__nv_bfloat16>(ws, L.dhzk), err, s));
+  // key side of the linear branch
+  BwdKeysArgs ka;
+  ka.K = static_cast<const __nv_bfloat16*>(K);
+  ka.V = static_cast<const __nv_bfloat16*>(V);
+  for (int i = 0; i < 3; ++i) {
+    ka.sk[i] = p->stride_k[i];
+    ka.sv[i] = p->stride_v[i];
+  }
+  ka.proj_w = alpha_mode ? nullptr : proj_w;
+  ka.dhz = at<__nv_bfloat16>(ws, L.dhzk);
+  ka.dk_lin = at<float>(ws, L.dklin);
+  ka.dv_lin = at<float>(ws, L.dvlin);
+  ka.dproj_w = alpha_mode ? nullptr : dproj_w;
+  ka.BH = pl.BH;
+  ka.H = pl.H;
+  ka.N = pl.N;
+  ka.Tkv = pl.Tkv;
+  ka.NN = pl.NN;
+  ka.phi = pl.phi;
+  SLA_TRY(cuda_status(launch_bwd_keys(ka, pl.d, s)));
+  // sparse branch
+  int32_t* rcnt = at<int32_t>(ws, L.rcnt);
+  int32_t* rptr = at<int32_t>(ws, L.rptr);
+  int32_t* rows = at<int32_t>(ws, L.rows);
+  SLA_TRY(cuda_status(launch_rlut(mc, rcnt, rptr, rows, pl.BH, pl.Tq, pl.Tkv, pl.nh, s)));
+  BwdSparseArgs sa;
+  sa.lut = lut;
+  sa.rptr = rptr;
+  sa.rows = rows;
+  sa.lse = lse;
+  sa.Drow = ra.Drow;
+  sa.alpha = alpha_mode ? alpha : nullptr;
+  sa.err = err;
+  sa.H = pl.H;
+  sa.N = pl.N;
+  sa.Tq = pl.Tq;
+  sa.Tkv = pl.Tkv;
+  sa.nh = pl.nh;
+  sa.combine = p->combine;
+  sa.scale = (float)(1.0 / std::sqrt((double)pl.d));
+  sa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)pl.d));
+  {
+    CUtensorMap mq, mdo, mk, mv;
+    if (!map_bhnd(&mq, Q, pl, p->stride_q, 128) || !map_bhnd(&mdo, dO, pl, p->stride_o, 128) ||
+        !map_bhnd(&mk, K, pl, p->stride_k, 64) || !map_bhnd(&mv, V, pl, p->stride_v, 64))
+      return SLA_ERR_CUDA;
+    BwdSparseArgs qa = sa;
+    qa.q_lin = ra.dq_lin;
+    qa.v_lin = nullptr;
+    qa.out0 = static_cast<__nv_bfloat16*>(dQ);
+    qa.out1 = nullptr;
+    for (int i = 0; i < 3; ++i) qa.s0[i] = qa.s1[i] = p->stride_q[i];
+    SLA_TRY(cuda_status(launch_bwd_dq(mq, mdo, mk, mv, qa, pl.d, pl.BH, s)));
+  }
+  {
+    CUtensorMap mk2, mv2, mq1, mdo1;
+    if (!map_bhnd(&mk2, K, pl, p->stride_k, 128) || !map_bhnd(&mv2, V, pl, p->stride_v, 128) ||
+        !map_bhnd(&mq1, Q, pl, p->stride_q, 64) || !map_bhnd(&mdo1, dO, pl, p->stride_o, 64))
+      return SLA_ERR_CUDA;
+    BwdSparseArgs kb = sa;
+    kb.q_lin = ka.dk_lin;
+    kb.v_lin = ka.dv_lin;
+    kb.out0 = static_cast<__nv_bfloat16*>(dK);
+    kb.out1 = static_cast<__nv_bfloat16*>(dV);
+    for (int i = 0; i < 3; ++i) {
+      kb.s0[i] = p->stride_k[i];
+      kb.s1[i] = p->stride_v[i];
+    }
+    SLA_TRY(cuda_status(launch_bwd_dkdv(mk2, mv2, mq1, mdo1, kb, pl.d, pl.BH, s)));
+  }
+  return SLA_OK;
 }
 
 }  // namespace
@@ -485,6 +663,23 @@ sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, co
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
+sla_status_t sla_forward_train(const sla_params_t* p, const void* Q, const void* K,
+                               const void* V, const int8_t* mc, const int32_t* lut,
+                               const void* hz, const float* proj_b, const float* alpha, void* O,
+                               float* lse, float* o_sparse, void* workspace,
+                               size_t workspace_bytes, sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !V || !mc || !lut || !hz || !O || !lse || !o_sparse) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(hz) ||
+      !aligned16(o_sparse))
+    return SLA_ERR_INVALID_ARG;
+  if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
+  return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, workspace,
+                      reinterpret_cast<cudaStream_t>(stream), lse, o_sparse);
+}
+
 sla_status_t sla_attention(const sla_params_t* p, const void* Q, const void* K, const void* V,
                            const float* proj_w, const float* proj_b, const float* alpha,
                            const float* Wq, const float* Wk, void* O, void* workspace,
@@ -555,15 +750,34 @@ sla_status_t sla_fused_forward(const sla_params_t* p, const void* Q, const void*
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
-sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, const void* V,
-                          const void* O, const void* dO, void* dQ, void* dK, void* dV,
-                          void* workspace, size_t workspace_bytes, sla_stream_t stream) {
-  (void)stream;
+sla_status_t sla_backward_workspace_size(const sla_params_t* p, size_t* bytes) {
   Plan pl;
   SLA_TRY(make_plan(p, &pl));
-  if (!Q || !K || !V || !O || !dO || !dQ || !dK || !dV) return SLA_ERR_INVALID_ARG;
-  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
-  return SLA_ERR_UNSUPPORTED;
+  if (!bytes) return SLA_ERR_INVALID_ARG;
+  *bytes = bwd_layout_of(pl).end;
+  return SLA_OK;
+}
+
+sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                          const int8_t* mc, const int32_t* lut, const void* hz,
+                          const float* proj_w, const float* proj_b, const float* alpha,
+                          const float* o_sparse, const float* lse, const void* dO, void* dQ,
+                          void* dK, void* dV, float* dproj_w, float* dproj_b, float* dalpha,
+                          void* workspace, size_t workspace_bytes, sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !V || !mc || !lut || !hz || !o_sparse || !lse || !dO || !dQ || !dK || !dV)
+    return SLA_ERR_INVALID_ARG;
+  for (const void* x : {Q, K, V, (const void*)o_sparse, dO, (const void*)dQ, (const void*)dK,
+                        (const void*)dV, hz})
+    if (!aligned16(x)) return SLA_ERR_INVALID_ARG;
+  if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
+  if (p->qk_prec != SLA_QK_BF16 && p->qk_prec != SLA_QK_FP8_E4M3) return SLA_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
+      workspace_bytes < bwd_layout_of(pl).end)
+    return SLA_ERR_WORKSPACE;
+  return backward_impl(pl, p, Q, K, V, mc, lut, hz, proj_w, proj_b, alpha, o_sparse, lse, dO, dQ, dK, dV,
+                       dproj_w, dproj_b, dalpha, workspace, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sla_status_t sla_get_device_status(void* workspace, sla_stream_t stream, int* detail) {

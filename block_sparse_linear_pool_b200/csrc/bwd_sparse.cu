@@ -1,0 +1,672 @@
+// Backward of the sparse branch ("SLA: Beyond Sparsity in Diffusion
+// Transformers via Fine-Tunable Sparse-Linear Attention", §4 check 6: the
+// sparse path's gradients follow the FlashAttention backward; §7: one kernel
+// for dQ and one for dK / dV).  Only critical (query block, key block) pairs
+// are visited, as in the forward.
+//
+// With P = exp(s - lse) the forward's probabilities over a row's critical
+// tokens (lse from the forward), dP = dO^s V^T, D_r = dO^s_r . o^s_r and
+// dS = P (dP - D):   dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d),  dV = P^T dO^s,
+// where dO^s = c_s dO (c_s = 1 for SLA, alpha for SLA2; applied to dP and to
+// the finished dV).  The linear branch's parts (fp32, from the linear
+// backward) are added in the epilogues.
+//
+//   rlut_*              reverse lists: for every key block, the query blocks
+//                       that have it critical (ascending), from M_c
+//   bwd_dq_kernel       CTA = query blocks 2p, 2p+1 (M = 128) over the union of
+//                       their critical lists: S = Q K^T and dP = dO V^T into
+//                       TMEM, dS by the row threads, dQ += dS K (dS read from TMEM)
+//   bwd_dkdv_kernel     CTA = key blocks 2p, 2p+1 (M = 128 key rows) over the
+//                       union of their reverse lists: S^T = K Q^T and
+//                       dP^T = V dO^T into TMEM, P^T and dS^T by the key-row
+//                       threads, dV += P^T dO and dK += dS^T Q
+// Both: warp 0 TMA producer, warp 1 MMA issuer, warps 2-5 one TMEM lane each.
+#include "kernels.cuh"
+
+namespace sla {
+
+namespace {
+constexpr float LOG2E_B = 1.4426950408889634f;
+
+__device__ __forceinline__ float ex2b(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Reverse lists.  rcnt[bh][j] = #query blocks with M_c = 1 at column j; rptr =
+// exclusive prefix sums (rptr[bh][T_kv] = T_q * n_h); rows = the query block
+// indices, ascending per column.
+// ---------------------------------------------------------------------------
+__global__ void rlut_count_kernel(const int8_t* __restrict__ mc, int32_t* __restrict__ rcnt, int Tq,
+                                  int Tkv) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x, bh = blockIdx.y;
+  if (j >= Tkv) return;
+  const int8_t* col = mc + (int64_t)bh * Tq * Tkv + j;
+  int c = 0;
+  for (int i = 0; i < Tq; ++i) c += col[(int64_t)i * Tkv] == 1;
+  rcnt[(int64_t)bh * Tkv + j] = c;
+}
+
+__global__ void __launch_bounds__(1024) rlut_scan_kernel(const int32_t* __restrict__ rcnt,
+                                                         int32_t* __restrict__ rptr, int Tkv) {
+  __shared__ int32_t part[1024];
+  const int bh = blockIdx.x, t = threadIdx.x;
+  const int per = (Tkv + 1023) / 1024;
+  const int j0 = t * per;
+  int s = 0;
+  for (int j = j0; j < min(j0 + per, Tkv); ++j) s += rcnt[(int64_t)bh * Tkv + j];
+  part[t] = s;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan of the per-thread sums
+    const int v = t >= o ? part[t - o] : 0;
+    __syncthreads();
+    part[t] += v;
+    __syncthreads();
+  }
+  int run = t > 0 ? part[t - 1] : 0;
+  int32_t* out = rptr + (int64_t)bh * (Tkv + 1);
+  for (int j = j0; j < min(j0 + per, Tkv); ++j) {
+    out[j] = run;
+    run += rcnt[(int64_t)bh * Tkv + j];
+  }
+  if (t == 1023) out[Tkv] = part[1023];
+}
+
+__global__ void rlut_fill_kernel(const int8_t* __restrict__ mc, const int32_t* __restrict__ rptr,
+                                 int32_t* __restrict__ rows, int Tq, int Tkv, int nh) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x, bh = blockIdx.y;
+  if (j >= Tkv) return;
+  const int8_t* col = mc + (int64_t)bh * Tq * Tkv + j;
+  int32_t* out = rows + (int64_t)bh * Tq * nh + rptr[(int64_t)bh * (Tkv + 1) + j];
+  int k = 0;
+  for (int i = 0; i < Tq; ++i)
+    if (col[(int64_t)i * Tkv] == 1) out[k++] = i;
+}
+
+cudaError_t launch_rlut(const int8_t* mc, int32_t* rcnt, int32_t* rptr, int32_t* rows, int BH,
+                        int Tq, int Tkv, int nh, cudaStream_t s) {
+  dim3 grid((Tkv + 127) / 128, BH);
+  rlut_count_kernel<<<grid, 128, 0, s>>>(mc, rcnt, Tq, Tkv);
+  rlut_scan_kernel<<<BH, 1024, 0, s>>>(rcnt, rptr, Tkv);
+  rlut_fill_kernel<<<grid, 128, 0, s>>>(mc, rptr, rows, Tq, Tkv, nh);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// dQ.  TMEM: S [0,64) (dS over its first 32 columns), dP [64,128), dQ [128,128+d).
+// Shared: Q tile, dO tile (128 rows), one K slot and one V slot (64 rows).
+// ---------------------------------------------------------------------------
+template <int D>
+struct DqSmem {
+  static constexpr int CH = D / 64;
+  static constexpr int T128 = 128 * D * 2;
+  static constexpr int T64 = 64 * D * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = OFF_Q + T128;
+  static constexpr int OFF_K = OFF_DO + T128;
+  static constexpr int OFF_V = OFF_K + T64;
+  static constexpr int OFF_BAR = OFF_V + T64;
+  static constexpr int OFF_U = OFF_BAR + 256;
+  static size_t bytes(int Tkv) { return (size_t)OFF_U + 5 * (size_t)((Tkv + 15) & ~15) + 1024; }
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 2)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapdO,
+                  const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
+                  BwdSparseArgs a) {
+  using L = DqSmem<D>;
+  constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint8_t* sQ = sm + L::OFF_Q;
+  uint8_t* sdO = sm + L::OFF_DO;
+  uint8_t* sK = sm + L::OFF_K;
+  uint8_t* sV = sm + L::OFF_V;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  uint64_t* in_full = bars + 0;   // Q and dO
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = bars + 2;
+  uint64_t* v_full = bars + 3;
+  uint64_t* v_empty = bars + 4;
+  uint64_t* sp_full = bars + 5;   // S and dP in TMEM
+  uint64_t* ds_ready = bars + 6;  // dS written by all row threads
+  uint64_t* dq_done = bars + 7;   // the last dQ MMA completed
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  int* s_count = reinterpret_cast<int*>(tslot + 1);
+  const int Tkvr = (a.Tkv + 15) & ~15;
+  uint8_t* fa = sm + L::OFF_U;
+  uint8_t* fb = fa + Tkvr;
+  uint8_t* uflag = fb + Tkvr;
+  uint16_t* uidx = reinterpret_cast<uint16_t*>(uflag + Tkvr);
+
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  const int p = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int ia = 2 * p, ib = 2 * p + 1;
+  const bool has_b = ib < a.Tq;
+
+  if (w == 1) {
+    tmem_alloc(tslot, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(in_full, 1);
+    mbar_init(k_full, 1);
+    mbar_init(k_empty, 1);
+    mbar_init(v_full, 1);
+    mbar_init(v_empty, 1);
+    mbar_init(sp_full, 1);
+    mbar_init(ds_ready, 128);
+    mbar_init(dq_done, 1);
+    fence_barrier_init();
+  }
+  for (int j = tid; j < 2 * Tkvr; j += blockDim.x) fa[j] = 0;
+  __syncthreads();
+  {
+    const int32_t* la = a.lut + ((int64_t)bh * a.Tq + ia) * a.nh;
+    const int32_t* lb = a.lut + ((int64_t)bh * a.Tq + (has_b ? ib : ia)) * a.nh;
+    const int tot = has_b ? 2 * a.nh : a.nh;
+    for (int e = tid; e < tot; e += blockDim.x) {
+      const bool second = e >= a.nh;
+      const int j = second ? lb[e - a.nh] : la[e];
+      if (j < 0 || j >= a.Tkv) {
+        atomicCAS(a.err, 0, DEV_BAD_INDEX);
+        continue;
+      }
+      (second ? fb : fa)[j] = 1;
+    }
+  }
+  __syncthreads();
+  if (w == 0) {
+    int base = 0;
+    const uint32_t lt = (1u << ln) - 1u;
+    for (int j0 = 0; j0 < a.Tkv; j0 += 32) {
+      const int j = j0 + ln;
+      const uint32_t f = (j < a.Tkv) ? (uint32_t)(fa[j] | (fb[j] << 1)) : 0u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, f != 0);
+      if (f) {
+        const int pos = base + __popc(bal & lt);
+        uidx[pos] = (uint16_t)j;
+        uflag[pos] = (uint8_t)f;
+      }
+      base += __popc(bal);
+    }
+    if (ln == 0) *s_count = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int U = *s_count;
+  const uint32_t tbase = *tslot;
+
+  if (w == 0) {
+    if (ln == 0) {
+      tma_prefetch_desc(&mapQ);
+      tma_prefetch_desc(&mapdO);
+      tma_prefetch_desc(&mapK);
+      tma_prefetch_desc(&mapV);
+      mbar_arrive_expect_tx(in_full, 2 * L::T128);
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c) {
+        tma_load_4d(sQ + c * 16384, &mapQ, in_full, c * 64, 128 * p, h, b);
+        tma_load_4d(sdO + c * 16384, &mapdO, in_full, c * 64, 128 * p, h, b);
+      }
+      bool ok = true;
+      for (int k = 0; k < U && ok; ++k) {
+        const int j = uidx[k];
+        if (k >= 1 && !mbar_wait(k_empty, (k - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
+        mbar_arrive_expect_tx(k_full, L::T64);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c) tma_load_4d(sK + c * 8192, &mapK, k_full, c * 64, 64 * j, h, b);
+        if (k >= 1 && !mbar_wait(v_empty, (k - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
+        mbar_arrive_expect_tx(v_full, L::T64);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c) tma_load_4d(sV + c * 8192, &mapV, v_full, c * 64, 64 * j, h, b);
+      }
+    }
+  } else if (w == 1) {
+    if (ln == 0) {
+      const uint32_t id_s = idesc_bf16(128, 64, false, false);
+      const uint32_t id_q = idesc_bf16(128, D, false, true);
+      const uint32_t q0 = smem_u32(sQ), o0 = smem_u32(sdO), kt = smem_u32(sK), vt = smem_u32(sV);
+      bool ok = mbar_wait(in_full, 0, a.err, DEV_TIMEOUT_TMA);
+      for (int k = 0; k < U && ok; ++k) {
+        if (!mbar_wait(k_full, k & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        if (!mbar_wait(v_full, k & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        tc_fence_after();
+        // S and dP overwrite dS_{k-1}: its dQ MMA was issued earlier by this
+        // thread, and tcgen05.mma operations of one thread execute in order
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32, offk = (kk / 4) * 8192 + (kk % 4) * 32;
+          umma_ss(tbase + COL_S, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kt + offk, 16, 1024), id_s,
+                  kk > 0 ? 1u : 0u);
+          umma_ss(tbase + COL_DP, sdesc_sw128(o0 + off, 16, 1024), sdesc_sw128(vt + offk, 16, 1024), id_s,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(sp_full);
+        umma_commit(v_empty);
+        if (!mbar_wait(ds_ready, k & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
+        tc_fence_after();
+        // dQ += dS K: dS (bf16 pairs) from TMEM, K as the MN-major B operand
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ts(tbase + COL_DQ, tbase + COL_S + 8 * kk, sdesc_sw128(kt + kk * 2048, 8192, 1024), id_q,
+                  (k > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(k_empty);
+      }
+      if (ok) umma_commit(dq_done);
+    }
+  } else {
+    // ---------------- one query row per thread
+    const int q4 = w & 3;
+    const int r = 32 * q4 + ln;
+    const int half = r >> 6;
+    const uint32_t bit = 1u << half;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
+    const int n = 128 * p + r;
+    const bool valid = (n < a.N) && (half == 0 || has_b);
+    const float lse2 = valid ? a.lse[(int64_t)bh * a.N + n] * LOG2E_B : INFINITY;  // P = 0 when invalid
+    const float Dr = valid ? a.Drow[(int64_t)bh * a.N + n] : 0.f;
+    const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
+    const float sl2 = a.scale_log2;
+    bool ok = true;
+    for (int k = 0; k < U; ++k) {
+      if (!__all_sync(0xffffffffu, mbar_wait(sp_full, k & 1, a.err, DEV_TIMEOUT_MMA))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool crit = (uflag[k] & bit) != 0;
+      uint32_t pk[32];
+      if (crit) {
+        uint32_t s0[32], s1[32], d0[32], d1[32];
+        tmem_ld32(tl + COL_S, s0);
+        tmem_ld32(tl + COL_S + 32, s1);
+        tmem_ld32(tl + COL_DP, d0);
+        tmem_ld32(tl + COL_DP + 32, d1);
+        tmem_ld_wait();
+        const int nvalid = a.N - 64 * (int)uidx[k];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          float ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int col = (e < 2) ? 2 * c + e : 32 + 2 * c + (e - 2);
+            const float sv = __uint_as_float(e < 2 ? s0[2 * c + e] : s1[2 * c + e - 2]);
+            const float dv = __uint_as_float(e < 2 ? d0[2 * c + e] : d1[2 * c + e - 2]);
+            const float pr = col < nvalid ? ex2b(fmaf(sv, sl2, -lse2)) : 0.f;
+            ds[e] = pr * (cs * dv - Dr);
+          }
+          pk[c] = pack_bf16x2(ds[0], ds[1]);
+          pk[16 + c] = pack_bf16x2(ds[2], ds[3]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+      }
+      tmem_st32(tl + COL_S, pk);  // dS_k over the first 32 columns of S_k
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_ready);
+    }
+    if (ok && U >= 1) ok = __all_sync(0xffffffffu, mbar_wait(dq_done, 0, a.err, DEV_TIMEOUT_MMA));
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* orow = a.out0 + (int64_t)b * a.s0[0] + (int64_t)h * a.s0[1] + (int64_t)n * a.s0[2];
+      const float* lin = a.q_lin + ((int64_t)bh * a.N + n) * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t v[32];
+        if (U >= 1) {
+          tmem_ld32(tl + COL_DQ + c0, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) v[c] = 0u;
+        }
+        if (valid) {
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(v[8 * q8 + e]) * a.scale + lin[c0 + 8 * q8 + e];
+            *reinterpret_cast<uint4*>(orow + c0 + 8 * q8) =
+                make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                           pack_bf16x2(y[6], y[7]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV.  TMEM (512 columns, one CTA per SM): S^T [0,64) (P^T over its first
+// 32 columns), dP^T [64,128) (dS^T over its first 32), dV [128,128+d),
+// dK [256,256+d).  Shared: K pair and V pair (128 rows), one Q slot and one dO
+// slot (64 rows).
+// ---------------------------------------------------------------------------
+template <int D>
+struct DkvSmem {
+  static constexpr int CH = D / 64;
+  static constexpr int T128 = 128 * D * 2;
+  static constexpr int T64 = 64 * D * 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + T128;
+  static constexpr int OFF_Q = OFF_V + T128;
+  static constexpr int OFF_DO = OFF_Q + T64;
+  static constexpr int OFF_BAR = OFF_DO + T64;
+  static constexpr int OFF_U = OFF_BAR + 256;
+  // at least 120 KB so that a second CTA (which would wait for the 512 TMEM
+  // columns) is never placed on the same SM
+  static size_t bytes(int Tq) {
+    const size_t b = (size_t)OFF_U + 5 * (size_t)((Tq + 15) & ~15) + 1024;
+    return b < 120 * 1024 ? 120 * 1024 : b;
+  }
+};
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mapK2, const __grid_constant__ CUtensorMap mapV2,
+                    const __grid_constant__ CUtensorMap mapQ1, const __grid_constant__ CUtensorMap mapdO1,
+                    BwdSparseArgs a) {
+  using L = DkvSmem<D>;
+  constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DV = 128, COL_DK = 256;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint8_t* sK = sm + L::OFF_K;
+  uint8_t* sV = sm + L::OFF_V;
+  uint8_t* sQ = sm + L::OFF_Q;
+  uint8_t* sdO = sm + L::OFF_DO;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  uint64_t* kv_full = bars + 0;
+  uint64_t* q_full = bars + 1;
+  uint64_t* q_empty = bars + 2;
+  uint64_t* sp_full = bars + 3;
+  uint64_t* ds_ready = bars + 4;
+  uint64_t* kv_done = bars + 5;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6);
+  int* s_count = reinterpret_cast<int*>(tslot + 1);
+  const int Tqr = (a.Tq + 15) & ~15;
+  uint8_t* fa = sm + L::OFF_U;
+  uint8_t* fb = fa + Tqr;
+  uint8_t* uflag = fb + Tqr;
+  uint16_t* uidx = reinterpret_cast<uint16_t*>(uflag + Tqr);
+
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  const int p = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int ja = 2 * p, jb = 2 * p + 1;
+  const bool has_b = jb < a.Tkv;
+
+  if (w == 1) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    mbar_init(sp_full, 1);
+    mbar_init(ds_ready, 128);
+    mbar_init(kv_done, 1);
+    fence_barrier_init();
+  }
+  for (int i = tid; i < 2 * Tqr; i += blockDim.x) fa[i] = 0;
+  __syncthreads();
+  {
+    const int32_t* rp = a.rptr + (int64_t)bh * (a.Tkv + 1);
+    const int32_t* rl = a.rows + (int64_t)bh * a.Tq * a.nh;
+    for (int t = 0; t < (has_b ? 2 : 1); ++t) {
+      const int j = t == 0 ? ja : jb;
+      const int e0 = rp[j], e1 = rp[j + 1];
+      for (int e = e0 + tid; e < e1; e += blockDim.x) {
+        const int i = rl[e];
+        if (i < 0 || i >= a.Tq) {
+          atomicCAS(a.err, 0, DEV_BAD_INDEX);
+          continue;
+        }
+        (t == 0 ? fa : fb)[i] = 1;
+      }
+    }
+  }
+  __syncthreads();
+  if (w == 0) {
+    int base = 0;
+    const uint32_t lt = (1u << ln) - 1u;
+    for (int i0 = 0; i0 < a.Tq; i0 += 32) {
+      const int i = i0 + ln;
+      const uint32_t f = (i < a.Tq) ? (uint32_t)(fa[i] | (fb[i] << 1)) : 0u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, f != 0);
+      if (f) {
+        const int pos = base + __popc(bal & lt);
+        uidx[pos] = (uint16_t)i;
+        uflag[pos] = (uint8_t)f;
+      }
+      base += __popc(bal);
+    }
+    if (ln == 0) *s_count = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int U = *s_count;
+  const uint32_t tbase = *tslot;
+
+  if (w == 0) {
+    if (ln == 0) {
+      tma_prefetch_desc(&mapK2);
+      tma_prefetch_desc(&mapV2);
+      tma_prefetch_desc(&mapQ1);
+      tma_prefetch_desc(&mapdO1);
+      mbar_arrive_expect_tx(kv_full, 2 * L::T128);
+#pragma unroll
+      for (int c = 0; c < L::CH; ++c) {
+        tma_load_4d(sK + c * 16384, &mapK2, kv_full, c * 64, 128 * p, h, b);
+        tma_load_4d(sV + c * 16384, &mapV2, kv_full, c * 64, 128 * p, h, b);
+      }
+      bool ok = true;
+      for (int e = 0; e < U && ok; ++e) {
+        const int i = uidx[e];
+        if (e >= 1 && !mbar_wait(q_empty, (e - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
+        mbar_arrive_expect_tx(q_full, 2 * L::T64);
+#pragma unroll
+        for (int c = 0; c < L::CH; ++c) {
+          tma_load_4d(sQ + c * 8192, &mapQ1, q_full, c * 64, 64 * i, h, b);
+          tma_load_4d(sdO + c * 8192, &mapdO1, q_full, c * 64, 64 * i, h, b);
+        }
+      }
+    }
+  } else if (w == 1) {
+    if (ln == 0) {
+      const uint32_t id_s = idesc_bf16(128, 64, false, false);
+      const uint32_t id_o = idesc_bf16(128, D, false, true);
+      const uint32_t k0 = smem_u32(sK), v0 = smem_u32(sV), qt = smem_u32(sQ), ot = smem_u32(sdO);
+      bool ok = mbar_wait(kv_full, 0, a.err, DEV_TIMEOUT_TMA);
+      for (int e = 0; e < U && ok; ++e) {
+        if (!mbar_wait(q_full, e & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        tc_fence_after();
+        // S^T = K Q_i^T and dP^T = V dO_i^T (M = 128 key rows, N = 64 query rows)
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off2 = (kk / 4) * 16384 + (kk % 4) * 32, off1 = (kk / 4) * 8192 + (kk % 4) * 32;
+          umma_ss(tbase + COL_S, sdesc_sw128(k0 + off2, 16, 1024), sdesc_sw128(qt + off1, 16, 1024), id_s,
+                  kk > 0 ? 1u : 0u);
+          umma_ss(tbase + COL_DP, sdesc_sw128(v0 + off2, 16, 1024), sdesc_sw128(ot + off1, 16, 1024), id_s,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(sp_full);
+        if (!mbar_wait(ds_ready, e & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
+        tc_fence_after();
+        // dV += P^T dO_i and dK += dS^T Q_i (P^T, dS^T bf16 pairs from TMEM)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          umma_ts(tbase + COL_DV, tbase + COL_S + 8 * kk, sdesc_sw128(ot + kk * 2048, 8192, 1024), id_o,
+                  (e > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tbase + COL_DK, tbase + COL_DP + 8 * kk, sdesc_sw128(qt + kk * 2048, 8192, 1024), id_o,
+                  (e > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(q_empty);
+      }
+      if (ok) umma_commit(kv_done);
+    }
+  } else {
+    // ---------------- one key row per thread
+    const int q4 = w & 3;
+    const int t = 32 * q4 + ln;
+    const int half = t >> 6;
+    const uint32_t bit = 1u << half;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
+    const int n = 128 * p + t;
+    const bool valid = (n < a.N) && (half == 0 || has_b);
+    const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
+    const float sl2 = a.scale_log2;
+    const float* lse = a.lse + (int64_t)bh * a.N;
+    const float* Dv = a.Drow + (int64_t)bh * a.N;
+    bool ok = true;
+    for (int e = 0; e < U; ++e) {
+      if (!__all_sync(0xffffffffu, mbar_wait(sp_full, e & 1, a.err, DEV_TIMEOUT_MMA))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool crit = (uflag[e] & bit) != 0;
+      uint32_t pp[32], pd[32];
+      if (crit) {
+        uint32_t s0[32], s1[32], d0[32], d1[32];
+        tmem_ld32(tl + COL_S, s0);
+        tmem_ld32(tl + COL_S + 32, s1);
+        tmem_ld32(tl + COL_DP, d0);
+        tmem_ld32(tl + COL_DP + 32, d1);
+        tmem_ld_wait();
+        const int r0 = 64 * (int)uidx[e];
+        const int rvalid = a.N - r0;  // query rows of this block that exist
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          float pv[4], ds[4];
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const int col = (e4 < 2) ? 2 * c + e4 : 32 + 2 * c + (e4 - 2);
+            const float sv = __uint_as_float(e4 < 2 ? s0[2 * c + e4] : s1[2 * c + e4 - 2]);
+            const float dv = __uint_as_float(e4 < 2 ? d0[2 * c + e4] : d1[2 * c + e4 - 2]);
+            float pr = 0.f, dr = 0.f;
+            if (col < rvalid) {
+              pr = ex2b(fmaf(sv, sl2, -lse[r0 + col] * LOG2E_B));
+              dr = Dv[r0 + col];
+            }
+            pv[e4] = pr;
+            ds[e4] = pr * (cs * dv - dr);
+          }
+          pp[c] = pack_bf16x2(pv[0], pv[1]);
+          pp[16 + c] = pack_bf16x2(pv[2], pv[3]);
+          pd[c] = pack_bf16x2(ds[0], ds[1]);
+          pd[16 + c] = pack_bf16x2(ds[2], ds[3]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pp[c] = pd[c] = 0u;
+      }
+      tmem_st32(tl + COL_S, pp);   // P^T over S^T
+      tmem_st32(tl + COL_DP, pd);  // dS^T over dP^T
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_ready);
+    }
+    if (ok && U >= 1) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, a.err, DEV_TIMEOUT_MMA));
+    if (ok) {
+      tc_fence_after();
+      for (int which = 0; which < 2; ++which) {
+        __nv_bfloat16* base = which == 0 ? a.out0 : a.out1;
+        const int64_t* st = which == 0 ? a.s0 : a.s1;
+        const float* lin = (which == 0 ? a.q_lin : a.v_lin) + ((int64_t)bh * a.N + n) * D;
+        const float f = which == 0 ? a.scale : cs;  // dK = acc / sqrt(d); dV = c_s acc
+        __nv_bfloat16* orow = base + (int64_t)b * st[0] + (int64_t)h * st[1] + (int64_t)n * st[2];
+        const uint32_t col = which == 0 ? COL_DK : COL_DV;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t v[32];
+          if (U >= 1) {
+            tmem_ld32(tl + col + c0, v);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) v[c] = 0u;
+          }
+          if (valid) {
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              float y[8];
+#pragma unroll
+              for (int e8 = 0; e8 < 8; ++e8) y[e8] = __uint_as_float(v[8 * q8 + e8]) * f + lin[c0 + 8 * q8 + e8];
+              *reinterpret_cast<uint4*>(orow + c0 + 8 * q8) =
+                  make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                             pack_bf16x2(y[6], y[7]));
+            }
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+template <class Kern>
+static cudaError_t set_smem(Kern k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+cudaError_t launch_bwd_dq(const CUtensorMap& mapQ, const CUtensorMap& mapdO, const CUtensorMap& mapK,
+                          const CUtensorMap& mapV, const BwdSparseArgs& a, int D, int BH,
+                          cudaStream_t s) {
+  dim3 grid((a.Tq + 1) / 2, BH);
+  if (D == 128) {
+    const size_t smem = DqSmem<128>::bytes(a.Tkv);
+    cudaError_t e = set_smem(bwd_dq_kernel<128>, smem);
+    if (e != cudaSuccess) return e;
+    bwd_dq_kernel<128><<<grid, 192, smem, s>>>(mapQ, mapdO, mapK, mapV, a);
+  } else {
+    const size_t smem = DqSmem<64>::bytes(a.Tkv);
+    cudaError_t e = set_smem(bwd_dq_kernel<64>, smem);
+    if (e != cudaSuccess) return e;
+    bwd_dq_kernel<64><<<grid, 192, smem, s>>>(mapQ, mapdO, mapK, mapV, a);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkdv(const CUtensorMap& mapK2, const CUtensorMap& mapV2,
+                            const CUtensorMap& mapQ1, const CUtensorMap& mapdO1,
+                            const BwdSparseArgs& a, int D, int BH, cudaStream_t s) {
+  dim3 grid((a.Tkv + 1) / 2, BH);
+  if (D == 128) {
+    const size_t smem = DkvSmem<128>::bytes(a.Tq);
+    cudaError_t e = set_smem(bwd_dkdv_kernel<128>, smem);
+    if (e != cudaSuccess) return e;
+    bwd_dkdv_kernel<128><<<grid, 192, smem, s>>>(mapK2, mapV2, mapQ1, mapdO1, a);
+  } else {
+    const size_t smem = DkvSmem<64>::bytes(a.Tq);
+    cudaError_t e = set_smem(bwd_dkdv_kernel<64>, smem);
+    if (e != cudaSuccess) return e;
+    bwd_dkdv_kernel<64><<<grid, 192, smem, s>>>(mapK2, mapV2, mapQ1, mapdO1, a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -501,6 +501,9 @@ __global__ void __launch_bounds__(192, 2)
       const int n = 128 * p + r;
       const bool store = (n < a.N) && (half == 0 || has_b);
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      // log-sum-exp of the row's scaled critical scores, for the backward:
+      // sum_t exp(s_t) = 2^m * l with m in log2 units
+      if (a.lse && store) a.lse[(int64_t)bh * a.N + n] = (m + log2f(l)) * 0.6931471805599453f;
       const float inv_den = 1.f / (edotz + esum * a.eps);
       float wa, wl;
       if (a.combine == 1) {
@@ -531,6 +534,13 @@ __global__ void __launch_bounds__(192, 2)
             }
             dst[v] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
                                 pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+          }
+          if (a.os) {  // the sparse branch's output in fp32, for the backward
+            float4* od = reinterpret_cast<float4*>(a.os + ((int64_t)bh * a.N + n) * D + c0);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              od[v] = make_float4(__uint_as_float(ov[4 * v]) * inv_l, __uint_as_float(ov[4 * v + 1]) * inv_l,
+                                  __uint_as_float(ov[4 * v + 2]) * inv_l, __uint_as_float(ov[4 * v + 3]) * inv_l);
           }
         }
       }

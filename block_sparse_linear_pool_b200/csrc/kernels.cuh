@@ -71,7 +71,68 @@ struct FusedArgs {
   const float* scale_q;   // FP8 path: per (head, query block) scale of Q, else nullptr
   const float* scale_k;   // FP8 path: per (head, key block) scale of K, else nullptr
   int phi;                // 0 softmax over d, 1 elu + 1
+  float* lse;             // [BH][N] natural-log sum of exp of the scaled critical scores, or nullptr
+  float* os;              // [BH][N][d] the sparse branch's output o^s (fp32), or nullptr
 };
+
+// ---- backward
+struct BwdRowsArgs {
+  const __nv_bfloat16* Q;
+  int64_t sq[3];
+  const float* os;          // [BH][N][d] the forward's sparse-branch output (fp32)
+  const __nv_bfloat16* dO;
+  int64_t so[3];            // strides of dO
+  const __nv_bfloat16* hagg;  // [BH][Tq][NN] forward's [H'_i^T | Z_i]
+  const float* alpha;       // [BH] (SLA2) or nullptr
+  float* Drow;              // [BH][N] out: dO^s . o^s
+  float* dq_lin;            // [BH][N][d] out
+  __nv_bfloat16* dhz;       // [BH][Tq][NN] out: [dH'_i^T | dZ_i]
+  float* dalpha;            // [BH] accumulated (SLA2) or nullptr
+  float* dproj_b;           // [d] accumulated (SLA) or nullptr
+  int H, N, Tq, NN, combine, phi;
+  float eps;
+};
+
+struct BwdKeysArgs {
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  int64_t sk[3], sv[3];
+  const float* proj_w;      // [d][d] (SLA) or nullptr (identity)
+  const __nv_bfloat16* dhz; // [BH][Tkv][NN] [dh'_j^T | dz_j]
+  float* dk_lin;            // [BH][N][d] out
+  float* dv_lin;            // [BH][N][d] out
+  float* dproj_w;           // [d][d] accumulated (SLA) or nullptr
+  int BH, H, N, Tkv, NN, phi;
+};
+
+struct BwdSparseArgs {
+  const int32_t* lut;       // [BH][Tq][nh]
+  const int32_t* rptr;      // [BH][Tkv + 1] reverse lists: query blocks with j critical
+  const int32_t* rows;      // [BH][Tq * nh]
+  const float* lse;         // [BH][N]
+  const float* Drow;        // [BH][N]
+  const float* alpha;       // [BH] (SLA2) or nullptr
+  const float* q_lin;       // [BH][N][d] dq (linear part), or dk (linear) for the key kernel
+  const float* v_lin;       // [BH][N][d] dv (linear part) for the key kernel
+  __nv_bfloat16* out0;      // dQ, or dK for the key kernel
+  __nv_bfloat16* out1;      // dV for the key kernel
+  int64_t s0[3], s1[3];     // strides of out0, out1
+  int* err;
+  int H, N, Tq, Tkv, nh, combine;
+  float scale_log2;         // log2(e) / sqrt(d)
+  float scale;              // 1 / sqrt(d)
+};
+
+cudaError_t launch_bwd_rows(const BwdRowsArgs& a, int D, int BH, cudaStream_t s);
+cudaError_t launch_bwd_keys(const BwdKeysArgs& a, int D, cudaStream_t s);
+cudaError_t launch_rlut(const int8_t* mc, int32_t* rcnt, int32_t* rptr, int32_t* rows, int BH,
+                        int Tq, int Tkv, int nh, cudaStream_t s);
+cudaError_t launch_bwd_dq(const CUtensorMap& mapQ, const CUtensorMap& mapdO, const CUtensorMap& mapK,
+                          const CUtensorMap& mapV, const BwdSparseArgs& a, int D, int BH,
+                          cudaStream_t s);
+cudaError_t launch_bwd_dkdv(const CUtensorMap& mapK2, const CUtensorMap& mapV2,
+                            const CUtensorMap& mapQ1, const CUtensorMap& mapdO1,
+                            const BwdSparseArgs& a, int D, int BH, cudaStream_t s);
 
 cudaError_t launch_pool(const PoolArgs& a, int D, int BH, cudaStream_t s);
 cudaError_t launch_router(const float* Qc, const float* Kc, float* Qr, float* Kr, float* kmean,
@@ -86,6 +147,8 @@ cudaError_t launch_kv_prep(const CUtensorMap& mapK, const CUtensorMap& mapV, con
 
 cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int Tq, int Tkv,
                                int Tkvp, bool all, cudaStream_t s);
+cudaError_t launch_marg_matrix_t(const int8_t* mc, __nv_bfloat16* mt, int BH, int Tq, int Tkv,
+                                 int Tqp, bool all, cudaStream_t s);
 cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const MargArgs& a,
                              int BH, cudaStream_t s);
 

@@ -30,6 +30,22 @@ __global__ void marg_matrix_kernel(const int8_t* __restrict__ mc, __nv_bfloat16*
   }
 }
 
+// The transpose for the backward: MmargT[bh][j][i] = Mmarg[bh][i][j], rows
+// padded to T_qp (the dh_j = sum_i dH_i product of the linear backward).
+__global__ void marg_matrix_t_kernel(const int8_t* __restrict__ mc, __nv_bfloat16* __restrict__ mt,
+                                     int BH, int Tq, int Tkv, int Tqp, bool all) {
+  const int64_t total = (int64_t)BH * Tkv * Tqp;
+  const __nv_bfloat16 one = __float2bfloat16(1.f), zero = __float2bfloat16(0.f);
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(e % Tqp);
+    const int64_t r = e / Tqp;  // bh * Tkv + j
+    const int j = (int)(r % Tkv);
+    const int64_t bh = r / Tkv;
+    mt[e] = (i < Tq && (all || mc[(bh * Tq + i) * Tkv + j] == 0)) ? one : zero;
+  }
+}
+
 namespace {
 constexpr int BM = 128, BN = 256, BK = 64, NST = 4;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
@@ -185,6 +201,14 @@ cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int 
   const int64_t total = (int64_t)BH * Tq * Tkvp;
   const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
   marg_matrix_kernel<<<blocks, 256, 0, s>>>(mc, mm, BH, Tq, Tkv, Tkvp, all);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_marg_matrix_t(const int8_t* mc, __nv_bfloat16* mt, int BH, int Tq, int Tkv,
+                                 int Tqp, bool all, cudaStream_t s) {
+  const int64_t total = (int64_t)BH * Tkv * Tqp;
+  const int blocks = (int)std::min<int64_t>((total + 255) / 256, 148 * 16);
+  marg_matrix_t_kernel<<<blocks, 256, 0, s>>>(mc, mt, BH, Tq, Tkv, Tqp, all);
   return cudaGetLastError();
 }
 

@@ -160,6 +160,19 @@ sla_status_t sla_forward(const sla_params_t* p, const void* Q, const void* K, co
                          size_t workspace_bytes, sla_stream_t stream);
 
 /*
+ * sla_forward that also keeps what sla_backward needs (device, caller-allocated):
+ *   lse       fp32 [B*H][N]: per query row, log(sum over its critical tokens t of
+ *             exp(q_n . k_t / sqrt(d))) (natural log);
+ *   o_sparse  fp32 [B*H][N][d]: the sparse branch's output o^s of every row (the
+ *             backward needs it apart from the combined O, in full precision).
+ */
+sla_status_t sla_forward_train(const sla_params_t* p, const void* Q, const void* K,
+                               const void* V, const int8_t* mc, const int32_t* lut,
+                               const void* hz, const float* proj_b, const float* alpha, void* O,
+                               float* lse, float* o_sparse, void* workspace,
+                               size_t workspace_bytes, sla_stream_t stream);
+
+/*
  * The two halves of sla_forward, for callers that schedule or time them
  * separately (sla_forward is exactly sla_aggregate_marginal followed by
  * sla_fused_forward on the same stream and workspace).
@@ -234,12 +247,41 @@ sla_status_t sla_predict_mask_noalloc(const sla_params_t* p, const void* Q, cons
                                       int32_t* lut, sla_stream_t stream);
 
 /*
- * Backward of the forward above ([SLA2] App. A; [SLA] §4 check 6).  Not
- * implemented in this build: returns SLA_ERR_UNSUPPORTED after validating
- * its arguments.
+ * Backward of sla_forward_train ([SLA2] App. A; [SLA] §4 check 6): the
+ * gradients of L = sum(O * dO) for fixed mc (hard Top-k has no gradient;
+ * SLA2's router is trained through a soft Top-k that is not part of this
+ * library, so Wq / Wk get none).
+ *   sparse branch  the FlashAttention backward over the critical blocks only:
+ *                  P = exp(q.k / sqrt(d) - lse), dS = P (dP - D) with
+ *                  D_r = dO^s_r . o^s_r; one kernel for dQ (per query-block
+ *                  pair, over its critical lists) and one for dK, dV (per
+ *                  key-block pair, over the query blocks that have it critical);
+ *   linear branch  per query block dH_i, dZ_i, summed into every marginal key
+ *                  block's dh_j, dz_j (the forward's 0/1 product, transposed),
+ *                  then back through h_j = phi(K_j)^T V_j, z_j and phi;
+ *   combine        SLA: dO^s = dO, the linear branch sees dO W;
+ *                  dproj_w = dO^T o_l, dproj_b = sum dO.
+ *                  SLA2: dO^s = alpha dO, dO^l = (1 - alpha) dO,
+ *                  dalpha = sum (o^s - o^l) . dO per head.
+ * Inputs (device): Q, K, V and params as given to the forward; mc, lut from
+ *   sla_predict_mask; hz from sla_precompute_linear (Proj's W folded in for
+ *   SLA); proj_w fp32 [d][d] (SLA), proj_b fp32 [d] or NULL (SLA), alpha fp32
+ *   [B*H] (SLA2); o_sparse and lse from sla_forward_train; dO bf16 [B,H,N,d]
+ *   with the strides of O (stride_o).
+ * Outputs (device, caller-allocated, overwritten): dQ, dK, dV bf16 with the
+ *   strides of Q, K, V; dproj_w fp32 [d][d] and dproj_b fp32 [d] (SLA; either
+ *   may be NULL); dalpha fp32 [B*H] (SLA2; may be NULL).
+ * Workspace: sla_backward_workspace_size bytes, 256-byte aligned; its first
+ *   word is the device error word (zero it once; sla_get_device_status reads
+ *   and clears it).  Q K^T is recomputed in bf16 also for qk_prec = FP8
+ *   ([SLA2] §5 keeps the backward in full precision).
  */
+sla_status_t sla_backward_workspace_size(const sla_params_t* p, size_t* bytes);
 sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, const void* V,
-                          const void* O, const void* dO, void* dQ, void* dK, void* dV,
+                          const int8_t* mc, const int32_t* lut, const void* hz,
+                          const float* proj_w, const float* proj_b, const float* alpha,
+                          const float* o_sparse, const float* lse, const void* dO, void* dQ,
+                          void* dK, void* dV, float* dproj_w, float* dproj_b, float* dalpha,
                           void* workspace, size_t workspace_bytes, sla_stream_t stream);
 
 /* Reads the device error word of `workspace` (synchronises `stream`) and

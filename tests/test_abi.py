@@ -84,10 +84,13 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
     # workspace too small
     assert L.sla_forward(ctypes.byref(p), dummy, dummy, dummy, dummy, dummy, dummy, None, None,
                          dummy, ctypes.c_void_p(4096), 16, None) == 3
-    # backward is declared but not implemented
-    need = bnd.sla_workspace_size(p)
-    assert L.sla_backward(ctypes.byref(p), dummy, dummy, dummy, dummy, dummy, dummy, dummy, dummy,
-                          ctypes.c_void_p(1 << 20), need, None) == 2
+    # backward: NULL gradient outputs, then a workspace that is too small
+    args = [dummy] * 12 + [None] * 6
+    assert L.sla_backward(ctypes.byref(p), *args[:9], dummy, dummy, dummy, None, None, None, None,
+                          None, None, ctypes.c_void_p(1 << 20), 1 << 40, None) == 1
+    need = bnd.sla_backward_workspace_size(p)
+    assert L.sla_backward(ctypes.byref(p), *[dummy] * 15, None, None, None,
+                          ctypes.c_void_p(1 << 20), need - 1, None) == 3
 
 
 def test_defaults_are_the_pages_main_method(L):
