@@ -422,7 +422,7 @@ BwdLayout bwd_layout_of(const Plan& p) {
   L.err = o;   o = align_up(o + 256);
   L.mm = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkvp * 2);
   L.hagg = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.NN * 2);
-  L.drow = o;  o = align_up(o + (size_t)p.BH * p.N * 4);
+  L.drow = o;  o = align_up(o + (size_t)p.BH * p.Tq * 64 * 8);
   L.dqlin = o; o = align_up(o + act32);
   L.dhzq = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.NN * 2);
   L.mmt = o;   o = align_up(o + (size_t)p.BH * p.Tkv * Tqp * 2);
@@ -470,7 +470,8 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   }
   ra.hagg = hagg;
   ra.alpha = alpha_mode ? alpha : nullptr;
-  ra.Drow = at<float>(ws, L.drow);
+  ra.lse = lse;
+  ra.ld2 = at<float2>(ws, L.drow);
   ra.dq_lin = at<float>(ws, L.dqlin);
   ra.dhz = at<__nv_bfloat16>(ws, L.dhzq);
   ra.dalpha = alpha_mode ? dalpha : nullptr;
@@ -516,8 +517,7 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   sa.lut = lut;
   sa.rptr = rptr;
   sa.rows = rows;
-  sa.lse = lse;
-  sa.Drow = ra.Drow;
+  sa.ld2 = ra.ld2;
   sa.alpha = alpha_mode ? alpha : nullptr;
   sa.err = err;
   sa.H = pl.H;

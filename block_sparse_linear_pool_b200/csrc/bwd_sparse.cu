@@ -18,15 +18,14 @@
 //                       TMEM, dS by the row threads, dQ += dS K (dS read from TMEM)
 //   bwd_dkdv_kernel     CTA = key blocks 2p, 2p+1 (M = 128 key rows) over the
 //                       union of their reverse lists: S^T = K Q^T and
-//                       dP^T = V dO^T into TMEM, P^T and dS^T by the key-row
-//                       threads, dV += P^T dO and dK += dS^T Q
+//                       dP^T = V dO^T into TMEM (two buffers), P^T and dS^T by
+//                       the key-row threads, dV += P^T dO and dK += dS^T Q
 // Both: warp 0 TMA producer, warp 1 MMA issuer, warps 2-5 one TMEM lane each.
 #include "kernels.cuh"
 
 namespace sla {
 
 namespace {
-constexpr float LOG2E_B = 1.4426950408889634f;
 
 __device__ __forceinline__ float ex2b(float x) {
   float y;
@@ -271,8 +270,9 @@ __global__ void __launch_bounds__(192, 2)
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
     const int n = 128 * p + r;
     const bool valid = (n < a.N) && (half == 0 || has_b);
-    const float lse2 = valid ? a.lse[(int64_t)bh * a.N + n] * LOG2E_B : INFINITY;  // P = 0 when invalid
-    const float Dr = valid ? a.Drow[(int64_t)bh * a.N + n] : 0.f;
+    // (lse log2 e, D) of this row; P = 0 on rows that do not exist
+    const float2 ld = valid ? a.ld2[(int64_t)bh * a.Tq * 64 + n] : make_float2(INFINITY, 0.f);
+    const float lse2 = ld.x, Dr = ld.y;
     const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
     const float sl2 = a.scale_log2;
     bool ok = true;
@@ -353,10 +353,12 @@ __global__ void __launch_bounds__(192, 2)
 }
 
 // ---------------------------------------------------------------------------
-// dK, dV.  TMEM (512 columns, one CTA per SM): S^T [0,64) (P^T over its first
-// 32 columns), dP^T [64,128) (dS^T over its first 32), dV [128,128+d),
-// dK [256,256+d).  Shared: K pair and V pair (128 rows), one Q slot and one dO
-// slot (64 rows).
+// dK, dV.  TMEM (512 columns, one CTA per SM): two score buffers x = 0, 1 with
+// S^T at [128x, 128x + 64) (P^T over its first 32 columns) and dP^T at
+// [128x + 64, 128x + 128) (dS^T over its first 32), dV [256, 256 + d),
+// dK [384, 384 + d).  S^T, dP^T of entry e+1 are computed while the key-row
+// threads work on entry e.  Shared: K pair and V pair (128 rows), a 2-slot
+// ring of (Q_i, dO_i, the 64 (lse log2 e, D) pairs of block i).
 // ---------------------------------------------------------------------------
 template <int D>
 struct DkvSmem {
@@ -365,9 +367,10 @@ struct DkvSmem {
   static constexpr int T64 = 64 * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + T128;
-  static constexpr int OFF_Q = OFF_V + T128;
-  static constexpr int OFF_DO = OFF_Q + T64;
-  static constexpr int OFF_BAR = OFF_DO + T64;
+  static constexpr int OFF_Q = OFF_V + T128;        // [2] slots
+  static constexpr int OFF_DO = OFF_Q + 2 * T64;    // [2]
+  static constexpr int OFF_LD = OFF_DO + 2 * T64;   // [2][64] float2
+  static constexpr int OFF_BAR = OFF_LD + 2 * 64 * 8;
   static constexpr int OFF_U = OFF_BAR + 256;
   // at least 120 KB so that a second CTA (which would wait for the 512 TMEM
   // columns) is never placed on the same SM
@@ -383,7 +386,7 @@ __global__ void __launch_bounds__(192, 1)
                     const __grid_constant__ CUtensorMap mapQ1, const __grid_constant__ CUtensorMap mapdO1,
                     BwdSparseArgs a) {
   using L = DkvSmem<D>;
-  constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DV = 128, COL_DK = 256;
+  constexpr uint32_t COL_DV = 256, COL_DK = 384;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -391,14 +394,15 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sV = sm + L::OFF_V;
   uint8_t* sQ = sm + L::OFF_Q;
   uint8_t* sdO = sm + L::OFF_DO;
+  float2* sLD = reinterpret_cast<float2*>(sm + L::OFF_LD);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;
-  uint64_t* q_empty = bars + 2;
-  uint64_t* sp_full = bars + 3;
-  uint64_t* ds_ready = bars + 4;
-  uint64_t* kv_done = bars + 5;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6);
+  uint64_t* q_full = bars + 1;    // [2] ring slots
+  uint64_t* q_empty = bars + 3;   // [2]
+  uint64_t* sp_full = bars + 5;   // [2] score buffers
+  uint64_t* ds_ready = bars + 7;  // [2]
+  uint64_t* kv_done = bars + 9;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 10);
   int* s_count = reinterpret_cast<int*>(tslot + 1);
   const int Tqr = (a.Tq + 15) & ~15;
   uint8_t* fa = sm + L::OFF_U;
@@ -418,10 +422,12 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (tid == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
-    mbar_init(sp_full, 1);
-    mbar_init(ds_ready, 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&sp_full[x], 1);
+      mbar_init(&ds_ready[x], 128);
+    }
     mbar_init(kv_done, 1);
     fence_barrier_init();
   }
@@ -480,47 +486,62 @@ __global__ void __launch_bounds__(192, 1)
       }
       bool ok = true;
       for (int e = 0; e < U && ok; ++e) {
-        const int i = uidx[e];
-        if (e >= 1 && !mbar_wait(q_empty, (e - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
-        mbar_arrive_expect_tx(q_full, 2 * L::T64);
+        const int i = uidx[e], x = e & 1;
+        if (e >= 2 && !mbar_wait(&q_empty[x], ((e - 2) >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&q_full[x], 2 * L::T64 + 64 * 8);
 #pragma unroll
         for (int c = 0; c < L::CH; ++c) {
-          tma_load_4d(sQ + c * 8192, &mapQ1, q_full, c * 64, 64 * i, h, b);
-          tma_load_4d(sdO + c * 8192, &mapdO1, q_full, c * 64, 64 * i, h, b);
+          tma_load_4d(sQ + x * L::T64 + c * 8192, &mapQ1, &q_full[x], c * 64, 64 * i, h, b);
+          tma_load_4d(sdO + x * L::T64 + c * 8192, &mapdO1, &q_full[x], c * 64, 64 * i, h, b);
         }
+        bulk_load(sLD + x * 64, a.ld2 + (int64_t)bh * a.Tq * 64 + 64 * i, 64 * 8, &q_full[x]);
       }
     }
   } else if (w == 1) {
     if (ln == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
       const uint32_t id_o = idesc_bf16(128, D, false, true);
-      const uint32_t k0 = smem_u32(sK), v0 = smem_u32(sV), qt = smem_u32(sQ), ot = smem_u32(sdO);
+      const uint32_t k0 = smem_u32(sK), v0 = smem_u32(sV);
       bool ok = mbar_wait(kv_full, 0, a.err, DEV_TIMEOUT_TMA);
-      for (int e = 0; e < U && ok; ++e) {
-        if (!mbar_wait(q_full, e & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+      // dV += P^T dO_e and dK += dS^T Q_e (P^T, dS^T bf16 pairs from TMEM buffer e & 1)
+      auto issue_grads = [&](int e) -> bool {
+        const int x = e & 1;
+        if (!mbar_wait(&ds_ready[x], (e >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
         tc_fence_after();
-        // S^T = K Q_i^T and dP^T = V dO_i^T (M = 128 key rows, N = 64 query rows)
+        const uint32_t qt = smem_u32(sQ + x * L::T64), ot = smem_u32(sdO + x * L::T64);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          umma_ts(tbase + COL_DV, tbase + 128 * x + 8 * kk, sdesc_sw128(ot + kk * 2048, 8192, 1024), id_o,
+                  (e > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tbase + COL_DK, tbase + 128 * x + 64 + 8 * kk, sdesc_sw128(qt + kk * 2048, 8192, 1024),
+                  id_o, (e > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&q_empty[x]);
+        return true;
+      };
+      for (int e = 0; e < U && ok; ++e) {
+        const int x = e & 1;
+        if (!mbar_wait(&q_full[x], (e >> 1) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        tc_fence_after();
+        // S^T = K Q_e^T and dP^T = V dO_e^T (M = 128 key rows, N = 64 query rows) into
+        // buffer x; its previous contents (entry e - 2) were consumed by MMAs issued
+        // earlier by this thread, which execute in order
+        const uint32_t qt = smem_u32(sQ + x * L::T64), ot = smem_u32(sdO + x * L::T64);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off2 = (kk / 4) * 16384 + (kk % 4) * 32, off1 = (kk / 4) * 8192 + (kk % 4) * 32;
-          umma_ss(tbase + COL_S, sdesc_sw128(k0 + off2, 16, 1024), sdesc_sw128(qt + off1, 16, 1024), id_s,
+          umma_ss(tbase + 128 * x, sdesc_sw128(k0 + off2, 16, 1024), sdesc_sw128(qt + off1, 16, 1024), id_s,
                   kk > 0 ? 1u : 0u);
-          umma_ss(tbase + COL_DP, sdesc_sw128(v0 + off2, 16, 1024), sdesc_sw128(ot + off1, 16, 1024), id_s,
-                  kk > 0 ? 1u : 0u);
+          umma_ss(tbase + 128 * x + 64, sdesc_sw128(v0 + off2, 16, 1024), sdesc_sw128(ot + off1, 16, 1024),
+                  id_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(sp_full);
-        if (!mbar_wait(ds_ready, e & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
-        tc_fence_after();
-        // dV += P^T dO_i and dK += dS^T Q_i (P^T, dS^T bf16 pairs from TMEM)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          umma_ts(tbase + COL_DV, tbase + COL_S + 8 * kk, sdesc_sw128(ot + kk * 2048, 8192, 1024), id_o,
-                  (e > 0 || kk > 0) ? 1u : 0u);
-          umma_ts(tbase + COL_DK, tbase + COL_DP + 8 * kk, sdesc_sw128(qt + kk * 2048, 8192, 1024), id_o,
-                  (e > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(q_empty);
+        umma_commit(&sp_full[x]);
+        if (e >= 1 && !issue_grads(e - 1)) { ok = false; break; }
       }
+      if (ok && U >= 1) ok = issue_grads(U - 1);
       if (ok) umma_commit(kv_done);
     }
   } else {
@@ -534,26 +555,25 @@ __global__ void __launch_bounds__(192, 1)
     const bool valid = (n < a.N) && (half == 0 || has_b);
     const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
     const float sl2 = a.scale_log2;
-    const float* lse = a.lse + (int64_t)bh * a.N;
-    const float* Dv = a.Drow + (int64_t)bh * a.N;
     bool ok = true;
     for (int e = 0; e < U; ++e) {
-      if (!__all_sync(0xffffffffu, mbar_wait(sp_full, e & 1, a.err, DEV_TIMEOUT_MMA))) {
+      const int x = e & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sp_full[x], (e >> 1) & 1, a.err, DEV_TIMEOUT_MMA))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const bool crit = (uflag[e] & bit) != 0;
+      const uint32_t ts = tl + 128 * x;
       uint32_t pp[32], pd[32];
       if (crit) {
         uint32_t s0[32], s1[32], d0[32], d1[32];
-        tmem_ld32(tl + COL_S, s0);
-        tmem_ld32(tl + COL_S + 32, s1);
-        tmem_ld32(tl + COL_DP, d0);
-        tmem_ld32(tl + COL_DP + 32, d1);
+        tmem_ld32(ts, s0);
+        tmem_ld32(ts + 32, s1);
+        tmem_ld32(ts + 64, d0);
+        tmem_ld32(ts + 96, d1);
         tmem_ld_wait();
-        const int r0 = 64 * (int)uidx[e];
-        const int rvalid = a.N - r0;  // query rows of this block that exist
+        const float2* ldv = sLD + x * 64;  // (lse log2 e, D) of the 64 query rows
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
           float pv[4], ds[4];
@@ -562,13 +582,10 @@ __global__ void __launch_bounds__(192, 1)
             const int col = (e4 < 2) ? 2 * c + e4 : 32 + 2 * c + (e4 - 2);
             const float sv = __uint_as_float(e4 < 2 ? s0[2 * c + e4] : s1[2 * c + e4 - 2]);
             const float dv = __uint_as_float(e4 < 2 ? d0[2 * c + e4] : d1[2 * c + e4 - 2]);
-            float pr = 0.f, dr = 0.f;
-            if (col < rvalid) {
-              pr = ex2b(fmaf(sv, sl2, -lse[r0 + col] * LOG2E_B));
-              dr = Dv[r0 + col];
-            }
+            const float2 l2 = ldv[col];
+            const float pr = ex2b(fmaf(sv, sl2, -l2.x));
             pv[e4] = pr;
-            ds[e4] = pr * (cs * dv - dr);
+            ds[e4] = pr * (cs * dv - l2.y);
           }
           pp[c] = pack_bf16x2(pv[0], pv[1]);
           pp[16 + c] = pack_bf16x2(pv[2], pv[3]);
@@ -579,11 +596,11 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int c = 0; c < 32; ++c) pp[c] = pd[c] = 0u;
       }
-      tmem_st32(tl + COL_S, pp);   // P^T over S^T
-      tmem_st32(tl + COL_DP, pd);  // dS^T over dP^T
+      tmem_st32(ts, pp);       // P^T over S^T
+      tmem_st32(ts + 64, pd);  // dS^T over dP^T
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ds_ready);
+      mbar_arrive(&ds_ready[x]);
     }
     if (ok && U >= 1) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, a.err, DEV_TIMEOUT_MMA));
     if (ok) {
