@@ -483,7 +483,26 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   ra.combine = p->combine;
   ra.phi = pl.phi;
   ra.eps = p->eps;
-  SLA_TRY(cuda_status(launch_bwd_rows(ra, pl.d, pl.BH, s)));
+  if (pl.d == 128) {
+    // tensor-core version: both query blocks of a pair per CTA
+    CUtensorMap mh, mz;
+    const uint64_t dh[4] = {(uint64_t)pl.d, (uint64_t)pl.d, (uint64_t)pl.Tq, (uint64_t)pl.BH};
+    const uint64_t sh[3] = {(uint64_t)pl.d * 2, (uint64_t)pl.NN * 2, (uint64_t)pl.Tq * pl.NN * 2};
+    const uint32_t bxh[4] = {64, (uint32_t)pl.d, 1, 1};
+    const uint64_t dz[3] = {(uint64_t)pl.NN, (uint64_t)pl.Tq, (uint64_t)pl.BH};
+    const uint64_t sz[2] = {(uint64_t)pl.NN * 2, (uint64_t)pl.Tq * pl.NN * 2};
+    const uint32_t bxz[3] = {64, 1, 1};
+    if (!encode(&mh, hagg, 4, dh, sh, bxh) || !encode(&mz, hagg, 3, dz, sz, bxz, false))
+      return SLA_ERR_CUDA;
+    BwdRowsArgs rt = ra;
+    rt.dproj_b = nullptr;
+    SLA_TRY(cuda_status(launch_bwd_rows_tc(mh, mz, rt, err, pl.BH, s)));
+    if (!alpha_mode && dproj_b)
+      SLA_TRY(cuda_status(launch_colsum(static_cast<const __nv_bfloat16*>(dO), p->stride_o, pl.H,
+                                        pl.N, pl.BH, pl.d, dproj_b, s)));
+  } else {
+    SLA_TRY(cuda_status(launch_bwd_rows(ra, pl.d, pl.BH, s)));
+  }
   // dh'_j = sum of dH'_i over the query blocks that have j marginal
   __nv_bfloat16* mmt = at<__nv_bfloat16>(ws, L.mmt);
   SLA_TRY(cuda_status(launch_marg_matrix_t(mc, mmt, pl.BH, pl.Tq, pl.Tkv, Tqp, pl.all, s)));

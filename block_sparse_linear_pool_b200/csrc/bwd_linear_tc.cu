@@ -1,0 +1,357 @@
+// Query side of the linear-branch backward on the tensor cores (d = 128).
+// Same quantities as bwd_rows_kernel (see bwd_linear.cu for the formulas);
+// here a CTA takes query blocks 2p and 2p+1 (128 rows, one TMEM lane each) and
+// the three products run as tcgen05.mma:
+//   G1  NUM_t  = phi(Q) H'_t           M = 128 rows, N = d, K = d   (t = 0, 1)
+//   G2  dphi_t = gp H'_t^T             M = 128 rows, N = d, K = d
+//   G3  dH'_t  = phi(Q_t)^T gp_t       M = d, N = d, K = 64 rows of block t
+// G1 and G2 are computed for all 128 rows against both blocks' H' (each row
+// keeps the half of its own block), so every per-row scalar (den, o'_r . dO_r,
+// D_r) stays with the thread that owns the row.  H'_t arrives by TMA as the
+// forward's [H_i^T | Z_i] row ([o][a], a contiguous): the K-major B operand of
+// G1 and, read the other way, the MN-major B operand of G2.
+//
+//   warp 0      TMA: both blocks' H' tiles and Z rows
+//   warp 1      tcgen05.mma issuer
+//   warps 2-5   one row each: phi(q) -> shared (bf16, swizzled), den; then o',
+//               D, gp -> shared, gden; then dq (linear part); finally one column
+//               a of dH'_t each (G3's lanes are a) and dZ_t[a]
+// TMEM (512 columns, one CTA per SM): G1 and then G2 at [0, 2d), G3 at [2d, 4d).
+#include "kernels.cuh"
+
+namespace sla {
+
+namespace {
+constexpr int TD = 128;                       // d
+constexpr int TILE = TD * 128;                // one [128 rows][128 B] chunk
+constexpr int OFF_H = 0;                      // [2 a-chunks][2 blocks][TD o][128 B]
+constexpr int OFF_F = OFF_H + 4 * TILE;       // phi(Q): [2 a-chunks][128 rows][128 B]
+constexpr int OFF_G = OFF_F + 2 * TILE;       // gp:     [2 o-chunks][128 rows][128 B]
+constexpr int OFF_Z = OFF_G + 2 * TILE;       // Z_t: [2][TD] bf16
+constexpr int OFF_GD = OFF_Z + 2 * TD * 2;    // gden [128] fp32
+constexpr int OFF_BAR = OFF_GD + 128 * 4;
+constexpr int SMEM_TC = OFF_BAR + 256 + 1024;
+constexpr float LOG2E_T = 1.4426950408889634f;
+
+__device__ __forceinline__ float bfv(uint32_t packed, int hi) {
+  return __uint_as_float(hi ? (packed & 0xffff0000u) : (packed << 16));
+}
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap mapH, const __grid_constant__ CUtensorMap mapZ,
+                       BwdRowsArgs a, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint8_t* sH = sm + OFF_H;
+  uint8_t* sF = sm + OFF_F;
+  uint8_t* sG = sm + OFF_G;
+  const __nv_bfloat16* sZ = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_Z);
+  float* sgden = reinterpret_cast<float*>(sm + OFF_GD);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
+  uint64_t* h_full = bars + 0;
+  uint64_t* fq_ready = bars + 1;
+  uint64_t* num_full = bars + 2;
+  uint64_t* gp_ready = bars + 3;
+  uint64_t* dphi_full = bars + 4;
+  uint64_t* dh_full = bars + 5;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6);
+
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  const int p = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int i0 = 2 * p, i1 = 2 * p + 1;
+  const bool has1 = i1 < a.Tq;
+
+  if (w == 1) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(h_full, 1);
+    mbar_init(fq_ready, 128);
+    mbar_init(num_full, 1);
+    mbar_init(gp_ready, 128);
+    mbar_init(dphi_full, 1);
+    mbar_init(dh_full, 1);
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+
+  if (w == 0) {
+    if (ln == 0) {
+      tma_prefetch_desc(&mapH);
+      tma_prefetch_desc(&mapZ);
+      mbar_arrive_expect_tx(h_full, 2 * (2 * TILE + TD * 2));
+      for (int t = 0; t < 2; ++t) {
+        const int i = (t == 1 && has1) ? i1 : i0;  // a missing second block reuses the first
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tma_load_4d(sH + c * 2 * TILE + t * TILE, &mapH, h_full, c * 64, 0, i, bh);
+          tma_load_3d(sm + OFF_Z + t * TD * 2 + c * 128, &mapZ, h_full, TD * TD + c * 64, i, bh);
+        }
+      }
+    }
+  } else if (w == 1) {
+    if (ln == 0) {
+      const uint32_t id_kk = idesc_bf16(128, TD, false, false);  // A, B K-major
+      const uint32_t id_km = idesc_bf16(128, TD, false, true);   // B MN-major
+      const uint32_t id_mm = idesc_bf16(128, TD, true, true);    // A, B MN-major
+      const uint32_t h0 = smem_u32(sH), f0 = smem_u32(sF), g0 = smem_u32(sG);
+      bool ok = mbar_wait(h_full, 0, err, DEV_TIMEOUT_TMA) && mbar_wait(fq_ready, 0, err, DEV_TIMEOUT_SYNC);
+      if (ok) {
+        tc_fence_after();
+        // G1: NUM_t[r][o] = sum_a F[r][a] H'_t[a][o]   (B rows o, K = a contiguous)
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int kk = 0; kk < TD / 16; ++kk)
+            umma_ss(tbase + TD * t, sdesc_sw128(f0 + (kk / 4) * TILE + (kk % 4) * 32, 16, 1024),
+                    sdesc_sw128(h0 + (kk / 4) * 2 * TILE + t * TILE + (kk % 4) * 32, 16, 1024), id_kk,
+                    kk > 0 ? 1u : 0u);
+        umma_commit(num_full);
+        ok = mbar_wait(gp_ready, 0, err, DEV_TIMEOUT_SYNC);
+      }
+      if (ok) {
+        tc_fence_after();
+        // G2: dphi_t[r][a] = sum_o GP[r][o] H'_t[a][o]   (B: N = a contiguous, K = o rows)
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int kk = 0; kk < TD / 16; ++kk)
+            umma_ss(tbase + TD * t, sdesc_sw128(g0 + (kk / 4) * TILE + (kk % 4) * 32, 16, 1024),
+                    sdesc_sw128(h0 + t * TILE + kk * 2048, 2 * TILE, 1024), id_km, kk > 0 ? 1u : 0u);
+        umma_commit(dphi_full);
+        // G3: dH'_t[a][o] = sum_{r in block t} F[r][a] GP[r][o]  (A: M = a contiguous; B: N = o contiguous)
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ss(tbase + 2 * TD + TD * t, sdesc_sw128(f0 + t * 8192 + kk * 2048, TILE, 1024),
+                    sdesc_sw128(g0 + t * 8192 + kk * 2048, TILE, 1024), id_mm, kk > 0 ? 1u : 0u);
+        umma_commit(dh_full);
+      }
+    }
+  } else {
+    const int q4 = w & 3;
+    const int r = 32 * q4 + ln;          // row (and, for G3, the column a)
+    const int t = r >> 6;                // block of this row
+    const int i = t == 0 ? i0 : i1;
+    const int n = 64 * i + (r & 63);
+    const bool valid = (t == 0 || has1) && n < a.N;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
+    const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
+    const float cl = a.combine == 1 ? 1.f - a.alpha[bh] : 1.f;
+    const __nv_bfloat16* qrow = a.Q + (int64_t)b * a.sq[0] + (int64_t)h * a.sq[1] + (int64_t)n * a.sq[2];
+    bool ok = __all_sync(0xffffffffu, mbar_wait(h_full, 0, err, DEV_TIMEOUT_TMA));
+    // ---- phase 1: phi(q) (bf16) into sF, den = phi(q) . Z_t + eps
+    float m = -INFINITY, s = 0.f;
+    if (valid && a.phi == 0) {
+      for (int c = 0; c < TD; c += 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(qrow + c);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, bfv(u[e / 2], e & 1));
+      }
+      for (int c = 0; c < TD; c += 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(qrow + c);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += exp2f((bfv(u[e / 2], e & 1) - m) * LOG2E_T);
+      }
+    }
+    const float inv_s = (a.phi == 0 && s > 0.f) ? 1.f / s : 1.f;
+    auto phi_of = [&](float x) {
+      return a.phi == 1 ? (x > 0.f ? x + 1.f : exp2f(x * LOG2E_T)) : exp2f((x - m) * LOG2E_T) * inv_s;
+    };
+    float den = a.eps;
+    if (ok) {
+      const __nv_bfloat16* z = sZ + t * TD;
+      for (int c = 0; c < TD; c += 8) {
+        uint32_t o4[4] = {0u, 0u, 0u, 0u};
+        if (valid) {
+          const uint4 v = *reinterpret_cast<const uint4*>(qrow + c);
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            o4[e] = pack_bf16x2(phi_of(bfv(u[e], 0)), phi_of(bfv(u[e], 1)));
+            den = fmaf(bfv(o4[e], 0), __bfloat162float(z[c + 2 * e]),
+                       fmaf(bfv(o4[e], 1), __bfloat162float(z[c + 2 * e + 1]), den));
+          }
+        }
+        *reinterpret_cast<uint4*>(sF + (c / 64) * TILE + sw128_offset(r, (c % 64) * 2)) =
+            make_uint4(o4[0], o4[1], o4[2], o4[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(fq_ready);
+    // ---- phase 2: o' = NUM / den, D, gp (bf16) into sG, gden
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(num_full, 0, err, DEV_TIMEOUT_MMA));
+    float dd = 0.f, dol = 0.f, da = 0.f;
+    if (ok) {
+      tc_fence_after();
+      const __nv_bfloat16* drow = a.dO + (int64_t)b * a.so[0] + (int64_t)h * a.so[1] + (int64_t)n * a.so[2];
+      const float* osrow = a.os + ((int64_t)bh * a.N + n) * TD;
+      const float inv_den = 1.f / den;
+#pragma unroll 1
+      for (int c0 = 0; c0 < TD; c0 += 32) {
+        uint32_t nv[32];
+        tmem_ld32(tl + TD * t + c0, nv);
+        tmem_ld_wait();
+        uint32_t gpk[16];
+#pragma unroll
+        for (int c8 = 0; c8 < 32; c8 += 8) {
+          float dov[8], osv[8];
+          if (valid) {
+            const uint4 v = *reinterpret_cast<const uint4*>(drow + c0 + c8);
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dov[e] = bfv(u[e / 2], e & 1);
+            const float4 o0 = *reinterpret_cast<const float4*>(osrow + c0 + c8);
+            const float4 o1 = *reinterpret_cast<const float4*>(osrow + c0 + c8 + 4);
+            osv[0] = o0.x; osv[1] = o0.y; osv[2] = o0.z; osv[3] = o0.w;
+            osv[4] = o1.x; osv[5] = o1.y; osv[6] = o1.z; osv[7] = o1.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) dov[e] = osv[e] = 0.f;
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float ol = __uint_as_float(nv[c8 + e]) * inv_den;  // o'_r
+            dd = fmaf(cs * dov[e], osv[e], dd);
+            dol = fmaf(dov[e], ol, dol);
+            da = fmaf(osv[e] - ol, dov[e], da);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; e += 2)
+            gpk[(c8 + e) / 2] = pack_bf16x2(cl * dov[e] * inv_den, cl * dov[e + 1] * inv_den);
+        }
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          *reinterpret_cast<uint4*>(sG + (c0 / 64) * TILE + sw128_offset(r, ((c0 % 64) + 8 * v4) * 2)) =
+              make_uint4(gpk[4 * v4], gpk[4 * v4 + 1], gpk[4 * v4 + 2], gpk[4 * v4 + 3]);
+      }
+    }
+    const float gden = valid ? -cl * dol / den : 0.f;
+    sgden[r] = gden;
+    if (valid) a.ld2[(int64_t)bh * a.Tq * 64 + n] = make_float2(a.lse[(int64_t)bh * a.N + n] * LOG2E_T, dd);
+    else if (t == 0 || has1) a.ld2[(int64_t)bh * a.Tq * 64 + n] = make_float2(INFINITY, 0.f);
+    if (a.combine == 1 && a.dalpha) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) da += __shfl_xor_sync(0xffffffffu, da, o);
+      if (ln == 0) atomicAdd(a.dalpha + bh, da);
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(gp_ready);
+    // ---- phase 3: dq (linear part) = phi backward of dphi = G2 + gden Z_t
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dphi_full, 0, err, DEV_TIMEOUT_MMA));
+    if (ok) {
+      tc_fence_after();
+      const __nv_bfloat16* z = sZ + t * TD;
+      float dot = 0.f;
+      if (a.phi == 0) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < TD; c0 += 32) {
+          uint32_t dv[32];
+          tmem_ld32(tl + TD * t + c0, dv);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float f = phi_of(__bfloat162float(qrow[c0 + e]));
+              dot = fmaf(f, __uint_as_float(dv[e]) + gden * __bfloat162float(z[c0 + e]), dot);
+            }
+          }
+        }
+      }
+      float* out = a.dq_lin + ((int64_t)bh * a.N + n) * TD;
+#pragma unroll 1
+      for (int c0 = 0; c0 < TD; c0 += 32) {
+        uint32_t dv[32];
+        tmem_ld32(tl + TD * t + c0, dv);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int e4 = 0; e4 < 32; e4 += 4) {
+            float y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x = __bfloat162float(qrow[c0 + e4 + e]);
+              const float dphi = __uint_as_float(dv[e4 + e]) + gden * __bfloat162float(z[c0 + e4 + e]);
+              y[e] = a.phi == 1 ? dphi * (x > 0.f ? 1.f : exp2f(x * LOG2E_T)) : phi_of(x) * (dphi - dot);
+            }
+            *reinterpret_cast<float4*>(out + c0 + e4) = make_float4(y[0], y[1], y[2], y[3]);
+          }
+        }
+      }
+    }
+    // ---- phase 4: thread r owns column a = r of dH'_t (G3's lanes) and dZ_t[a];
+    // the waits on fq_ready / gp_ready order the other rows' phi(q) and gden writes
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dh_full, 0, err, DEV_TIMEOUT_MMA) &&
+                                             mbar_wait(fq_ready, 0, err, DEV_TIMEOUT_SYNC) &&
+                                             mbar_wait(gp_ready, 0, err, DEV_TIMEOUT_SYNC));
+    if (ok) {
+      tc_fence_after();
+      const int aa = r;
+      for (int tt = 0; tt < (has1 ? 2 : 1); ++tt) {
+        const int it = tt == 0 ? i0 : i1;
+        __nv_bfloat16* dst = a.dhz + ((int64_t)bh * a.Tq + it) * a.NN;
+#pragma unroll 1
+        for (int c0 = 0; c0 < TD; c0 += 32) {
+          uint32_t hv[32];
+          tmem_ld32(tl + 2 * TD + TD * tt + c0, hv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) dst[(int64_t)(c0 + e) * TD + aa] = __float2bfloat16(__uint_as_float(hv[e]));
+        }
+        // dZ_t[a] = sum_{rows of block tt} gden_r phi(q_r)[a]
+        float dz = 0.f;
+        for (int rr = 64 * tt; rr < 64 * tt + 64; ++rr) {
+          const __nv_bfloat16* fp = reinterpret_cast<const __nv_bfloat16*>(
+              sF + (aa / 64) * TILE + sw128_offset(rr, (aa % 64) * 2));
+          dz = fmaf(sgden[rr], __bfloat162float(*fp), dz);
+        }
+        dst[TD * TD + aa] = __float2bfloat16(dz);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+cudaError_t launch_bwd_rows_tc(const CUtensorMap& mapH, const CUtensorMap& mapZ, const BwdRowsArgs& a,
+                               int* err, int BH, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(bwd_rows_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM_TC);
+  if (e != cudaSuccess) return e;
+  bwd_rows_tc_kernel<<<dim3((a.Tq + 1) / 2, BH), 192, SMEM_TC, s>>>(mapH, mapZ, a, err);
+  return cudaGetLastError();
+}
+
+// Column sums of dO over every row of every head (d bias of Proj): one CTA of
+// d threads per 256 rows, one atomic per column and CTA.
+__global__ void colsum_kernel(const __nv_bfloat16* __restrict__ dO, const int64_t s0, const int64_t s1,
+                              const int64_t s2, int H, int N, int64_t rows, int D, float* __restrict__ out) {
+  const int c = threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.x * 256;
+  float acc = 0.f;
+  for (int64_t r = r0; r < min(r0 + 256, rows); ++r) {
+    const int64_t bh = r / N, n = r % N;
+    acc += __bfloat162float(dO[(bh / H) * s0 + (bh % H) * s1 + n * s2 + c]);
+  }
+  atomicAdd(out + c, acc);
+}
+
+cudaError_t launch_colsum(const __nv_bfloat16* dO, const int64_t* so, int H, int N, int BH, int D,
+                          float* out, cudaStream_t s) {
+  const int64_t rows = (int64_t)BH * N;
+  colsum_kernel<<<(unsigned)((rows + 255) / 256), D, 0, s>>>(dO, so[0], so[1], so[2], H, N, rows, D, out);
+  return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -125,6 +125,10 @@ struct BwdSparseArgs {
 
 cudaError_t launch_bwd_rows(const BwdRowsArgs& a, int D, int BH, cudaStream_t s);
 cudaError_t launch_bwd_keys(const BwdKeysArgs& a, int D, cudaStream_t s);
+cudaError_t launch_bwd_rows_tc(const CUtensorMap& mapH, const CUtensorMap& mapZ, const BwdRowsArgs& a,
+                               int* err, int BH, cudaStream_t s);
+cudaError_t launch_colsum(const __nv_bfloat16* dO, const int64_t* so, int H, int N, int BH, int D,
+                          float* out, cudaStream_t s);
 cudaError_t launch_rlut(const int8_t* mc, int32_t* rcnt, int32_t* rptr, int32_t* rows, int BH,
                         int Tq, int Tkv, int nh, cudaStream_t s);
 cudaError_t launch_bwd_dq(const CUtensorMap& mapQ, const CUtensorMap& mapdO, const CUtensorMap& mapK,
