@@ -411,7 +411,7 @@ sla_status_t attention_impl(const Plan& pl, const sla_params_t* p, const void* Q
 // Backward
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-  size_t err, mm, hagg, drow, dqlin, dhzq, mmt, dhzk, dklin, dvlin, rcnt, rptr, rows, end;
+  size_t err, mm, hagg, drow, dqlin, dhzq, mmt, dhzk, dklin, dvlin, ubuf, rcnt, rptr, rows, end;
 };
 
 BwdLayout bwd_layout_of(const Plan& p) {
@@ -429,6 +429,7 @@ BwdLayout bwd_layout_of(const Plan& p) {
   L.dhzk = o;  o = align_up(o + (size_t)p.BH * p.Tkv * p.NN * 2);
   L.dklin = o; o = align_up(o + act32);
   L.dvlin = o; o = align_up(o + act32);
+  L.ubuf = o;  o = align_up(o + (size_t)p.BH * p.Tkv * 64 * p.d * 2);
   L.rcnt = o;  o = align_up(o + (size_t)p.BH * p.Tkv * 4);
   L.rptr = o;  o = align_up(o + (size_t)p.BH * (p.Tkv + 1) * 4);
   L.rows = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
@@ -526,7 +527,30 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   ka.Tkv = pl.Tkv;
   ka.NN = pl.NN;
   ka.phi = pl.phi;
-  SLA_TRY(cuda_status(launch_bwd_keys(ka, pl.d, s)));
+  if (pl.d == 128) {
+    // tensor-core version: both key blocks of a pair per CTA; dW by a split-K product
+    __nv_bfloat16* dhzk = at<__nv_bfloat16>(ws, L.dhzk);
+    __nv_bfloat16* ubuf = at<__nv_bfloat16>(ws, L.ubuf);
+    CUtensorMap mg, mz, mk2, mv2, mu;
+    const uint64_t dg[4] = {(uint64_t)pl.d, (uint64_t)pl.d, (uint64_t)pl.Tkv, (uint64_t)pl.BH};
+    const uint64_t sg[3] = {(uint64_t)pl.d * 2, (uint64_t)pl.NN * 2, (uint64_t)pl.Tkv * pl.NN * 2};
+    const uint32_t bxg[4] = {64, (uint32_t)pl.d, 1, 1};
+    const uint64_t dz[3] = {(uint64_t)pl.NN, (uint64_t)pl.Tkv, (uint64_t)pl.BH};
+    const uint64_t sz[2] = {(uint64_t)pl.NN * 2, (uint64_t)pl.Tkv * pl.NN * 2};
+    const uint32_t bxz[3] = {64, 1, 1};
+    const uint64_t du[3] = {(uint64_t)pl.d, (uint64_t)pl.Tkv * 64, (uint64_t)pl.BH};
+    const uint64_t su[2] = {(uint64_t)pl.d * 2, (uint64_t)pl.Tkv * 64 * pl.d * 2};
+    const uint32_t bxu[3] = {64, 128, 1};
+    if (!encode(&mg, dhzk, 4, dg, sg, bxg) || !encode(&mz, dhzk, 3, dz, sz, bxz, false) ||
+        !map_bhnd(&mk2, K, pl, p->stride_k, 128) || !map_bhnd(&mv2, V, pl, p->stride_v, 128) ||
+        !encode(&mu, ubuf, 3, du, su, bxu))
+      return SLA_ERR_CUDA;
+    const bool want_dw = !alpha_mode && proj_w && dproj_w;
+    SLA_TRY(cuda_status(launch_bwd_keys_tc(mg, mz, mk2, mv2, ka, want_dw ? ubuf : nullptr, err, s)));
+    if (want_dw) SLA_TRY(cuda_status(launch_dw(mu, mv2, pl.H, pl.BH, pl.Tkv, dproj_w, err, s)));
+  } else {
+    SLA_TRY(cuda_status(launch_bwd_keys(ka, pl.d, s)));
+  }
   // sparse branch
   int32_t* rcnt = at<int32_t>(ws, L.rcnt);
   int32_t* rptr = at<int32_t>(ws, L.rptr);

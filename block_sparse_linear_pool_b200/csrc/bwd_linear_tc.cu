@@ -355,3 +355,419 @@ cudaError_t launch_colsum(const __nv_bfloat16* dO, const int64_t* so, int H, int
 }
 
 }  // namespace sla
+
+namespace sla {
+
+// ---------------------------------------------------------------------------
+// Key side of the linear-branch backward on the tensor cores (d = 128).  A CTA
+// takes key blocks 2p and 2p+1 (128 key rows, one TMEM lane each):
+//   G1  U_t    = phi(K) dh'_t          M = 128 rows, N = d, K = d  (t = 0, 1)
+//   G3  w      = V W~^T                M = 128 rows, N = d, K = d  (SLA; w = V for SLA2)
+//   G2  dv     = U W~                  M = 128 rows, N = d, K = d  (SLA; dv = U for SLA2)
+//   G4  dphi_t = w dh'_t^T             M = 128 rows, N = d, K = d
+// then dk = phi backward of dphi + dz.  dW = sum_t u_t v_t^T is left to
+// dw_kernel: U (bf16, rows of every head) goes to a buffer.
+// TMEM (512 columns): G1 and then G4 at [0, 2d), G3 and then G2 at [2d, 3d).
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int K_OFF_G = 0;                     // dh': [2 a-chunks][2 blocks][TD o][128 B]
+constexpr int K_OFF_F = K_OFF_G + 4 * TILE;    // phi(K), then w: [2 chunks][128 rows][128 B]
+constexpr int K_OFF_V = K_OFF_F + 2 * TILE;    // V pair
+constexpr int K_OFF_U = K_OFF_V + 2 * TILE;    // U (bf16)
+constexpr int K_OFF_W = K_OFF_U + 2 * TILE;    // W~ (bf16): [2 c-chunks][TD o][128 B]
+constexpr int K_OFF_Z = K_OFF_W + 2 * TILE;    // dz_t: [2][TD] bf16
+constexpr int K_OFF_BAR = K_OFF_Z + 2 * TD * 2;
+constexpr int K_SMEM = K_OFF_BAR + 256 + 1024;
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap mapG, const __grid_constant__ CUtensorMap mapZ,
+                       const __grid_constant__ CUtensorMap mapK2, const __grid_constant__ CUtensorMap mapV2,
+                       BwdKeysArgs a, __nv_bfloat16* ubuf, int* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                           ~uintptr_t(1023));
+  uint8_t* sG = sm + K_OFF_G;
+  uint8_t* sF = sm + K_OFF_F;
+  uint8_t* sV = sm + K_OFF_V;
+  uint8_t* sU = sm + K_OFF_U;
+  uint8_t* sW = sm + K_OFF_W;
+  const __nv_bfloat16* sZ = reinterpret_cast<const __nv_bfloat16*>(sm + K_OFF_Z);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + K_OFF_BAR);
+  uint64_t* in_full = bars + 0;
+  uint64_t* fk_ready = bars + 1;
+  uint64_t* g1_full = bars + 2;
+  uint64_t* u_ready = bars + 3;
+  uint64_t* g2_full = bars + 4;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 5);
+
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  const int p = blockIdx.x, bh = blockIdx.y;
+  const int b = bh / a.H, h = bh % a.H;
+  const int j0 = 2 * p, j1 = 2 * p + 1;
+  const bool has1 = j1 < a.Tkv;
+  const bool proj = a.proj_w != nullptr;
+
+  if (w == 1) {
+    tmem_alloc(tslot, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(in_full, 1);
+    mbar_init(fk_ready, 128);
+    mbar_init(g1_full, 1);
+    mbar_init(u_ready, 128);
+    mbar_init(g2_full, 1);
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tslot;
+
+  if (w == 0) {
+    if (ln == 0) {
+      tma_prefetch_desc(&mapG);
+      tma_prefetch_desc(&mapZ);
+      tma_prefetch_desc(&mapK2);
+      tma_prefetch_desc(&mapV2);
+      mbar_arrive_expect_tx(in_full, 2 * (2 * TILE + TD * 2) + 4 * TILE);
+      for (int t = 0; t < 2; ++t) {
+        const int j = (t == 1 && has1) ? j1 : j0;  // a missing second block reuses the first
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tma_load_4d(sG + c * 2 * TILE + t * TILE, &mapG, in_full, c * 64, 0, j, bh);
+          tma_load_3d(sm + K_OFF_Z + t * TD * 2 + c * 128, &mapZ, in_full, TD * TD + c * 64, j, bh);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tma_load_4d(sF + c * TILE, &mapK2, in_full, c * 64, 128 * p, h, b);
+        tma_load_4d(sV + c * TILE, &mapV2, in_full, c * 64, 128 * p, h, b);
+      }
+    }
+  } else if (w == 1) {
+    if (ln == 0) {
+      const uint32_t id_kk = idesc_bf16(128, TD, false, false);
+      const uint32_t id_km = idesc_bf16(128, TD, false, true);
+      const uint32_t g0 = smem_u32(sG), f0 = smem_u32(sF), v0 = smem_u32(sV), u0 = smem_u32(sU),
+                     w0 = smem_u32(sW);
+      bool ok = mbar_wait(fk_ready, 0, err, DEV_TIMEOUT_SYNC);
+      if (ok) {
+        tc_fence_after();
+        // G1: U_t[r][o] = sum_a F[r][a] dh'_t[a][o]
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int kk = 0; kk < TD / 16; ++kk)
+            umma_ss(tbase + TD * t, sdesc_sw128(f0 + (kk / 4) * TILE + (kk % 4) * 32, 16, 1024),
+                    sdesc_sw128(g0 + (kk / 4) * 2 * TILE + t * TILE + (kk % 4) * 32, 16, 1024), id_kk,
+                    kk > 0 ? 1u : 0u);
+        // G3: w[r][o] = sum_c V[r][c] W[o][c]
+        if (proj)
+#pragma unroll
+          for (int kk = 0; kk < TD / 16; ++kk)
+            umma_ss(tbase + 2 * TD, sdesc_sw128(v0 + (kk / 4) * TILE + (kk % 4) * 32, 16, 1024),
+                    sdesc_sw128(w0 + (kk / 4) * TILE + (kk % 4) * 32, 16, 1024), id_kk, kk > 0 ? 1u : 0u);
+        umma_commit(g1_full);
+        ok = mbar_wait(u_ready, 0, err, DEV_TIMEOUT_SYNC);
+      }
+      if (ok) {
+        tc_fence_after();
+        // G2: dv[r][c] = sum_o U[r][o] W[o][c]   (B: N = c contiguous, K = o rows)
+        if (proj)
+#pragma unroll
+          for (int kk = 0; kk < TD / 16; ++kk)
+            umma_ss(tbase + 2 * TD, sdesc_sw128(u0 + (kk / 4) * TILE + (kk % 4) * 32, 16, 1024),
+                    sdesc_sw128(w0 + kk * 2048, TILE, 1024), id_km, kk > 0 ? 1u : 0u);
+        // G4: dphi_t[r][a] = sum_o w[r][o] dh'_t[a][o]   (w in sF for SLA, V itself for SLA2)
+        const uint32_t ws = proj ? f0 : v0;
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+          for (int kk = 0; kk < TD / 16; ++kk)
+            umma_ss(tbase + TD * t, sdesc_sw128(ws + (kk / 4) * TILE + (kk % 4) * 32, 16, 1024),
+                    sdesc_sw128(g0 + t * TILE + kk * 2048, 2 * TILE, 1024), id_km, kk > 0 ? 1u : 0u);
+        umma_commit(g2_full);
+      }
+    }
+  } else {
+    const int q4 = w & 3;
+    const int r = 32 * q4 + ln;  // key row of the pair
+    const int t = r >> 6;
+    const int n = 128 * p + r;
+    const bool valid = (t == 0 || has1) && n < a.N;
+    const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
+    // W~ as bf16 into sW (row o = r), the K-major B operand of G3 / MN-major B of G2
+    if (proj) {
+      const float* wr = a.proj_w + (int64_t)r * TD;
+      for (int c = 0; c < TD; c += 8) {
+        const float4 x0 = *reinterpret_cast<const float4*>(wr + c);
+        const float4 x1 = *reinterpret_cast<const float4*>(wr + c + 4);
+        *reinterpret_cast<uint4*>(sW + (c / 64) * TILE + sw128_offset(r, (c % 64) * 2)) =
+            make_uint4(pack_bf16x2(x0.x, x0.y), pack_bf16x2(x0.z, x0.w), pack_bf16x2(x1.x, x1.y),
+                       pack_bf16x2(x1.z, x1.w));
+      }
+    }
+    bool ok = __all_sync(0xffffffffu, mbar_wait(in_full, 0, err, DEV_TIMEOUT_TMA));
+    // ---- phi(K) in place (bf16); rows that do not exist get 0
+    const __nv_bfloat16* krow = a.K + (int64_t)b * a.sk[0] + (int64_t)h * a.sk[1] + (int64_t)n * a.sk[2];
+    float m = -INFINITY, s = 0.f;
+    if (valid && a.phi == 0) {
+      for (int c = 0; c < TD; c += 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(krow + c);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, bfv(u[e / 2], e & 1));
+      }
+      for (int c = 0; c < TD; c += 8) {
+        const uint4 v = *reinterpret_cast<const uint4*>(krow + c);
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += exp2f((bfv(u[e / 2], e & 1) - m) * LOG2E_T);
+      }
+    }
+    const float inv_s = (a.phi == 0 && s > 0.f) ? 1.f / s : 1.f;
+    auto phi_of = [&](float x) {
+      return a.phi == 1 ? (x > 0.f ? x + 1.f : exp2f(x * LOG2E_T)) : exp2f((x - m) * LOG2E_T) * inv_s;
+    };
+    if (ok) {
+      for (int c = 0; c < TD; c += 8) {
+        uint8_t* dst = sF + (c / 64) * TILE + sw128_offset(r, (c % 64) * 2);
+        uint32_t o4[4] = {0u, 0u, 0u, 0u};
+        if (valid) {
+          const uint4 v = *reinterpret_cast<const uint4*>(dst);  // K as loaded (bf16)
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o4[e] = pack_bf16x2(phi_of(bfv(u[e], 0)), phi_of(bfv(u[e], 1)));
+        }
+        *reinterpret_cast<uint4*>(dst) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(fk_ready);
+    // ---- U (own block's half) -> sU (and the U buffer for dW, SLA); dv = U for SLA2;
+    //      w -> sF (SLA)
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(g1_full, 0, err, DEV_TIMEOUT_MMA));
+    if (ok) {
+      tc_fence_after();
+      __nv_bfloat16* urow = ubuf ? ubuf + ((int64_t)bh * a.Tkv * 64 + n) * TD : nullptr;
+      float* dvrow = a.dv_lin + ((int64_t)bh * a.N + n) * TD;
+#pragma unroll 1
+      for (int c0 = 0; c0 < TD; c0 += 32) {
+        uint32_t uv[32];
+        tmem_ld32(tl + TD * t + c0, uv);
+        tmem_ld_wait();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[e] = valid ? pack_bf16x2(__uint_as_float(uv[2 * e]), __uint_as_float(uv[2 * e + 1])) : 0u;
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          const uint4 q = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          *reinterpret_cast<uint4*>(sU + (c0 / 64) * TILE + sw128_offset(r, ((c0 % 64) + 8 * v4) * 2)) = q;
+          if (urow && (t == 0 || has1) && n < a.Tkv * 64) reinterpret_cast<uint4*>(urow + c0)[v4] = q;
+        }
+        if (!proj && valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dvrow + c0 + e) =
+                make_float4(__uint_as_float(uv[e]), __uint_as_float(uv[e + 1]), __uint_as_float(uv[e + 2]),
+                            __uint_as_float(uv[e + 3]));
+        }
+      }
+      if (proj) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < TD; c0 += 32) {
+          uint32_t wv[32];
+          tmem_ld32(tl + 2 * TD + c0, wv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            uint32_t q[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              q[e] = pack_bf16x2(__uint_as_float(wv[8 * v4 + 2 * e]), __uint_as_float(wv[8 * v4 + 2 * e + 1]));
+            *reinterpret_cast<uint4*>(sF + (c0 / 64) * TILE + sw128_offset(r, ((c0 % 64) + 8 * v4) * 2)) =
+                make_uint4(q[0], q[1], q[2], q[3]);
+          }
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(u_ready);
+    // ---- dv (SLA) and dk = phi backward of dphi_t + dz_t.  tcgen05.ld is a
+    // warp-wide instruction: every lane runs it, only valid rows store.
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(g2_full, 0, err, DEV_TIMEOUT_MMA));
+    if (ok) {
+      tc_fence_after();
+      if (proj) {
+        float* dvrow = a.dv_lin + ((int64_t)bh * a.N + n) * TD;
+#pragma unroll 1
+        for (int c0 = 0; c0 < TD; c0 += 32) {
+          uint32_t dv[32];
+          tmem_ld32(tl + 2 * TD + c0, dv);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4*>(dvrow + c0 + e) =
+                  make_float4(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1]), __uint_as_float(dv[e + 2]),
+                              __uint_as_float(dv[e + 3]));
+          }
+        }
+      }
+      const __nv_bfloat16* z = sZ + t * TD;
+      float dot = 0.f;
+      if (a.phi == 0) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < TD; c0 += 32) {
+          uint32_t dv[32];
+          tmem_ld32(tl + TD * t + c0, dv);
+          tmem_ld_wait();
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              dot = fmaf(phi_of(__bfloat162float(krow[c0 + e])),
+                         __uint_as_float(dv[e]) + __bfloat162float(z[c0 + e]), dot);
+          }
+        }
+      }
+      float* out = a.dk_lin + ((int64_t)bh * a.N + n) * TD;
+#pragma unroll 1
+      for (int c0 = 0; c0 < TD; c0 += 32) {
+        uint32_t dv[32];
+        tmem_ld32(tl + TD * t + c0, dv);
+        tmem_ld_wait();
+        if (valid) {
+#pragma unroll
+          for (int e4 = 0; e4 < 32; e4 += 4) {
+            float y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float x = __bfloat162float(krow[c0 + e4 + e]);
+              const float dphi = __uint_as_float(dv[e4 + e]) + __bfloat162float(z[c0 + e4 + e]);
+              y[e] = a.phi == 1 ? dphi * (x > 0.f ? 1.f : exp2f(x * LOG2E_T)) : phi_of(x) * (dphi - dot);
+            }
+            *reinterpret_cast<float4*>(out + c0 + e4) = make_float4(y[0], y[1], y[2], y[3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dW = sum over every token row of u_t v_t^T (SLA's Proj weight gradient):
+// persistent, CTA c sums 128-row tiles c, c + G, ... of all heads into one
+// 128 x 128 TMEM accumulator (A = U^T and B = V, both MN-major: the rows are
+// the reduction), then adds it to dproj_w with one atomic per element.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(192, 1)
+    dw_kernel(const __grid_constant__ CUtensorMap mapU, const __grid_constant__ CUtensorMap mapV2,
+              int H, int Tkv, int ntiles_head, int ntiles, float* __restrict__ dW, int* err) {
+  extern __shared__ uint8_t smem_dw[];  // 2 stages of (U tile, V tile), 1024-byte aligned
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dw) + 1023) & ~uintptr_t(1023));
+  (void)Tkv;
+  __shared__ uint64_t full[2], empty[2], done;
+  __shared__ uint32_t tslot;
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  if (w == 1) {
+    tmem_alloc(&tslot, 128);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&full[x], 1);
+      mbar_init(&empty[x], 1);
+    }
+    mbar_init(&done, 1);
+    fence_barrier_init();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tslot;
+  int my = 0;
+  for (int tt = blockIdx.x; tt < ntiles; tt += gridDim.x) ++my;
+  if (w == 0 && ln == 0) {
+    bool ok = true;
+    int k = 0;
+    for (int tt = blockIdx.x; tt < ntiles && ok; tt += gridDim.x, ++k) {
+      const int x = k & 1;
+      if (k >= 2 && !mbar_wait(&empty[x], ((k - 2) >> 1) & 1, err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
+      const int bh = tt / ntiles_head, r0 = 128 * (tt % ntiles_head);
+      uint8_t* st = sm + x * 4 * TILE;
+      mbar_arrive_expect_tx(&full[x], 4 * TILE);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tma_load_3d(st + c * TILE, &mapU, &full[x], c * 64, r0, bh);
+        tma_load_4d(st + 2 * TILE + c * TILE, &mapV2, &full[x], c * 64, r0, bh % H, bh / H);
+      }
+    }
+  } else if (w == 1 && ln == 0) {
+    const uint32_t id_mm = idesc_bf16(128, TD, true, true);
+    bool ok = true;
+    for (int k = 0; k < my && ok; ++k) {
+      const int x = k & 1;
+      if (!mbar_wait(&full[x], (k >> 1) & 1, err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t st = smem_u32(sm + x * 4 * TILE);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        umma_ss(tbase, sdesc_sw128(st + kk * 2048, TILE, 1024), sdesc_sw128(st + 2 * TILE + kk * 2048, TILE, 1024),
+                id_mm, (k > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(&empty[x]);
+    }
+    if (ok) umma_commit(&done);
+  } else if (w >= 2) {
+    const int q4 = w & 3;
+    const int o = 32 * q4 + ln;
+    if (my > 0 && __all_sync(0xffffffffu, mbar_wait(&done, 0, err, DEV_TIMEOUT_MMA))) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < TD; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tbase + ((uint32_t)(32 * q4) << 16) + c0, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) atomicAdd(dW + (int64_t)o * TD + c0 + e, __uint_as_float(v[e]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 128);
+  }
+}
+
+cudaError_t launch_bwd_keys_tc(const CUtensorMap& mapG, const CUtensorMap& mapZ, const CUtensorMap& mapK2,
+                               const CUtensorMap& mapV2, const BwdKeysArgs& a, __nv_bfloat16* ubuf, int* err,
+                               cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(bwd_keys_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, K_SMEM);
+  if (e != cudaSuccess) return e;
+  bwd_keys_tc_kernel<<<dim3((a.Tkv + 1) / 2, a.BH), 192, K_SMEM, s>>>(mapG, mapZ, mapK2, mapV2, a, ubuf, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dw(const CUtensorMap& mapU, const CUtensorMap& mapV2, int H, int BH, int Tkv, float* dW,
+                      int* err, cudaStream_t s) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int per_head = (Tkv * 64 + 127) / 128;
+  const int ntiles = per_head * BH;
+  const int smem = 2 * 4 * TILE + 1024;
+  cudaError_t e = cudaFuncSetAttribute(dw_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  dw_kernel<<<ntiles < sms ? ntiles : sms, 192, smem, s>>>(mapU, mapV2, H, Tkv, per_head, ntiles, dW, err);
+  return cudaGetLastError();
+}
+
+}  // namespace sla

@@ -127,6 +127,11 @@ cudaError_t launch_bwd_rows(const BwdRowsArgs& a, int D, int BH, cudaStream_t s)
 cudaError_t launch_bwd_keys(const BwdKeysArgs& a, int D, cudaStream_t s);
 cudaError_t launch_bwd_rows_tc(const CUtensorMap& mapH, const CUtensorMap& mapZ, const BwdRowsArgs& a,
                                int* err, int BH, cudaStream_t s);
+cudaError_t launch_bwd_keys_tc(const CUtensorMap& mapG, const CUtensorMap& mapZ, const CUtensorMap& mapK2,
+                               const CUtensorMap& mapV2, const BwdKeysArgs& a, __nv_bfloat16* ubuf, int* err,
+                               cudaStream_t s);
+cudaError_t launch_dw(const CUtensorMap& mapU, const CUtensorMap& mapV2, int H, int BH, int Tkv, float* dW,
+                      int* err, cudaStream_t s);
 cudaError_t launch_colsum(const __nv_bfloat16* dO, const int64_t* so, int H, int N, int BH, int D,
                           float* out, cudaStream_t s);
 cudaError_t launch_rlut(const int8_t* mc, int32_t* rcnt, int32_t* rptr, int32_t* rows, int BH,
