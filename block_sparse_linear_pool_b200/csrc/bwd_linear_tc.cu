@@ -29,7 +29,8 @@ constexpr int OFF_F = OFF_H + 4 * TILE;       // phi(Q): [2 a-chunks][128 rows][
 constexpr int OFF_G = OFF_F + 2 * TILE;       // gp:     [2 o-chunks][128 rows][128 B]
 constexpr int OFF_Z = OFF_G + 2 * TILE;       // Z_t: [2][TD] bf16
 constexpr int OFF_GD = OFF_Z + 2 * TD * 2;    // gden [128] fp32
-constexpr int OFF_BAR = OFF_GD + 128 * 4;
+constexpr int OFF_PHI = OFF_GD + 128 * 4;     // phi(q) fp32 [128 rows][TD + 1]
+constexpr int OFF_BAR = OFF_PHI + 128 * (TD + 1) * 4;
 constexpr int SMEM_TC = OFF_BAR + 256 + 1024;
 constexpr float LOG2E_T = 1.4426950408889634f;
 
@@ -49,6 +50,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sG = sm + OFF_G;
   const __nv_bfloat16* sZ = reinterpret_cast<const __nv_bfloat16*>(sm + OFF_Z);
   float* sgden = reinterpret_cast<float*>(sm + OFF_GD);
+  float* sphi = reinterpret_cast<float*>(sm + OFF_PHI);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_BAR);
   uint64_t* h_full = bars + 0;
   uint64_t* fq_ready = bars + 1;
@@ -175,7 +177,10 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            o4[e] = pack_bf16x2(phi_of(bfv(u[e], 0)), phi_of(bfv(u[e], 1)));
+            const float f0 = phi_of(bfv(u[e], 0)), f1 = phi_of(bfv(u[e], 1));
+            sphi[r * (TD + 1) + c + 2 * e] = f0;
+            sphi[r * (TD + 1) + c + 2 * e + 1] = f1;
+            o4[e] = pack_bf16x2(f0, f1);
             den = fmaf(bfv(o4[e], 0), __bfloat162float(z[c + 2 * e]),
                        fmaf(bfv(o4[e], 1), __bfloat162float(z[c + 2 * e + 1]), den));
           }
@@ -258,10 +263,9 @@ __global__ void __launch_bounds__(192, 1)
           tmem_ld_wait();
           if (valid) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const float f = phi_of(__bfloat162float(qrow[c0 + e]));
-              dot = fmaf(f, __uint_as_float(dv[e]) + gden * __bfloat162float(z[c0 + e]), dot);
-            }
+            for (int e = 0; e < 32; ++e)
+              dot = fmaf(sphi[r * (TD + 1) + c0 + e], __uint_as_float(dv[e]) + gden * __bfloat162float(z[c0 + e]),
+                         dot);
           }
         }
       }
@@ -277,9 +281,10 @@ __global__ void __launch_bounds__(192, 1)
             float y[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float x = __bfloat162float(qrow[c0 + e4 + e]);
+              const float f = sphi[r * (TD + 1) + c0 + e4 + e];
               const float dphi = __uint_as_float(dv[e4 + e]) + gden * __bfloat162float(z[c0 + e4 + e]);
-              y[e] = a.phi == 1 ? dphi * (x > 0.f ? 1.f : exp2f(x * LOG2E_T)) : phi_of(x) * (dphi - dot);
+              // elu + 1: d phi / dx = 1 where x > 0 (phi > 1), else e^x = phi
+              y[e] = a.phi == 1 ? dphi * (f > 1.f ? 1.f : f) : f * (dphi - dot);
             }
             *reinterpret_cast<float4*>(out + c0 + e4) = make_float4(y[0], y[1], y[2], y[3]);
           }
@@ -333,24 +338,39 @@ cudaError_t launch_bwd_rows_tc(const CUtensorMap& mapH, const CUtensorMap& mapZ,
   return cudaGetLastError();
 }
 
-// Column sums of dO over every row of every head (d bias of Proj): one CTA of
-// d threads per 256 rows, one atomic per column and CTA.
-__global__ void colsum_kernel(const __nv_bfloat16* __restrict__ dO, const int64_t s0, const int64_t s1,
-                              const int64_t s2, int H, int N, int64_t rows, int D, float* __restrict__ out) {
-  const int c = threadIdx.x;
-  const int64_t r0 = (int64_t)blockIdx.x * 256;
-  float acc = 0.f;
-  for (int64_t r = r0; r < min(r0 + 256, rows); ++r) {
+// Column sums of dO over every row of every head (d bias of Proj).  256
+// threads = 16 row lanes x 16 groups of 8 columns (16-byte loads); a CTA sums
+// 1024 rows, reduces its 16 row lanes in shared memory and adds one atomic per
+// column.
+__global__ void __launch_bounds__(256) colsum_kernel(const __nv_bfloat16* __restrict__ dO, const int64_t s0,
+                                                     const int64_t s1, const int64_t s2, int H, int N,
+                                                     int64_t rows, float* __restrict__ out) {
+  __shared__ float red[16][TD + 4];
+  const int cg = threadIdx.x & 15, rl = threadIdx.x >> 4;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  const int64_t r0 = (int64_t)blockIdx.x * 1024;
+  for (int64_t r = r0 + rl; r < min(r0 + 1024, rows); r += 16) {
     const int64_t bh = r / N, n = r % N;
-    acc += __bfloat162float(dO[(bh / H) * s0 + (bh % H) * s1 + n * s2 + c]);
+    const uint4 v = *reinterpret_cast<const uint4*>(dO + (bh / H) * s0 + (bh % H) * s1 + n * s2 + 8 * cg);
+    const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += bfv(u[e / 2], e & 1);
   }
-  atomicAdd(out + c, acc);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[rl][8 * cg + e] = acc[e];
+  __syncthreads();
+  if (threadIdx.x < TD) {
+    float t = 0.f;
+    for (int k = 0; k < 16; ++k) t += red[k][threadIdx.x];
+    atomicAdd(out + threadIdx.x, t);
+  }
 }
 
 cudaError_t launch_colsum(const __nv_bfloat16* dO, const int64_t* so, int H, int N, int BH, int D,
                           float* out, cudaStream_t s) {
+  if (D != TD) return cudaErrorInvalidValue;
   const int64_t rows = (int64_t)BH * N;
-  colsum_kernel<<<(unsigned)((rows + 255) / 256), D, 0, s>>>(dO, so[0], so[1], so[2], H, N, rows, D, out);
+  colsum_kernel<<<(unsigned)((rows + 1023) / 1024), 256, 0, s>>>(dO, so[0], so[1], so[2], H, N, rows, out);
   return cudaGetLastError();
 }
 
@@ -367,7 +387,8 @@ namespace sla {
 //   G4  dphi_t = w dh'_t^T             M = 128 rows, N = d, K = d
 // then dk = phi backward of dphi + dz.  dW = sum_t u_t v_t^T is left to
 // dw_kernel: U (bf16, rows of every head) goes to a buffer.
-// TMEM (512 columns): G1 and then G4 at [0, 2d), G3 and then G2 at [2d, 3d).
+// TMEM (512 columns): G1 and then G4 at [0, 2d), G3 and then G2 at [2d, 3d),
+// phi(K) in fp32 at [3d, 4d).
 // ---------------------------------------------------------------------------
 namespace {
 constexpr int K_OFF_G = 0;                     // dh': [2 a-chunks][2 blocks][TD o][128 B]
@@ -529,18 +550,35 @@ __global__ void __launch_bounds__(192, 1)
     auto phi_of = [&](float x) {
       return a.phi == 1 ? (x > 0.f ? x + 1.f : exp2f(x * LOG2E_T)) : exp2f((x - m) * LOG2E_T) * inv_s;
     };
+    // phi(K) in place in sF (bf16, the MMA operand) and in fp32 in TMEM columns
+    // [3d, 4d) of this row's lane, for the phi backward at the end
     if (ok) {
-      for (int c = 0; c < TD; c += 8) {
-        uint8_t* dst = sF + (c / 64) * TILE + sw128_offset(r, (c % 64) * 2);
-        uint32_t o4[4] = {0u, 0u, 0u, 0u};
-        if (valid) {
-          const uint4 v = *reinterpret_cast<const uint4*>(dst);  // K as loaded (bf16)
-          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll 1
+      for (int c0 = 0; c0 < TD; c0 += 32) {
+        uint32_t fv[32];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o4[e] = pack_bf16x2(phi_of(bfv(u[e], 0)), phi_of(bfv(u[e], 1)));
+        for (int c8 = 0; c8 < 32; c8 += 8) {
+          uint8_t* dst = sF + (c0 / 64) * TILE + sw128_offset(r, ((c0 % 64) + c8) * 2);
+          uint32_t o4[4] = {0u, 0u, 0u, 0u};
+          if (valid) {
+            const uint4 v = *reinterpret_cast<const uint4*>(dst);  // K as loaded (bf16)
+            const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float f0 = phi_of(bfv(u[e], 0)), f1 = phi_of(bfv(u[e], 1));
+              fv[c8 + 2 * e] = __float_as_uint(f0);
+              fv[c8 + 2 * e + 1] = __float_as_uint(f1);
+              o4[e] = pack_bf16x2(f0, f1);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) fv[c8 + e] = 0u;
+          }
+          *reinterpret_cast<uint4*>(dst) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
         }
-        *reinterpret_cast<uint4*>(dst) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        tmem_st32(tl + 3 * TD + c0, fv);
       }
+      tmem_st_wait();
     }
     fence_proxy_async_smem();
     mbar_arrive(fk_ready);
@@ -620,22 +658,23 @@ __global__ void __launch_bounds__(192, 1)
       if (a.phi == 0) {
 #pragma unroll 1
         for (int c0 = 0; c0 < TD; c0 += 32) {
-          uint32_t dv[32];
+          uint32_t dv[32], fv[32];
           tmem_ld32(tl + TD * t + c0, dv);
+          tmem_ld32(tl + 3 * TD + c0, fv);
           tmem_ld_wait();
           if (valid) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              dot = fmaf(phi_of(__bfloat162float(krow[c0 + e])),
-                         __uint_as_float(dv[e]) + __bfloat162float(z[c0 + e]), dot);
+              dot = fmaf(__uint_as_float(fv[e]), __uint_as_float(dv[e]) + __bfloat162float(z[c0 + e]), dot);
           }
         }
       }
       float* out = a.dk_lin + ((int64_t)bh * a.N + n) * TD;
 #pragma unroll 1
       for (int c0 = 0; c0 < TD; c0 += 32) {
-        uint32_t dv[32];
+        uint32_t dv[32], fv[32];
         tmem_ld32(tl + TD * t + c0, dv);
+        tmem_ld32(tl + 3 * TD + c0, fv);
         tmem_ld_wait();
         if (valid) {
 #pragma unroll
@@ -643,9 +682,10 @@ __global__ void __launch_bounds__(192, 1)
             float y[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float x = __bfloat162float(krow[c0 + e4 + e]);
+              const float f = __uint_as_float(fv[e4 + e]);
               const float dphi = __uint_as_float(dv[e4 + e]) + __bfloat162float(z[c0 + e4 + e]);
-              y[e] = a.phi == 1 ? dphi * (x > 0.f ? 1.f : exp2f(x * LOG2E_T)) : phi_of(x) * (dphi - dot);
+              // elu + 1: d phi / dx = 1 where x > 0 (phi > 1), else e^x = phi
+              y[e] = a.phi == 1 ? dphi * (f > 1.f ? 1.f : f) : f * (dphi - dot);
             }
             *reinterpret_cast<float4*>(out + c0 + e4) = make_float4(y[0], y[1], y[2], y[3]);
           }

@@ -15,12 +15,14 @@
 //                       that have it critical (ascending), from M_c
 //   bwd_dq_kernel       CTA = query blocks 2p, 2p+1 (M = 128) over the union of
 //                       their critical lists: S = Q K^T and dP = dO V^T into
-//                       TMEM, dS by the row threads, dQ += dS K (dS read from TMEM)
+//                       TMEM (two buffers), dS by the row threads, dQ += dS K
+//                       (dS read from TMEM)
 //   bwd_dkdv_kernel     CTA = key blocks 2p, 2p+1 (M = 128 key rows) over the
 //                       union of their reverse lists: S^T = K Q^T and
 //                       dP^T = V dO^T into TMEM (two buffers), P^T and dS^T by
 //                       the key-row threads, dV += P^T dO and dK += dS^T Q
-// Both: warp 0 TMA producer, warp 1 MMA issuer, warps 2-5 one TMEM lane each.
+// Both: warp 0 TMA producer, warp 1 MMA issuer, warps 2-9 two threads per TMEM
+// lane (each takes half of the 64 columns of a score tile).
 #include "kernels.cuh"
 
 namespace sla {
@@ -95,30 +97,39 @@ cudaError_t launch_rlut(const int8_t* mc, int32_t* rcnt, int32_t* rptr, int32_t*
 }
 
 // ---------------------------------------------------------------------------
-// dQ.  TMEM: S [0,64) (dS over its first 32 columns), dP [64,128), dQ [128,128+d).
-// Shared: Q tile, dO tile (128 rows), one K slot and one V slot (64 rows).
+// dQ.  TMEM (512 columns, one CTA per SM): two score buffers x = 0, 1 with S at
+// [128x, 128x + 64) (dS over its first 32 columns) and dP at [128x + 64,
+// 128x + 128); dQ at [256, 256 + d).  S, dP of entry k+1 are computed while the
+// row threads turn entry k into dS.  Shared: Q and dO tiles (128 rows), a
+// 3-slot K ring (K_k serves S_k and, later, dQ += dS_k K_k) and a 2-slot V ring.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DqSmem {
   static constexpr int CH = D / 64;
   static constexpr int T128 = 128 * D * 2;
   static constexpr int T64 = 64 * D * 2;
+  static constexpr int NK = 3, NV = 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_DO = OFF_Q + T128;
   static constexpr int OFF_K = OFF_DO + T128;
-  static constexpr int OFF_V = OFF_K + T64;
-  static constexpr int OFF_BAR = OFF_V + T64;
+  static constexpr int OFF_V = OFF_K + NK * T64;
+  static constexpr int OFF_BAR = OFF_V + NV * T64;
   static constexpr int OFF_U = OFF_BAR + 256;
-  static size_t bytes(int Tkv) { return (size_t)OFF_U + 5 * (size_t)((Tkv + 15) & ~15) + 1024; }
+  // at least 120 KB: one CTA per SM (it holds all 512 TMEM columns)
+  static size_t bytes(int Tkv) {
+    const size_t b = (size_t)OFF_U + 5 * (size_t)((Tkv + 15) & ~15) + 1024;
+    return b < 120 * 1024 ? 120 * 1024 : b;
+  }
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 2)
+__global__ void __launch_bounds__(320, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapdO,
                   const __grid_constant__ CUtensorMap mapK, const __grid_constant__ CUtensorMap mapV,
                   BwdSparseArgs a) {
   using L = DqSmem<D>;
-  constexpr uint32_t COL_S = 0, COL_DP = 64, COL_DQ = 128;
+  constexpr int NK = L::NK, NV = L::NV;
+  constexpr uint32_t COL_DQ = 256;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -127,15 +138,15 @@ __global__ void __launch_bounds__(192, 2)
   uint8_t* sK = sm + L::OFF_K;
   uint8_t* sV = sm + L::OFF_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
-  uint64_t* in_full = bars + 0;   // Q and dO
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = bars + 2;
-  uint64_t* v_full = bars + 3;
-  uint64_t* v_empty = bars + 4;
-  uint64_t* sp_full = bars + 5;   // S and dP in TMEM
-  uint64_t* ds_ready = bars + 6;  // dS written by all row threads
-  uint64_t* dq_done = bars + 7;   // the last dQ MMA completed
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 8);
+  uint64_t* in_full = bars + 0;    // Q and dO
+  uint64_t* k_full = bars + 1;     // [NK]
+  uint64_t* k_empty = bars + 4;    // [NK]
+  uint64_t* v_full = bars + 7;     // [NV]
+  uint64_t* v_empty = bars + 9;    // [NV]
+  uint64_t* sp_full = bars + 11;   // [2] S and dP of buffer x
+  uint64_t* ds_ready = bars + 13;  // [2] dS written by all row threads
+  uint64_t* dq_done = bars + 15;   // the last dQ MMA completed
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 16);
   int* s_count = reinterpret_cast<int*>(tslot + 1);
   const int Tkvr = (a.Tkv + 15) & ~15;
   uint8_t* fa = sm + L::OFF_U;
@@ -150,17 +161,23 @@ __global__ void __launch_bounds__(192, 2)
   const bool has_b = ib < a.Tq;
 
   if (w == 1) {
-    tmem_alloc(tslot, 256);
+    tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
     mbar_init(in_full, 1);
-    mbar_init(k_full, 1);
-    mbar_init(k_empty, 1);
-    mbar_init(v_full, 1);
-    mbar_init(v_empty, 1);
-    mbar_init(sp_full, 1);
-    mbar_init(ds_ready, 128);
+    for (int x = 0; x < NK; ++x) {
+      mbar_init(&k_full[x], 1);
+      mbar_init(&k_empty[x], 1);
+    }
+    for (int x = 0; x < NV; ++x) {
+      mbar_init(&v_full[x], 1);
+      mbar_init(&v_empty[x], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&sp_full[x], 1);
+      mbar_init(&ds_ready[x], 256);
+    }
     mbar_init(dq_done, 1);
     fence_barrier_init();
   }
@@ -217,53 +234,73 @@ __global__ void __launch_bounds__(192, 2)
       }
       bool ok = true;
       for (int k = 0; k < U && ok; ++k) {
-        const int j = uidx[k];
-        if (k >= 1 && !mbar_wait(k_empty, (k - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
-        mbar_arrive_expect_tx(k_full, L::T64);
+        const int j = uidx[k], sk = k % NK, sv = k % NV;
+        if (k >= NK && !mbar_wait(&k_empty[sk], ((k / NK) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&k_full[sk], L::T64);
 #pragma unroll
-        for (int c = 0; c < L::CH; ++c) tma_load_4d(sK + c * 8192, &mapK, k_full, c * 64, 64 * j, h, b);
-        if (k >= 1 && !mbar_wait(v_empty, (k - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
-        mbar_arrive_expect_tx(v_full, L::T64);
+        for (int c = 0; c < L::CH; ++c)
+          tma_load_4d(sK + sk * L::T64 + c * 8192, &mapK, &k_full[sk], c * 64, 64 * j, h, b);
+        if (k >= NV && !mbar_wait(&v_empty[sv], ((k / NV) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[sv], L::T64);
 #pragma unroll
-        for (int c = 0; c < L::CH; ++c) tma_load_4d(sV + c * 8192, &mapV, v_full, c * 64, 64 * j, h, b);
+        for (int c = 0; c < L::CH; ++c)
+          tma_load_4d(sV + sv * L::T64 + c * 8192, &mapV, &v_full[sv], c * 64, 64 * j, h, b);
       }
     }
   } else if (w == 1) {
     if (ln == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
       const uint32_t id_q = idesc_bf16(128, D, false, true);
-      const uint32_t q0 = smem_u32(sQ), o0 = smem_u32(sdO), kt = smem_u32(sK), vt = smem_u32(sV);
+      const uint32_t q0 = smem_u32(sQ), o0 = smem_u32(sdO);
       bool ok = mbar_wait(in_full, 0, a.err, DEV_TIMEOUT_TMA);
-      for (int k = 0; k < U && ok; ++k) {
-        if (!mbar_wait(k_full, k & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
-        if (!mbar_wait(v_full, k & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+      // dQ += dS_k K_k: dS (bf16 pairs) from TMEM buffer k & 1, K as the MN-major B operand
+      auto issue_dq = [&](int k) -> bool {
+        const int x = k & 1, sk = k % NK;
+        if (!mbar_wait(&ds_ready[x], (k >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
         tc_fence_after();
-        // S and dP overwrite dS_{k-1}: its dQ MMA was issued earlier by this
-        // thread, and tcgen05.mma operations of one thread execute in order
+        const uint32_t kt = smem_u32(sK + sk * L::T64);
+        // keys 16 kk .. 16 kk + 15: packed at columns 32 (kk / 2) + 8 (kk % 2)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ts(tbase + COL_DQ, tbase + 128 * x + 32 * (kk / 2) + 8 * (kk % 2),
+                  sdesc_sw128(kt + kk * 2048, 8192, 1024), id_q, (k > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&k_empty[sk]);
+        return true;
+      };
+      for (int k = 0; k < U && ok; ++k) {
+        const int x = k & 1, sk = k % NK, sv = k % NV;
+        if (!mbar_wait(&k_full[sk], (k / NK) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        if (!mbar_wait(&v_full[sv], (k / NV) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        tc_fence_after();
+        // S and dP into buffer x; its previous contents (entry k - 2) were consumed
+        // by the dQ MMA issued earlier by this thread (in-order execution)
+        const uint32_t kt = smem_u32(sK + sk * L::T64), vt = smem_u32(sV + sv * L::T64);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32, offk = (kk / 4) * 8192 + (kk % 4) * 32;
-          umma_ss(tbase + COL_S, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kt + offk, 16, 1024), id_s,
+          umma_ss(tbase + 128 * x, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kt + offk, 16, 1024), id_s,
                   kk > 0 ? 1u : 0u);
-          umma_ss(tbase + COL_DP, sdesc_sw128(o0 + off, 16, 1024), sdesc_sw128(vt + offk, 16, 1024), id_s,
-                  kk > 0 ? 1u : 0u);
+          umma_ss(tbase + 128 * x + 64, sdesc_sw128(o0 + off, 16, 1024), sdesc_sw128(vt + offk, 16, 1024),
+                  id_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(sp_full);
-        umma_commit(v_empty);
-        if (!mbar_wait(ds_ready, k & 1, a.err, DEV_TIMEOUT_SYNC)) { ok = false; break; }
-        tc_fence_after();
-        // dQ += dS K: dS (bf16 pairs) from TMEM, K as the MN-major B operand
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          umma_ts(tbase + COL_DQ, tbase + COL_S + 8 * kk, sdesc_sw128(kt + kk * 2048, 8192, 1024), id_q,
-                  (k > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(k_empty);
+        umma_commit(&sp_full[x]);
+        umma_commit(&v_empty[sv]);
+        if (k >= 1 && !issue_dq(k - 1)) { ok = false; break; }
       }
+      if (ok && U >= 1) ok = issue_dq(U - 1);
       if (ok) umma_commit(dq_done);
     }
   } else {
-    // ---------------- one query row per thread
+    // ---------------- two threads per query row (warps w and w + 4 share TMEM
+    // lanes); each turns 32 of the 64 key columns into dS
     const int q4 = w & 3;
+    const int hs = (w - 2) >> 2;
     const int r = 32 * q4 + ln;
     const int half = r >> 6;
     const uint32_t bit = 1u << half;
@@ -277,43 +314,42 @@ __global__ void __launch_bounds__(192, 2)
     const float sl2 = a.scale_log2;
     bool ok = true;
     for (int k = 0; k < U; ++k) {
-      if (!__all_sync(0xffffffffu, mbar_wait(sp_full, k & 1, a.err, DEV_TIMEOUT_MMA))) {
+      const int x = k & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sp_full[x], (k >> 1) & 1, a.err, DEV_TIMEOUT_MMA))) {
         ok = false;
         break;
       }
       tc_fence_after();
       const bool crit = (uflag[k] & bit) != 0;
-      uint32_t pk[32];
+      const uint32_t ts = tl + 128 * x;
+      uint32_t pk[16];
       if (crit) {
-        uint32_t s0[32], s1[32], d0[32], d1[32];
-        tmem_ld32(tl + COL_S, s0);
-        tmem_ld32(tl + COL_S + 32, s1);
-        tmem_ld32(tl + COL_DP, d0);
-        tmem_ld32(tl + COL_DP + 32, d1);
+        uint32_t s0[32], d0[32];
+        tmem_ld32(ts + 32 * hs, s0);
+        tmem_ld32(ts + 64 + 32 * hs, d0);
         tmem_ld_wait();
-        const int nvalid = a.N - 64 * (int)uidx[k];
+        const int nvalid = a.N - 64 * (int)uidx[k] - 32 * hs;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          float ds[4];
+          float ds[2];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int col = (e < 2) ? 2 * c + e : 32 + 2 * c + (e - 2);
-            const float sv = __uint_as_float(e < 2 ? s0[2 * c + e] : s1[2 * c + e - 2]);
-            const float dv = __uint_as_float(e < 2 ? d0[2 * c + e] : d1[2 * c + e - 2]);
-            const float pr = col < nvalid ? ex2b(fmaf(sv, sl2, -lse2)) : 0.f;
-            ds[e] = pr * (cs * dv - Dr);
+          for (int e = 0; e < 2; ++e) {
+            const int col = 2 * c + e;
+            const float pr = col < nvalid ? ex2b(fmaf(__uint_as_float(s0[col]), sl2, -lse2)) : 0.f;
+            ds[e] = pr * (cs * __uint_as_float(d0[col]) - Dr);
           }
           pk[c] = pack_bf16x2(ds[0], ds[1]);
-          pk[16 + c] = pack_bf16x2(ds[2], ds[3]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = 0u;
+        for (int c = 0; c < 16; ++c) pk[c] = 0u;
       }
-      tmem_st32(tl + COL_S, pk);  // dS_k over the first 32 columns of S_k
+      // dS for this thread's 32 keys (16 bf16 pairs) over the start of its own S
+      // columns: the other thread of the row never reads them
+      tmem_st16(ts + 32 * hs, pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(ds_ready);
+      mbar_arrive(&ds_ready[x]);
     }
     if (ok && U >= 1) ok = __all_sync(0xffffffffu, mbar_wait(dq_done, 0, a.err, DEV_TIMEOUT_MMA));
     if (ok) {
@@ -321,7 +357,7 @@ __global__ void __launch_bounds__(192, 2)
       __nv_bfloat16* orow = a.out0 + (int64_t)b * a.s0[0] + (int64_t)h * a.s0[1] + (int64_t)n * a.s0[2];
       const float* lin = a.q_lin + ((int64_t)bh * a.N + n) * D;
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 32) {
+      for (int c0 = (D / 2) * hs; c0 < (D / 2) * (hs + 1); c0 += 32) {  // this thread's half of the row
         uint32_t v[32];
         if (U >= 1) {
           tmem_ld32(tl + COL_DQ + c0, v);
@@ -348,7 +384,7 @@ __global__ void __launch_bounds__(192, 2)
   __syncthreads();
   if (w == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, 256);
+    tmem_dealloc(tbase, 512);
   }
 }
 
@@ -381,7 +417,7 @@ struct DkvSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap mapK2, const __grid_constant__ CUtensorMap mapV2,
                     const __grid_constant__ CUtensorMap mapQ1, const __grid_constant__ CUtensorMap mapdO1,
                     BwdSparseArgs a) {
@@ -426,7 +462,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&q_full[x], 1);
       mbar_init(&q_empty[x], 1);
       mbar_init(&sp_full[x], 1);
-      mbar_init(&ds_ready[x], 128);
+      mbar_init(&ds_ready[x], 256);
     }
     mbar_init(kv_done, 1);
     fence_barrier_init();
@@ -512,11 +548,13 @@ __global__ void __launch_bounds__(192, 1)
         if (!mbar_wait(&ds_ready[x], (e >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
         tc_fence_after();
         const uint32_t qt = smem_u32(sQ + x * L::T64), ot = smem_u32(sdO + x * L::T64);
+        // query rows 16 kk .. 16 kk + 15: packed at columns 32 (kk / 2) + 8 (kk % 2)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          umma_ts(tbase + COL_DV, tbase + 128 * x + 8 * kk, sdesc_sw128(ot + kk * 2048, 8192, 1024), id_o,
+          const uint32_t ca = 32 * (kk / 2) + 8 * (kk % 2);
+          umma_ts(tbase + COL_DV, tbase + 128 * x + ca, sdesc_sw128(ot + kk * 2048, 8192, 1024), id_o,
                   (e > 0 || kk > 0) ? 1u : 0u);
-          umma_ts(tbase + COL_DK, tbase + 128 * x + 64 + 8 * kk, sdesc_sw128(qt + kk * 2048, 8192, 1024),
+          umma_ts(tbase + COL_DK, tbase + 128 * x + 64 + ca, sdesc_sw128(qt + kk * 2048, 8192, 1024),
                   id_o, (e > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&q_empty[x]);
@@ -545,8 +583,10 @@ __global__ void __launch_bounds__(192, 1)
       if (ok) umma_commit(kv_done);
     }
   } else {
-    // ---------------- one key row per thread
+    // ---------------- two threads per key row (warps w and w + 4 share TMEM
+    // lanes); each handles 32 of the 64 query columns
     const int q4 = w & 3;
+    const int hs = (w - 2) >> 2;
     const int t = 32 * q4 + ln;
     const int half = t >> 6;
     const uint32_t bit = 1u << half;
@@ -565,39 +605,35 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const bool crit = (uflag[e] & bit) != 0;
       const uint32_t ts = tl + 128 * x;
-      uint32_t pp[32], pd[32];
+      uint32_t pp[16], pd[16];
       if (crit) {
-        uint32_t s0[32], s1[32], d0[32], d1[32];
-        tmem_ld32(ts, s0);
-        tmem_ld32(ts + 32, s1);
-        tmem_ld32(ts + 64, d0);
-        tmem_ld32(ts + 96, d1);
+        uint32_t s0[32], d0[32];
+        tmem_ld32(ts + 32 * hs, s0);
+        tmem_ld32(ts + 64 + 32 * hs, d0);
         tmem_ld_wait();
-        const float2* ldv = sLD + x * 64;  // (lse log2 e, D) of the 64 query rows
+        const float2* ldv = sLD + x * 64 + 32 * hs;  // (lse log2 e, D) of this thread's 32 query rows
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          float pv[4], ds[4];
+          float pv[2], ds[2];
 #pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const int col = (e4 < 2) ? 2 * c + e4 : 32 + 2 * c + (e4 - 2);
-            const float sv = __uint_as_float(e4 < 2 ? s0[2 * c + e4] : s1[2 * c + e4 - 2]);
-            const float dv = __uint_as_float(e4 < 2 ? d0[2 * c + e4] : d1[2 * c + e4 - 2]);
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int col = 2 * c + e2;
             const float2 l2 = ldv[col];
-            const float pr = ex2b(fmaf(sv, sl2, -l2.x));
-            pv[e4] = pr;
-            ds[e4] = pr * (cs * dv - l2.y);
+            const float pr = ex2b(fmaf(__uint_as_float(s0[col]), sl2, -l2.x));
+            pv[e2] = pr;
+            ds[e2] = pr * (cs * __uint_as_float(d0[col]) - l2.y);
           }
           pp[c] = pack_bf16x2(pv[0], pv[1]);
-          pp[16 + c] = pack_bf16x2(pv[2], pv[3]);
           pd[c] = pack_bf16x2(ds[0], ds[1]);
-          pd[16 + c] = pack_bf16x2(ds[2], ds[3]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pp[c] = pd[c] = 0u;
+        for (int c = 0; c < 16; ++c) pp[c] = pd[c] = 0u;
       }
-      tmem_st32(ts, pp);       // P^T over S^T
-      tmem_st32(ts + 64, pd);  // dS^T over dP^T
+      // P^T and dS^T for this thread's 32 query rows over the start of its own
+      // S^T and dP^T columns (the other thread of the row never reads them)
+      tmem_st16(ts + 32 * hs, pp);
+      tmem_st16(ts + 64 + 32 * hs, pd);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&ds_ready[x]);
@@ -613,7 +649,7 @@ __global__ void __launch_bounds__(192, 1)
         __nv_bfloat16* orow = base + (int64_t)b * st[0] + (int64_t)h * st[1] + (int64_t)n * st[2];
         const uint32_t col = which == 0 ? COL_DK : COL_DV;
 #pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
+        for (int c0 = (D / 2) * hs; c0 < (D / 2) * (hs + 1); c0 += 32) {  // this thread's half
           uint32_t v[32];
           if (U >= 1) {
             tmem_ld32(tl + col + c0, v);
@@ -658,12 +694,12 @@ cudaError_t launch_bwd_dq(const CUtensorMap& mapQ, const CUtensorMap& mapdO, con
     const size_t smem = DqSmem<128>::bytes(a.Tkv);
     cudaError_t e = set_smem(bwd_dq_kernel<128>, smem);
     if (e != cudaSuccess) return e;
-    bwd_dq_kernel<128><<<grid, 192, smem, s>>>(mapQ, mapdO, mapK, mapV, a);
+    bwd_dq_kernel<128><<<grid, 320, smem, s>>>(mapQ, mapdO, mapK, mapV, a);
   } else {
     const size_t smem = DqSmem<64>::bytes(a.Tkv);
     cudaError_t e = set_smem(bwd_dq_kernel<64>, smem);
     if (e != cudaSuccess) return e;
-    bwd_dq_kernel<64><<<grid, 192, smem, s>>>(mapQ, mapdO, mapK, mapV, a);
+    bwd_dq_kernel<64><<<grid, 320, smem, s>>>(mapQ, mapdO, mapK, mapV, a);
   }
   return cudaGetLastError();
 }
@@ -676,12 +712,12 @@ cudaError_t launch_bwd_dkdv(const CUtensorMap& mapK2, const CUtensorMap& mapV2,
     const size_t smem = DkvSmem<128>::bytes(a.Tq);
     cudaError_t e = set_smem(bwd_dkdv_kernel<128>, smem);
     if (e != cudaSuccess) return e;
-    bwd_dkdv_kernel<128><<<grid, 192, smem, s>>>(mapK2, mapV2, mapQ1, mapdO1, a);
+    bwd_dkdv_kernel<128><<<grid, 320, smem, s>>>(mapK2, mapV2, mapQ1, mapdO1, a);
   } else {
     const size_t smem = DkvSmem<64>::bytes(a.Tq);
     cudaError_t e = set_smem(bwd_dkdv_kernel<64>, smem);
     if (e != cudaSuccess) return e;
-    bwd_dkdv_kernel<64><<<grid, 192, smem, s>>>(mapK2, mapV2, mapQ1, mapdO1, a);
+    bwd_dkdv_kernel<64><<<grid, 320, smem, s>>>(mapK2, mapV2, mapQ1, mapdO1, a);
   }
   return cudaGetLastError();
 }
