@@ -342,7 +342,7 @@ def run_e2e(ctx, steps):
             "api": "sla_attention_host (pinned host Q, K, V, O)"}
 
 
-def run_train(ctx, steps=10):
+def run_train(ctx, steps=10, warmup=3, dense=True):
     """Forward + backward of the same workload (the fine-tuning step): the four
     forward stages with the LSE output, then sla_backward with dO ~ N(0, 1) bf16.
     Also times dense attention's forward + backward (torch SDPA) on the same inputs."""
@@ -396,7 +396,7 @@ def run_train(ctx, steps=10):
         if ev is not None:
             ev[4].record()
 
-    for _ in range(3):
+    for _ in range(max(warmup, 1)):
         step()
     torch.cuda.synchronize()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps)]
@@ -412,6 +412,8 @@ def run_train(ctx, steps=10):
            "ms_per_step": round(sum(stage_ms), 4),
            "stage_ms": {n: round(x, 4) for n, x in zip(names, stage_ms)}}
     # dense attention forward + backward on the same inputs
+    if not dense:
+        return res
     try:
         from torch.nn.attention import SDPBackend, sdpa_kernel
         q, k_, v = (t.detach().clone().requires_grad_(True) for t in (Q, K, V))
@@ -430,6 +432,27 @@ def run_train(ctx, steps=10):
     except Exception as e:  # backend not available for this shape
         res["dense_fwd_bwd_ms"] = f"unavailable: {type(e).__name__}"
     return res
+
+
+def run_train_main(args):
+    """`--train`: the forward + backward step of the workload as its own JSON line."""
+    dev = 0
+    torch.cuda.set_device(dev)
+    over = {} if args.heads is None else {"H": args.heads}
+    data, w = I.make_workload(args.workload, device=f"cuda:{dev}", **over)
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"])
+    Q, K, V = (data[k].to(dev) for k in ("Q", "K", "V"))
+    f32 = lambda t: None if t is None else t.to(dev).float().contiguous()  # noqa: E731
+    params = tuple(f32(data.get(k)) for k in ("proj_w", "proj_b", "alpha", "Wq", "Wk"))
+    ctx = dict(Q=Q, K=K, V=V, cfg=cfg, dev=dev, params=params)
+    r = run_train(ctx, steps=args.steps, warmup=args.warmup, dense=not args.no_extras)
+    B, H, N, d = Q.shape
+    return {"metric": "SLA forward + backward step ms", "value": r["ms_per_step"], "unit": "ms",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": False,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{args.workload} (B={B}, H={H}, N={N}, d={d}) forward + backward, "
+                                   "dO ~ N(0, 1) bf16"},
+            **{k: v for k, v in r.items() if k not in ("workload", "ms_per_step")}}
 
 
 def run_dense(ctx, iters=10):
@@ -544,6 +567,9 @@ def main():
                     help="precision of Q K^T on critical blocks (fp8_e4m3: d = 128 only)")
     ap.add_argument("--heads", type=int, default=None, help="override the workload's head count "
                     "(profiling runs only; the bench line uses the workload as named)")
+    ap.add_argument("--train", action="store_true",
+                    help="time the training step (forward with the backward's residuals + sla_backward) "
+                         "instead of the forward; one GPU")
     ap.add_argument("--burn", type=float, default=0.5,
                     help="seconds of untimed steps before the timed region (clock sampling)")
     args = ap.parse_args()
@@ -559,6 +585,10 @@ def main():
         return
 
     bnd.lib()
+    if args.train:
+        if rank == 0:
+            print(json.dumps(run_train_main(args)), flush=True)
+        return
     if world > 1:
         import datetime
         torch.cuda.set_device(local)
