@@ -20,6 +20,8 @@ from .sla import (  # noqa: F401
     feature_map,
     linear_block_stats,
     quantize_e4m3,
+    pv_fp8_scales,
+    sparse_branch_fp8_pv,
     forward_given_mask,
     forward,
     mask_grading,

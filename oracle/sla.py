@@ -36,8 +36,8 @@ Readings taken where the pages are silent:
   * the backward treats M_c as a constant (hard Top-k has no gradient) and
     returns gradients for Q, K, V and the combine's parameters only.
 
-Parity unpinned: the FP8 path's exact values (only the tolerance bound is
-checked against this oracle's unquantised result).
+Parity unpinned: the FP8 paths' exact values at full size (the quantiser is
+pinned; the emulations are pinned only on cases where they must be exact).
 """
 from __future__ import annotations
 
@@ -259,9 +259,41 @@ def _fp8_dequant_tile(X: np.ndarray) -> np.ndarray:
     return quantize_e4m3(X / s) * s
 
 
+def pv_fp8_scales(Vh: np.ndarray) -> np.ndarray:
+    """Per-channel scale of one head's V for the FP8 P V product: max_t |V[t, c]| / 448
+    (1 where a channel is all zero).  [SLA2] §5 quantises P and V with scales and
+    dequantises their product; with one scale per channel and P on the fixed scale
+    448 (P <= 1), both scales factor out of the sum over keys."""
+    amax = np.abs(Vh).max(axis=0)
+    return np.where(amax > 0, amax / 448.0, 1.0)
+
+
+def sparse_branch_fp8_pv(q, keys_blocks, vhat_blocks, scale):
+    """o^s of one query block with the FP8 P V product ([SLA2] §5), step by step:
+    critical blocks in ascending order with an online row maximum m (P = exp(s - m)
+    <= 1); on every increase of m the accumulator and the row sum are rescaled;
+    P is quantised as E4M3(448 P); the row sum l uses the unquantised P.
+    Returns (acc, l): o^s = acc * s_V / 448 / l."""
+    rows = q.shape[0]
+    m = np.full(rows, -np.inf)
+    l = np.zeros(rows)
+    acc = np.zeros((rows, vhat_blocks[0].shape[1]))
+    for kj, vj in zip(keys_blocks, vhat_blocks):
+        s = (q @ kj.T) * scale
+        mj = np.maximum(m, s.max(axis=1))
+        f = np.where(np.isfinite(m), np.exp(m - mj), 0.0)
+        acc *= f[:, None]
+        l *= f
+        P = np.exp(s - mj[:, None])
+        l += P.sum(axis=1)
+        acc += quantize_e4m3(448.0 * P) @ vj
+        m = mj
+    return acc, l
+
+
 def forward_given_mask(Q, K, V, Mc, p: OracleParams, proj_w=None, proj_b=None, alpha=None,
                        qblocks: Optional[Sequence[int]] = None, heads: Optional[Sequence] = None,
-                       qk_fp8: bool = False, return_branches: bool = False):
+                       qk_fp8: bool = False, return_branches: bool = False, pv_fp8: bool = False):
     """SLA / SLA2 output for a given compressed mask M_c.
 
     Q, K, V: [B, H, N, d] (any float dtype; upcast to float64).
@@ -277,7 +309,8 @@ def forward_given_mask(Q, K, V, Mc, p: OracleParams, proj_w=None, proj_b=None, a
       "alpha": O = alpha_h O^s + (1 - alpha_h) O^l
     `qblocks` / `heads` restrict the work to a sample (rows of other blocks are
     left as NaN).  `qk_fp8` quantises Q and K per 64-row tile to E4M3 before
-    Q K^T ([SLA2] §5); diagnosis only.
+    Q K^T ([SLA2] §5); `pv_fp8` computes the sparse branch's P V with E4M3 P and V
+    (``sparse_branch_fp8_pv``); both are emulations of the low-bit path.
     """
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -300,6 +333,9 @@ def forward_given_mask(Q, K, V, Mc, p: OracleParams, proj_w=None, proj_b=None, a
     for (bb, hh) in heads:
         h_stats, z_stats = linear_block_stats(K[bb, hh], V[bb, hh], p.b_kv, p.phi)
         fQ = feature_map(Q[bb, hh], p.phi)
+        if pv_fp8:
+            sV = pv_fp8_scales(V[bb, hh])
+            Vhat = quantize_e4m3(V[bb, hh] / sV[None, :])
         for i in qsel:
             qs, qe = block_range(i, p.b_q, N)
             q = Q[bb, hh, qs:qe]
@@ -316,7 +352,11 @@ def forward_given_mask(Q, K, V, Mc, p: OracleParams, proj_w=None, proj_b=None, a
                     kj = _fp8_dequant_tile(kj)
                 keys.append(kj)
                 vals.append(V[bb, hh, ks:ke])
-            if keys:
+            if keys and pv_fp8:
+                vhat = [Vhat[slice(*block_range(int(j), p.b_kv, N))] for j in crit]
+                acc, lsum = sparse_branch_fp8_pv(q, keys, vhat, scale)
+                o_s = acc * sV[None, :] / 448.0 / lsum[:, None]
+            elif keys:
                 kk = np.concatenate(keys, axis=0)
                 vv = np.concatenate(vals, axis=0)
                 s = (q @ kk.T) * scale

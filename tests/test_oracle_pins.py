@@ -288,3 +288,56 @@ def test_mask_grading_excludes_near_ties():
     g = O.mask_grading(L, 2, 1)
     # thresholds: top-2 -> midpoint(1.00005, 1.0); bottom-1 -> midpoint(-3, 0)
     np.testing.assert_array_equal(g[0], [True, False, False, True, True])
+
+
+# ---------------------------------------------------------------- FP8 P V emulation
+def test_fp8_pv_is_exact_when_p_and_v_are_on_the_grid():
+    # Q = 0: every score is 0, so P = 1 (E4M3(448) is exact); V in {0, +-1, 2, 4, 8} has
+    # per-channel amax 8 and V / s_V in {0, +-56, 112, 224, 448}, all E4M3 values.
+    rng = np.random.default_rng(11)
+    B, H, N, d = 1, 1, 192, 8
+    Q = np.zeros((B, H, N, d))
+    K = rng.standard_normal((B, H, N, d))
+    V = rng.choice([-8.0, -4.0, -2.0, -1.0, 0.0, 1.0, 2.0, 4.0, 8.0], size=(B, H, N, d))
+    V[..., 0, :] = 8.0  # every channel reaches 8
+    T = O.num_blocks(N, 64)
+    Mc = np.full((B, H, T, T), -1, dtype=np.int8)
+    Mc[..., 0] = 1
+    Mc[..., 1] = 1
+    p = O.OracleParams(combine="alpha")
+    a = np.ones((B, H))
+    exact = O.forward_given_mask(Q, K, V, Mc, p, alpha=a)
+    fp8 = O.forward_given_mask(Q, K, V, Mc, p, alpha=a, pv_fp8=True)
+    np.testing.assert_allclose(fp8, exact, rtol=0, atol=1e-12)
+
+
+def test_fp8_pv_online_form_equals_softmax_without_rounding(monkeypatch):
+    # with the quantiser replaced by the identity, the online step-by-step form is
+    # plain softmax attention over the critical tokens
+    rng = np.random.default_rng(12)
+    B, H, N, d = 1, 2, 200, 16
+    Q, K, V = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    T = O.num_blocks(N, 64)
+    Mc = np.zeros((B, H, T, T), dtype=np.int8)
+    Mc[..., ::2] = 1
+    p = O.OracleParams(combine="alpha")
+    a = np.ones((B, H))
+    exact = O.forward_given_mask(Q, K, V, Mc, p, alpha=a)
+    import oracle.sla as S
+    monkeypatch.setattr(S, "quantize_e4m3", lambda x: np.asarray(x, dtype=np.float64))
+    online = S.forward_given_mask(Q, K, V, Mc, p, alpha=a, pv_fp8=True)
+    np.testing.assert_allclose(online, exact, rtol=1e-10, atol=1e-12)
+
+
+def test_fp8_pv_rounds_something_on_generic_inputs():
+    rng = np.random.default_rng(13)
+    B, H, N, d = 1, 1, 128, 16
+    Q, K, V = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    T = O.num_blocks(N, 64)
+    Mc = np.ones((B, H, T, T), dtype=np.int8)
+    p = O.OracleParams(k_h=1.0, k_l=0.0, combine="alpha")
+    a = np.ones((B, H))
+    exact = O.forward_given_mask(Q, K, V, Mc, p, alpha=a)
+    fp8 = O.forward_given_mask(Q, K, V, Mc, p, alpha=a, pv_fp8=True)
+    err = np.abs(fp8 - exact).max() / np.abs(exact).max()
+    assert 1e-4 < err < 0.1
