@@ -53,7 +53,7 @@ class sla_params_t(ctypes.Structure):
         ("eps", ctypes.c_float),
         ("stride_q", ctypes.c_int64 * 3), ("stride_k", ctypes.c_int64 * 3),
         ("stride_v", ctypes.c_int64 * 3), ("stride_o", ctypes.c_int64 * 3),
-        ("phi", ctypes.c_int), ("linear_over_all", ctypes.c_int),
+        ("phi", ctypes.c_int), ("linear_over_all", ctypes.c_int), ("pv_prec", ctypes.c_int),
     ]
 
 
@@ -128,6 +128,7 @@ class SlaConfig:
     eps: float = 1e-5
     phi: str = "softmax"      # "softmax" ([SLA] Fig. 4) or "elu1" ([SLA] Table 2 ablation)
     linear_over_all: bool = False  # linear branch over every key block ([SLA] §7 item 2)
+    pv: str = "bf16"          # "bf16" or "fp8_e4m3" (P V of critical blocks, [SLA2] §5)
 
 
 def make_params(Q: torch.Tensor, cfg: SlaConfig, K=None, V=None, O=None) -> sla_params_t:
@@ -142,6 +143,9 @@ def make_params(Q: torch.Tensor, cfg: SlaConfig, K=None, V=None, O=None) -> sla_
         raise ValueError(f"phi must be 'softmax' or 'elu1', not {cfg.phi!r}")
     p.phi = SLA_PHI_SOFTMAX if cfg.phi == "softmax" else SLA_PHI_ELU1
     p.linear_over_all = int(cfg.linear_over_all)
+    if cfg.pv not in ("bf16", "fp8_e4m3"):
+        raise ValueError(f"pv must be 'bf16' or 'fp8_e4m3', not {cfg.pv!r}")
+    p.pv_prec = 0 if cfg.pv == "bf16" else 1
     p.stride_q = _strides(Q)
     p.stride_k = _strides(K if K is not None else Q)
     p.stride_v = _strides(V if V is not None else Q)

@@ -21,6 +21,7 @@ constexpr size_t kAlign = 256;
 struct Plan {
   int B, H, N, d, BH, Tq, Tkv, nh, nl, NN, Tkvp;
   bool fp8;  // Q K^T on E4M3 with per-block scales
+  bool pv8;  // P V on E4M3 (P on the fixed scale 448, V per (head, channel))
   int phi;   // sla_phi_t
   bool all;  // linear branch over every key block
 };
@@ -29,7 +30,7 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t err, qc, kc, qr, kr, kmean, keys, mm, hagg;      // sla_workspace_size ...
-  size_t q8, k8, scq, sck, end;                           // ... (+ FP8 operands)
+  size_t q8, k8, scq, sck, v8t, vmax, end;                // ... (+ FP8 operands)
   size_t mc, lut, hz, end_attn;                           // + sla_attention extras
   size_t hq, hk, hv, ho, end_host;                        // + sla_attention_host staging
 };
@@ -52,6 +53,8 @@ Layout layout_of(const Plan& p) {
   L.k8 = o;    o = align_up(o + k8);
   L.scq = o;   o = align_up(o + (p.fp8 ? (size_t)p.BH * p.Tq * 4 : 0));
   L.sck = o;   o = align_up(o + (p.fp8 ? (size_t)p.BH * p.Tkv * 4 : 0));
+  L.v8t = o;   o = align_up(o + (p.pv8 ? (size_t)p.BH * p.Tkv * p.d * 128 : 0));
+  L.vmax = o;  o = align_up(o + (p.pv8 ? (size_t)p.BH * p.d * 4 : 0));
   L.end = o;
   L.mc = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkv);
   L.lut = o;   o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
@@ -94,6 +97,8 @@ sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
   if (p->linear_over_all != 0 && p->linear_over_all != 1) return SLA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if (p->qk_prec == SLA_QK_FP8_E4M3 && p->d != 128) return SLA_ERR_UNSUPPORTED;
+  if (p->pv_prec != SLA_PV_BF16 && p->pv_prec != SLA_PV_FP8_E4M3) return SLA_ERR_INVALID_ARG;
+  if (p->pv_prec == SLA_PV_FP8_E4M3 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if (p->b_q != 64 || p->b_kv != 64) return SLA_ERR_UNSUPPORTED;
   if (p->N > kMaxN || (int64_t)p->B * p->H > 65535) return SLA_ERR_UNSUPPORTED;
   if (!stride_ok(p->stride_q, p->d) || !stride_ok(p->stride_k, p->d) ||
@@ -110,6 +115,7 @@ sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
   pl->NN = p->d * p->d + p->d;
   pl->Tkvp = (pl->Tkv + 7) & ~7;
   pl->fp8 = p->qk_prec == SLA_QK_FP8_E4M3;
+  pl->pv8 = p->pv_prec == SLA_PV_FP8_E4M3;
   pl->phi = p->phi;
   pl->all = p->linear_over_all != 0;
   return SLA_OK;
@@ -348,6 +354,19 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
     scq = qa.scale_q;
     sck = qa.scale_k;
   }
+  const unsigned int* vmax = nullptr;
+  if (pl.pv8) {
+    // V^ [BH][T_kv][d rows][128 B] and the per-(head, channel) maxima
+    uint8_t* v8t = at<uint8_t>(ws, L.v8t);
+    unsigned int* vm = at<unsigned int>(ws, L.vmax);
+    SLA_TRY(cuda_status(launch_vquant_fp8(static_cast<const __nv_bfloat16*>(V), p->stride_v, pl.H, pl.N,
+                                          pl.Tkv, pl.BH, pl.d, vm, v8t, s)));
+    const uint64_t dv[3] = {128, (uint64_t)pl.Tkv * pl.d, (uint64_t)pl.BH};
+    const uint64_t sv[2] = {128, (uint64_t)pl.Tkv * pl.d * 128};
+    const uint32_t bv[3] = {128, (uint32_t)pl.d, 1};
+    if (!encode(&mv, v8t, 3, dv, sv, bv, true, CU_TENSOR_MAP_DATA_TYPE_UINT8)) return SLA_ERR_CUDA;
+    vmax = vm;
+  }
   FusedArgs a;
   a.lut = lut;
   a.Hz = hagg;
@@ -372,7 +391,8 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.phi = pl.phi;
   a.lse = lse;
   a.os = o_sparse;
-  return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, pl.fp8, pl.BH, s));
+  a.vmax = vmax;
+  return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, pl.fp8, pl.pv8, pl.BH, s));
 }
 
 sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
@@ -625,6 +645,7 @@ void sla_params_default(sla_params_t* p, int B, int H, int N, int d, float k_h, 
   p->eps = 1e-5f;
   p->phi = SLA_PHI_SOFTMAX;
   p->linear_over_all = 0;
+  p->pv_prec = SLA_PV_BF16;
   const int64_t s[3] = {(int64_t)H * N * d, (int64_t)N * d, (int64_t)d};
   for (int i = 0; i < 3; ++i) {
     p->stride_q[i] = s[i];
@@ -853,6 +874,6 @@ const char* sla_status_string(sla_status_t s) {
   return "SLA_ERR_UNKNOWN";
 }
 
-int sla_abi_version(void) { return 101; }
+int sla_abi_version(void) { return 102; }
 
 }  // extern "C"

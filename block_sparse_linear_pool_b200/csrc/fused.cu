@@ -32,7 +32,7 @@
 //
 // Low-bit variant ([SLA2] §5): Q and K arrive as E4M3 with one scale per
 // (head, 64-row block) and S = Q^ K^^T runs as tcgen05.mma kind::f8f6f4; the
-// softmax multiplies the scores by s_Q s_K.  P V stays in bf16.  The FP8 Q tile
+// softmax multiplies the scores by s_Q s_K.  The FP8 Q tile
 // and K ring are half the size, so the bf16 Q tile (needed for phi(Q)) fits
 // beside them and H_a loads over the FP8 Q tile and K ring.
 //
@@ -40,6 +40,16 @@
 // and s = sum_a e_a, phi(q) = e / s, so
 //     phi(q) H / (phi(q) Z + eps) = (e H) / (e Z + s eps)      exactly.
 // With the elu + 1 feature map ([SLA] Table 2 ablation) e = phi(q) and s = 1.
+//
+// FP8 P V (PV8, [SLA2] §5: P and V quantised, their product dequantised): V
+// arrives as E4M3 with one scale per (head, channel), transposed per key block
+// ([d rows][64 tokens, padded to 128 B]: the K-major B operand); the running
+// maximum is updated on every increase (no lazy rescale), so P <= 1 and
+// P^ = E4M3(448 P) is written over S (four values per TMEM column); O += P^ V^
+// runs as kind::f8f6f4 with P^ read from TMEM, and the epilogue applies
+// s_V[c] / 448.  The row sum l uses the unquantised P.
+#include <cuda_fp8.h>
+
 #include "kernels.cuh"
 
 namespace sla {
@@ -81,13 +91,14 @@ __device__ __forceinline__ float ex2(float x) {
 }
 }  // namespace
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool PV8>
 __global__ void __launch_bounds__(192, 2)
     sla_fused_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                      const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH,
                      const __grid_constant__ CUtensorMap mapZ, const __grid_constant__ CUtensorMap mapQ8,
                      const __grid_constant__ CUtensorMap mapK8, FusedArgs a) {
   static_assert(!FP8 || D == 128, "the FP8 path is built for d = 128");
+  static_assert(!PV8 || D == 128, "the FP8 P V path is built for d = 128");
   using L = FusedSmem<D, FP8>;
   constexpr int NR = L::NR;
   extern __shared__ uint8_t smem_raw[];
@@ -235,9 +246,13 @@ __global__ void __launch_bounds__(192, 2)
           }
           const int j = uidx[kv];
           mbar_arrive_expect_tx(&v_full[s], L::KT_BYTES);
+          if (PV8) {  // V^ of block j: [d rows][128 B], the same 16 KB as a bf16 V tile
+            tma_load_3d(sV + s * L::KT_BYTES, &mapV, &v_full[s], 0, D * j, bh);
+          } else {
 #pragma unroll
-          for (int c = 0; c < L::CH; ++c)
-            tma_load_4d(sV + s * L::KT_BYTES + c * 8192, &mapV, &v_full[s], c * 64, 64 * j, h, b);
+            for (int c = 0; c < L::CH; ++c)
+              tma_load_4d(sV + s * L::KT_BYTES + c * 8192, &mapV, &v_full[s], c * 64, 64 * j, h, b);
+          }
         }
       }
       // H_a (+ Z_a) into the K ring once its last S MMAs completed, H_b (+ Z_b)
@@ -268,6 +283,7 @@ __global__ void __launch_bounds__(192, 2)
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
       const uint32_t id_s8 = idesc_e4m3(128, 64);
       const uint32_t id_pv = idesc_bf16(128, D, false, true);
+      const uint32_t id_pv8 = idesc_e4m3(128, D);
       const uint32_t id_l = idesc_bf16(128, D, false, false);
       const uint32_t q0 = smem_u32(sQ);
       bool ok = mbar_wait(q_full, 0, a.err, DEV_TIMEOUT_TMA);
@@ -277,11 +293,19 @@ __global__ void __launch_bounds__(192, 2)
         if (!mbar_wait(&v_full[sv], (kp / NR) & 1, a.err, DEV_TIMEOUT_TMA)) return false;
         tc_fence_after();
         const uint32_t vt = smem_u32(sV + sv * L::KT_BYTES);
+        if (PV8) {
+          // P^ (E4M3, 4 per column) from TMEM, V^ K-major: 32 tokens per instruction
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = sdesc_sw128(vt + kk * 2048, 8192, 1024);
-          umma_ts(tbase + COL_O, tbase + COL_S + 64 * (kp & 1) + 8 * kk, bd, id_pv,
-                  (kp > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 2; ++kk)
+            umma_ts_f8(tbase + COL_O, tbase + COL_S + 64 * (kp & 1) + 8 * kk, sdesc_sw128(vt + kk * 32, 16, 1024),
+                       id_pv8, (kp > 0 || kk > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sdesc_sw128(vt + kk * 2048, 8192, 1024);
+            umma_ts(tbase + COL_O, tbase + COL_S + 64 * (kp & 1) + 8 * kk, bd, id_pv,
+                    (kp > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&pv_done[kp & 1]);
         umma_commit(&v_empty[sv]);
@@ -382,7 +406,7 @@ __global__ void __launch_bounds__(192, 2)
         const float mx = t[0] * sc;
         // lazy rescale: keep the running max unless it grows by more than 2^8
         const bool first = (m == -INFINITY);
-        const bool grow = !first && (mx - m > RESCALE_THRESHOLD);
+        const bool grow = !first && (mx - m > (PV8 ? 0.f : RESCALE_THRESHOLD));
         if (first) m = mx;  // O and l of this row are still exactly 0
         if (__any_sync(0xffffffffu, grow)) {
           // O must hold P_{k-1} V_{k-1} before it is rescaled
@@ -418,9 +442,19 @@ __global__ void __launch_bounds__(192, 2)
           const float p3 = ex2(fmaf(__uint_as_float(s1[2 * c + 1]), sc, nm));
           u[c] = p0 + p1;
           u[16 + c] = p2 + p3;
-          pk[c] = pack_bf16x2(p0, p1);
-          pk[16 + c] = pack_bf16x2(p2, p3);
+          if (PV8) {  // E4M3(448 p), four tokens per 32-bit column
+            const __nv_fp8x2_storage_t a01 =
+                __nv_cvt_float2_to_fp8x2(make_float2(448.f * p0, 448.f * p1), __NV_SATFINITE, __NV_E4M3);
+            const __nv_fp8x2_storage_t a23 =
+                __nv_cvt_float2_to_fp8x2(make_float2(448.f * p2, 448.f * p3), __NV_SATFINITE, __NV_E4M3);
+            pk[c] = (uint32_t)a01;        // tokens 2c, 2c+1
+            pk[16 + c] = (uint32_t)a23;   // tokens 32+2c, 33+2c
+          } else {
+            pk[c] = pack_bf16x2(p0, p1);
+            pk[16 + c] = pack_bf16x2(p2, p3);
+          }
         }
+
 #pragma unroll
         for (int st = 16; st >= 1; st >>= 1)
 #pragma unroll
@@ -430,7 +464,16 @@ __global__ void __launch_bounds__(192, 2)
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
       }
-      tmem_st32(ts, pk);  // P_k over the first 32 columns of S_k
+      if (PV8) {
+        // pk[c] holds tokens 2c, 2c+1 in its low 16 bits (c < 32, token order);
+        // TMEM column q takes tokens 4q .. 4q+3, lowest token in the lowest byte
+        uint32_t p16[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) p16[q] = (pk[2 * q] & 0xffffu) | (pk[2 * q + 1] << 16);
+        tmem_st16(ts, p16);  // P^_k over the first 16 columns of S_k
+      } else {
+        tmem_st32(ts, pk);  // P_k over the first 32 columns of S_k
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&p_ready[sb]);
@@ -521,6 +564,12 @@ __global__ void __launch_bounds__(192, 2)
         tmem_ld32(tl + COL_O + c0, ov);
         tmem_ld32(tl + COL_L + c0, lv);
         tmem_ld_wait();
+        if (PV8) {  // dequantise P^ V^: s_V[c] / 448 with s_V = max|V[:, c]| / 448
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            ov[c] = __float_as_uint(__uint_as_float(ov[c]) *
+                                    (__uint_as_float(a.vmax[(int64_t)bh * D + c0 + c]) * (1.f / 200704.f)));
+        }
         if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
@@ -558,28 +607,31 @@ __global__ void __launch_bounds__(192, 2)
   }
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool PV8>
 static cudaError_t launch_fused_t(const CUtensorMap& mapQ, const CUtensorMap& mapK,
                                   const CUtensorMap& mapV, const CUtensorMap& mapH,
                                   const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
                                   const CUtensorMap& mapK8, const FusedArgs& a, int BH,
                                   cudaStream_t s) {
   const size_t smem = FusedSmem<D, FP8>::bytes(a.Tkv);
-  cudaError_t e = cudaFuncSetAttribute(sla_fused_kernel<D, FP8>,
+  cudaError_t e = cudaFuncSetAttribute(sla_fused_kernel<D, FP8, PV8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.Tq + 1) / 2, BH);
-  sla_fused_kernel<D, FP8><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a);
+  sla_fused_kernel<D, FP8, PV8><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                          const CUtensorMap& mapH, const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
-                         const CUtensorMap& mapK8, const FusedArgs& a, int D, bool fp8, int BH,
+                         const CUtensorMap& mapK8, const FusedArgs& a, int D, bool fp8, bool pv8, int BH,
                          cudaStream_t s) {
-  if (fp8) return launch_fused_t<128, true>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
-  return D == 128 ? launch_fused_t<128, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s)
-                  : launch_fused_t<64, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
+  if (pv8)
+    return fp8 ? launch_fused_t<128, true, true>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s)
+               : launch_fused_t<128, false, true>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
+  if (fp8) return launch_fused_t<128, true, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
+  return D == 128 ? launch_fused_t<128, false, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s)
+                  : launch_fused_t<64, false, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
 }
 
 }  // namespace sla

@@ -73,6 +73,7 @@ struct FusedArgs {
   int phi;                // 0 softmax over d, 1 elu + 1
   float* lse;             // [BH][N] natural-log sum of exp of the scaled critical scores, or nullptr
   float* os;              // [BH][N][d] the sparse branch's output o^s (fp32), or nullptr
+  const unsigned int* vmax;  // FP8 P V: per (head, channel) max |V| (float bits), else nullptr
 };
 
 // ---- backward
@@ -162,11 +163,13 @@ cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, c
                              int BH, cudaStream_t s);
 
 cudaError_t launch_quant_fp8(const QuantArgs& a, int BH, cudaStream_t s);
+cudaError_t launch_vquant_fp8(const __nv_bfloat16* V, const int64_t* sv, int H, int N, int T, int BH, int D,
+                              unsigned int* vmax, uint8_t* V8T, cudaStream_t s);
 
 // mapQ8 / mapK8 are used only when fp8 is set (d = 128 only).
 cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                          const CUtensorMap& mapH, const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
-                         const CUtensorMap& mapK8, const FusedArgs& a, int D, bool fp8, int BH,
+                         const CUtensorMap& mapK8, const FusedArgs& a, int D, bool fp8, bool pv8, int BH,
                          cudaStream_t s);
 
 }  // namespace sla

@@ -61,6 +61,14 @@ typedef enum {
 } sla_qk_prec_t;
 
 typedef enum {
+  SLA_PV_BF16 = 0,      /* P V of critical blocks in bf16, fp32 accumulate */
+  SLA_PV_FP8_E4M3 = 1   /* [SLA2] §5: P and V quantised to E4M3, product dequantised:
+                           P on the fixed scale 448 (P <= 1: the running maximum is
+                           updated on every increase), V with one scale per
+                           (head, channel) max|V[:, c]| / 448 */
+} sla_pv_prec_t;
+
+typedef enum {
   SLA_PHI_SOFTMAX = 0,  /* phi(x) = softmax of x over the head dimension ([SLA] Fig. 4) */
   SLA_PHI_ELU1 = 1      /* phi(x) = elu(x) + 1, the ablation of [SLA] Table 2 */
 } sla_phi_t;
@@ -82,10 +90,11 @@ typedef struct {
   int phi;             /* sla_phi_t: the linear branch's feature map, for K and Q */
   int linear_over_all; /* 1: H_i, Z_i sum h_j, z_j over every key block instead of the
                           marginal ones (the released code's variant, [SLA] §7 item 2) */
+  int pv_prec;         /* sla_pv_prec_t (FP8: d = 128 only) */
 } sla_params_t;
 
 /* Fills a params struct for contiguous [B,H,N,d] tensors, b = 64, eps = 1e-5,
- * bf16 Q K^T, softmax feature map, linear branch over the marginal blocks. */
+ * bf16 Q K^T and P V, softmax feature map, linear branch over the marginal blocks. */
 void sla_params_default(sla_params_t* p, int B, int H, int N, int d, float k_h, float k_l,
                         int combine);
 

@@ -71,6 +71,12 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
     p.linear_over_all = 7
     assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == 1
     p = _params()
+    p.pv_prec = 3
+    assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == 1
+    p = _params(d=64)
+    p.pv_prec = 1  # FP8 P V is built for d = 128
+    assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == 2
+    p = _params()
     ws = (ctypes.c_uint8 * 1024)()
     # NULL tensors
     assert L.sla_predict_mask(ctypes.byref(p), None, None, None, None, None, None, ws, 1024, None) == 1
@@ -95,7 +101,7 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
 
 def test_defaults_are_the_pages_main_method(L):
     p = _params()
-    assert (p.phi, p.linear_over_all, p.qk_prec, p.smooth_k) == (0, 0, 0, 0)
+    assert (p.phi, p.linear_over_all, p.qk_prec, p.smooth_k, p.pv_prec) == (0, 0, 0, 0, 0)
     assert abs(p.eps - 1e-5) < 1e-12
 
 
@@ -110,4 +116,4 @@ def test_workspace_sizes_grow_with_the_problem(L):
 def test_status_strings(L):
     for code, name in bnd.STATUS.items():
         assert L.sla_status_string(code).decode() == name
-    assert L.sla_abi_version() == 101
+    assert L.sla_abi_version() == 102

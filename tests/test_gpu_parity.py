@@ -84,14 +84,15 @@ def _run(data, cfg, qblocks=None, heads=None):
     Mc = mc.cpu().numpy().reshape(B, H, T, T)
     ref = O.forward_given_mask(_np(Q), _np(K), _np(V), Mc, _oparams(cfg), proj_w=_np(proj_w),
                                proj_b=_np(proj_b), alpha=_np(alpha), qblocks=qblocks, heads=heads)
-    if cfg.qk == "bf16":
+    if cfg.qk == "bf16" and cfg.pv == "bf16":
         rel = _check_out(out, ref, "forward")
     else:
-        # The bf16 bounds against the oracle's own E4M3 rounding of Q and K (the
-        # CUDA path computes what the method computes) ...
+        # The bf16 bounds against the oracle's own E4M3 rounding (Q, K per 64-row
+        # block; P and V for the FP8 P V product): the CUDA path computes what the
+        # method computes ...
         ref8 = O.forward_given_mask(_np(Q), _np(K), _np(V), Mc, _oparams(cfg), proj_w=_np(proj_w),
                                     proj_b=_np(proj_b), alpha=_np(alpha), qblocks=qblocks,
-                                    heads=heads, qk_fp8=True)
+                                    heads=heads, qk_fp8=cfg.qk != "bf16", pv_fp8=cfg.pv != "bf16")
         _check_out(out, ref8, "fp8 forward vs emulated fp8")
         # ... and against the unquantised oracle: the stated max-abs bound, or the
         # method's own quantisation error where that is larger (per-64-row-block
@@ -167,6 +168,19 @@ def test_small_shapes(B, H, N, d, kh, kl, combine):
 def test_code_variants(B, H, N, d, kh, kl, combine, phi, over_all):
     data = _small(B, H, N, d, seed=N + d + 7)
     cfg = bnd.SlaConfig(k_h=kh, k_l=kl, combine=combine, phi=phi, linear_over_all=over_all)
+    if combine == "proj":
+        data["Wq"] = data["Wk"] = None
+    _run(data, cfg)
+
+
+@pytest.mark.parametrize("B,H,N,d,kh,kl,combine,qk", [
+    (1, 2, 1000, 128, 0.10, 0.50, "alpha", "bf16"),      # FP8 P V, ragged tail
+    (1, 1, 3000, 128, 0.10, 0.40, "proj", "bf16"),
+    (2, 1, 2049, 128, 0.05, 0.70, "alpha", "fp8_e4m3"),  # FP8 Q K^T and P V, tail of 1 token
+])
+def test_fp8_pv(B, H, N, d, kh, kl, combine, qk):
+    data = _small(B, H, N, d, seed=N + 5)
+    cfg = bnd.SlaConfig(k_h=kh, k_l=kl, combine=combine, qk=qk, pv="fp8_e4m3")
     if combine == "proj":
         data["Wq"] = data["Wk"] = None
     _run(data, cfg)
@@ -264,9 +278,18 @@ def test_fp8_qk_wan14b_720p_sla2_full_size_sampled():
     _run(data, cfg, qblocks=[0, 590, 1181], heads=[(0, 0), (0, 39)])
 
 
+def test_fp8_qk_and_pv_wan14b_720p_sla2_full_size_sampled():
+    data, w = I.make_workload("wan14b_720p_sla2")
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine="alpha", qk="fp8_e4m3", pv="fp8_e4m3")
+    _run(data, cfg, qblocks=[0, 590, 1181], heads=[(0, 0), (0, 39)])
+
+
 def test_fp8_requires_d128():
     Q = torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16, device="cuda")
     cfg = bnd.SlaConfig(k_h=0.5, k_l=0.0, qk="fp8_e4m3")
     with pytest.raises(bnd.SlaError) as e:
         bnd.sla_attention(Q, Q, Q, cfg)
+    assert e.value.code == 2
+    with pytest.raises(bnd.SlaError) as e:
+        bnd.sla_attention(Q, Q, Q, bnd.SlaConfig(k_h=0.5, k_l=0.0, pv="fp8_e4m3"))
     assert e.value.code == 2
