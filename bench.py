@@ -187,7 +187,7 @@ def run_ours(args, rank, world, dev):
     torch.cuda.set_device(dev)
     over = {} if args.heads is None else {"H": args.heads}
     data, w = I.make_workload(args.workload, device=f"cuda:{dev}", problem=rank, **over)
-    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"], qk=args.qk)
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"], qk=args.qk, pv=args.pv)
     Q, K, V = (data[k].to(dev) for k in ("Q", "K", "V"))
     O = torch.empty_like(Q)
     f32 = lambda t: None if t is None else t.to(dev).float().contiguous()  # noqa: E731
@@ -221,7 +221,7 @@ def run_ours(args, rank, world, dev):
     names = ["predict_mask", "precompute_linear", "aggregate_marginal", "fused_forward"]
     launches_per_step = {"predict_mask": 3 + (2 if Wq is not None or Wk is not None else 0),
                          "precompute_linear": 1, "aggregate_marginal": 2,
-                         "fused_forward": 1 + (1 if args.qk != "bf16" else 0)}
+                         "fused_forward": 1 + (1 if args.qk != "bf16" else 0) + (2 if args.pv != "bf16" else 0)}
 
     def step(ev=None):
         for i in range(4):
@@ -280,12 +280,13 @@ def run_ours(args, rank, world, dev):
         fused_ms = stage_ms[3]
         ach = fl["fused_alg"] / (fused_ms * 1e-3) / 1e12
         peak = float(peaks["bf16_tflops"])
-        traffic = fused_traffic_per_launch(args.workload, H, args.qk)
+        traffic = fused_traffic_per_launch(args.workload, H, args.qk if args.pv == "bf16" else "fp8 P V")
         result = {
             "metric": METRIC, "value": round(job_flops / (ms_total * 1e-3 / args.steps) / 1e12, 3),
             "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if args.qk == "bf16" else "bf16+e4m3",
+            "vs_baseline": None,
+            "dtype": "bf16" if args.qk == "bf16" and args.pv == "bf16" else "bf16+e4m3",
             "data": "synthetic",
             "config": {"workload": f"{args.workload} (B={B}, H={H}, N={N}, d={d}, k_h={cfg.k_h}, "
                                    f"k_l={cfg.k_l}, {cfg.combine} combine)",
@@ -565,6 +566,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, dense baseline and CPU baseline")
     ap.add_argument("--qk", choices=["bf16", "fp8_e4m3"], default="bf16",
                     help="precision of Q K^T on critical blocks (fp8_e4m3: d = 128 only)")
+    ap.add_argument("--pv", choices=["bf16", "fp8_e4m3"], default="bf16",
+                    help="precision of P V on critical blocks (fp8_e4m3: d = 128 only)")
     ap.add_argument("--heads", type=int, default=None, help="override the workload's head count "
                     "(profiling runs only; the bench line uses the workload as named)")
     ap.add_argument("--train", action="store_true",

@@ -35,6 +35,7 @@ EXPORTS = (
     "sla_attention_host_workspace_size", "sla_attention_host", "sla_backward",
     "sla_get_device_status", "sla_status_string", "sla_abi_version",
     "sla_predict_mask_noalloc", "sla_forward_train", "sla_backward_workspace_size",
+    "sla_selftest_wait_timeout",
 )
 
 
@@ -88,6 +89,7 @@ def lib() -> ctypes.CDLL:
         L.sla_forward_train.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_backward.argtypes = [P] + [vp] * 18 + [vp, sz, vp]
         L.sla_get_device_status.argtypes = [vp, vp, ip]
+        L.sla_selftest_wait_timeout.argtypes = [vp, vp]
         L.sla_status_string.argtypes = [ctypes.c_int]
         L.sla_status_string.restype = ctypes.c_char_p
         for f in EXPORTS:

@@ -623,6 +623,19 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   return SLA_OK;
 }
 
+// One thread waits on an mbarrier that nothing arrives at: the bounded wait gives
+// up after SLA_WAIT_TIMEOUT_NS, records the timeout in the error word and the
+// kernel returns (the failure path of every wait in the library, without a fault).
+__global__ void selftest_wait_kernel(int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, err, DEV_TIMEOUT_SYNC);
+}
+
 }  // namespace
 
 extern "C" {
@@ -842,6 +855,12 @@ sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, c
     return SLA_ERR_WORKSPACE;
   return backward_impl(pl, p, Q, K, V, mc, lut, hz, proj_w, proj_b, alpha, o_sparse, lse, dO, dQ, dK, dV,
                        dproj_w, dproj_b, dalpha, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sla_status_t sla_selftest_wait_timeout(void* workspace, sla_stream_t stream) {
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return SLA_ERR_WORKSPACE;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(static_cast<int*>(workspace));
+  return cuda_status(cudaGetLastError());
 }
 
 sla_status_t sla_get_device_status(void* workspace, sla_stream_t stream, int* detail) {

@@ -293,6 +293,16 @@ sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, c
                           void* dK, void* dV, float* dproj_w, float* dproj_b, float* dalpha,
                           void* workspace, size_t workspace_bytes, sla_stream_t stream);
 
+/*
+ * Diagnostic (no counterpart on the pages): launches one thread that waits on a
+ * barrier nothing completes.  The wait gives up after one second, records a
+ * timeout in the error word of `workspace` (any workspace of this library, or
+ * 256 zeroed bytes) and the kernel returns; sla_get_device_status then reports
+ * SLA_ERR_DEVICE_TIMEOUT.  It exercises the failure path that every wait of
+ * every kernel takes, without faulting the GPU.
+ */
+sla_status_t sla_selftest_wait_timeout(void* workspace, sla_stream_t stream);
+
 /* Reads the device error word of `workspace` (synchronises `stream`) and
  * clears it.  Returns SLA_OK, SLA_ERR_DEVICE_TIMEOUT or
  * SLA_ERR_DEVICE_BAD_INDEX; *detail (may be NULL) receives the raw code. */
