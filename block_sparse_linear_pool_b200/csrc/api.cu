@@ -30,7 +30,7 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t err, qc, kc, qr, kr, kmean, keys, mm, hagg;      // sla_workspace_size ...
-  size_t q8, k8, scq, sck, v8t, vmax, end;                // ... (+ FP8 operands)
+  size_t q8, k8, scq, sck, v8t, vmax, pairs, end;         // ... (+ FP8 operands)
   size_t mc, lut, hz, end_attn;                           // + sla_attention extras
   size_t hq, hk, hv, ho, end_host;                        // + sla_attention_host staging
 };
@@ -55,6 +55,7 @@ Layout layout_of(const Plan& p) {
   L.sck = o;   o = align_up(o + (p.fp8 ? (size_t)p.BH * p.Tkv * 4 : 0));
   L.v8t = o;   o = align_up(o + (p.pv8 ? (size_t)p.BH * p.Tkv * p.d * 128 : 0));
   L.vmax = o;  o = align_up(o + (p.pv8 ? (size_t)p.BH * p.d * 4 : 0));
+  L.pairs = o; o = align_up(o + (size_t)p.BH * ((p.Tq + 1) / 2) * 8);
   L.end = o;
   L.mc = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkv);
   L.lut = o;   o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
@@ -307,9 +308,12 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   const Layout L = layout_of(pl);
   __nv_bfloat16* hagg = at<__nv_bfloat16>(ws, L.hagg);
   CUtensorMap mq, mk, mv, mh, mz;
-  if (!map_bhnd(&mq, Q, pl, p->stride_q, 128) || !map_bhnd(&mk, K, pl, p->stride_k, 64) ||
+  if (!map_bhnd(&mq, Q, pl, p->stride_q, 64) || !map_bhnd(&mk, K, pl, p->stride_k, 64) ||
       !map_bhnd(&mv, V, pl, p->stride_v, 64))
     return SLA_ERR_CUDA;
+  // which two query blocks share a CTA (similar critical lists: a smaller union)
+  int2* pairs = at<int2>(ws, L.pairs);
+  SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pairs, s)));
   {
     // H_i^T as (a, b, i, bh) tiles of d x d; Z_i as one unswizzled row of d
     const uint64_t dh[4] = {(uint64_t)pl.d, (uint64_t)pl.d, (uint64_t)pl.Tq, (uint64_t)pl.BH};
@@ -344,7 +348,7 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
     SLA_TRY(cuda_status(launch_quant_fp8(qa, pl.BH, s)));
     const uint64_t dq[3] = {(uint64_t)pl.d, (uint64_t)pl.Tq * 64, (uint64_t)pl.BH};
     const uint64_t sq[2] = {(uint64_t)pl.d, (uint64_t)pl.Tq * 64 * pl.d};
-    const uint32_t bq[3] = {(uint32_t)pl.d, 128, 1};
+    const uint32_t bq[3] = {(uint32_t)pl.d, 64, 1};
     const uint64_t dk[3] = {(uint64_t)pl.d, (uint64_t)pl.Tkv * 64, (uint64_t)pl.BH};
     const uint64_t sk[2] = {(uint64_t)pl.d, (uint64_t)pl.Tkv * 64 * pl.d};
     const uint32_t bk[3] = {(uint32_t)pl.d, 64, 1};
@@ -392,6 +396,7 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.lse = lse;
   a.os = o_sparse;
   a.vmax = vmax;
+  a.pairs = pairs;
   return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, pl.fp8, pl.pv8, pl.BH, s));
 }
 

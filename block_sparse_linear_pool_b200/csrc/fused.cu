@@ -3,10 +3,11 @@
 // Attention", §2 Q2 steps 3-4 and Fig. 4 "Fused kernel"; "SLA2: Sparse-Linear
 // Attention with Learnable Routing and QAT", §3).
 //
-// A CTA owns 128 query rows = query blocks 2p and 2p+1 of one head, so every
-// tcgen05.mma runs at M = 128.  It walks the union of the two blocks' critical
-// lists (ascending); a key block that is critical for only one of the two
-// query blocks is masked out of the other half (its probabilities are 0).
+// A CTA owns 128 query rows = two query blocks of one head (chosen by
+// pairing_kernel for similar critical lists), so every tcgen05.mma runs at
+// M = 128.  It walks the union of the two blocks' critical lists (ascending); a
+// key block that is critical for only one of the two query blocks is masked out
+// of the other half (its probabilities are 0).
 //
 //   warp 0      TMA producer: Q tile, then K_j and V_j per union entry through
 //               two separate rings (a K slot frees when its S MMA completes, a
@@ -89,6 +90,7 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
 }  // namespace
 
 template <int D, bool FP8, bool PV8>
@@ -137,8 +139,11 @@ __global__ void __launch_bounds__(192, 2)
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const int p = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int ia = 2 * p, ib = 2 * p + 1;
-  const bool has_b = ib < a.Tq;
+  // the CTA's two query blocks (rows 0-63: ia, rows 64-127: ib); ib < 0: none
+  const int2 pair = a.pairs[(int64_t)bh * ((a.Tq + 1) / 2) + p];
+  const int ia = pair.x, ib = pair.y;
+  const bool has_b = ib >= 0;
+  const int ibl = has_b ? ib : ia;  // block loaded into the second half
 
   // ---------------- set-up: TMEM, barriers, union of the two critical lists
   if (w == 1) {
@@ -217,8 +222,14 @@ __global__ void __launch_bounds__(192, 2)
       if (FP8) tma_prefetch_desc(&mapQ8), tma_prefetch_desc(&mapK8);
       mbar_arrive_expect_tx(q_full, L::Q_BYTES + L::Q8_BYTES);
 #pragma unroll
-      for (int c = 0; c < L::CH; ++c) tma_load_4d(sQ + c * 16384, &mapQ, q_full, c * 64, 128 * p, h, b);
-      if (FP8) tma_load_3d(sQ8, &mapQ8, q_full, 0, 128 * p, bh);
+      for (int c = 0; c < L::CH; ++c) {
+        tma_load_4d(sQ + c * 16384, &mapQ, q_full, c * 64, 64 * ia, h, b);
+        tma_load_4d(sQ + c * 16384 + 8192, &mapQ, q_full, c * 64, 64 * ibl, h, b);
+      }
+      if (FP8) {
+        tma_load_3d(sQ8, &mapQ8, q_full, 0, 64 * ia, bh);
+        tma_load_3d(sQ8 + 8192, &mapQ8, q_full, 0, 64 * ibl, bh);
+      }
       bool ok = true;
       // K_k is issued one step ahead of V_{k-1}
       for (int k = 0; k <= U && ok; ++k) {
@@ -541,7 +552,7 @@ __global__ void __launch_bounds__(192, 2)
                                                    DEV_TIMEOUT_MMA));
     if (ok) {
       tc_fence_after();
-      const int n = 128 * p + r;
+      const int n = 64 * (half == 0 ? ia : ibl) + (r & 63);
       const bool store = (n < a.N) && (half == 0 || has_b);
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       // log-sum-exp of the row's scaled critical scores, for the backward:

@@ -74,6 +74,7 @@ struct FusedArgs {
   float* lse;             // [BH][N] natural-log sum of exp of the scaled critical scores, or nullptr
   float* os;              // [BH][N][d] the sparse branch's output o^s (fp32), or nullptr
   const unsigned int* vmax;  // FP8 P V: per (head, channel) max |V| (float bits), else nullptr
+  const int2* pairs;      // [BH][ceil(Tq / 2)] the two query blocks of each CTA (b = -1: none)
 };
 
 // ---- backward
@@ -115,6 +116,7 @@ struct BwdSparseArgs {
   const float* alpha;       // [BH] (SLA2) or nullptr
   const float* q_lin;       // [BH][N][d] dq (linear part), or dk (linear) for the key kernel
   const float* v_lin;       // [BH][N][d] dv (linear part) for the key kernel
+  const int2* pairs;        // [BH][ceil(Tq / 2)] query-block pairs of the dQ kernel
   __nv_bfloat16* out0;      // dQ, or dK for the key kernel
   __nv_bfloat16* out1;      // dV for the key kernel
   int64_t s0[3], s1[3];     // strides of out0, out1
@@ -145,6 +147,7 @@ cudaError_t launch_bwd_dkdv(const CUtensorMap& mapK2, const CUtensorMap& mapV2,
                             const BwdSparseArgs& a, int D, int BH, cudaStream_t s);
 
 cudaError_t launch_pool(const PoolArgs& a, int D, int BH, cudaStream_t s);
+cudaError_t launch_pairing(const int32_t* lut, int BH, int Tq, int nh, int2* pairs, cudaStream_t s);
 cudaError_t launch_router(const float* Qc, const float* Kc, float* Qr, float* Kr, float* kmean,
                           const float* Wq, const float* Wk, bool smooth, int BH, int Tq, int Tk,
                           int N, int bs, int D, cudaStream_t s);
