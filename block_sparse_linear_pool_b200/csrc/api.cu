@@ -436,7 +436,7 @@ sla_status_t attention_impl(const Plan& pl, const sla_params_t* p, const void* Q
 // Backward
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-  size_t err, mm, hagg, drow, dqlin, dhzq, mmt, dhzk, dklin, dvlin, ubuf, rcnt, rptr, rows, end;
+  size_t err, mm, hagg, drow, dqlin, dhzq, mmt, dhzk, dklin, dvlin, ubuf, rcnt, rptr, rows, pairs, kpairs, end;
 };
 
 BwdLayout bwd_layout_of(const Plan& p) {
@@ -458,6 +458,8 @@ BwdLayout bwd_layout_of(const Plan& p) {
   L.rcnt = o;  o = align_up(o + (size_t)p.BH * p.Tkv * 4);
   L.rptr = o;  o = align_up(o + (size_t)p.BH * (p.Tkv + 1) * 4);
   L.rows = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
+  L.pairs = o; o = align_up(o + (size_t)p.BH * ((p.Tq + 1) / 2) * 8);
+  L.kpairs = o; o = align_up(o + (size_t)p.BH * ((p.Tkv + 1) / 2) * 8);
   L.end = o;
   return L;
 }
@@ -581,12 +583,19 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   int32_t* rptr = at<int32_t>(ws, L.rptr);
   int32_t* rows = at<int32_t>(ws, L.rows);
   SLA_TRY(cuda_status(launch_rlut(mc, rcnt, rptr, rows, pl.BH, pl.Tq, pl.Tkv, pl.nh, s)));
+  // the dQ kernel's query-block pairs (as in the forward) and the dK / dV
+  // kernel's key-block pairs (by overlap of the reverse lists)
+  int2* pairs = at<int2>(ws, L.pairs);
+  int2* kpairs = at<int2>(ws, L.kpairs);
+  SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pairs, s)));
+  SLA_TRY(cuda_status(launch_pairing_csr(rows, rptr, (int64_t)pl.Tq * pl.nh, pl.BH, pl.Tkv, kpairs, s)));
   BwdSparseArgs sa;
   sa.lut = lut;
   sa.rptr = rptr;
   sa.rows = rows;
   sa.ld2 = ra.ld2;
   sa.alpha = alpha_mode ? alpha : nullptr;
+  sa.pairs = nullptr;
   sa.err = err;
   sa.H = pl.H;
   sa.N = pl.N;
@@ -598,10 +607,11 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   sa.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)pl.d));
   {
     CUtensorMap mq, mdo, mk, mv;
-    if (!map_bhnd(&mq, Q, pl, p->stride_q, 128) || !map_bhnd(&mdo, dO, pl, p->stride_o, 128) ||
+    if (!map_bhnd(&mq, Q, pl, p->stride_q, 64) || !map_bhnd(&mdo, dO, pl, p->stride_o, 64) ||
         !map_bhnd(&mk, K, pl, p->stride_k, 64) || !map_bhnd(&mv, V, pl, p->stride_v, 64))
       return SLA_ERR_CUDA;
     BwdSparseArgs qa = sa;
+    qa.pairs = pairs;
     qa.q_lin = ra.dq_lin;
     qa.v_lin = nullptr;
     qa.out0 = static_cast<__nv_bfloat16*>(dQ);
@@ -611,10 +621,11 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   }
   {
     CUtensorMap mk2, mv2, mq1, mdo1;
-    if (!map_bhnd(&mk2, K, pl, p->stride_k, 128) || !map_bhnd(&mv2, V, pl, p->stride_v, 128) ||
+    if (!map_bhnd(&mk2, K, pl, p->stride_k, 64) || !map_bhnd(&mv2, V, pl, p->stride_v, 64) ||
         !map_bhnd(&mq1, Q, pl, p->stride_q, 64) || !map_bhnd(&mdo1, dO, pl, p->stride_o, 64))
       return SLA_ERR_CUDA;
     BwdSparseArgs kb = sa;
+    kb.pairs = kpairs;
     kb.q_lin = ka.dk_lin;
     kb.v_lin = ka.dv_lin;
     kb.out0 = static_cast<__nv_bfloat16*>(dK);

@@ -13,12 +13,14 @@
 //
 //   rlut_*              reverse lists: for every key block, the query blocks
 //                       that have it critical (ascending), from M_c
-//   bwd_dq_kernel       CTA = query blocks 2p, 2p+1 (M = 128) over the union of
-//                       their critical lists: S = Q K^T and dP = dO V^T into
+//   bwd_dq_kernel       CTA = two query blocks (M = 128; the forward's pairing
+//                       by critical-list overlap) over the union of their
+//                       critical lists: S = Q K^T and dP = dO V^T into
 //                       TMEM (two buffers), dS by the row threads, dQ += dS K
 //                       (dS read from TMEM)
-//   bwd_dkdv_kernel     CTA = key blocks 2p, 2p+1 (M = 128 key rows) over the
-//                       union of their reverse lists: S^T = K Q^T and
+//   bwd_dkdv_kernel     CTA = two key blocks (M = 128 key rows, paired by
+//                       reverse-list overlap) over the union of their reverse
+//                       lists: S^T = K Q^T and
 //                       dP^T = V dO^T into TMEM (two buffers), P^T and dS^T by
 //                       the key-row threads, dV += P^T dO and dK += dS^T Q
 // Both: warp 0 TMA producer, warp 1 MMA issuer, warps 2-9 two threads per TMEM
@@ -157,8 +159,11 @@ __global__ void __launch_bounds__(320, 1)
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const int p = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int ia = 2 * p, ib = 2 * p + 1;
-  const bool has_b = ib < a.Tq;
+  // the CTA's two query blocks (rows 0-63: ia, rows 64-127: ib); ib < 0: none
+  const int2 pair = a.pairs[(int64_t)bh * ((a.Tq + 1) / 2) + p];
+  const int ia = pair.x, ib = pair.y;
+  const bool has_b = ib >= 0;
+  const int ibl = has_b ? ib : ia;  // block loaded into the second half
 
   if (w == 1) {
     tmem_alloc(tslot, 512);
@@ -185,7 +190,7 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   {
     const int32_t* la = a.lut + ((int64_t)bh * a.Tq + ia) * a.nh;
-    const int32_t* lb = a.lut + ((int64_t)bh * a.Tq + (has_b ? ib : ia)) * a.nh;
+    const int32_t* lb = a.lut + ((int64_t)bh * a.Tq + ibl) * a.nh;
     const int tot = has_b ? 2 * a.nh : a.nh;
     for (int e = tid; e < tot; e += blockDim.x) {
       const bool second = e >= a.nh;
@@ -229,8 +234,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive_expect_tx(in_full, 2 * L::T128);
 #pragma unroll
       for (int c = 0; c < L::CH; ++c) {
-        tma_load_4d(sQ + c * 16384, &mapQ, in_full, c * 64, 128 * p, h, b);
-        tma_load_4d(sdO + c * 16384, &mapdO, in_full, c * 64, 128 * p, h, b);
+        tma_load_4d(sQ + c * 16384, &mapQ, in_full, c * 64, 64 * ia, h, b);
+        tma_load_4d(sQ + c * 16384 + 8192, &mapQ, in_full, c * 64, 64 * ibl, h, b);
+        tma_load_4d(sdO + c * 16384, &mapdO, in_full, c * 64, 64 * ia, h, b);
+        tma_load_4d(sdO + c * 16384 + 8192, &mapdO, in_full, c * 64, 64 * ibl, h, b);
       }
       bool ok = true;
       for (int k = 0; k < U && ok; ++k) {
@@ -305,7 +312,7 @@ __global__ void __launch_bounds__(320, 1)
     const int half = r >> 6;
     const uint32_t bit = 1u << half;
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
-    const int n = 128 * p + r;
+    const int n = 64 * (half == 0 ? ia : ibl) + (r & 63);
     const bool valid = (n < a.N) && (half == 0 || has_b);
     // (lse log2 e, D) of this row; P = 0 on rows that do not exist
     const float2 ld = valid ? a.ld2[(int64_t)bh * a.Tq * 64 + n] : make_float2(INFINITY, 0.f);
@@ -449,8 +456,11 @@ __global__ void __launch_bounds__(320, 1)
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const int p = blockIdx.x, bh = blockIdx.y;
   const int b = bh / a.H, h = bh % a.H;
-  const int ja = 2 * p, jb = 2 * p + 1;
-  const bool has_b = jb < a.Tkv;
+  // the CTA's two key blocks (rows 0-63: ja, rows 64-127: jb); jb < 0: none
+  const int2 pair = a.pairs[(int64_t)bh * ((a.Tkv + 1) / 2) + p];
+  const int ja = pair.x, jb = pair.y;
+  const bool has_b = jb >= 0;
+  const int jbl = has_b ? jb : ja;  // block loaded into the second half
 
   if (w == 1) {
     tmem_alloc(tslot, 512);
@@ -517,8 +527,10 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive_expect_tx(kv_full, 2 * L::T128);
 #pragma unroll
       for (int c = 0; c < L::CH; ++c) {
-        tma_load_4d(sK + c * 16384, &mapK2, kv_full, c * 64, 128 * p, h, b);
-        tma_load_4d(sV + c * 16384, &mapV2, kv_full, c * 64, 128 * p, h, b);
+        tma_load_4d(sK + c * 16384, &mapK2, kv_full, c * 64, 64 * ja, h, b);
+        tma_load_4d(sK + c * 16384 + 8192, &mapK2, kv_full, c * 64, 64 * jbl, h, b);
+        tma_load_4d(sV + c * 16384, &mapV2, kv_full, c * 64, 64 * ja, h, b);
+        tma_load_4d(sV + c * 16384 + 8192, &mapV2, kv_full, c * 64, 64 * jbl, h, b);
       }
       bool ok = true;
       for (int e = 0; e < U && ok; ++e) {
@@ -591,7 +603,7 @@ __global__ void __launch_bounds__(320, 1)
     const int half = t >> 6;
     const uint32_t bit = 1u << half;
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
-    const int n = 128 * p + t;
+    const int n = 64 * (half == 0 ? ja : jbl) + (t & 63);
     const bool valid = (n < a.N) && (half == 0 || has_b);
     const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
     const float sl2 = a.scale_log2;

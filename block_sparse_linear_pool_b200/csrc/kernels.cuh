@@ -116,7 +116,7 @@ struct BwdSparseArgs {
   const float* alpha;       // [BH] (SLA2) or nullptr
   const float* q_lin;       // [BH][N][d] dq (linear part), or dk (linear) for the key kernel
   const float* v_lin;       // [BH][N][d] dv (linear part) for the key kernel
-  const int2* pairs;        // [BH][ceil(Tq / 2)] query-block pairs of the dQ kernel
+  const int2* pairs;        // [BH][ceil(T / 2)] block pairs: query blocks (dQ) or key blocks (dK / dV)
   __nv_bfloat16* out0;      // dQ, or dK for the key kernel
   __nv_bfloat16* out1;      // dV for the key kernel
   int64_t s0[3], s1[3];     // strides of out0, out1
@@ -148,6 +148,8 @@ cudaError_t launch_bwd_dkdv(const CUtensorMap& mapK2, const CUtensorMap& mapV2,
 
 cudaError_t launch_pool(const PoolArgs& a, int D, int BH, cudaStream_t s);
 cudaError_t launch_pairing(const int32_t* lut, int BH, int Tq, int nh, int2* pairs, cudaStream_t s);
+cudaError_t launch_pairing_csr(const int32_t* rows, const int32_t* ptr, int64_t stride, int BH, int T,
+                               int2* pairs, cudaStream_t s);
 cudaError_t launch_router(const float* Qc, const float* Kc, float* Qr, float* Kr, float* kmean,
                           const float* Wq, const float* Wk, bool smooth, int BH, int Tq, int Tk,
                           int N, int bs, int D, cudaStream_t s);
