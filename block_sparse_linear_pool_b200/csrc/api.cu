@@ -30,7 +30,7 @@ inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
   size_t err, qc, kc, qr, kr, kmean, keys, mm, hagg;      // sla_workspace_size ...
-  size_t q8, k8, scq, sck, v8t, vmax, pairs, end;         // ... (+ FP8 operands)
+  size_t q8, k8, scq, sck, v8t, vmax, pairs, pov, end;    // ... (+ FP8 operands)
   size_t mc, lut, hz, end_attn;                           // + sla_attention extras
   size_t hq, hk, hv, ho, end_host;                        // + sla_attention_host staging
 };
@@ -56,6 +56,7 @@ Layout layout_of(const Plan& p) {
   L.v8t = o;   o = align_up(o + (p.pv8 ? (size_t)p.BH * p.Tkv * p.d * 128 : 0));
   L.vmax = o;  o = align_up(o + (p.pv8 ? (size_t)p.BH * p.d * 4 : 0));
   L.pairs = o; o = align_up(o + (size_t)p.BH * ((p.Tq + 1) / 2) * 8);
+  L.pov = o;   o = align_up(o + pairing_overlap_bytes(p.BH, p.Tq));
   L.end = o;
   L.mc = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkv);
   L.lut = o;   o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
@@ -313,7 +314,7 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
     return SLA_ERR_CUDA;
   // which two query blocks share a CTA (similar critical lists: a smaller union)
   int2* pairs = at<int2>(ws, L.pairs);
-  SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pairs, s)));
+  SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pl.Tkv, at<uint16_t>(ws, L.pov), pairs, s)));
   {
     // H_i^T as (a, b, i, bh) tiles of d x d; Z_i as one unswizzled row of d
     const uint64_t dh[4] = {(uint64_t)pl.d, (uint64_t)pl.d, (uint64_t)pl.Tq, (uint64_t)pl.BH};
@@ -436,7 +437,7 @@ sla_status_t attention_impl(const Plan& pl, const sla_params_t* p, const void* Q
 // Backward
 // ---------------------------------------------------------------------------
 struct BwdLayout {
-  size_t err, mm, hagg, drow, dqlin, dhzq, mmt, dhzk, dklin, dvlin, ubuf, rcnt, rptr, rows, pairs, kpairs, end;
+  size_t err, mm, hagg, drow, dqlin, dhzq, mmt, dhzk, dklin, dvlin, ubuf, rcnt, rptr, rows, pairs, kpairs, pov, end;
 };
 
 BwdLayout bwd_layout_of(const Plan& p) {
@@ -460,6 +461,7 @@ BwdLayout bwd_layout_of(const Plan& p) {
   L.rows = o;  o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
   L.pairs = o; o = align_up(o + (size_t)p.BH * ((p.Tq + 1) / 2) * 8);
   L.kpairs = o; o = align_up(o + (size_t)p.BH * ((p.Tkv + 1) / 2) * 8);
+  L.pov = o;   o = align_up(o + pairing_overlap_bytes(p.BH, std::max(p.Tq, p.Tkv)));
   L.end = o;
   return L;
 }
@@ -587,8 +589,10 @@ sla_status_t backward_impl(const Plan& pl, const sla_params_t* p, const void* Q,
   // kernel's key-block pairs (by overlap of the reverse lists)
   int2* pairs = at<int2>(ws, L.pairs);
   int2* kpairs = at<int2>(ws, L.kpairs);
-  SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pairs, s)));
-  SLA_TRY(cuda_status(launch_pairing_csr(rows, rptr, (int64_t)pl.Tq * pl.nh, pl.BH, pl.Tkv, kpairs, s)));
+  uint16_t* pov = at<uint16_t>(ws, L.pov);  // used by one pairing at a time (stream order)
+  SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pl.Tkv, pov, pairs, s)));
+  SLA_TRY(cuda_status(launch_pairing_csr(rows, rptr, (int64_t)pl.Tq * pl.nh, pl.BH, pl.Tkv, pl.Tq, pov, kpairs,
+                                         s)));
   BwdSparseArgs sa;
   sa.lut = lut;
   sa.rptr = rptr;

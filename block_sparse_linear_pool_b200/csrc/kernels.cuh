@@ -147,9 +147,12 @@ cudaError_t launch_bwd_dkdv(const CUtensorMap& mapK2, const CUtensorMap& mapV2,
                             const BwdSparseArgs& a, int D, int BH, cudaStream_t s);
 
 cudaError_t launch_pool(const PoolArgs& a, int D, int BH, cudaStream_t s);
-cudaError_t launch_pairing(const int32_t* lut, int BH, int Tq, int nh, int2* pairs, cudaStream_t s);
+// ov: scratch of pairing_overlap_bytes(BH, T); ncol: the range of the list entries
+size_t pairing_overlap_bytes(int BH, int T);
+cudaError_t launch_pairing(const int32_t* lut, int BH, int Tq, int nh, int ncol, uint16_t* ov, int2* pairs,
+                           cudaStream_t s);
 cudaError_t launch_pairing_csr(const int32_t* rows, const int32_t* ptr, int64_t stride, int BH, int T,
-                               int2* pairs, cudaStream_t s);
+                               int ncol, uint16_t* ov, int2* pairs, cudaStream_t s);
 cudaError_t launch_router(const float* Qc, const float* Kc, float* Qr, float* Kr, float* kmean,
                           const float* Wq, const float* Wk, bool smooth, int BH, int Tq, int Tk,
                           int N, int bs, int D, cudaStream_t s);
