@@ -6,11 +6,13 @@
 // With the SLA combine, Proj's weight W is folded in (h_j W^T is stored):
 // Proj(O^l) = phi(Q) (H W^T) / den + b because den is a per-row scalar.
 //
-// One CTA (4 warps) walks key blocks of 64 tokens persistently through two
-// shared-memory stages, the next block's K_j, V_j loading while the current one
-// is processed:
+// One CTA (4 warps, two per SM) walks key blocks of 64 tokens persistently
+// through three shared-memory stages, the next two blocks' K_j, V_j loading
+// while the current one is processed:
 //   TMA      K_j, V_j  -> stage (128B-swizzled, d contiguous)
-//   tcgen05  D1 = W V_j^T          (M = d, N = 64, K = d)   [SLA only]
+//   tcgen05  D1 = W V_j^T          (M = d, N = 64, K = d)   [SLA only; for
+//            d = 128 W is the A operand from TMEM, which leaves the shared
+//            memory to the three stages]
 //   threads  phi(K_j) in place of K_j; V'^T = D1 in place of V_j (bf16)
 //   tcgen05  D2 = V'^T phi(K_j)    (M = d, N = d, K = 64)  = (h_j W^T)^T
 //   threads  z_j = column sums of phi(K_j); D2 -> the stage as a swizzled
@@ -22,12 +24,14 @@ namespace sla {
 template <int D>
 struct KvSmem {
   static constexpr int CH = D / 64;                 // 64-column chunks of d
-  static constexpr int W_BYTES = D * D * 2;         // W, K-major [CH][D rows][128B]
+  static constexpr bool W_TMEM = D == 128;          // W in TMEM columns [192, 256) as bf16 pairs
+  static constexpr int W_BYTES = W_TMEM ? 0 : D * D * 2;  // else W, K-major [CH][D rows][128B]
   static constexpr int T_BYTES = 64 * D * 2;        // one 64-token tile
   static constexpr int STAGE = 2 * T_BYTES;         // K (then phi) | V (then V'^T); then the h tile
+  static constexpr int NST = 3;                     // stages
   static constexpr int OFF_W = 0;
   static constexpr int OFF_ST = OFF_W + W_BYTES;
-  static constexpr int OFF_BAR = OFF_ST + 2 * STAGE;
+  static constexpr int OFF_BAR = OFF_ST + NST * STAGE;
   static constexpr int BYTES = OFF_BAR + 64;
   static constexpr int ALLOC = BYTES + 1024;        // slack for 1024-byte alignment
 };
@@ -44,9 +48,9 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
   uint8_t* sW = sm + L::OFF_W;
-  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);  // [2]
-  uint64_t* mma_bar = tma_bar + 2;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(tma_bar + 3);
+  uint64_t* tma_bar = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);  // [NST]
+  uint64_t* mma_bar = tma_bar + L::NST;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(mma_bar + 1);
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const bool proj = a.proj_w != nullptr;
 
@@ -55,15 +59,14 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&tma_bar[0], 1);
-    mbar_init(&tma_bar[1], 1);
+    for (int x = 0; x < L::NST; ++x) mbar_init(&tma_bar[x], 1);
     mbar_init(mma_bar, 1);
     fence_barrier_init();
     tma_prefetch_desc(&mapK);
     tma_prefetch_desc(&mapV);
     tma_prefetch_desc(&mapO);
   }
-  if (proj) {  // W (fp32 [o][b]) -> bf16, K-major over b
+  if (proj && !L::W_TMEM) {  // W (fp32 [o][b]) -> bf16, K-major over b
     for (int g = tid; g < D * D / 8; g += 128) {
       const int o = g / (D / 8), b0 = (g % (D / 8)) * 8;
       const float4 x0 = __ldg(reinterpret_cast<const float4*>(a.proj_w + o * D + b0));
@@ -83,7 +86,29 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
   const uint32_t tbase = *tslot;
   const uint32_t tD1 = tbase;       // 64 columns
   const uint32_t tD2 = tbase + 64;  // D columns
+  const uint32_t tW = tbase + 192;  // d = 128: W, row o in lane o, bf16 pairs along b
   const uint32_t lane_off = (uint32_t)(32 * (w & 3)) << 16;
+  if (proj && L::W_TMEM) {  // thread tid holds row o = tid (lane tid)
+    const float* wr = a.proj_w + (int64_t)tid * D;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t r[32];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float4 x0 = __ldg(reinterpret_cast<const float4*>(wr + 64 * half + 8 * c));
+        const float4 x1 = __ldg(reinterpret_cast<const float4*>(wr + 64 * half + 8 * c + 4));
+        r[4 * c + 0] = pack_bf16x2(x0.x, x0.y);
+        r[4 * c + 1] = pack_bf16x2(x0.z, x0.w);
+        r[4 * c + 2] = pack_bf16x2(x1.x, x1.y);
+        r[4 * c + 3] = pack_bf16x2(x1.z, x1.w);
+      }
+      tmem_st32(tW + lane_off + 32 * half, r);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
   // Row of the M = D accumulators held by this thread (M = 64 packs rows
   // 16 per 32-lane quarter).
   const int my_row = (D == 128) ? tid : ((ln < 16) ? 16 * w + ln : -1);
@@ -99,34 +124,39 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       tma_load_4d(st + L::T_BYTES + c * 8192, &mapV, &tma_bar[s], c * 64, j * 64, h, b);
     }
   };
-  if (tid == 0 && (int)blockIdx.x < a.nitems) issue_load(blockIdx.x, 0);
+  int n_issued = 0;  // loads issued (thread 0)
+  if (tid == 0) {
+    for (int x = 0; x < L::NST - 1; ++x)
+      if ((int)blockIdx.x + x * (int)gridDim.x < a.nitems) {
+        issue_load(blockIdx.x + x * gridDim.x, x);
+        ++n_issued;
+      }
+  }
 
   uint32_t mma_phase = 0;
   int n = 0;
   // Every wait result is agreed on by the whole CTA (__syncthreads_and), so a
   // timeout makes all threads leave the loop at the same point.
   for (int item = blockIdx.x; item < a.nitems; item += gridDim.x, ++n) {
-    const int s = n & 1;
+    const int s = n % L::NST;
     uint8_t* sK = sm + L::OFF_ST + s * L::STAGE;
     uint8_t* sV = sK + L::T_BYTES;
     const int bh = item / a.Tkv, j = item % a.Tkv;
     const int cnt = min(64, a.N - j * 64);
-    // next block into the other stage, once the store that last used it has
-    // finished reading shared memory
-    if (tid == 0 && item + (int)gridDim.x < a.nitems) {
-      bulk_wait_read_all();
-      issue_load(item + gridDim.x, s ^ 1);
-    }
-    if (!__syncthreads_and(mbar_wait(&tma_bar[s], (n >> 1) & 1, a.err, DEV_TIMEOUT_TMA))) break;
+    if (!__syncthreads_and(mbar_wait(&tma_bar[s], (n / L::NST) & 1, a.err, DEV_TIMEOUT_TMA))) break;
     if (proj && tid == 0) {
       tc_fence_after();
       const uint32_t id = idesc_bf16(D, 64, false, false);
 #pragma unroll
       for (int k = 0; k < D / 16; ++k) {
         const uint32_t off = (k % 4) * 32;
-        const uint64_t ad = sdesc_sw128(smem_u32(sW) + (k / 4) * (D * 128) + off, 16, 1024);
         const uint64_t bd = sdesc_sw128(smem_u32(sV) + (k / 4) * 8192 + off, 16, 1024);
-        umma_ss(tD1, ad, bd, id, k > 0);
+        if (L::W_TMEM) {  // b = 16 k .. 16 k + 15: columns 8 k .. 8 k + 7 of W
+          umma_ts(tD1, tW + 8 * k, bd, id, k > 0);
+        } else {
+          const uint64_t ad = sdesc_sw128(smem_u32(sW) + (k / 4) * (D * 128) + off, 16, 1024);
+          umma_ss(tD1, ad, bd, id, k > 0);
+        }
       }
       umma_commit(mma_bar);
     }
@@ -218,6 +248,14 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
         umma_ss(tD2, ad, bd, id, k > 0);
       }
       umma_commit(mma_bar);
+      // the block two ahead into the stage that the previous block used, once
+      // that block's store has finished reading it
+      const int nx = item + 2 * (int)gridDim.x;
+      if (nx < a.nitems) {
+        bulk_wait_read_all();
+        issue_load(nx, (n + 2) % L::NST);
+        ++n_issued;
+      }
     }
     // z_j = column sums of phi(K_j) (the bf16 values the MMA consumes)
     float z = 0.f;
@@ -266,7 +304,12 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
       bulk_commit_group();
     }
   }
-  if (tid == 0) bulk_wait_all();
+  if (tid == 0) {
+    // loads still in flight after an early exit land before the CTA leaves
+    for (int k = n; k < n_issued; ++k)
+      if (!mbar_wait(&tma_bar[k % L::NST], (k / L::NST) & 1, a.err, DEV_TIMEOUT_TMA)) break;
+    bulk_wait_all();
+  }
   tc_fence_before();
   __syncthreads();
   if (w == 0) {
