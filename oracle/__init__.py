@@ -15,6 +15,7 @@ from .sla import (  # noqa: F401
     compressed_logits,
     compressed_attention,
     classify,
+    soft_topk,
     predict_mask,
     critical_lut,
     feature_map,

@@ -36,6 +36,9 @@ Readings taken where the pages are silent:
   * the backward treats M_c as a constant (hard Top-k has no gradient) and
     returns gradients for Q, K, V and the combine's parameters only.
 
+  * SoftTop-k ([SLA2] §4, §6) keeps n_h (the hard Top-k's count) per row and
+    applies its sigmoid to P_c.
+
 Parity unpinned: the FP8 paths' exact values at full size (the quantiser is
 pinned; the emulations are pinned only on cases where they must be exact).
 """
@@ -164,6 +167,44 @@ def classify(Pc: np.ndarray, n_h: int, n_l: int) -> np.ndarray:
         if n_l > 0:
             Mc[r, rank >= T - n_l] = -1
     return Mc.reshape(Pc.shape)
+
+
+def soft_topk(Pc: np.ndarray, n_h: int, tau: float, iters: int = 200):
+    """SLA2's SoftTop-k, the differentiable stand-in for the router's hard
+    row-wise Top-k during training ([SLA2] §4 Learnable Router, §6 Training with
+    SLA2: a sigmoid with temperature tau and a per-row threshold lambda_i found
+    by binary search so that the row keeps the Top-k row sum).
+
+    M[i, j] = sigmoid((Pc[i, j] - lambda_i) / tau), with lambda_i the root of
+    f(lambda) = sum_j sigmoid((Pc[i, j] - lambda) / tau) - n_h.  f falls
+    monotonically from T (lambda -> -inf) to 0 (lambda -> +inf), so bisection on
+    [min_j Pc - 50 tau, max_j Pc + 50 tau] (where every term is within e^-50 of
+    1, respectively 0) finds it; `iters` halvings run it to fp64 resolution.
+
+    Readings: the target row sum is n_h, the hard Top-k's count, so that
+    tau -> 0 gives back the hard mask's critical set; the sigmoid acts on P_c,
+    the quantity the hard Top-k ranks.  Returns (M, lambda) in float64.
+    """
+    from scipy.special import expit
+    if not tau > 0:
+        raise ValueError("tau must be positive")
+    Pc = np.asarray(Pc, dtype=np.float64)
+    T = Pc.shape[-1]
+    flat = Pc.reshape(-1, T)
+    M = np.empty_like(flat)
+    lam = np.empty(flat.shape[0])
+    for r in range(flat.shape[0]):
+        row = flat[r]
+        lo, hi = row.min() - 50.0 * tau, row.max() + 50.0 * tau
+        for _ in range(iters):
+            mid = 0.5 * (lo + hi)
+            if expit((row - mid) / tau).sum() > n_h:
+                lo = mid
+            else:
+                hi = mid
+        lam[r] = 0.5 * (lo + hi)
+        M[r] = expit((row - lam[r]) / tau)
+    return M.reshape(Pc.shape), lam.reshape(Pc.shape[:-1])
 
 
 def predict_mask(Q, K, p: OracleParams, Wq=None, Wk=None):
