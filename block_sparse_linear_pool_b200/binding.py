@@ -35,7 +35,7 @@ EXPORTS = (
     "sla_attention_host_workspace_size", "sla_attention_host", "sla_backward",
     "sla_get_device_status", "sla_status_string", "sla_abi_version",
     "sla_predict_mask_noalloc", "sla_forward_train", "sla_backward_workspace_size",
-    "sla_selftest_wait_timeout",
+    "sla_selftest_wait_timeout", "sla_router_probs", "sla_soft_topk",
 )
 
 
@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
         L.sla_backward.argtypes = [P] + [vp] * 18 + [vp, sz, vp]
         L.sla_get_device_status.argtypes = [vp, vp, ip]
         L.sla_selftest_wait_timeout.argtypes = [vp, vp]
+        L.sla_router_probs.argtypes = [P, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_soft_topk.argtypes = [P, vp, ctypes.c_float, vp, vp, vp]
         L.sla_status_string.argtypes = [ctypes.c_int]
         L.sla_status_string.restype = ctypes.c_char_p
         for f in EXPORTS:
@@ -201,6 +203,34 @@ def sla_predict_mask(Q, K, cfg: SlaConfig, Wq=None, Wk=None, workspace=None):
     _check(lib().sla_predict_mask(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(Wq), _ptr(Wk), _ptr(mc),
                                   _ptr(lut), _ptr(ws), ws.numel(), _stream()), "sla_predict_mask")
     return mc, lut
+
+
+def sla_router_probs(Q, K, cfg: SlaConfig, Wq=None, Wk=None, workspace=None):
+    """P_c fp32 [B*H, T_q, T_kv]: the row softmax of the router's compressed logits."""
+    p = make_params(Q, cfg, K=K)
+    Tq, Tkv, _, _ = sla_block_counts(p)
+    BH = Q.shape[0] * Q.shape[1]
+    Pc = torch.empty((BH, Tq, Tkv), dtype=torch.float32, device=Q.device)
+    ws = workspace if workspace is not None else new_workspace(sla_workspace_size(p), Q.device)
+    Wq, Wk = _f32(Wq, Q.device), _f32(Wk, Q.device)
+    _check(lib().sla_router_probs(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(Wq), _ptr(Wk), _ptr(Pc),
+                                  _ptr(ws), ws.numel(), _stream()), "sla_router_probs")
+    return Pc
+
+
+def sla_soft_topk(Pc, Q, cfg: SlaConfig, tau: float):
+    """SoftTop-k of P_c ([B*H, T_q, T_kv] fp32; Q gives the problem's shape):
+    returns (M fp32 like Pc, lambda fp32 [B*H, T_q])."""
+    p = make_params(Q, cfg)
+    Tq, Tkv, _, _ = sla_block_counts(p)
+    BH = Q.shape[0] * Q.shape[1]
+    if tuple(Pc.shape) != (BH, Tq, Tkv) or Pc.dtype != torch.float32 or not Pc.is_contiguous():
+        raise ValueError(f"Pc must be contiguous fp32 {(BH, Tq, Tkv)}")
+    M = torch.empty_like(Pc)
+    lam = torch.empty((BH, Tq), dtype=torch.float32, device=Pc.device)
+    _check(lib().sla_soft_topk(ctypes.byref(p), _ptr(Pc), ctypes.c_float(tau), _ptr(M), _ptr(lam),
+                               _stream()), "sla_soft_topk")
+    return M, lam
 
 
 def sla_precompute_linear(K, V, cfg: SlaConfig, proj_w=None, workspace=None):

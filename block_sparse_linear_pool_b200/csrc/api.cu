@@ -193,9 +193,11 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-sla_status_t predict_mask_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
-                               const float* Wq, const float* Wk, int8_t* mc, int32_t* lut,
-                               void* ws, cudaStream_t s) {
+// a1 and the router part of a2: pooled (smoothed, projected) Q_c, K_c in the
+// workspace; *qsrc, *ksrc point at the ones the logits use
+sla_status_t router_inputs(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
+                           const float* Wq, const float* Wk, void* ws, cudaStream_t s,
+                           const float** qsrc_out, const float** ksrc_out) {
   const Layout L = layout_of(pl);
   PoolArgs pa;
   pa.Q = static_cast<const __nv_bfloat16*>(Q);
@@ -220,6 +222,17 @@ sla_status_t predict_mask_impl(const Plan& pl, const sla_params_t* p, const void
     qsrc = at<float>(ws, L.qr);
     ksrc = at<float>(ws, L.kr);
   }
+  *qsrc_out = qsrc;
+  *ksrc_out = ksrc;
+  return SLA_OK;
+}
+
+sla_status_t predict_mask_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
+                               const float* Wq, const float* Wk, int8_t* mc, int32_t* lut,
+                               void* ws, cudaStream_t s) {
+  const Layout L = layout_of(pl);
+  const float *qsrc = nullptr, *ksrc = nullptr;
+  SLA_TRY(router_inputs(pl, p, Q, K, Wq, Wk, ws, s, &qsrc, &ksrc));
   SelectArgs sa;
   sa.Qc = qsrc;
   sa.Kc = ksrc;
@@ -734,6 +747,39 @@ sla_status_t sla_predict_mask(const sla_params_t* p, const void* Q, const void* 
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
+sla_status_t sla_router_probs(const sla_params_t* p, const void* Q, const void* K, const float* Wq,
+                              const float* Wk, float* Pc, void* workspace, size_t workspace_bytes,
+                              sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !Pc || !aligned16(Q) || !aligned16(K) || !aligned16(Pc)) return SLA_ERR_INVALID_ARG;
+  if ((Wq && !aligned16(Wq)) || (Wk && !aligned16(Wk))) return SLA_ERR_INVALID_ARG;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const Layout L = layout_of(pl);
+  const float *qsrc = nullptr, *ksrc = nullptr;
+  SLA_TRY(router_inputs(pl, p, Q, K, Wq, Wk, workspace, s, &qsrc, &ksrc));
+  LogitArgs la;
+  la.Qc = qsrc;
+  la.Kc = ksrc;
+  la.keys = at<uint32_t>(workspace, L.keys);
+  la.d = pl.d;
+  la.Tq = pl.Tq;
+  la.Tkv = pl.Tkv;
+  SLA_TRY(cuda_status(launch_logits(la, pl.BH, s)));
+  return cuda_status(launch_router_probs(la.keys, Pc, pl.Tkv, (int64_t)pl.BH * pl.Tq, s));
+}
+
+sla_status_t sla_soft_topk(const sla_params_t* p, const float* Pc, float tau, float* M, float* lambda,
+                           sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Pc || !M || !lambda || !aligned16(Pc) || !aligned16(M)) return SLA_ERR_INVALID_ARG;
+  if (!(tau > 0.f) || !std::isfinite(tau)) return SLA_ERR_INVALID_ARG;
+  return cuda_status(launch_soft_topk(Pc, M, lambda, pl.Tkv, (int64_t)pl.BH * pl.Tq, pl.nh, tau,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 sla_status_t sla_precompute_linear(const sla_params_t* p, const void* K, const void* V,
                                    const float* proj_w, void* hz, void* workspace,
                                    size_t workspace_bytes, sla_stream_t stream) {
@@ -913,6 +959,6 @@ const char* sla_status_string(sla_status_t s) {
   return "SLA_ERR_UNKNOWN";
 }
 
-int sla_abi_version(void) { return 102; }
+int sla_abi_version(void) { return 103; }
 
 }  // extern "C"

@@ -147,6 +147,10 @@ cudaError_t launch_bwd_dkdv(const CUtensorMap& mapK2, const CUtensorMap& mapV2,
                             const BwdSparseArgs& a, int D, int BH, cudaStream_t s);
 
 cudaError_t launch_pool(const PoolArgs& a, int D, int BH, cudaStream_t s);
+cudaError_t launch_logits(const LogitArgs& a, int BH, cudaStream_t s);
+cudaError_t launch_router_probs(const uint32_t* keys, float* Pc, int Tkv, int64_t rows, cudaStream_t s);
+cudaError_t launch_soft_topk(const float* Pc, float* M, float* lam, int Tkv, int64_t rows, int nh, float tau,
+                             cudaStream_t s);
 // ov: scratch of pairing_overlap_bytes(BH, T); ncol: the range of the list entries
 size_t pairing_overlap_bytes(int BH, int T);
 cudaError_t launch_pairing(const int32_t* lut, int BH, int Tq, int nh, int ncol, uint16_t* ov, int2* pairs,

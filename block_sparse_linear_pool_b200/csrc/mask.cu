@@ -399,6 +399,11 @@ size_t select_smem_bytes(int Tk) {
   return (size_t)select_rows_per_cta(Tk) * 2 * Tk * sizeof(uint32_t);
 }
 
+cudaError_t launch_logits(const LogitArgs& la, int BH, cudaStream_t s) {
+  logits_kernel<<<dim3((la.Tkv + LT - 1) / LT, (la.Tq + LT - 1) / LT, BH), 256, 0, s>>>(la);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_select(const SelectArgs& a, int BH, cudaStream_t s) {
   LogitArgs la;
   la.Qc = a.Qc;
@@ -407,8 +412,7 @@ cudaError_t launch_select(const SelectArgs& a, int BH, cudaStream_t s) {
   la.d = a.d;
   la.Tq = a.Tq;
   la.Tkv = a.Tkv;
-  logits_kernel<<<dim3((a.Tkv + LT - 1) / LT, (a.Tq + LT - 1) / LT, BH), 256, 0, s>>>(la);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_logits(la, BH, s);
   if (e != cudaSuccess) return e;
   const size_t smem = select_smem_bytes(a.Tkv);
   e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

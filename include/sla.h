@@ -131,6 +131,37 @@ sla_status_t sla_predict_mask(const sla_params_t* p, const void* Q, const void* 
                               void* workspace, size_t workspace_bytes, sla_stream_t stream);
 
 /*
+ * The router's compressed attention ([SLA2] §4 Learnable Router; [SLA] Fig. 4):
+ * P_c = row softmax of the logits that sla_predict_mask ranks (the same pooling,
+ * smooth-K and Wq / Wk projections, the same fp32 logits).
+ * Output (device, caller-allocated, 16-byte aligned):
+ *   Pc  fp32 [B*H][T_q][T_kv]
+ * Uses the workspace of sla_workspace_size.  Errors: SLA_ERR_INVALID_ARG for
+ * NULL or misaligned pointers, SLA_ERR_WORKSPACE, SLA_ERR_CUDA.
+ */
+sla_status_t sla_router_probs(const sla_params_t* p, const void* Q, const void* K,
+                              const float* Wq, const float* Wk, float* Pc, void* workspace,
+                              size_t workspace_bytes, sla_stream_t stream);
+
+/*
+ * SoftTop-k, the training-time replacement of the router's hard row-wise Top-k
+ * ([SLA2] §4 Learnable Router, §6 Training with SLA2):
+ *   M[i][j] = sigmoid((Pc[i][j] - lambda_i) / tau),
+ * lambda_i chosen per row by bisection so that sum_j M[i][j] = n_h (the hard
+ * Top-k's count, sla_block_counts), 40 halvings of [min Pc - 50 tau,
+ * max Pc + 50 tau] in fp32.  As tau -> 0, M becomes the hard mask's critical
+ * set.  The pages fix the sigmoid, tau, the binary search and the row sum;
+ * the target n_h and the input P_c are this library's readings.
+ * Inputs (device): Pc fp32 [B*H][T_q][T_kv] (e.g. from sla_router_probs), tau > 0.
+ * Outputs (device, caller-allocated): M fp32 [B*H][T_q][T_kv], lambda fp32
+ * [B*H][T_q].  Pc and M 16-byte aligned.  No workspace.
+ * Errors: SLA_ERR_INVALID_ARG (NULL or misaligned pointers, tau not a positive
+ * finite number), SLA_ERR_CUDA.
+ */
+sla_status_t sla_soft_topk(const sla_params_t* p, const float* Pc, float tau, float* M,
+                           float* lambda, sla_stream_t stream);
+
+/*
  * Per-key-block linear-attention statistics ([SLA] §2 Q2 step 3, Fig. 4
  * "Linear Attention Precomputation"):
  *   h_j = phi(K_j)^T V_j  (d x d),   z_j = rowsum(phi(K_j)^T)  (d),

@@ -97,6 +97,16 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
     need = bnd.sla_backward_workspace_size(p)
     assert L.sla_backward(ctypes.byref(p), *[dummy] * 15, None, None, None,
                           ctypes.c_void_p(1 << 20), need - 1, None) == 3
+    # router probabilities and SoftTop-k: NULL / misaligned buffers, tau not positive and finite
+    assert L.sla_router_probs(ctypes.byref(p), dummy, dummy, None, None, None, ws, 1024, None) == 1
+    assert L.sla_router_probs(ctypes.byref(p), dummy, dummy, None, None, ctypes.c_void_p(4100), ws,
+                              1024, None) == 1
+    assert L.sla_router_probs(ctypes.byref(p), dummy, dummy, None, None, dummy,
+                              ctypes.c_void_p(4096), 16, None) == 3
+    for tau in (0.0, -1.0, float("nan"), float("inf")):
+        assert L.sla_soft_topk(ctypes.byref(p), dummy, ctypes.c_float(tau), dummy, dummy, None) == 1
+    assert L.sla_soft_topk(ctypes.byref(p), None, ctypes.c_float(0.1), dummy, dummy, None) == 1
+    assert L.sla_soft_topk(ctypes.byref(p), dummy, ctypes.c_float(0.1), dummy, None, None) == 1
 
 
 def test_defaults_are_the_pages_main_method(L):
@@ -116,4 +126,4 @@ def test_workspace_sizes_grow_with_the_problem(L):
 def test_status_strings(L):
     for code, name in bnd.STATUS.items():
         assert L.sla_status_string(code).decode() == name
-    assert L.sla_abi_version() == 102
+    assert L.sla_abi_version() == 103
