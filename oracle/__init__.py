@@ -21,7 +21,12 @@ from .sla import (  # noqa: F401
     feature_map,
     linear_block_stats,
     quantize_e4m3,
+    quantize_int8,
+    LOWBIT_MAX,
+    LOG2E,
+    lowbit_tile,
     pv_fp8_scales,
+    pv_fp8_values,
     sparse_branch_fp8_pv,
     forward_given_mask,
     forward,

@@ -39,8 +39,9 @@ Readings taken where the pages are silent:
   * SoftTop-k ([SLA2] §4, §6) keeps n_h (the hard Top-k's count) per row and
     applies its sigmoid to P_c.
 
-Parity unpinned: the FP8 paths' exact values at full size (the quantiser is
-pinned; the emulations are pinned only on cases where they must be exact).
+Low-bit emulations ([SLA2] §5): ``lowbit_tile`` (Q, K per 64-row tile, E4M3
+or INT8) and ``sparse_branch_fp8_pv`` (E4M3 P and V) are pinned against
+torch's float8_e4m3fn cast, hand-worked values and N x N brute force.
 """
 from __future__ import annotations
 
@@ -290,51 +291,83 @@ def quantize_e4m3(x: np.ndarray) -> np.ndarray:
     return np.sign(x) * q
 
 
-def _fp8_dequant_tile(X: np.ndarray) -> np.ndarray:
-    """Quantise one 64-row tile with scale max|X|/448 and return the
-    dequantised values ([SLA2] §5: tensors mapped to FP8 with scales)."""
-    amax = np.abs(X).max()
+def quantize_int8(y: np.ndarray) -> np.ndarray:
+    """Round to the nearest integer (ties to even) and clamp to [-127, 127]: the
+    symmetric INT8 code of a value already divided by its scale ([SLA2] §5 names
+    INT8 beside FP8 as the low-bit format)."""
+    return np.clip(np.round(np.asarray(y, dtype=np.float64)), -127.0, 127.0)
+
+
+LOWBIT_MAX = {"fp8_e4m3": 448.0, "int8": 127.0}
+
+
+def lowbit_tile(X: np.ndarray, fmt: str) -> np.ndarray:
+    """Quantise one 64-row tile of Q or K with one scale per tile and return the
+    dequantised values ([SLA2] §5: Q and K are mapped to a low-bit format with
+    scales before Q K^T, and the product is rescaled).
+
+    The scale is s = max|X| / R with R = 448 (the largest finite E4M3 value) or
+    127 (symmetric INT8).  The code of each element is an integer decision, so it
+    is taken on the fp32 value X * (R / max|X|) (both factors and the product
+    rounded to fp32), which is the precision a GPU kernel takes it in; the
+    dequantised value is code * s."""
+    R = np.float32(LOWBIT_MAX[fmt])
+    X32 = np.asarray(X, dtype=np.float32)
+    amax = np.float32(np.abs(X32).max()) if X32.size else np.float32(0)
     if amax == 0:
-        return np.zeros_like(X)
-    s = amax / 448.0
-    return quantize_e4m3(X / s) * s
+        return np.zeros(X32.shape, dtype=np.float64)
+    inv = R / amax                       # fp32 division
+    y = (X32 * inv).astype(np.float64)   # fp32 product, exact in fp64
+    code = quantize_e4m3(y) if fmt == "fp8_e4m3" else quantize_int8(y)
+    return code * np.float64(amax / R)
 
 
 def pv_fp8_scales(Vh: np.ndarray) -> np.ndarray:
     """Per-channel scale of one head's V for the FP8 P V product: max_t |V[t, c]| / 448
     (1 where a channel is all zero).  [SLA2] §5 quantises P and V with scales and
-    dequantises their product; with one scale per channel and P on the fixed scale
-    448 (P <= 1), both scales factor out of the sum over keys."""
-    amax = np.abs(Vh).max(axis=0)
-    return np.where(amax > 0, amax / 448.0, 1.0)
+    dequantises their product; with one scale per channel both scales factor out of
+    the sum over keys."""
+    amax = np.abs(np.asarray(Vh, dtype=np.float32)).max(axis=0)
+    return np.where(amax > 0, amax.astype(np.float64) / 448.0, 1.0)
 
 
-def sparse_branch_fp8_pv(q, keys_blocks, vhat_blocks, scale):
-    """o^s of one query block with the FP8 P V product ([SLA2] §5), step by step:
-    critical blocks in ascending order with an online row maximum m (P = exp(s - m)
-    <= 1); on every increase of m the accumulator and the row sum are rescaled;
-    P is quantised as E4M3(448 P); the row sum l uses the unquantised P.
-    Returns (acc, l): o^s = acc * s_V / 448 / l."""
-    rows = q.shape[0]
-    m = np.full(rows, -np.inf)
-    l = np.zeros(rows)
-    acc = np.zeros((rows, vhat_blocks[0].shape[1]))
-    for kj, vj in zip(keys_blocks, vhat_blocks):
-        s = (q @ kj.T) * scale
-        mj = np.maximum(m, s.max(axis=1))
-        f = np.where(np.isfinite(m), np.exp(m - mj), 0.0)
-        acc *= f[:, None]
-        l *= f
-        P = np.exp(s - mj[:, None])
-        l += P.sum(axis=1)
-        acc += quantize_e4m3(448.0 * P) @ vj
-        m = mj
-    return acc, l
+def pv_fp8_values(Vh: np.ndarray) -> np.ndarray:
+    """E4M3 codes of one head's V on its per-channel scale, V / s_V, the division
+    taken as the fp32 product V * (448 / max|V[:, c]|) (an integer decision in
+    the kernel's precision)."""
+    V32 = np.asarray(Vh, dtype=np.float32)
+    amax = np.abs(V32).max(axis=0)
+    inv = np.where(amax > 0, np.float32(448.0) / np.where(amax > 0, amax, np.float32(1)), np.float32(0))
+    return quantize_e4m3((V32 * inv.astype(np.float32)).astype(np.float64))
+
+
+LOG2E = 1.4426950408889634
+
+
+def sparse_branch_fp8_pv(s: np.ndarray, vhat: np.ndarray, sV: np.ndarray) -> np.ndarray:
+    """o^s of a set of query rows with the FP8 P V product ([SLA2] §5: P and V are
+    quantised with scales and their product is dequantised).
+
+    s: the rows' scaled scores over their critical tokens [rows, C]; vhat: the
+    E4M3 codes of those tokens' V on the per-channel scale sV [C, d].
+    Per row, P is taken against the row's maximum score rounded up to a whole
+    power of two: with x = s log2(e) and M = ceil(max x), P = 2^(x - M), so
+    1/2 < max P <= 1 and the row's P scale is an exact power of two.  P is
+    quantised as E4M3(448 P), the product with V^ is dequantised by sV / 448,
+    and the row sum uses the unquantised P:
+        o^s = (E4M3(448 P) V^) sV / 448 / sum(P).
+    The result depends only on the set of critical tokens, not on the order in
+    which a kernel visits them."""
+    x = np.asarray(s, dtype=np.float64) * LOG2E
+    M = np.ceil(x.max(axis=1, keepdims=True))
+    P = np.exp2(x - M)
+    acc = quantize_e4m3(448.0 * P) @ np.asarray(vhat, dtype=np.float64)
+    return acc * np.asarray(sV, dtype=np.float64)[None, :] / 448.0 / P.sum(axis=1, keepdims=True)
 
 
 def forward_given_mask(Q, K, V, Mc, p: OracleParams, proj_w=None, proj_b=None, alpha=None,
                        qblocks: Optional[Sequence[int]] = None, heads: Optional[Sequence] = None,
-                       qk_fp8: bool = False, return_branches: bool = False, pv_fp8: bool = False):
+                       qk: str = "bf16", return_branches: bool = False, pv_fp8: bool = False):
     """SLA / SLA2 output for a given compressed mask M_c.
 
     Q, K, V: [B, H, N, d] (any float dtype; upcast to float64).
@@ -349,9 +382,10 @@ def forward_given_mask(Q, K, V, Mc, p: OracleParams, proj_w=None, proj_b=None, a
       "proj":  O = O^s + O^l W^T + b
       "alpha": O = alpha_h O^s + (1 - alpha_h) O^l
     `qblocks` / `heads` restrict the work to a sample (rows of other blocks are
-    left as NaN).  `qk_fp8` quantises Q and K per 64-row tile to E4M3 before
-    Q K^T ([SLA2] §5); `pv_fp8` computes the sparse branch's P V with E4M3 P and V
-    (``sparse_branch_fp8_pv``); both are emulations of the low-bit path.
+    left as NaN).  `qk` = "fp8_e4m3" or "int8" quantises Q and K per 64-row
+    tile (``lowbit_tile``) before Q K^T ([SLA2] §5); `pv_fp8` computes the sparse
+    branch's P V with E4M3 P and V (``sparse_branch_fp8_pv``); both emulate the
+    low-bit path.
     """
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
@@ -376,31 +410,34 @@ def forward_given_mask(Q, K, V, Mc, p: OracleParams, proj_w=None, proj_b=None, a
         fQ = feature_map(Q[bb, hh], p.phi)
         if pv_fp8:
             sV = pv_fp8_scales(V[bb, hh])
-            Vhat = quantize_e4m3(V[bb, hh] / sV[None, :])
+            Vhat = pv_fp8_values(V[bb, hh])
+        if qk not in ("bf16", "fp8_e4m3", "int8"):
+            raise ValueError(qk)
         for i in qsel:
             qs, qe = block_range(i, p.b_q, N)
             q = Q[bb, hh, qs:qe]
             row = Mc[bb, hh, i]
             # --- sparse branch over critical blocks
             crit = np.nonzero(row == 1)[0]
-            if qk_fp8:
-                q = _fp8_dequant_tile(q)
-            keys, vals = [], []
+            if qk != "bf16":
+                q = lowbit_tile(q, qk)
+            keys, vals, vhat = [], [], []
             for j in crit:
                 ks, ke = block_range(int(j), p.b_kv, N)
                 kj = K[bb, hh, ks:ke]
-                if qk_fp8:
-                    kj = _fp8_dequant_tile(kj)
+                if qk != "bf16":
+                    kj = lowbit_tile(kj, qk)
                 keys.append(kj)
                 vals.append(V[bb, hh, ks:ke])
-            if keys and pv_fp8:
-                vhat = [Vhat[slice(*block_range(int(j), p.b_kv, N))] for j in crit]
-                acc, lsum = sparse_branch_fp8_pv(q, keys, vhat, scale)
-                o_s = acc * sV[None, :] / 448.0 / lsum[:, None]
-            elif keys:
+                if pv_fp8:
+                    vhat.append(Vhat[ks:ke])
+            if keys:
                 kk = np.concatenate(keys, axis=0)
-                vv = np.concatenate(vals, axis=0)
                 s = (q @ kk.T) * scale
+            if keys and pv_fp8:
+                o_s = sparse_branch_fp8_pv(s, np.concatenate(vhat, axis=0), sV)
+            elif keys:
+                vv = np.concatenate(vals, axis=0)
                 m = s.max(axis=1, keepdims=True)
                 e = np.exp(s - m)
                 o_s = (e @ vv) / e.sum(axis=1, keepdims=True)

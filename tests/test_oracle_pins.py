@@ -290,10 +290,163 @@ def test_mask_grading_excludes_near_ties():
     np.testing.assert_array_equal(g[0], [True, False, False, True, True])
 
 
+# ---------------------------------------------------------------- low-bit Q, K tiles
+def _tiles_with_different_ranges(seed, d=32):
+    """Three 64-row tiles and a partial one whose magnitudes differ by orders of
+    magnitude, so that a per-tensor scale or a scale taken over the wrong rows
+    cannot pass."""
+    rng = np.random.default_rng(seed)
+    parts = [rng.standard_normal((64, d)) * s for s in (0.01, 1.0, 40.0)] + [rng.standard_normal((20, d)) * 3.0]
+    X = np.concatenate(parts)
+    return torch.from_numpy(X).to(torch.bfloat16).double().numpy()  # bf16 values, as the kernels see them
+
+
+def _torch_tile_dequant(X, fmt):
+    """Per-64-row-tile quantisation with torch: E4M3 through the float8_e4m3fn cast,
+    INT8 through round-half-even and clamping; scale max|tile| / R."""
+    R = 448.0 if fmt == "fp8_e4m3" else 127.0
+    out = np.empty_like(X)
+    for s in range(0, X.shape[0], 64):
+        t = torch.from_numpy(X[s:s + 64]).float()
+        amax = t.abs().max()
+        y = t * (torch.tensor(R, dtype=torch.float32) / amax)
+        code = y.to(torch.float8_e4m3fn).double() if fmt == "fp8_e4m3" else torch.round(y).clamp(-127, 127).double()
+        out[s:s + 64] = (code * (amax / R).double()).numpy()
+    return out
+
+
+@pytest.mark.parametrize("fmt", ["fp8_e4m3", "int8"])
+def test_lowbit_tile_per_64_row_tile_against_torch(fmt):
+    X = _tiles_with_different_ranges(40)
+    got = np.concatenate([O.lowbit_tile(X[s:s + 64], fmt) for s in range(0, X.shape[0], 64)])
+    np.testing.assert_array_equal(got, _torch_tile_dequant(X, fmt))
+
+
+@pytest.mark.parametrize("fmt", ["fp8_e4m3", "int8"])
+def test_lowbit_tile_error_bounds_and_range(fmt):
+    # each tile's largest element maps to the format's largest code, and every
+    # element is within the format's rounding bound of its own tile's scale:
+    # E4M3 half a step (2^-4 relative in the normal range, 2^-10 s below it),
+    # INT8 half a step (s / 2).  A swapped (448 / max) or per-tensor scale breaks both.
+    X = _tiles_with_different_ranges(41)
+    R = O.LOWBIT_MAX[fmt]
+    for s in range(0, X.shape[0], 64):
+        t = X[s:s + 64]
+        q = O.lowbit_tile(t, fmt)
+        amax = np.abs(t).max()
+        sc = amax / R
+        assert abs(np.abs(q).max() - amax) <= 1e-6 * amax
+        err = np.abs(q - t)
+        if fmt == "int8":
+            assert (err <= 0.5 * sc * (1 + 1e-4)).all()  # + the fp32 rounding of x * (R / max)
+            codes = q / np.float64(np.float32(amax) / np.float32(R))
+            np.testing.assert_allclose(codes, np.round(codes), atol=1e-9)
+        else:
+            normal = np.abs(t) >= 2.0 ** -6 * sc
+            assert (err[normal] <= 2.0 ** -4 * np.abs(t[normal]) * (1 + 1e-4)).all()
+            assert (err[~normal] <= 2.0 ** -10 * sc * (1 + 1e-4)).all()
+
+
+def test_lowbit_tile_int8_exact_on_its_grid():
+    c = 0.37
+    ints = np.random.default_rng(42).integers(-127, 128, size=(64, 16)).astype(np.float64)
+    ints[0, 0] = 127.0
+    X = ints * c
+    np.testing.assert_allclose(O.lowbit_tile(X, "int8"), X, rtol=1e-6, atol=0)
+
+
+def _sparse_case(seed, N=200, d=16, alpha_one=True):
+    rng = np.random.default_rng(seed)
+    B, H = 1, 1
+    T = O.num_blocks(N, 64)
+    Q = np.concatenate([rng.standard_normal((B, H, 64, d)) * s for s in (0.3, 2.0, 0.05, 8.0)], axis=2)[:, :, :N]
+    K = np.concatenate([rng.standard_normal((B, H, 64, d)) * s for s in (5.0, 0.1, 1.0, 0.7)], axis=2)[:, :, :N]
+    V = rng.standard_normal((B, H, N, d)) * np.linspace(0.2, 3.0, d)
+    Q, K, V = (torch.from_numpy(x).to(torch.bfloat16).double().numpy() for x in (Q, K, V))
+    Mc = np.full((B, H, T, T), -1, dtype=np.int8)
+    for i in range(T):  # two critical blocks per row (no marginal ones), a different pair per row
+        Mc[0, 0, i, [(i + 1) % T, (3 * i) % T if (3 * i) % T != (i + 1) % T else (i + 2) % T]] = 1
+    return Q, K, V, Mc
+
+
+@pytest.mark.parametrize("fmt", ["fp8_e4m3", "int8"])
+def test_lowbit_qk_forward_is_block_sparse_attention_on_dequantised_tiles(fmt):
+    # brute force: Q, K dequantised tile by tile with torch, N x N scores with -inf
+    # outside the critical blocks, torch SDPA; alpha = 1 and no marginal blocks.
+    Q, K, V, Mc = _sparse_case(43)
+    N = Q.shape[2]
+    Qd = _torch_tile_dequant(Q[0, 0], fmt)
+    Kd = _torch_tile_dequant(K[0, 0], fmt)
+    allow = torch.from_numpy(_token_mask(Mc[0, 0], 1, 64, N))
+    ref = F.scaled_dot_product_attention(torch.from_numpy(Qd)[None], torch.from_numpy(Kd)[None],
+                                         torch.from_numpy(V[0, 0])[None], attn_mask=allow)[0].numpy()
+    p = O.OracleParams(combine="alpha")
+    got = O.forward_given_mask(Q, K, V, Mc, p, alpha=np.ones((1, 1)), qk=fmt)[0, 0]
+    np.testing.assert_allclose(got, ref, rtol=1e-10, atol=1e-12)
+    # and the quantisation is not the identity
+    plain = O.forward_given_mask(Q, K, V, Mc, p, alpha=np.ones((1, 1)))[0, 0]
+    assert np.abs(got - plain).max() > 1e-4 * np.abs(plain).max()
+
+
 # ---------------------------------------------------------------- FP8 P V emulation
+def _golden_fp8_pv():
+    vals = {}
+    for line in open(os.path.join(GOLDEN, "fp8_pv_tiny.txt")):
+        line = line.split("#")[0].strip()
+        if line:
+            k, rest = line.split(None, 1)
+            vals[k] = np.array([[float(x) for x in r.split()] for r in rest.split("|")])
+    return vals
+
+
+def test_fp8_pv_hand_worked_case():
+    g = _golden_fp8_pv()
+    V = g["V"]
+    np.testing.assert_array_equal(O.pv_fp8_values(V), g["Vhat"])
+    np.testing.assert_array_equal(O.pv_fp8_scales(V), [1 / 448, 3 / 448])
+    s = g["x"] * math.log(2.0)  # scores in natural-log units
+    got = O.sparse_branch_fp8_pv(s, g["Vhat"], O.pv_fp8_scales(V))
+    np.testing.assert_allclose(got, g["o"], rtol=1e-13)
+
+
+def test_fp8_pv_forward_against_n_by_n_brute_force():
+    # the whole N x N score matrix, -inf outside the critical blocks; per row
+    # M = ceil(max s log2 e), P = 2^(s log2 e - M); E4M3 by torch's float8 cast
+    Q, K, V, Mc = _sparse_case(44)
+    N, d = Q.shape[2], Q.shape[3]
+    allow = _token_mask(Mc[0, 0], 1, 64, N)
+    S = np.where(allow, (Q[0, 0] @ K[0, 0].T) / math.sqrt(d), -np.inf)
+    x = S * math.log2(math.e)
+    M = np.ceil(x.max(axis=1, keepdims=True))
+    P = np.where(allow, np.exp2(x - M), 0.0)
+    f8 = lambda a: torch.from_numpy(a).to(torch.float8_e4m3fn).double().numpy()  # noqa: E731
+    V32 = torch.from_numpy(V[0, 0]).float()
+    amax = V32.abs().max(dim=0).values
+    Vhat = f8((V32 * (torch.tensor(448.0) / amax)).double().numpy())
+    ref = (f8(448.0 * P) @ Vhat) * (amax.double().numpy() / 448.0) / 448.0 / P.sum(axis=1, keepdims=True)
+    p = O.OracleParams(combine="alpha")
+    got = O.forward_given_mask(Q, K, V, Mc, p, alpha=np.ones((1, 1)), pv_fp8=True)[0, 0]
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-13)
+
+
+def test_fp8_pv_is_independent_of_token_order_and_whole_power_of_two_shifts():
+    rng = np.random.default_rng(45)
+    s = rng.standard_normal((8, 300)) * 3.0
+    V = rng.standard_normal((300, 16))
+    vh, sV = O.pv_fp8_values(V), O.pv_fp8_scales(V)
+    base = O.sparse_branch_fp8_pv(s, vh, sV)
+    perm = rng.permutation(300)
+    np.testing.assert_allclose(O.sparse_branch_fp8_pv(s[:, perm], vh[perm], sV), base, rtol=1e-13, atol=1e-15)
+    # adding 3 ln 2 to a row moves M by exactly 3 and leaves every P (and o) unchanged
+    np.testing.assert_allclose(O.sparse_branch_fp8_pv(s + 3 * math.log(2.0), vh, sV), base, rtol=1e-13, atol=1e-15)
+    # ... while a shift that is not a whole power of two changes the rounding
+    assert np.abs(O.sparse_branch_fp8_pv(s + 0.3, vh, sV) - base).max() > 0
+
+
 def test_fp8_pv_is_exact_when_p_and_v_are_on_the_grid():
-    # Q = 0: every score is 0, so P = 1 (E4M3(448) is exact); V in {0, +-1, 2, 4, 8} has
-    # per-channel amax 8 and V / s_V in {0, +-56, 112, 224, 448}, all E4M3 values.
+    # Q = 0: every score is 0, so M = 0 and P = 1 (E4M3(448) is exact); V in
+    # {0, +-1, 2, 4, 8} has per-channel amax 8 and V / s_V in {0, +-56, 112, 224, 448},
+    # all E4M3 values.
     rng = np.random.default_rng(11)
     B, H, N, d = 1, 1, 192, 8
     Q = np.zeros((B, H, N, d))
@@ -311,9 +464,9 @@ def test_fp8_pv_is_exact_when_p_and_v_are_on_the_grid():
     np.testing.assert_allclose(fp8, exact, rtol=0, atol=1e-12)
 
 
-def test_fp8_pv_online_form_equals_softmax_without_rounding(monkeypatch):
-    # with the quantiser replaced by the identity, the online step-by-step form is
-    # plain softmax attention over the critical tokens
+def test_fp8_pv_without_rounding_is_softmax_attention(monkeypatch):
+    # with the quantiser replaced by the identity, the FP8 P V form is plain softmax
+    # attention over the critical tokens (up to the fp32 rounding of V * 448 / max|V|)
     rng = np.random.default_rng(12)
     B, H, N, d = 1, 2, 200, 16
     Q, K, V = (rng.standard_normal((B, H, N, d)) for _ in range(3))
@@ -325,19 +478,5 @@ def test_fp8_pv_online_form_equals_softmax_without_rounding(monkeypatch):
     exact = O.forward_given_mask(Q, K, V, Mc, p, alpha=a)
     import oracle.sla as S
     monkeypatch.setattr(S, "quantize_e4m3", lambda x: np.asarray(x, dtype=np.float64))
-    online = S.forward_given_mask(Q, K, V, Mc, p, alpha=a, pv_fp8=True)
-    np.testing.assert_allclose(online, exact, rtol=1e-10, atol=1e-12)
-
-
-def test_fp8_pv_rounds_something_on_generic_inputs():
-    rng = np.random.default_rng(13)
-    B, H, N, d = 1, 1, 128, 16
-    Q, K, V = (rng.standard_normal((B, H, N, d)) for _ in range(3))
-    T = O.num_blocks(N, 64)
-    Mc = np.ones((B, H, T, T), dtype=np.int8)
-    p = O.OracleParams(k_h=1.0, k_l=0.0, combine="alpha")
-    a = np.ones((B, H))
-    exact = O.forward_given_mask(Q, K, V, Mc, p, alpha=a)
-    fp8 = O.forward_given_mask(Q, K, V, Mc, p, alpha=a, pv_fp8=True)
-    err = np.abs(fp8 - exact).max() / np.abs(exact).max()
-    assert 1e-4 < err < 0.1
+    ident = S.forward_given_mask(Q, K, V, Mc, p, alpha=a, pv_fp8=True)
+    np.testing.assert_allclose(ident, exact, rtol=1e-6, atol=1e-6)
