@@ -565,8 +565,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(I.WORKLOADS))
     ap.add_argument("--no-extras", action="store_true", help="skip e2e, dense baseline and CPU baseline")
-    ap.add_argument("--qk", choices=["bf16", "fp8_e4m3"], default="bf16",
-                    help="precision of Q K^T on critical blocks (fp8_e4m3: d = 128 only)")
+    ap.add_argument("--qk", choices=["bf16", "fp8_e4m3", "int8"], default="bf16",
+                    help="precision of Q K^T on critical blocks (fp8_e4m3, int8: d = 128 only)")
     ap.add_argument("--pv", choices=["bf16", "fp8_e4m3"], default="bf16",
                     help="precision of P V on critical blocks (fp8_e4m3: d = 128 only)")
     ap.add_argument("--heads", type=int, default=None, help="override the workload's head count "

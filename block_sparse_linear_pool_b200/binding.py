@@ -19,7 +19,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsla.so")
 
 SLA_COMBINE_PROJ, SLA_COMBINE_ALPHA = 0, 1
-SLA_QK_BF16, SLA_QK_FP8_E4M3 = 0, 1
+SLA_QK_BF16, SLA_QK_FP8_E4M3, SLA_QK_INT8 = 0, 1, 2
+_QK_PREC = {"bf16": SLA_QK_BF16, "fp8_e4m3": SLA_QK_FP8_E4M3, "int8": SLA_QK_INT8}
 SLA_PHI_SOFTMAX, SLA_PHI_ELU1 = 0, 1
 
 STATUS = {
@@ -127,7 +128,7 @@ class SlaConfig:
     k_h: float
     k_l: float
     combine: str = "proj"     # "proj" (SLA) or "alpha" (SLA2)
-    qk: str = "bf16"          # "bf16" or "fp8_e4m3"
+    qk: str = "bf16"          # "bf16", "fp8_e4m3" or "int8" (Q K^T of critical blocks, [SLA2] §5)
     smooth_k: bool = False
     eps: float = 1e-5
     phi: str = "softmax"      # "softmax" ([SLA] Fig. 4) or "elu1" ([SLA] Table 2 ablation)
@@ -140,7 +141,9 @@ def make_params(Q: torch.Tensor, cfg: SlaConfig, K=None, V=None, O=None) -> sla_
     p = sla_params_t()
     lib().sla_params_default(ctypes.byref(p), B, H, N, d, cfg.k_h, cfg.k_l,
                              SLA_COMBINE_PROJ if cfg.combine == "proj" else SLA_COMBINE_ALPHA)
-    p.qk_prec = SLA_QK_BF16 if cfg.qk == "bf16" else SLA_QK_FP8_E4M3
+    if cfg.qk not in _QK_PREC:
+        raise ValueError(f"qk must be one of {sorted(_QK_PREC)}, not {cfg.qk!r}")
+    p.qk_prec = _QK_PREC[cfg.qk]
     p.smooth_k = int(cfg.smooth_k)
     p.eps = cfg.eps
     if cfg.phi not in ("softmax", "elu1"):

@@ -20,7 +20,8 @@ constexpr size_t kAlign = 256;
 
 struct Plan {
   int B, H, N, d, BH, Tq, Tkv, nh, nl, NN, Tkvp;
-  bool fp8;  // Q K^T on E4M3 with per-block scales
+  bool fp8;  // Q K^T on 8-bit codes (E4M3 or INT8) with per-block scales
+  bool qk_int8;  // ... INT8 (else E4M3)
   bool pv8;  // P V on E4M3 (P on the fixed scale 448, V per (head, channel))
   int phi;   // sla_phi_t
   bool all;  // linear branch over every key block
@@ -94,11 +95,12 @@ sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
   if (!(p->k_h >= 0.f && p->k_h <= 1.f && p->k_l >= 0.f && p->k_l <= 1.f)) return SLA_ERR_INVALID_ARG;
   if (!(p->eps >= 0.f) || !std::isfinite(p->eps)) return SLA_ERR_INVALID_ARG;
   if (p->combine != SLA_COMBINE_PROJ && p->combine != SLA_COMBINE_ALPHA) return SLA_ERR_INVALID_ARG;
-  if (p->qk_prec != SLA_QK_BF16 && p->qk_prec != SLA_QK_FP8_E4M3) return SLA_ERR_INVALID_ARG;
+  if (p->qk_prec != SLA_QK_BF16 && p->qk_prec != SLA_QK_FP8_E4M3 && p->qk_prec != SLA_QK_INT8)
+    return SLA_ERR_INVALID_ARG;
   if (p->phi != SLA_PHI_SOFTMAX && p->phi != SLA_PHI_ELU1) return SLA_ERR_INVALID_ARG;
   if (p->linear_over_all != 0 && p->linear_over_all != 1) return SLA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return SLA_ERR_UNSUPPORTED;
-  if (p->qk_prec == SLA_QK_FP8_E4M3 && p->d != 128) return SLA_ERR_UNSUPPORTED;
+  if (p->qk_prec != SLA_QK_BF16 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if (p->pv_prec != SLA_PV_BF16 && p->pv_prec != SLA_PV_FP8_E4M3) return SLA_ERR_INVALID_ARG;
   if (p->pv_prec == SLA_PV_FP8_E4M3 && p->d != 128) return SLA_ERR_UNSUPPORTED;
   if (p->b_q != 64 || p->b_kv != 64) return SLA_ERR_UNSUPPORTED;
@@ -116,7 +118,8 @@ sla_status_t make_plan(const sla_params_t* p, Plan* pl) {
   counts(pl->Tkv, p->k_h, p->k_l, &pl->nh, &pl->nl);
   pl->NN = p->d * p->d + p->d;
   pl->Tkvp = (pl->Tkv + 7) & ~7;
-  pl->fp8 = p->qk_prec == SLA_QK_FP8_E4M3;
+  pl->fp8 = p->qk_prec != SLA_QK_BF16;
+  pl->qk_int8 = p->qk_prec == SLA_QK_INT8;
   pl->pv8 = p->pv_prec == SLA_PV_FP8_E4M3;
   pl->phi = p->phi;
   pl->all = p->linear_over_all != 0;
@@ -359,6 +362,7 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
     qa.N = pl.N;
     qa.Tq = pl.Tq;
     qa.Tkv = pl.Tkv;
+    qa.int8 = pl.qk_int8 ? 1 : 0;
     SLA_TRY(cuda_status(launch_quant_fp8(qa, pl.BH, s)));
     const uint64_t dq[3] = {(uint64_t)pl.d, (uint64_t)pl.Tq * 64, (uint64_t)pl.BH};
     const uint64_t sq[2] = {(uint64_t)pl.d, (uint64_t)pl.Tq * 64 * pl.d};
@@ -411,7 +415,8 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.os = o_sparse;
   a.vmax = vmax;
   a.pairs = pairs;
-  return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, pl.fp8, pl.pv8, pl.BH, s));
+  const int qk8 = pl.fp8 ? (pl.qk_int8 ? 2 : 1) : 0;
+  return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, qk8, pl.pv8, pl.BH, s));
 }
 
 sla_status_t forward_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
@@ -775,7 +780,9 @@ sla_status_t sla_soft_topk(const sla_params_t* p, const float* Pc, float tau, fl
   Plan pl;
   SLA_TRY(make_plan(p, &pl));
   if (!Pc || !M || !lambda || !aligned16(Pc) || !aligned16(M)) return SLA_ERR_INVALID_ARG;
-  if (!(tau > 0.f) || !std::isfinite(tau)) return SLA_ERR_INVALID_ARG;
+  // the kernel divides by tau in fp32: tau below the normal range (or whose
+  // reciprocal overflows) would turn (P - lambda) / tau into inf * 0 = NaN
+  if (!(tau >= 1.1754944e-38f) || !std::isfinite(tau) || !std::isfinite(1.f / tau)) return SLA_ERR_INVALID_ARG;
   return cuda_status(launch_soft_topk(Pc, M, lambda, pl.Tkv, (int64_t)pl.BH * pl.Tq, pl.nh, tau,
                                       reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -915,7 +922,6 @@ sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, c
                         (const void*)dV, hz})
     if (!aligned16(x)) return SLA_ERR_INVALID_ARG;
   if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
-  if (p->qk_prec != SLA_QK_BF16 && p->qk_prec != SLA_QK_FP8_E4M3) return SLA_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
       workspace_bytes < bwd_layout_of(pl).end)
     return SLA_ERR_WORKSPACE;

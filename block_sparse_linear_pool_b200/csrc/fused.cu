@@ -31,11 +31,12 @@
 // O [128,128+d).  After the last P V the S/P region [0,d) holds L_a; once the
 // rows of query block 2p have been written out it holds L_b.
 //
-// Low-bit variant ([SLA2] §5): Q and K arrive as E4M3 with one scale per
-// (head, 64-row block) and S = Q^ K^^T runs as tcgen05.mma kind::f8f6f4; the
-// softmax multiplies the scores by s_Q s_K.  The FP8 Q tile
-// and K ring are half the size, so the bf16 Q tile (needed for phi(Q)) fits
-// beside them and H_a loads over the FP8 Q tile and K ring.
+// Low-bit variant ([SLA2] §5): Q and K arrive as 8-bit codes (E4M3, or
+// symmetric INT8) with one scale per (head, 64-row block) and S = Q^ K^^T runs
+// as tcgen05.mma kind::f8f6f4 (fp32 accumulate) or kind::i8 (int32 accumulate);
+// the softmax multiplies the scores by s_Q s_K.  The 8-bit Q tile and K ring are
+// half the size, so the bf16 Q tile (needed for phi(Q)) fits beside them and
+// H_a loads over the 8-bit Q tile and K ring.
 //
 // Linear branch with unnormalised feature map: for e_a = 2^((q_a - max q) log2 e)
 // and s = sum_a e_a, phi(q) = e / s, so
@@ -45,7 +46,8 @@
 // FP8 P V (PV8, [SLA2] §5: P and V quantised, their product dequantised): V
 // arrives as E4M3 with one scale per (head, channel), transposed per key block
 // ([d rows][64 tokens, padded to 128 B]: the K-major B operand); the running
-// maximum is updated on every increase (no lazy rescale), so P <= 1 and
+// maximum is kept in whole log2 units and raised on every increase (no lazy
+// rescale), so P <= 1, every rescale of O is an exact power of two, and
 // P^ = E4M3(448 P) is written over S (four values per TMEM column); O += P^ V^
 // runs as kind::f8f6f4 with P^ read from TMEM, and the epilogue applies
 // s_V[c] / 448.  The row sum l uses the unquantised P.
@@ -91,15 +93,22 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^n for a whole number n <= 0, exactly (0 below the normal range)
+__device__ __forceinline__ float exp2_whole(float n) {
+  const int e = 127 + __float2int_rn(n);
+  return e > 0 ? __int_as_float(e << 23) : 0.f;
+}
+
 }  // namespace
 
-template <int D, bool FP8, bool PV8>
+template <int D, int QK8, bool PV8>
 __global__ void __launch_bounds__(192, 2)
     sla_fused_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                      const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapH,
                      const __grid_constant__ CUtensorMap mapZ, const __grid_constant__ CUtensorMap mapQ8,
                      const __grid_constant__ CUtensorMap mapK8, FusedArgs a) {
-  static_assert(!FP8 || D == 128, "the FP8 path is built for d = 128");
+  constexpr bool FP8 = QK8 != 0;  // 8-bit Q K^T: 1 E4M3 (kind::f8f6f4), 2 INT8 (kind::i8)
+  static_assert(!FP8 || D == 128, "the 8-bit Q K^T path is built for d = 128");
   static_assert(!PV8 || D == 128, "the FP8 P V path is built for d = 128");
   using L = FusedSmem<D, FP8>;
   constexpr int NR = L::NR;
@@ -292,7 +301,7 @@ __global__ void __launch_bounds__(192, 2)
     // ---------------- MMA issuer
     if (ln == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
-      const uint32_t id_s8 = idesc_e4m3(128, 64);
+      const uint32_t id_s8 = QK8 == 2 ? idesc_s8(128, 64) : idesc_e4m3(128, 64);
       const uint32_t id_pv = idesc_bf16(128, D, false, true);
       const uint32_t id_pv8 = idesc_e4m3(128, D);
       const uint32_t id_l = idesc_bf16(128, D, false, false);
@@ -337,7 +346,10 @@ __global__ void __launch_bounds__(192, 2)
           for (int kk = 0; kk < D / 32; ++kk) {
             const uint64_t ad = sdesc_sw128(q8 + kk * 32, 16, 1024);
             const uint64_t bd = sdesc_sw128(kt + kk * 32, 16, 1024);
-            umma_ss_f8(tbase + COL_S + 64 * (k & 1), ad, bd, id_s8, kk > 0 ? 1u : 0u);
+            if (QK8 == 2)
+              umma_ss_i8(tbase + COL_S + 64 * (k & 1), ad, bd, id_s8, kk > 0 ? 1u : 0u);
+            else
+              umma_ss_f8(tbase + COL_S + 64 * (k & 1), ad, bd, id_s8, kk > 0 ? 1u : 0u);
           }
         } else {
 #pragma unroll
@@ -397,6 +409,13 @@ __global__ void __launch_bounds__(192, 2)
         tmem_ld32(ts, s0);
         tmem_ld32(ts + 32, s1);
         tmem_ld_wait();
+        if (QK8 == 2) {  // int32 dot products of the INT8 codes (exact in fp32: |S| < 2^24)
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            s0[c] = __float_as_uint((float)(int)s0[c]);
+            s1[c] = __float_as_uint((float)(int)s1[c]);
+          }
+        }
         const int nvalid = a.N - 64 * (int)uidx[k];
         if (nvalid < 64) {  // partial last key block: padding columns get -inf
 #pragma unroll
@@ -412,13 +431,17 @@ __global__ void __launch_bounds__(192, 2)
         for (int st = 16; st >= 1; st >>= 1)
 #pragma unroll
           for (int c = 0; c < st; ++c) t[c] = fmaxf(t[c], t[c + st]);
-        // FP8 scores carry the two block scales: s = (q^ . k^) s_Q s_K
+        // 8-bit scores carry the two block scales: s = (q^ . k^) s_Q s_K
         const float sc = FP8 ? sl2 * sq_half * usk[k] : sl2;
         const float mx = t[0] * sc;
-        // lazy rescale: keep the running max unless it grows by more than 2^8
+        // lazy rescale: keep the running max unless it grows by more than 2^8.
+        // FP8 P V: the running max is kept in whole log2 units (the row max
+        // rounded up), so every rescale is an exact power of two and the final
+        // E4M3(448 P) values do not depend on the order of the critical blocks.
+        const float mt = PV8 ? ceilf(mx) : mx;
         const bool first = (m == -INFINITY);
-        const bool grow = !first && (mx - m > (PV8 ? 0.f : RESCALE_THRESHOLD));
-        if (first) m = mx;  // O and l of this row are still exactly 0
+        const bool grow = !first && (mt - m > (PV8 ? 0.f : RESCALE_THRESHOLD));
+        if (first) m = mt;  // O and l of this row are still exactly 0
         if (__any_sync(0xffffffffu, grow)) {
           // O must hold P_{k-1} V_{k-1} before it is rescaled
           if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[(k - 1) & 1], ((k - 1) >> 1) & 1, a.err,
@@ -427,7 +450,7 @@ __global__ void __launch_bounds__(192, 2)
             break;
           }
           tc_fence_after();
-          const float f = grow ? ex2(m - mx) : 1.f;
+          const float f = grow ? (PV8 ? exp2_whole(m - mt) : ex2(m - mx)) : 1.f;
 #pragma unroll 1
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
@@ -440,7 +463,7 @@ __global__ void __launch_bounds__(192, 2)
           tmem_st_wait();
           if (grow) {
             l *= f;
-            m = mx;
+            m = mt;
           }
         }
         const float nm = -m;
@@ -618,31 +641,31 @@ __global__ void __launch_bounds__(192, 2)
   }
 }
 
-template <int D, bool FP8, bool PV8>
+template <int D, int QK8, bool PV8>
 static cudaError_t launch_fused_t(const CUtensorMap& mapQ, const CUtensorMap& mapK,
                                   const CUtensorMap& mapV, const CUtensorMap& mapH,
                                   const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
                                   const CUtensorMap& mapK8, const FusedArgs& a, int BH,
                                   cudaStream_t s) {
-  const size_t smem = FusedSmem<D, FP8>::bytes(a.Tkv);
-  cudaError_t e = cudaFuncSetAttribute(sla_fused_kernel<D, FP8, PV8>,
+  const size_t smem = FusedSmem<D, (QK8 != 0)>::bytes(a.Tkv);
+  cudaError_t e = cudaFuncSetAttribute(sla_fused_kernel<D, QK8, PV8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.Tq + 1) / 2, BH);
-  sla_fused_kernel<D, FP8, PV8><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a);
+  sla_fused_kernel<D, QK8, PV8><<<grid, 192, smem, s>>>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                          const CUtensorMap& mapH, const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
-                         const CUtensorMap& mapK8, const FusedArgs& a, int D, bool fp8, bool pv8, int BH,
+                         const CUtensorMap& mapK8, const FusedArgs& a, int D, int qk8, bool pv8, int BH,
                          cudaStream_t s) {
-  if (pv8)
-    return fp8 ? launch_fused_t<128, true, true>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s)
-               : launch_fused_t<128, false, true>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
-  if (fp8) return launch_fused_t<128, true, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
-  return D == 128 ? launch_fused_t<128, false, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s)
-                  : launch_fused_t<64, false, false>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s);
+#define SLA_FUSED(d_, q_, p_) launch_fused_t<d_, q_, p_>(mapQ, mapK, mapV, mapH, mapZ, mapQ8, mapK8, a, BH, s)
+  if (pv8) return qk8 == 2 ? SLA_FUSED(128, 2, true) : (qk8 == 1 ? SLA_FUSED(128, 1, true) : SLA_FUSED(128, 0, true));
+  if (qk8 == 2) return SLA_FUSED(128, 2, false);
+  if (qk8 == 1) return SLA_FUSED(128, 1, false);
+  return D == 128 ? SLA_FUSED(128, 0, false) : SLA_FUSED(64, 0, false);
+#undef SLA_FUSED
 }
 
 }  // namespace sla

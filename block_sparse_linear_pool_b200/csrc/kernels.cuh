@@ -54,6 +54,7 @@ struct QuantArgs {
   float* scale_q;      // [BH][T_q]
   float* scale_k;      // [BH][T_kv]
   int H, N, Tq, Tkv;
+  int int8;            // 1: symmetric INT8 codes (scale max/127), 0: E4M3 (scale max/448)
 };
 
 struct FusedArgs {
@@ -68,8 +69,8 @@ struct FusedArgs {
   int combine;            // 0 proj, 1 alpha
   float scale_log2;       // log2(e) / sqrt(d)
   float eps;
-  const float* scale_q;   // FP8 path: per (head, query block) scale of Q, else nullptr
-  const float* scale_k;   // FP8 path: per (head, key block) scale of K, else nullptr
+  const float* scale_q;   // 8-bit Q K^T: per (head, query block) scale of Q, else nullptr
+  const float* scale_k;   // 8-bit Q K^T: per (head, key block) scale of K, else nullptr
   int phi;                // 0 softmax over d, 1 elu + 1
   float* lse;             // [BH][N] natural-log sum of exp of the scaled critical scores, or nullptr
   float* os;              // [BH][N][d] the sparse branch's output o^s (fp32), or nullptr
@@ -178,10 +179,10 @@ cudaError_t launch_quant_fp8(const QuantArgs& a, int BH, cudaStream_t s);
 cudaError_t launch_vquant_fp8(const __nv_bfloat16* V, const int64_t* sv, int H, int N, int T, int BH, int D,
                               unsigned int* vmax, uint8_t* V8T, cudaStream_t s);
 
-// mapQ8 / mapK8 are used only when fp8 is set (d = 128 only).
+// qk8: 0 bf16 Q K^T, 1 E4M3, 2 INT8; mapQ8 / mapK8 are used only for qk8 != 0 (d = 128 only).
 cudaError_t launch_fused(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
                          const CUtensorMap& mapH, const CUtensorMap& mapZ, const CUtensorMap& mapQ8,
-                         const CUtensorMap& mapK8, const FusedArgs& a, int D, bool fp8, bool pv8, int BH,
+                         const CUtensorMap& mapK8, const FusedArgs& a, int D, int qk8, bool pv8, int BH,
                          cudaStream_t s);
 
 }  // namespace sla

@@ -2,9 +2,11 @@
 // Learnable Routing and QAT", §5: Q and K are mapped to FP8 with scales before
 // Q K^T, and the product is rescaled).
 //
-// One scale per (head, 64-row block): s = max|x| / 448 (448 = largest finite
-// E4M3 value), x_q = round-to-nearest-even(x / s) with saturation.  Rows past N
-// in the last block are written as zeros, so every block occupies 64 rows.
+// One scale per (head, 64-row block): s = max|x| / R with R = 448 (the largest
+// finite E4M3 value) or 127 (symmetric INT8, the other low-bit format the page
+// names); the code is the round-to-nearest-even of x * (R / max|x|) (E4M3 with
+// saturation; INT8 clamped to [-127, 127]).  Rows past N in the last block are
+// written as zeros, so every block occupies 64 rows.
 #include <cuda_fp8.h>
 
 #include "kernels.cuh"
@@ -45,9 +47,29 @@ __global__ void __launch_bounds__(128) quant_fp8_kernel(QuantArgs a) {
   if ((t & 31) == 0) red[t >> 5] = amax;
   __syncthreads();
   amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  const float s = amax > 0.f ? amax / 448.f : 1.f;
-  const float inv = amax > 0.f ? 448.f / amax : 0.f;
+  const float R = a.int8 ? 127.f : 448.f;
+  const float s = amax > 0.f ? amax / R : 1.f;
+  const float inv = amax > 0.f ? R / amax : 0.f;
   uint8_t* out = dst + ((int64_t)bh * T * 64 + 64 * blk + row) * 128 + c0;
+  if (a.int8) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      uint32_t w[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        uint32_t word = 0;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int c = min(max(__float2int_rn(x[16 * v + 4 * u + b] * inv), -127), 127);
+          word |= (uint32_t)(c & 0xff) << (8 * b);
+        }
+        w[u] = word;
+      }
+      reinterpret_cast<uint4*>(out)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (t == 0) scale[(int64_t)bh * T + blk] = s;
+    return;
+  }
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
     uint32_t w[4];

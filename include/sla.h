@@ -56,16 +56,20 @@ typedef enum {
 
 typedef enum {
   SLA_QK_BF16 = 0,      /* Q K^T of critical blocks in bf16, fp32 accumulate */
-  SLA_QK_FP8_E4M3 = 1   /* [SLA2] §5: Q, K quantised to E4M3 with one scale per
+  SLA_QK_FP8_E4M3 = 1,  /* [SLA2] §5: Q, K quantised to E4M3 with one scale per
                            64-row block (max|x|/448) before Q K^T */
+  SLA_QK_INT8 = 2       /* [SLA2] §5 (low-bit tensors "such as INT8 or FP8"): Q, K
+                           quantised to symmetric INT8 codes in [-127, 127] with one
+                           scale per 64-row block (max|x|/127), integer Q K^T with
+                           int32 accumulation, rescaled by the two block scales */
 } sla_qk_prec_t;
 
 typedef enum {
   SLA_PV_BF16 = 0,      /* P V of critical blocks in bf16, fp32 accumulate */
   SLA_PV_FP8_E4M3 = 1   /* [SLA2] §5: P and V quantised to E4M3, product dequantised:
-                           P on the fixed scale 448 (P <= 1: the running maximum is
-                           updated on every increase), V with one scale per
-                           (head, channel) max|V[:, c]| / 448 */
+                           P = 2^(s log2 e - M) with M the row maximum rounded up to
+                           whole log2 units, stored as E4M3(448 P); V with one scale
+                           per (head, channel) max|V[:, c]| / 448 */
 } sla_pv_prec_t;
 
 typedef enum {
@@ -155,8 +159,8 @@ sla_status_t sla_router_probs(const sla_params_t* p, const void* Q, const void* 
  * Inputs (device): Pc fp32 [B*H][T_q][T_kv] (e.g. from sla_router_probs), tau > 0.
  * Outputs (device, caller-allocated): M fp32 [B*H][T_q][T_kv], lambda fp32
  * [B*H][T_q].  Pc and M 16-byte aligned.  No workspace.
- * Errors: SLA_ERR_INVALID_ARG (NULL or misaligned pointers, tau not a positive
- * finite number), SLA_ERR_CUDA.
+ * Errors: SLA_ERR_INVALID_ARG (NULL or misaligned pointers, tau not a finite
+ * number >= FLT_MIN, the smallest normal fp32 value), SLA_ERR_CUDA.
  */
 sla_status_t sla_soft_topk(const sla_params_t* p, const float* Pc, float tau, float* M,
                            float* lambda, sla_stream_t stream);
@@ -288,9 +292,9 @@ sla_status_t sla_predict_mask_noalloc(const sla_params_t* p, const void* Q, cons
 
 /*
  * Backward of sla_forward_train ([SLA2] App. A; [SLA] §4 check 6): the
- * gradients of L = sum(O * dO) for fixed mc (hard Top-k has no gradient;
- * SLA2's router is trained through a soft Top-k that is not part of this
- * library, so Wq / Wk get none).
+ * gradients of L = sum(O * dO) for fixed mc (hard Top-k has no gradient).
+ * SLA2's router is trained through SoftTop-k; its forward is sla_soft_topk,
+ * but its gradient is not built, so Wq / Wk get no gradient here.
  *   sparse branch  the FlashAttention backward over the critical blocks only:
  *                  P = exp(q.k / sqrt(d) - lse), dS = P (dP - D) with
  *                  D_r = dO^s_r . o^s_r; one kernel for dQ (per query-block
@@ -313,8 +317,8 @@ sla_status_t sla_predict_mask_noalloc(const sla_params_t* p, const void* Q, cons
  *   may be NULL); dalpha fp32 [B*H] (SLA2; may be NULL).
  * Workspace: sla_backward_workspace_size bytes, 256-byte aligned; its first
  *   word is the device error word (zero it once; sla_get_device_status reads
- *   and clears it).  Q K^T is recomputed in bf16 also for qk_prec = FP8
- *   ([SLA2] §5 keeps the backward in full precision).
+ *   and clears it).  Q K^T is recomputed in bf16 also when the forward ran
+ *   it on 8-bit codes ([SLA2] §5 keeps the backward in full precision).
  */
 sla_status_t sla_backward_workspace_size(const sla_params_t* p, size_t* bytes);
 sla_status_t sla_backward(const sla_params_t* p, const void* Q, const void* K, const void* V,

@@ -76,6 +76,13 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
     p = _params(d=64)
     p.pv_prec = 1  # FP8 P V is built for d = 128
     assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == 2
+    for qk, want in ((1, 2), (2, 2), (3, 1)):  # 8-bit Q K^T is built for d = 128; no format 3
+        p = _params(d=64)
+        p.qk_prec = qk
+        assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == want
+    p = _params(d=128)
+    p.qk_prec = 2  # INT8 Q K^T at d = 128
+    assert L.sla_block_counts(ctypes.byref(p), None, None, None, None) == 0
     p = _params()
     ws = (ctypes.c_uint8 * 1024)()
     # NULL tensors
@@ -103,7 +110,8 @@ def test_invalid_arguments_are_rejected_before_any_launch(L):
                               1024, None) == 1
     assert L.sla_router_probs(ctypes.byref(p), dummy, dummy, None, None, dummy,
                               ctypes.c_void_p(4096), 16, None) == 3
-    for tau in (0.0, -1.0, float("nan"), float("inf")):
+    # (a subnormal tau would make 1 / tau overflow in the kernel's fp32 arithmetic)
+    for tau in (0.0, -1.0, float("nan"), float("inf"), 1e-39, 1e-45):
         assert L.sla_soft_topk(ctypes.byref(p), dummy, ctypes.c_float(tau), dummy, dummy, None) == 1
     assert L.sla_soft_topk(ctypes.byref(p), None, ctypes.c_float(0.1), dummy, dummy, None) == 1
     assert L.sla_soft_topk(ctypes.byref(p), dummy, ctypes.c_float(0.1), dummy, None, None) == 1
