@@ -137,45 +137,64 @@ def fused_traffic_per_launch(workload: str, heads: int, qk: str):
         return None
 
 
-# --------------------------------------------------------------------------- FLOP accounting
-def flop_model(cfg, dims, lut_np):
-    """Executed and algorithmic FLOPs of one step.
+# --------------------------------------------------------------------------- work accounting
+def work_model(cfg, dims, lut_np, pairs_np=None):
+    """Algorithmic and issued work of one step.
 
-    Executed = every tensor-core MMA the kernels issue (union entries of the fused
-    kernel, padded GEMM tiles) plus the fp32 logits; algorithmic (fused) = QK^T and
-    PV over the critical pairs plus phi(Q)H per query row."""
+    Algorithmic FLOPs (what the method needs, counted once):
+      fused     Q K^T + P V over the critical pairs, 4*64*64*d each, plus
+                phi(Q) H (2 d^2 per query row) and, for the SLA combine, the Proj
+                product (2 d^2 per row; folded into h_j here, executed by kv_prep);
+      kv_prep   h_j = phi(K_j)^T V_j, 2 d^2 per key token;
+      marginal  one add per (query block, marginal key block, element of [h|z]);
+      logits    pooled Q_c K_c^T, 2 d per (query block, key block), plus the
+                router's two d x d maps per pooled row (SLA2).
+    Issued FLOPs add what the kernels execute beyond that: the fused kernel's
+    masked halves (a tile walks the union of its two blocks' critical lists:
+    U entries per tile, counted on the pairs the kernel used) and the dense
+    0/1 aggregation GEMM (128 x 256 tiles, K padded to 64)."""
     BH, N, d, Tq, Tkv, nh, nl = (dims[k] for k in ("BH", "N", "d", "Tq", "Tkv", "nh", "nl"))
     NN = d * d + d
-    # fused kernel: per CTA (pair of query blocks) U union entries x (S + PV), + 2 phi(Q)H tiles
     lut = lut_np.reshape(BH, Tq, nh)
+    if pairs_np is None:  # adjacent pairs
+        pairs_np = np.stack([np.arange(0, Tq, 2), np.where(np.arange(1, Tq + 1, 2) < Tq,
+                                                           np.arange(1, Tq + 1, 2), -1)], axis=1)
+        pairs_np = np.broadcast_to(pairs_np, (BH,) + pairs_np.shape)
     U = 0
     for bh in range(BH):
-        for p in range(0, Tq, 2):
-            s = set(lut[bh, p].tolist())
-            if p + 1 < Tq:
-                s |= set(lut[bh, p + 1].tolist())
+        for a, b in pairs_np[bh].tolist():
+            s = set(lut[bh, a].tolist())
+            if b >= 0:
+                s |= set(lut[bh, b].tolist())
             U += len(s)
-    n_cta = BH * ((Tq + 1) // 2)
-    fused_exec = U * 2 * (2 * 128 * 64 * d) + n_cta * 2 * (2 * 128 * d * d)
-    fused_alg = 4 * 64 * 64 * d * Tq * nh * BH + 2 * N * d * d * BH
-    # marginal aggregation GEMM: 128 x 256 tiles, K padded to 64
-    marg_exec = 2 * (math.ceil(Tq / 128) * 128) * (math.ceil(NN / 256) * 256) * \
-        (math.ceil(Tkv / 64) * 64) * BH
-    marg_alg = Tq * (Tkv - nh - nl) * NN * BH  # one add per marginal (i, j, element)
-    kv_exec = BH * Tkv * ((2 * 64 * d * d) * (2 if cfg.combine == "proj" else 1))
-    select = 2 * Tq * Tkv * d * BH + (4 * Tq * d * d * BH if cfg.combine == "alpha" else 0)
-    return {"fused_exec": fused_exec, "fused_alg": fused_alg, "marg_exec": marg_exec,
-            "marg_alg": marg_alg, "kv_exec": kv_exec, "select": select, "union_total": U,
-            "n_cta_fused": n_cta,
-            "step_exec": fused_exec + marg_exec + kv_exec + select,
-            "dense_equiv": 4 * N * N * d * BH}
+    n_cta = int(pairs_np.shape[0] * pairs_np.shape[1])
+    proj = cfg.combine == "proj"
+    fused_pairs = 4 * 64 * 64 * d * Tq * nh * BH
+    fused_alg = fused_pairs + 2 * N * d * d * BH
+    fused_issued = U * 2 * (2 * 128 * 64 * d) + n_cta * 2 * (2 * 128 * d * d)
+    kv_alg = 2 * N * d * d * BH + (2 * N * d * d * BH if proj else 0)
+    n_m = Tkv - nh - nl
+    marg_alg = Tq * n_m * NN * BH
+    marg_issued = 2 * (math.ceil(Tq / 128) * 128) * (math.ceil(NN / 256) * 256) * (math.ceil(Tkv / 64) * 64) * BH
+    logits = 2 * Tq * Tkv * d * BH + (4 * Tq * d * d * BH if cfg.combine == "alpha" else 0)
+    step_alg = fused_alg + kv_alg + marg_alg + logits
+    act = BH * N * d * 2  # one bf16 [B, H, N, d] tensor
+    hz_bytes = BH * Tkv * NN * 2
+    return {"fused_alg": fused_alg, "fused_pairs_alg": fused_pairs, "fused_issued": fused_issued,
+            "kv_alg": kv_alg, "marg_alg": marg_alg, "marg_issued": marg_issued, "logits": logits,
+            "step_alg": step_alg, "step_issued": fused_issued + kv_alg + marg_issued + logits,
+            "union_total": U, "n_tiles": n_cta, "critical_entries": Tq * nh * BH,
+            "dense_equiv": 4 * N * N * d * BH,
+            # algorithmic HBM bytes of the bandwidth-bound stages
+            "bytes": {"predict_mask": 2 * act, "precompute_linear": 2 * act + hz_bytes,
+                      "aggregate_marginal": 2 * hz_bytes}}
 
 
 # --------------------------------------------------------------------------- our arm
 def reduce_over_ranks(ms_total: float, flops_per_step: float, device):
     """Whole-job figures of a data-parallel run: the slowest rank's timed-region
-    duration (max over ranks) and the executed FLOPs of one step summed over the
-    ranks' independent problems.  Every rank must call this, in the same order."""
+    duration (max over ranks) and the algorithmic FLOPs of one step summed over
+    the ranks' independent problems.  Every rank must call this, in the same order."""
     t_ms = torch.tensor([ms_total], dtype=torch.float64, device=device)
     t_fl = torch.tensor([flops_per_step], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t_ms, op=torch.distributed.ReduceOp.MAX)
@@ -183,11 +202,17 @@ def reduce_over_ranks(ms_total: float, flops_per_step: float, device):
     return float(t_ms.item()), float(t_fl.item())
 
 
-def run_ours(args, rank, world, dev):
+STAGES = ["predict_mask", "precompute_linear", "aggregate_marginal", "pair_query_blocks", "fused_kernel"]
+
+
+def measure(workload, qk, pv, steps, warmup, dev, rank=0, world=1, heads=None, burn=0.0, sampler=None,
+            keep=False):
+    """Times `steps` steps of one workload on this rank's GPU.  Returns a record
+    (ms per step, stage ms, work, fused roofline) and, with keep, the inputs."""
     torch.cuda.set_device(dev)
-    over = {} if args.heads is None else {"H": args.heads}
-    data, w = I.make_workload(args.workload, device=f"cuda:{dev}", problem=rank, **over)
-    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"], qk=args.qk, pv=args.pv)
+    over = {} if heads is None else {"H": heads}
+    data, w = I.make_workload(workload, device=f"cuda:{dev}", problem=rank, **over)
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"], qk=qk, pv=pv)
     Q, K, V = (data[k].to(dev) for k in ("Q", "K", "V"))
     O = torch.empty_like(Q)
     f32 = lambda t: None if t is None else t.to(dev).float().contiguous()  # noqa: E731
@@ -204,115 +229,114 @@ def run_ours(args, rank, world, dev):
     hz = torch.empty((BH, Tkv, d * d + d), dtype=torch.bfloat16, device=dev)
     P = bnd._ptr
     pw = proj_w if cfg.combine == "proj" else None
-    st = lambda: bnd._stream()  # noqa: E731
+    st = bnd._stream
     wsz = ws.numel()
-
-    def stage(i):
-        if i == 0:
-            return L.sla_predict_mask(bnd.ctypes.byref(p), P(Q), P(K), P(Wq), P(Wk), P(mc), P(lut),
-                                      P(ws), wsz, st())
-        if i == 1:
-            return L.sla_precompute_linear(bnd.ctypes.byref(p), P(K), P(V), P(pw), P(hz), P(ws), wsz, st())
-        if i == 2:
-            return L.sla_aggregate_marginal(bnd.ctypes.byref(p), P(mc), P(hz), P(ws), wsz, st())
-        return L.sla_fused_forward(bnd.ctypes.byref(p), P(Q), P(K), P(V), P(lut), P(proj_b), P(alpha),
-                                   P(O), P(ws), wsz, st())
-
-    names = ["predict_mask", "precompute_linear", "aggregate_marginal", "fused_forward"]
-    launches_per_step = {"predict_mask": 3 + (2 if Wq is not None or Wk is not None else 0),
-                         "precompute_linear": 1, "aggregate_marginal": 2,
-                         "fused_forward": 3 + (1 if args.qk != "bf16" else 0) + (2 if args.pv != "bf16" else 0)}
+    pp = bnd.ctypes.byref(p)
+    calls = [
+        lambda: L.sla_predict_mask(pp, P(Q), P(K), P(Wq), P(Wk), P(mc), P(lut), P(ws), wsz, st()),
+        lambda: L.sla_precompute_linear(pp, P(K), P(V), P(pw), P(hz), P(ws), wsz, st()),
+        lambda: L.sla_aggregate_marginal(pp, P(mc), P(hz), P(ws), wsz, st()),
+        lambda: L.sla_pair_query_blocks(pp, P(lut), P(ws), wsz, st()),
+        lambda: L.sla_fused_forward_paired(pp, P(Q), P(K), P(V), P(lut), P(proj_b), P(alpha), P(O), P(ws),
+                                           wsz, st()),
+    ]
+    router = Wq is not None or Wk is not None
+    launches = {"predict_mask": 3 + (1 if router else 0), "precompute_linear": 1, "aggregate_marginal": 2,
+                "pair_query_blocks": 3 if (qk == "bf16" and pv == "bf16") else 2,
+                "fused_kernel": 1 + (1 if qk != "bf16" else 0) + (2 if pv != "bf16" else 0)}
 
     def step(ev=None):
-        for i in range(4):
+        for i, c in enumerate(calls):
             if ev is not None:
                 ev[i].record()
-            code = stage(i)
+            code = c()
             if code != 0:
-                raise bnd.SlaError(code, names[i])
+                raise bnd.SlaError(code, STAGES[i])
         if ev is not None:
-            ev[4].record()
+            ev[len(calls)].record()
 
-    for _ in range(max(args.warmup, 3)):
+    for _ in range(max(warmup, 3)):
         step()
     torch.cuda.synchronize()
     code, detail = bnd.sla_get_device_status(ws)
     if code != 0:
         raise RuntimeError(f"device status {code} ({detail}) after warm-up")
-    fl = flop_model(cfg, dict(BH=BH, N=N, d=d, Tq=Tq, Tkv=Tkv, nh=nh, nl=nl), lut.cpu().numpy())
+    pairs = bnd.sla_workspace_pairs(p, ws).cpu().numpy()
+    wk = work_model(cfg, dict(BH=BH, N=N, d=d, Tq=Tq, Tkv=Tkv, nh=nh, nl=nl), lut.cpu().numpy(), pairs)
 
-    # keep the GPU busy ~0.5 s before timing so that the clock sampler sees the loaded state
-    sampler = ClockSampler(bus_id_of(dev) if rank == 0 else None)
-    if rank == 0:
+    if sampler is not None:
         sampler.start()
-    t_end = time.time() + args.burn
+    t_end = time.time() + burn
     while time.time() < t_end:
         step()
         torch.cuda.synchronize()
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    nst = len(calls) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     start.record()
-    for k in range(args.steps):
+    for k in range(steps):
         step(evs[k])
     end.record()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
-    clocks = sampler.stop() if rank == 0 else None
+    clocks = sampler.stop() if sampler is not None else None
     ms_total = start.elapsed_time(end)
-    stage_ms = [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(args.steps)) / args.steps
-                for i in range(4)]
-    job_flops = fl["step_exec"]
-    if world > 1:
-        ms_total, job_flops = reduce_over_ranks(ms_total, fl["step_exec"], torch.device(f"cuda:{dev}"))
+    stage_ms = [sum(evs[k][i].elapsed_time(evs[k][i + 1]) for k in range(steps)) / steps
+                for i in range(len(calls))]
     code, detail = bnd.sla_get_device_status(ws)
     if code != 0:
         raise RuntimeError(f"device status {code} ({detail}) after timing")
-    ms_step = ms_total / args.steps
+    rec = {"workload": workload, "qk": qk, "pv": pv, "B": B, "H": H, "N": N, "d": d, "T": Tq, "n_h": nh,
+           "n_l": nl, "sparsity": round(1 - nh / Tkv, 4), "ms_total": ms_total, "steps": steps,
+           "ms_per_step": ms_total / steps, "stage_ms": dict(zip(STAGES, stage_ms)), "work": wk,
+           "launches_per_step": launches, "clocks": clocks}
+    ctx = None
+    if keep:
+        ctx = dict(Q=Q, K=K, V=V, cfg=cfg, data=data, w=w, wk=wk, params=(proj_w, proj_b, alpha, Wq, Wk),
+                   dev=dev)
+    return rec, ctx
 
-    result = None
-    if rank == 0:
-        peaks, peak_kind = load_peaks()
-        fused_ms = stage_ms[3]
-        ach = fl["fused_alg"] / (fused_ms * 1e-3) / 1e12
-        peak = float(peaks["bf16_tflops"])
-        traffic = fused_traffic_per_launch(args.workload, H, args.qk if args.pv == "bf16" else "fp8 P V")
-        result = {
-            "metric": METRIC, "value": round(job_flops / (ms_total * 1e-3 / args.steps) / 1e12, 3),
-            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "bf16" if args.qk == "bf16" and args.pv == "bf16" else "bf16+e4m3",
-            "data": "synthetic",
-            "config": {"workload": f"{args.workload} (B={B}, H={H}, N={N}, d={d}, k_h={cfg.k_h}, "
-                                   f"k_l={cfg.k_l}, {cfg.combine} combine)",
-                       "B": B, "H": H, "N": N, "d": d, "n_h": nh, "n_l": nl, "T": Tq,
-                       "sparsity": round(1 - nh / Tkv, 4),
-                       "l2": "inputs larger than L2 (Q, K, V = 302 MB vs 126 MB L2); no flush",
-                       "parallelism": f"{world} independent problems, one per GPU (no collective)"},
-            "stage_ms": {n: round(x, 4) for n, x in zip(names, stage_ms)},
-            "flops": {"step_executed": fl["step_exec"], "fused_executed": fl["fused_exec"],
-                      "fused_algorithmic": fl["fused_alg"], "marginal_gemm_executed": fl["marg_exec"],
-                      "dense_equivalent": fl["dense_equiv"], "fused_union_entries": fl["union_total"]},
-            "dense_equiv_tflops": round(fl["dense_equiv"] / (ms_step * 1e-3) / 1e12, 2),
-            "fused_executed_tflops": round(fl["fused_exec"] / (fused_ms * 1e-3) / 1e12, 2),
-            "fused_executed_frac": round(fl["fused_exec"] / (fused_ms * 1e-3) / 1e12 / peak, 4),
-            "roofline": {"kernel": "sla_fused_kernel<128>", "timed": "the fused_forward stage (pair_overlap_kernel "
-                         "+ pair_match_kernel + sla_fused_kernel)", "bound": "tensor", "achieved": round(ach, 2),
-                         "peak": peak, "unit": "TFLOP/s", "frac": round(ach / peak, 4),
-                         "traffic": traffic,
-                         "peak_note": f"dense bf16 GEMM burst peak ({peak_kind})",
-                         "per_launch_flops": fl["fused_alg"]},
-            "clocks": clocks,
-            "gpu_launches": sum(launches_per_step.values()) * args.steps,
-        }
-        result["_ctx"] = dict(Q=Q, K=K, V=V, cfg=cfg, data=data, w=w, fl=fl,
-                              params=(proj_w, proj_b, alpha, Wq, Wk), dev=dev)
-    return result
+
+def rooflines(rec, peaks, peak_kind):
+    """Achieved / peak per stage: the fused kernel against the bf16 tensor peak on
+    its algorithmic FLOPs (the FP8 / INT8 paths' own peak is twice that), the
+    bandwidth-bound stages against the HBM copy peak on their algorithmic bytes."""
+    wk, sm = rec["work"], rec["stage_ms"]
+    # an 8-bit product runs at twice the bf16 rate (the recipe's nominal ratio): the
+    # fused kernel's peak is the harmonic mix over Q K^T, P V and the bf16 phi(Q) H
+    half = wk["fused_pairs_alg"] / 2
+    rest = wk["fused_alg"] - 2 * half
+    t_unit = half / (2.0 if rec["qk"] != "bf16" else 1.0) + half / (2.0 if rec["pv"] != "bf16" else 1.0) + rest
+    tens = round(float(peaks["bf16_tflops"]) * wk["fused_alg"] / t_unit, 1)
+    hbm = float(peaks["hbm_gbs"])
+    out = {}
+    f_ms = sm["fused_kernel"]
+    ach = wk["fused_alg"] / (f_ms * 1e-3) / 1e12
+    out["fused_kernel"] = {"bound": "tensor", "achieved": round(ach, 2), "peak": tens, "unit": "TFLOP/s",
+                           "frac": round(ach / tens, 4),
+                           "issued_tflops": round(wk["fused_issued"] / (f_ms * 1e-3) / 1e12, 2),
+                           "issued_frac": round(wk["fused_issued"] / (f_ms * 1e-3) / 1e12 / tens, 4)}
+    for s in ("predict_mask", "precompute_linear", "aggregate_marginal"):
+        gbs = wk["bytes"][s] / (sm[s] * 1e-3) / 1e9
+        out[s] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                  "frac": round(gbs / hbm, 4)}
+    return out
+
+
+def workload_summary(rec, peaks, peak_kind):
+    ms = rec["ms_per_step"]
+    wk = rec["work"]
+    return {"workload": rec["workload"], "qk": rec["qk"], "pv": rec["pv"],
+            "shape": f"B={rec['B']}, H={rec['H']}, N={rec['N']}, d={rec['d']}, n_h={rec['n_h']}, "
+                     f"n_l={rec['n_l']}, sparsity {rec['sparsity']}",
+            "ms_per_step": round(ms, 4), "algorithmic_tflops": round(wk["step_alg"] / (ms * 1e-3) / 1e12, 2),
+            "dense_equiv_tflops": round(wk["dense_equiv"] / (ms * 1e-3) / 1e12, 1),
+            "stage_ms": {k: round(v, 4) for k, v in rec["stage_ms"].items()},
+            "roofline": rooflines(rec, peaks, peak_kind)}
 
 
 def run_e2e(ctx, steps):
@@ -339,7 +363,7 @@ def run_e2e(ctx, steps):
         raise RuntimeError(f"device status {code} in e2e")
     ms = a.elapsed_time(b) / steps
     act = Qh.numel() * Qh.element_size()
-    return {"value": round(ctx["fl"]["step_exec"] / (ms * 1e-3) / 1e12, 3), "unit": UNIT,
+    return {"value": round(ctx["wk"]["step_alg"] / (ms * 1e-3) / 1e12, 3), "unit": UNIT,
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": 3 * act, "d2h_bytes_per_step": act,
             "api": "sla_attention_host (pinned host Q, K, V, O)"}
 
@@ -413,6 +437,18 @@ def run_train(ctx, steps=10, warmup=3, dense=True):
     res = {"workload": "forward + backward of the bench workload, dO ~ N(0, 1) bf16",
            "ms_per_step": round(sum(stage_ms), 4),
            "stage_ms": {n: round(x, 4) for n, x in zip(names, stage_ms)}}
+    # the backward's algorithmic work: the sparse branch's FlashAttention backward over
+    # the critical pairs (dQ: S, dP, dS K = 6*64*64*d; dK, dV: S^T, dP^T, dV, dK =
+    # 8*64*64*d per pair) and the linear branch's d x d products (query side 3, key
+    # side 4, dW 1 per token: 16 N d^2 per head)
+    crit = Tq * nh * BH
+    bwd_alg = 14 * 64 * 64 * d * crit + 16 * N * d * d * BH
+    peaks, _ = load_peaks()
+    ach = bwd_alg / (stage_ms[3] * 1e-3) / 1e12
+    res["backward_roofline"] = {"kernels": "all of sla_backward", "bound": "tensor", "achieved": round(ach, 2),
+                                "peak": float(peaks["bf16_tflops"]), "unit": "TFLOP/s",
+                                "frac": round(ach / float(peaks["bf16_tflops"]), 4),
+                                "algorithmic_flops": bwd_alg}
     # dense attention forward + backward on the same inputs
     if not dense:
         return res
@@ -476,84 +512,95 @@ def run_dense(ctx, iters=10):
                 torch.cuda.synchronize()
             ms = a.elapsed_time(b) / iters
             out[name] = {"ms": round(ms, 3),
-                         "tflops": round(ctx["fl"]["dense_equiv"] / (ms * 1e-3) / 1e12, 1)}
+                         "tflops": round(ctx["wk"]["dense_equiv"] / (ms * 1e-3) / 1e12, 1)}
         except Exception as e:  # backend not available for this shape
             out[name] = {"error": str(e).splitlines()[0][:120]}
     return out
 
 
 # --------------------------------------------------------------------------- oracle arm
-def oracle_sample(data, w, heads, qblocks_per_head):
-    """Runs the fp64 oracle on `heads` heads and the first `qblocks_per_head` query
-    blocks of each; returns (seconds, fraction of the workload's (head, query
-    block) units covered)."""
+def oracle_head(data, w, hh):
+    """The fp64 oracle's whole forward of one head (mask prediction, linear
+    statistics, every query block); returns its seconds and BLAS threads."""
     import oracle as Or
     from threadpoolctl import threadpool_info
     p = Or.OracleParams(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"])
-    H = data["Q"].shape[1]
-    T = Or.num_blocks(data["Q"].shape[2], 64)
-    nb = min(qblocks_per_head, T)
+    np_ = lambda t: None if t is None else t.float().cpu().numpy().astype(np.float64)  # noqa: E731
+    sl = slice(hh, hh + 1)
+    Q, K, V = (np_(data[k][:, sl]) for k in ("Q", "K", "V"))
     t0 = time.perf_counter()
-    for hh in range(heads):
-        sl = slice(hh, hh + 1)
-        Q, K, V = (data[k][:, sl].float().numpy().astype(np.float64) for k in ("Q", "K", "V"))
-        np_ = lambda t: None if t is None else t.float().numpy().astype(np.float64)  # noqa: E731
-        Mc, _, _ = Or.predict_mask(Q, K, p, np_(data.get("Wq")), np_(data.get("Wk")))
-        alpha = data.get("alpha")
-        a = None if alpha is None else np_(alpha)[:, sl]
-        Or.forward_given_mask(Q, K, V, Mc, p, proj_w=np_(data.get("proj_w")),
-                              proj_b=np_(data.get("proj_b")), alpha=a, qblocks=range(nb))
+    Mc, _, _ = Or.predict_mask(Q, K, p, np_(data.get("Wq")), np_(data.get("Wk")))
+    alpha = data.get("alpha")
+    Or.forward_given_mask(Q, K, V, Mc, p, proj_w=np_(data.get("proj_w")), proj_b=np_(data.get("proj_b")),
+                          alpha=None if alpha is None else np_(alpha)[:, sl])
     secs = time.perf_counter() - t0
     cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    return secs, (heads * nb) / (H * T), cores
+    return secs, cores
 
 
-def cpu_baseline(ctx):
-    secs, frac, cores = oracle_sample(ctx["data"], ctx["w"], heads=4, qblocks_per_head=10 ** 9)
-    step_equiv = secs / frac
-    return {"value": round(ctx["fl"]["step_exec"] / step_equiv / 1e12, 6), "unit": UNIT,
-            "cores": cores, "kind": "oracle", "ms_per_step_equiv": round(step_equiv * 1e3, 1),
-            "sample": f"4 of {ctx['data']['Q'].shape[1]} heads, all query blocks, mask prediction "
-                      f"and linear statistics included ({secs:.1f} s); value = the step's executed "
-                      f"FLOPs scaled by the covered (head, query block) fraction {frac:.3f}"}
+def head_work(workload, data, w):
+    """Algorithmic FLOPs of one head of the workload (the unit both CPU legs time)."""
+    import oracle as Or
+    B, H, N, d = data["Q"].shape
+    T = Or.num_blocks(N, 64)
+    nh, nl = Or.block_counts(T, w["k_h"], w["k_l"])
+    cfg = bnd.SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"])
+    lut = np.zeros((1, T, nh), dtype=np.int32)  # the count of critical pairs is all that is used
+    wk = work_model(cfg, dict(BH=1, N=N, d=d, Tq=T, Tkv=T, nh=nh, nl=nl), lut,
+                    np.zeros((1, 0, 2), dtype=np.int64))
+    return wk["step_alg"], H
+
+
+SAMPLE_RULE = ("one whole head per sample (mask prediction, linear statistics and every query block of "
+               "that head), heads taken in order; value = that head's algorithmic FLOPs / its seconds")
+
+
+def cpu_baseline(ctx, budget_s=15.0):
+    """The oracle on the GPU machine's host cores, timed on whole heads until ~budget_s."""
+    flops_head, H = head_work(WORKLOAD, ctx["data"], ctx["w"])
+    tot, n, cores = 0.0, 0, 1
+    while n < H and (n == 0 or tot < budget_s):
+        s, cores = oracle_head(ctx["data"], ctx["w"], n)
+        tot += s
+        n += 1
+    return {"value": round(flops_head * n / tot / 1e12, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {H} heads ({tot:.1f} s); " + SAMPLE_RULE,
+            "s_per_head": round(tot / n, 3),
+            "full_step_s": {"value": round(tot / n * H, 1), "extrapolated": True}}
 
 
 def run_reference(args):
+    """`--impl reference`: the fp64 oracle (the pages ship no code; the oracle is
+    this build's reference arm) on the host cores, one whole head per step."""
     data, w = I.make_workload(args.workload)
     B, H, N, d = data["Q"].shape
-    # one step = 1 head, first 64 query blocks (about 1 s of fp64 work on 8 cores)
-    from block_sparse_linear_pool_b200.binding import SlaConfig
-    cfg = SlaConfig(k_h=w["k_h"], k_l=w["k_l"], combine=w["combine"])
-    import oracle as Or
-    T = Or.num_blocks(N, 64)
-    nh, nl = Or.block_counts(T, cfg.k_h, cfg.k_l)
-    Mc, _, _ = Or.predict_mask(data["Q"].float().numpy().astype(np.float64),
-                               data["K"].float().numpy().astype(np.float64),
-                               Or.OracleParams(k_h=w["k_h"], k_l=w["k_l"]),
-                               None if data.get("Wq") is None else data["Wq"].numpy().astype(np.float64),
-                               None if data.get("Wk") is None else data["Wk"].numpy().astype(np.float64))
-    lut = Or.critical_lut(Mc)
-    fl = flop_model(cfg, dict(BH=B * H, N=N, d=d, Tq=T, Tkv=T, nh=nh, nl=nl), lut)
-    for _ in range(args.warmup):
-        oracle_sample(data, w, 1, 64)
-    tot, frac, cores = 0.0, 0.0, 1
-    for _ in range(args.steps):
-        s, frac, cores = oracle_sample(data, w, 1, 64)
+    flops_head, _ = head_work(args.workload, data, w)
+    for k in range(args.warmup):
+        oracle_head(data, w, k % H)
+    tot, cores = 0.0, 1
+    for k in range(args.steps):
+        s, cores = oracle_head(data, w, k % H)
         tot += s
-    step_equiv = tot / args.steps / frac
-    value = fl["step_exec"] / step_equiv / 1e12
+    ms = tot / args.steps * 1e3
+    value = flops_head * args.steps / tot / 1e12
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(step_equiv * 1e3, 1), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": f"{args.workload} (B={B}, H={H}, N={N}, d={d}, k_h={w['k_h']}, "
-                                   f"k_l={w['k_l']}, {w['combine']} combine)"},
+                                   f"k_l={w['k_l']}, {w['combine']} combine)",
+                       "step": "one whole head of the workload (a bounded sample)"},
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": "per step: 1 head, its first 64 query blocks, mask prediction "
-                                       "and linear statistics of that head; value scaled by the "
-                                       f"covered (head, query block) fraction {frac:.4f}"},
+                             "sample": SAMPLE_RULE,
+                             "full_step_s": {"value": round(ms / 1e3 * H, 1), "extrapolated": True}},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
+
+
+# the other workloads of the metric, each as its own record in the bench line
+EXTRA_WORKLOADS = [("wan1.3b_sla2", "bf16", "bf16"), ("wan14b_720p_sla2", "bf16", "bf16"),
+                   ("wan14b_720p_sla2", "fp8_e4m3", "bf16"), ("wan14b_720p_sla2", "int8", "bf16"),
+                   ("wan14b_720p_sla2", "int8", "fp8_e4m3")]
 
 
 # --------------------------------------------------------------------------- main
@@ -564,7 +611,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(I.WORKLOADS))
-    ap.add_argument("--no-extras", action="store_true", help="skip e2e, dense baseline and CPU baseline")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip e2e, the other workloads, dense, training and CPU baselines")
     ap.add_argument("--qk", choices=["bf16", "fp8_e4m3", "int8"], default="bf16",
                     help="precision of Q K^T on critical blocks (fp8_e4m3, int8: d = 128 only)")
     ap.add_argument("--pv", choices=["bf16", "fp8_e4m3"], default="bf16",
@@ -598,17 +646,69 @@ def main():
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device(f"cuda:{local}"))
-    res = run_ours(args, rank, world, local)
+    sampler = ClockSampler(bus_id_of(local)) if rank == 0 else None
+    rec, ctx = measure(args.workload, args.qk, args.pv, args.steps, args.warmup, local, rank, world,
+                       args.heads, args.burn, sampler, keep=True)
+    ms_total, job_flops = rec["ms_total"], rec["work"]["step_alg"]
+    if world > 1:
+        ms_total, job_flops = reduce_over_ranks(ms_total, job_flops, torch.device(f"cuda:{local}"))
     if rank == 0:
-        ctx = res.pop("_ctx")
-        if not args.no_extras:
+        peaks, peak_kind = load_peaks()
+        wk = rec["work"]
+        ms_step = ms_total / args.steps
+        rl = rooflines(rec, peaks, peak_kind)
+        fr = rl["fused_kernel"]
+        B, H, N, d = rec["B"], rec["H"], rec["N"], rec["d"]
+        cfg = ctx["cfg"]
+        res = {
+            "metric": METRIC, "value": round(job_flops / (ms_step * 1e-3) / 1e12, 3),
+            "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if args.qk == "bf16" and args.pv == "bf16" else f"bf16+{args.qk}/{args.pv}",
+            "data": "synthetic",
+            "config": {"workload": f"{args.workload} (B={B}, H={H}, N={N}, d={d}, k_h={cfg.k_h}, "
+                                   f"k_l={cfg.k_l}, {cfg.combine} combine)",
+                       "B": B, "H": H, "N": N, "d": d, "n_h": rec["n_h"], "n_l": rec["n_l"], "T": rec["T"],
+                       "sparsity": rec["sparsity"],
+                       "l2": "inputs larger than L2 (Q, K, V = 302 MB vs 126 MB L2); no flush",
+                       "parallelism": f"{world} independent problems, one per GPU (no collective)"},
+            "value_note": "algorithmic FLOPs of the step (critical Q K^T + P V, phi(Q) H, Proj, h_j, "
+                          "marginal adds, compressed logits) / time; issued FLOPs are under 'work'",
+            "stage_ms": {n: round(x, 4) for n, x in rec["stage_ms"].items()},
+            "work": {"step_algorithmic_flops": wk["step_alg"], "step_issued_flops": wk["step_issued"],
+                     "fused_algorithmic_flops": wk["fused_alg"], "fused_issued_flops": wk["fused_issued"],
+                     "union_entries": wk["union_total"], "critical_entries": wk["critical_entries"],
+                     "tiles": wk["n_tiles"], "marginal_gemm_issued_flops": wk["marg_issued"],
+                     "dense_equivalent_flops": wk["dense_equiv"]},
+            "dense_equiv_tflops": round(wk["dense_equiv"] / (ms_step * 1e-3) / 1e12, 2),
+            "roofline": {"kernel": "sla_fused_kernel", "timed": "sla_fused_forward_paired alone (CUDA events "
+                         "around it inside the timed loop)", "bound": "tensor", "achieved": fr["achieved"],
+                         "peak": fr["peak"], "unit": "TFLOP/s", "frac": fr["frac"],
+                         "traffic": fused_traffic_per_launch(args.workload, H, args.qk if args.pv == "bf16"
+                                                             else "fp8 P V"),
+                         "peak_note": f"dense bf16 GEMM burst peak ({peak_kind})",
+                         "per_launch_flops": wk["fused_alg"], "issued_frac": fr["issued_frac"]},
+            "stage_roofline": {k: v for k, v in rl.items() if k != "fused_kernel"},
+            "clocks": rec["clocks"],
+            "gpu_launches": sum(rec["launches_per_step"].values()) * args.steps,
+        }
+        if not args.no_extras and world == 1:  # single-GPU measurements: no rank waits on them
             res["e2e"] = run_e2e(ctx, steps=min(args.steps, 10))
             res["dense_baseline"] = run_dense(ctx)
-            res["train_step"] = run_train(ctx)
             best = min((v["ms"] for v in res["dense_baseline"].values() if "ms" in v), default=None)
-            res["speedup_vs_dense"] = None if best is None else round(best / res["ms_per_step"], 2)
+            res["speedup_vs_dense"] = None if best is None else round(best / ms_step, 2)
+            res["train_step"] = run_train(ctx)
             if world == 1:
                 res["cpu_baseline"] = cpu_baseline(ctx)
+            del ctx
+            torch.cuda.empty_cache()
+            res["workloads"] = []
+            for (wl, qk, pv) in EXTRA_WORKLOADS:
+                r2, _ = measure(wl, qk, pv, 10, 3, local)
+                res["workloads"].append(workload_summary(r2, peaks, peak_kind))
+                del r2
+                torch.cuda.empty_cache()
         print(json.dumps(res), flush=True)
     if world > 1:
         torch.distributed.barrier()

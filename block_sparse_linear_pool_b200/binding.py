@@ -37,6 +37,7 @@ EXPORTS = (
     "sla_get_device_status", "sla_status_string", "sla_abi_version",
     "sla_predict_mask_noalloc", "sla_forward_train", "sla_backward_workspace_size",
     "sla_selftest_wait_timeout", "sla_router_probs", "sla_soft_topk",
+    "sla_pair_query_blocks", "sla_fused_forward_paired", "sla_workspace_pairs",
 )
 
 
@@ -85,6 +86,9 @@ def lib() -> ctypes.CDLL:
         L.sla_attention.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_aggregate_marginal.argtypes = [P, vp, vp, vp, sz, vp]
         L.sla_fused_forward.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_fused_forward_paired.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.sla_pair_query_blocks.argtypes = [P, vp, vp, sz, vp]
+        L.sla_workspace_pairs.argtypes = [P, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)]
         L.sla_attention_host.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.sla_predict_mask_noalloc.argtypes = [P, vp, vp, vp, vp, vp, vp, vp]
         L.sla_forward_train.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -336,6 +340,29 @@ def sla_fused_forward(p: sla_params_t, Q, K, V, lut, O, workspace, proj_b=None, 
     _check(lib().sla_fused_forward(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(lut), _ptr(proj_b),
                                    _ptr(alpha), _ptr(O), _ptr(workspace), workspace.numel(), _stream()),
            "sla_fused_forward")
+
+
+def sla_pair_query_blocks(p: sla_params_t, lut, workspace):
+    """Which two query blocks share a tile of the fused kernel (first step of
+    sla_fused_forward); the pairs stay in `workspace`."""
+    _check(lib().sla_pair_query_blocks(ctypes.byref(p), _ptr(lut), _ptr(workspace), workspace.numel(),
+                                       _stream()), "sla_pair_query_blocks")
+
+
+def sla_fused_forward_paired(p: sla_params_t, Q, K, V, lut, O, workspace, proj_b=None, alpha=None):
+    """The fused kernel on the pairs already in `workspace` (second step of sla_fused_forward)."""
+    _check(lib().sla_fused_forward_paired(ctypes.byref(p), _ptr(Q), _ptr(K), _ptr(V), _ptr(lut),
+                                          _ptr(proj_b), _ptr(alpha), _ptr(O), _ptr(workspace),
+                                          workspace.numel(), _stream()), "sla_fused_forward_paired")
+
+
+def sla_workspace_pairs(p: sla_params_t, workspace) -> torch.Tensor:
+    """The block pairs in `workspace` as an int32 [B*H, ceil(T_q / 2), 2] view."""
+    off, cnt = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib().sla_workspace_pairs(ctypes.byref(p), ctypes.byref(off), ctypes.byref(cnt)),
+           "sla_workspace_pairs")
+    B, H = p.B, p.H
+    return workspace[off.value:off.value + cnt.value * 8].view(torch.int32).view(B * H, -1, 2)
 
 
 def sla_attention_host(p: sla_params_t, Qh, Kh, Vh, Oh, workspace, proj_w=None, proj_b=None,

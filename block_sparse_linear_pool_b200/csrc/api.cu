@@ -29,9 +29,23 @@ struct Plan {
 
 inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
+// uint16 per tile-union record of the persistent fused kernel: count, 7 unused,
+// then up to min(2 n_h, T_kv) entries, rounded up to 16 bytes
+inline int union_record(const Plan& p) {
+  const int cap = 2 * p.nh < p.Tkv ? 2 * p.nh : p.Tkv;
+  return 8 + ((cap + 7) & ~7);
+}
+
+// The persistent fused kernel serves bf16 Q K^T and P V when two CTAs fit an SM
+// (its shared memory holds the union records); the other paths use the
+// per-tile kernel.
+inline bool pt_eligible(const Plan& p) {
+  return !p.fp8 && !p.pv8 && fused_pt_smem_bytes(p.d, union_record(p)) <= 113 * 1024;
+}
+
 struct Layout {
   size_t err, qc, kc, qr, kr, kmean, keys, mm, hagg;      // sla_workspace_size ...
-  size_t q8, k8, scq, sck, v8t, vmax, pairs, pov, end;    // ... (+ FP8 operands)
+  size_t q8, k8, scq, sck, v8t, vmax, pairs, pov, ulist, end;  // ... (+ 8-bit operands, tiles)
   size_t mc, lut, hz, end_attn;                           // + sla_attention extras
   size_t hq, hk, hv, ho, end_host;                        // + sla_attention_host staging
 };
@@ -58,6 +72,7 @@ Layout layout_of(const Plan& p) {
   L.vmax = o;  o = align_up(o + (p.pv8 ? (size_t)p.BH * p.d * 4 : 0));
   L.pairs = o; o = align_up(o + (size_t)p.BH * ((p.Tq + 1) / 2) * 8);
   L.pov = o;   o = align_up(o + pairing_overlap_bytes(p.BH, p.Tq));
+  L.ulist = o; o = align_up(o + (size_t)p.BH * ((p.Tq + 1) / 2) * union_record(p) * 2);
   L.end = o;
   L.mc = o;    o = align_up(o + (size_t)p.BH * p.Tq * p.Tkv);
   L.lut = o;   o = align_up(o + (size_t)p.BH * p.Tq * p.nh * 4);
@@ -318,10 +333,28 @@ sla_status_t zero_one_product(const Plan& pl, const __nv_bfloat16* A, int M, int
   return cuda_status(launch_marg_gemm(ma, mb, a, pl.BH, s));
 }
 
+// which two query blocks share a tile; for the persistent kernel also each tile's union list
+sla_status_t pairing_impl(const Plan& pl, const int32_t* lut, void* ws, cudaStream_t s) {
+  const Layout L = layout_of(pl);
+  int2* pairs = at<int2>(ws, L.pairs);
+  SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pl.Tkv, at<uint16_t>(ws, L.pov), pairs, s)));
+  if (pt_eligible(pl))
+    SLA_TRY(cuda_status(launch_tile_union(lut, pairs, pl.BH, pl.Tq, pl.Tkv, pl.nh, union_record(pl),
+                                          at<uint16_t>(ws, L.ulist), at<int>(ws, L.err), s)));
+  return SLA_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return n;
+}
+
 sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
                         const void* V, const int32_t* lut, const float* proj_b, const float* alpha,
                         void* O, void* ws, cudaStream_t s, float* lse = nullptr,
-                        float* o_sparse = nullptr) {
+                        float* o_sparse = nullptr, bool pair = true) {
   const Layout L = layout_of(pl);
   __nv_bfloat16* hagg = at<__nv_bfloat16>(ws, L.hagg);
   CUtensorMap mq, mk, mv, mh, mz;
@@ -330,7 +363,8 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
     return SLA_ERR_CUDA;
   // which two query blocks share a CTA (similar critical lists: a smaller union)
   int2* pairs = at<int2>(ws, L.pairs);
-  SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pl.Tkv, at<uint16_t>(ws, L.pov), pairs, s)));
+  const bool pt = pt_eligible(pl) && !lse && !o_sparse;
+  if (pair) SLA_TRY(pairing_impl(pl, lut, ws, s));
   {
     // H_i^T as (a, b, i, bh) tiles of d x d; Z_i as one unswizzled row of d
     const uint64_t dh[4] = {(uint64_t)pl.d, (uint64_t)pl.d, (uint64_t)pl.Tq, (uint64_t)pl.BH};
@@ -415,6 +449,14 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.os = o_sparse;
   a.vmax = vmax;
   a.pairs = pairs;
+  a.ulist = at<uint16_t>(ws, L.ulist);
+  a.urec = union_record(pl);
+  a.BH = pl.BH;
+  if (pt) {
+    const int nsm = sm_count();
+    if (nsm <= 0) return SLA_ERR_CUDA;
+    return cuda_status(launch_fused_pt(mq, mk, mv, mh, mz, a, pl.d, nsm, s));
+  }
   const int qk8 = pl.fp8 ? (pl.qk_int8 ? 2 : 1) : 0;
   return cuda_status(launch_fused(mq, mk, mv, mh, mz, mq8, mk8, a, pl.d, qk8, pl.pv8, pl.BH, s));
 }
@@ -900,6 +942,38 @@ sla_status_t sla_fused_forward(const sla_params_t* p, const void* Q, const void*
                     reinterpret_cast<cudaStream_t>(stream));
 }
 
+sla_status_t sla_pair_query_blocks(const sla_params_t* p, const int32_t* lut, void* workspace,
+                                   size_t workspace_bytes, sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!lut) return SLA_ERR_INVALID_ARG;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
+  return pairing_impl(pl, lut, workspace, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sla_status_t sla_fused_forward_paired(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                                      const int32_t* lut, const float* proj_b, const float* alpha,
+                                      void* O, void* workspace, size_t workspace_bytes,
+                                      sla_stream_t stream) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!Q || !K || !V || !lut || !O) return SLA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SLA_ERR_INVALID_ARG;
+  if (p->combine == SLA_COMBINE_ALPHA && !alpha) return SLA_ERR_INVALID_ARG;
+  SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_BASE));
+  return fused_impl(pl, p, Q, K, V, lut, proj_b, alpha, O, workspace,
+                    reinterpret_cast<cudaStream_t>(stream), nullptr, nullptr, false);
+}
+
+sla_status_t sla_workspace_pairs(const sla_params_t* p, size_t* offset, size_t* count) {
+  Plan pl;
+  SLA_TRY(make_plan(p, &pl));
+  if (!offset || !count) return SLA_ERR_INVALID_ARG;
+  *offset = layout_of(pl).pairs;
+  *count = (size_t)pl.BH * ((pl.Tq + 1) / 2);
+  return SLA_OK;
+}
+
 sla_status_t sla_backward_workspace_size(const sla_params_t* p, size_t* bytes) {
   Plan pl;
   SLA_TRY(make_plan(p, &pl));
@@ -965,6 +1039,6 @@ const char* sla_status_string(sla_status_t s) {
   return "SLA_ERR_UNKNOWN";
 }
 
-int sla_abi_version(void) { return 103; }
+int sla_abi_version(void) { return 104; }
 
 }  // extern "C"

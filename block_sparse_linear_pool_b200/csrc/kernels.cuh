@@ -76,6 +76,9 @@ struct FusedArgs {
   float* os;              // [BH][N][d] the sparse branch's output o^s (fp32), or nullptr
   const unsigned int* vmax;  // FP8 P V: per (head, channel) max |V| (float bits), else nullptr
   const int2* pairs;      // [BH][ceil(Tq / 2)] the two query blocks of each CTA (b = -1: none)
+  const uint16_t* ulist;  // persistent kernel: per tile the union record (tile_union_kernel)
+  int urec;               // uint16 per union record
+  int BH;
 };
 
 // ---- backward
@@ -176,6 +179,16 @@ cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, c
                              int BH, cudaStream_t s);
 
 cudaError_t launch_quant_fp8(const QuantArgs& a, int BH, cudaStream_t s);
+
+// Per tile of the persistent fused kernel: the union of its two query blocks'
+// critical lists (uint16 records of urec entries: count, then j | flag << 14 from 8).
+cudaError_t launch_tile_union(const int32_t* lut, const int2* pairs, int BH, int Tq, int Tkv, int nh, int urec,
+                              uint16_t* out, int* err, cudaStream_t s);
+// The persistent fused kernel (bf16 Q K^T and P V, no training outputs); nsm = SM count.
+cudaError_t launch_fused_pt(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                            const CUtensorMap& mapH, const CUtensorMap& mapZ, const FusedArgs& a, int D, int nsm,
+                            cudaStream_t s);
+size_t fused_pt_smem_bytes(int D, int urec);
 cudaError_t launch_vquant_fp8(const __nv_bfloat16* V, const int64_t* sv, int H, int N, int T, int BH, int D,
                               unsigned int* vmax, uint8_t* V8T, cudaStream_t s);
 

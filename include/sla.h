@@ -240,6 +240,34 @@ sla_status_t sla_fused_forward(const sla_params_t* p, const void* Q, const void*
                                sla_stream_t stream);
 
 /*
+ * The two steps of sla_fused_forward, for callers that time or schedule them
+ * apart (sla_fused_forward is exactly sla_pair_query_blocks followed by
+ * sla_fused_forward_paired on the same stream and workspace).
+ *
+ * sla_pair_query_blocks: chooses which two query blocks of a head share one
+ * 128-row tile of the fused kernel, from lut (blocks whose critical lists
+ * overlap most are paired, so the union of the two lists is small).  A pure
+ * scheduling choice: any pairing gives the same output.  The pairs stay in the
+ * workspace, int2 [B*H][ceil(T_q / 2)] (second block -1: a tile with one
+ * block) at the offset sla_workspace_pairs returns.
+ *
+ * sla_fused_forward_paired: the fused kernel on the pairs already in the
+ * workspace (requires sla_aggregate_marginal and sla_pair_query_blocks, in
+ * either order, on the same workspace and lut).
+ *
+ * sla_workspace_pairs: byte offset of the pairs in the workspace and their
+ * number (B*H*ceil(T_q / 2)), for callers that read them back.
+ * Errors: SLA_ERR_INVALID_ARG (NULL pointers), SLA_ERR_WORKSPACE, SLA_ERR_CUDA.
+ */
+sla_status_t sla_pair_query_blocks(const sla_params_t* p, const int32_t* lut, void* workspace,
+                                   size_t workspace_bytes, sla_stream_t stream);
+sla_status_t sla_fused_forward_paired(const sla_params_t* p, const void* Q, const void* K, const void* V,
+                                      const int32_t* lut, const float* proj_b, const float* alpha,
+                                      void* O, void* workspace, size_t workspace_bytes,
+                                      sla_stream_t stream);
+sla_status_t sla_workspace_pairs(const sla_params_t* p, size_t* offset, size_t* count);
+
+/*
  * The whole forward in one call: sla_predict_mask, sla_precompute_linear and
  * sla_forward, with mc, lut and hz kept in the workspace
  * (sla_attention_workspace_size bytes).  proj_w / proj_b are used by the SLA

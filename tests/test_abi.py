@@ -134,4 +134,4 @@ def test_workspace_sizes_grow_with_the_problem(L):
 def test_status_strings(L):
     for code, name in bnd.STATUS.items():
         assert L.sla_status_string(code).decode() == name
-    assert L.sla_abi_version() == 103
+    assert L.sla_abi_version() == 104

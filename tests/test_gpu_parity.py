@@ -347,6 +347,15 @@ def test_split_entry_points_and_host_buffers_match_forward():
     bnd.sla_aggregate_marginal(p, mc, hz, ws)
     O2 = torch.empty_like(Q)
     bnd.sla_fused_forward(p, Q, K, V, lut, O2, ws, proj_b=pb.float())
+    # the fused forward's two steps, pairing then the kernel on those pairs
+    O3 = torch.empty_like(Q)
+    bnd.sla_pair_query_blocks(p, lut, ws)
+    pairs = bnd.sla_workspace_pairs(p, ws).cpu().numpy()
+    bnd.sla_fused_forward_paired(p, Q, K, V, lut, O3, ws, proj_b=pb.float())
+    Tq = lut.shape[1]
+    for bh in range(pairs.shape[0]):  # every query block in exactly one tile
+        blocks = [b for b in pairs[bh].ravel().tolist() if b >= 0]
+        assert sorted(blocks) == list(range(Tq))
     # host-buffer variant
     Qh, Kh, Vh = (t.cpu().pin_memory() for t in (Q, K, V))
     Oh = torch.empty_like(Qh).pin_memory()
@@ -355,6 +364,7 @@ def test_split_entry_points_and_host_buffers_match_forward():
     bnd.sla_attention_host(ph, Qh, Kh, Vh, Oh, wsh, pw.float(), pb.float())
     torch.cuda.synchronize()
     assert torch.equal(O2, ref)
+    assert torch.equal(O3, ref)
     assert torch.equal(Oh, ref.cpu())
     assert bnd.sla_get_device_status(ws)[0] == 0 and bnd.sla_get_device_status(wsh)[0] == 0
 
