@@ -114,11 +114,11 @@ def bus_id_of(dev):
 
 
 def fused_traffic_per_launch(workload: str, heads: int, qk: str):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
-    or None if the summary is for another workload or the kernel source changed
-    since those counters were taken."""
-    path = os.path.join(ROOT, "profiles", f"fused_{workload}_traffic.txt")
-    src = os.path.join(ROOT, "block_sparse_linear_pool_b200", "csrc", "fused.cu")
+    """DRAM bytes per launch of the persistent fused kernel from the committed ncu
+    summary, or None if the summary is for another workload or the kernel source
+    changed since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", f"fused_pt_{workload}_traffic.txt")
+    src = os.path.join(ROOT, "block_sparse_linear_pool_b200", "csrc", "fused_pt.cu")
     if not os.path.exists(path):
         return None
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
@@ -127,7 +127,7 @@ def fused_traffic_per_launch(workload: str, heads: int, qk: str):
         if "=" in line and not line.startswith("#"):
             k, v = line.split("=", 1)
             vals[k.strip()] = v.strip()
-    if vals.get("fused_cu_sha256_16") != sha:
+    if vals.get("source_sha256_16") != sha:
         return None
     if vals.get("heads") != str(heads) or vals.get("qk", "bf16") != qk:
         return None

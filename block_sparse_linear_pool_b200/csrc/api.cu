@@ -3,6 +3,7 @@
 // allocates device memory or synchronises a stream (except
 // sla_get_device_status).
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -36,11 +37,27 @@ inline int union_record(const Plan& p) {
   return 8 + ((cap + 7) & ~7);
 }
 
-// The persistent fused kernel serves bf16 Q K^T and P V when two CTAs fit an SM
-// (its shared memory holds the union records); the other paths use the
-// per-tile kernel.
+// The persistent fused kernel serves bf16 Q K^T and P V (the inference and the
+// training forward) when two CTAs fit an SM (its shared memory holds the union
+// records); the 8-bit paths and the rest use the per-tile kernel.
 inline bool pt_eligible(const Plan& p) {
   return !p.fp8 && !p.pv8 && fused_pt_smem_bytes(p.d, union_record(p)) <= 113 * 1024;
+}
+
+// The split-union kernel (one tile per SM, two softmax warpgroups, a 6-stage
+// ring) needs up to 227 KB of shared memory.
+inline bool sk_eligible(const Plan& p) {
+  return !p.fp8 && !p.pv8 && fused_sk_smem_bytes(p.d, union_record(p)) <= 227 * 1024;
+}
+
+// Which bf16 kernel schedule runs: the SLA_FUSED_SCHEDULE environment variable
+// ("split" or "persistent") overrides the default (persistent), for comparisons.
+inline bool prefer_split() {
+  static const int v = [] {
+    const char* e = std::getenv("SLA_FUSED_SCHEDULE");
+    return (e && std::strcmp(e, "split") == 0) ? 1 : 0;
+  }();
+  return v != 0;
 }
 
 struct Layout {
@@ -288,6 +305,14 @@ sla_status_t precompute_impl(const Plan& pl, const sla_params_t* p, const void* 
   return cuda_status(launch_kv_prep(mk, mv, mo, a, pl.d, s));
 }
 
+// [BH][M][NN] bf16 rows as TMA store tiles of 64 columns x 128 rows (128-byte swizzle)
+bool map_rows_out(CUtensorMap* m, void* base, int M, const Plan& pl) {
+  const uint64_t dims[3] = {(uint64_t)pl.NN, (uint64_t)M, (uint64_t)pl.BH};
+  const uint64_t str[2] = {(uint64_t)pl.NN * 2, (uint64_t)M * pl.NN * 2};
+  const uint32_t box[3] = {64, 128, 1};
+  return encode(m, base, 3, dims, str, box);
+}
+
 sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, void* ws,
                             cudaStream_t s) {
   const Layout L = layout_of(pl);
@@ -301,6 +326,8 @@ sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, vo
   const uint64_t sb[2] = {(uint64_t)pl.NN * 2, (uint64_t)pl.Tkv * pl.NN * 2};
   const uint32_t bb[3] = {64, 64, 1};
   if (!encode(&ma, mm, 3, da, sa, ba) || !encode(&mb, hz, 3, db, sb, bb)) return SLA_ERR_CUDA;
+  CUtensorMap mo;
+  if (!map_rows_out(&mo, at<__nv_bfloat16>(ws, L.hagg), pl.Tq, pl)) return SLA_ERR_CUDA;
   MargArgs a;
   a.Hout = at<__nv_bfloat16>(ws, L.hagg);
   a.err = at<int>(ws, L.err);
@@ -308,7 +335,7 @@ sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, vo
   a.Tkv = pl.Tkv;
   a.NN = pl.NN;
   a.ktiles = (pl.Tkv + 63) / 64;
-  return cuda_status(launch_marg_gemm(ma, mb, a, pl.BH, s));
+  return cuda_status(launch_marg_gemm(ma, mb, mo, a, pl.BH, s));
 }
 
 // out[bh][m][:] = sum_k A[bh][m][k] B[bh][k][:] for the 0/1 matrix A (bf16
@@ -323,6 +350,8 @@ sla_status_t zero_one_product(const Plan& pl, const __nv_bfloat16* A, int M, int
   const uint64_t sb[2] = {(uint64_t)pl.NN * 2, (uint64_t)Kdim * pl.NN * 2};
   const uint32_t bb[3] = {64, 64, 1};
   if (!encode(&ma, A, 3, da, sa, ba) || !encode(&mb, B, 3, db, sb, bb)) return SLA_ERR_CUDA;
+  CUtensorMap mo;
+  if (!map_rows_out(&mo, out, M, pl)) return SLA_ERR_CUDA;
   MargArgs a;
   a.Hout = out;
   a.err = err;
@@ -330,7 +359,7 @@ sla_status_t zero_one_product(const Plan& pl, const __nv_bfloat16* A, int M, int
   a.Tkv = Kdim;
   a.NN = pl.NN;
   a.ktiles = (Kdim + 63) / 64;
-  return cuda_status(launch_marg_gemm(ma, mb, a, pl.BH, s));
+  return cuda_status(launch_marg_gemm(ma, mb, mo, a, pl.BH, s));
 }
 
 // which two query blocks share a tile; for the persistent kernel also each tile's union list
@@ -338,7 +367,7 @@ sla_status_t pairing_impl(const Plan& pl, const int32_t* lut, void* ws, cudaStre
   const Layout L = layout_of(pl);
   int2* pairs = at<int2>(ws, L.pairs);
   SLA_TRY(cuda_status(launch_pairing(lut, pl.BH, pl.Tq, pl.nh, pl.Tkv, at<uint16_t>(ws, L.pov), pairs, s)));
-  if (pt_eligible(pl))
+  if (pt_eligible(pl) || sk_eligible(pl))
     SLA_TRY(cuda_status(launch_tile_union(lut, pairs, pl.BH, pl.Tq, pl.Tkv, pl.nh, union_record(pl),
                                           at<uint16_t>(ws, L.ulist), at<int>(ws, L.err), s)));
   return SLA_OK;
@@ -363,7 +392,8 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
     return SLA_ERR_CUDA;
   // which two query blocks share a CTA (similar critical lists: a smaller union)
   int2* pairs = at<int2>(ws, L.pairs);
-  const bool pt = pt_eligible(pl) && !lse && !o_sparse;
+  const bool pt = pt_eligible(pl);
+  const bool sk = sk_eligible(pl) && (prefer_split() || !pt);
   if (pair) SLA_TRY(pairing_impl(pl, lut, ws, s));
   {
     // H_i^T as (a, b, i, bh) tiles of d x d; Z_i as one unswizzled row of d
@@ -452,9 +482,10 @@ sla_status_t fused_impl(const Plan& pl, const sla_params_t* p, const void* Q, co
   a.ulist = at<uint16_t>(ws, L.ulist);
   a.urec = union_record(pl);
   a.BH = pl.BH;
-  if (pt) {
+  if (sk || pt) {
     const int nsm = sm_count();
     if (nsm <= 0) return SLA_ERR_CUDA;
+    if (sk) return cuda_status(launch_fused_sk(mq, mk, mv, mh, a, pl.d, nsm, s));
     return cuda_status(launch_fused_pt(mq, mk, mv, mh, mz, a, pl.d, nsm, s));
   }
   const int qk8 = pl.fp8 ? (pl.qk_int8 ? 2 : 1) : 0;
@@ -894,6 +925,37 @@ sla_status_t sla_attention_host_workspace_size(const sla_params_t* p, size_t* by
   return SLA_OK;
 }
 
+// Copy streams and events of the host-buffer entry point, created once per device
+// (no device memory): chunk c's host-to-device copies run on `h2d`, its compute
+// on the caller's stream, its device-to-host copy on `d2h`.
+constexpr int kHostChunks = 6;
+struct HostPipes {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr, in[kHostChunks] = {}, out[kHostChunks] = {};
+  bool ok = false;
+};
+
+HostPipes* host_pipes() {
+  static std::mutex mu;
+  static HostPipes pipes[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  HostPipes& hp = pipes[dev];
+  if (!hp.ok) {
+    bool good = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming) == cudaSuccess &&
+                cudaEventCreateWithFlags(&hp.end, cudaEventDisableTiming) == cudaSuccess;
+    for (int c = 0; c < kHostChunks && good; ++c)
+      good = cudaEventCreateWithFlags(&hp.in[c], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&hp.out[c], cudaEventDisableTiming) == cudaSuccess;
+    if (!good) return nullptr;
+    hp.ok = true;
+  }
+  return &hp;
+}
+
 sla_status_t sla_attention_host(const sla_params_t* p, const void* Q_host, const void* K_host,
                                 const void* V_host, const float* proj_w, const float* proj_b,
                                 const float* alpha, const float* Wq, const float* Wk,
@@ -907,16 +969,49 @@ sla_status_t sla_attention_host(const sla_params_t* p, const void* Q_host, const
   SLA_TRY(check_ws(pl, workspace, workspace_bytes, WS_HOST));
   const Layout L = layout_of(pl);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const size_t act = (size_t)pl.BH * pl.N * pl.d * 2;
-  void* dq = at<void>(workspace, L.hq);
-  void* dk = at<void>(workspace, L.hk);
-  void* dv = at<void>(workspace, L.hv);
-  void* dout = at<void>(workspace, L.ho);
-  SLA_TRY(cuda_status(cudaMemcpyAsync(dq, Q_host, act, cudaMemcpyHostToDevice, s)));
-  SLA_TRY(cuda_status(cudaMemcpyAsync(dk, K_host, act, cudaMemcpyHostToDevice, s)));
-  SLA_TRY(cuda_status(cudaMemcpyAsync(dv, V_host, act, cudaMemcpyHostToDevice, s)));
-  SLA_TRY(attention_impl(pl, p, dq, dk, dv, proj_w, proj_b, alpha, Wq, Wk, dout, workspace, s));
-  return cuda_status(cudaMemcpyAsync(O_host, dout, act, cudaMemcpyDeviceToHost, s));
+  HostPipes* hp = host_pipes();
+  if (!hp) return SLA_ERR_CUDA;
+  uint8_t* dq = at<uint8_t>(workspace, L.hq);
+  uint8_t* dk = at<uint8_t>(workspace, L.hk);
+  uint8_t* dv = at<uint8_t>(workspace, L.hv);
+  uint8_t* dout = at<uint8_t>(workspace, L.ho);
+  const uint8_t* qh = static_cast<const uint8_t*>(Q_host);
+  const uint8_t* kh = static_cast<const uint8_t*>(K_host);
+  const uint8_t* vh = static_cast<const uint8_t*>(V_host);
+  uint8_t* oh = static_cast<uint8_t*>(O_host);
+  // The (batch, head) problems are independent: chunks of heads are copied in,
+  // computed and copied out in a pipeline, so the copies of one chunk overlap the
+  // compute of another (the chunks' computations share the workspace one after
+  // the other on `stream`).
+  const int nchunk = pl.BH < kHostChunks ? pl.BH : kHostChunks;
+  const size_t head_bytes = (size_t)pl.N * pl.d * 2;
+  SLA_TRY(cuda_status(cudaEventRecord(hp->start, s)));
+  SLA_TRY(cuda_status(cudaStreamWaitEvent(hp->h2d, hp->start, 0)));
+  SLA_TRY(cuda_status(cudaStreamWaitEvent(hp->d2h, hp->start, 0)));
+  for (int c = 0; c < nchunk; ++c) {
+    const int b0 = (int)((int64_t)pl.BH * c / nchunk), b1 = (int)((int64_t)pl.BH * (c + 1) / nchunk);
+    const size_t off = (size_t)b0 * head_bytes, bytes = (size_t)(b1 - b0) * head_bytes;
+    SLA_TRY(cuda_status(cudaMemcpyAsync(dq + off, qh + off, bytes, cudaMemcpyHostToDevice, hp->h2d)));
+    SLA_TRY(cuda_status(cudaMemcpyAsync(dk + off, kh + off, bytes, cudaMemcpyHostToDevice, hp->h2d)));
+    SLA_TRY(cuda_status(cudaMemcpyAsync(dv + off, vh + off, bytes, cudaMemcpyHostToDevice, hp->h2d)));
+    SLA_TRY(cuda_status(cudaEventRecord(hp->in[c], hp->h2d)));
+    SLA_TRY(cuda_status(cudaStreamWaitEvent(s, hp->in[c], 0)));
+    // the chunk as a problem of its own: B = 1, H = its heads, contiguous
+    sla_params_t sp = *p;
+    sp.B = 1;
+    sp.H = b1 - b0;
+    const int64_t st[3] = {(int64_t)sp.H * pl.N * pl.d, (int64_t)pl.N * pl.d, (int64_t)pl.d};
+    for (int i = 0; i < 3; ++i) sp.stride_q[i] = sp.stride_k[i] = sp.stride_v[i] = sp.stride_o[i] = st[i];
+    Plan sub;
+    SLA_TRY(make_plan(&sp, &sub));
+    SLA_TRY(attention_impl(sub, &sp, dq + off, dk + off, dv + off, proj_w, proj_b, alpha ? alpha + b0 : nullptr,
+                           Wq, Wk, dout + off, workspace, s));
+    SLA_TRY(cuda_status(cudaEventRecord(hp->out[c], s)));
+    SLA_TRY(cuda_status(cudaStreamWaitEvent(hp->d2h, hp->out[c], 0)));
+    SLA_TRY(cuda_status(cudaMemcpyAsync(oh + off, dout + off, bytes, cudaMemcpyDeviceToHost, hp->d2h)));
+  }
+  SLA_TRY(cuda_status(cudaEventRecord(hp->end, hp->d2h)));
+  return cuda_status(cudaStreamWaitEvent(s, hp->end, 0));
 }
 
 sla_status_t sla_aggregate_marginal(const sla_params_t* p, const int8_t* mc, const void* hz,

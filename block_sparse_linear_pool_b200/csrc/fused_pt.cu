@@ -31,7 +31,9 @@
 //   warp 1      MMA issuer: S, P V, and the two linear-branch chains
 //   warps 2-5   one query row per thread: online softmax with exp2 (lazy
 //               rescale of O only when the running max grows by more than 2^8),
-//               P over S in TMEM; then phi~(q), P', and the epilogue
+//               P over S in TMEM; then (training forward) the row's LSE and its
+//               sparse-branch output o^s from O before the linear term joins it,
+//               phi~(q), P', and the epilogue
 //
 // TMEM: S_0 in columns [0, 64), S_1 in [64, 128) (P', after the loop, over
 // [0, d)), O in [128, 128 + d).
@@ -508,6 +510,29 @@ __global__ void __launch_bounds__(192, 2)
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(q_full, it & 1, a.err, DEV_TIMEOUT_TMA));
       if (!ok) break;
       tc_fence_after();
+      const int n = 64 * blk + (r & 63);
+      const bool store = (n < a.N) && (half == 0 || has_b);
+      if (a.lse || a.os) {
+        // for the backward: the sparse branch alone (O holds only P V so far) and the
+        // log-sum-exp of the row's scaled critical scores, sum_t exp(s_t) = 2^m l
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        if (a.lse && store) a.lse[(int64_t)bh * a.N + n] = (m + log2f(l)) * 0.6931471805599453f;
+        if (a.os) {
+#pragma unroll 1
+          for (int c0o = 0; c0o < D; c0o += 32) {
+            uint32_t ov[32];
+            tmem_ld32(tO + c0o, ov);
+            tmem_ld_wait();
+            if (store) {
+              float4* od = reinterpret_cast<float4*>(a.os + ((int64_t)bh * a.N + n) * D + c0o);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                od[v] = make_float4(__uint_as_float(ov[4 * v]) * inv_l, __uint_as_float(ov[4 * v + 1]) * inv_l,
+                                    __uint_as_float(ov[4 * v + 2]) * inv_l, __uint_as_float(ov[4 * v + 3]) * inv_l);
+            }
+          }
+        }
+      }
       // e = phi~(q) as bf16 pairs; the denominator's sums use the rounded values
       uint32_t pe[D / 2];
       float esum = 0.f, edotz = 0.f;
@@ -573,8 +598,6 @@ __global__ void __launch_bounds__(192, 2)
       if (!__all_sync(0xffffffffu, mbar_wait(o_full, it & 1, a.err, DEV_TIMEOUT_MMA))) { ok = false; break; }
       tc_fence_after();
       {
-        const int n = 64 * blk + (r & 63);
-        const bool store = (n < a.N) && (half == 0 || has_b);
         const int b = bh / a.H, h = bh % a.H;
         __nv_bfloat16* orow = a.O + (int64_t)b * a.so0 + (int64_t)h * a.so1 + (int64_t)n * a.so2;
 #pragma unroll 1

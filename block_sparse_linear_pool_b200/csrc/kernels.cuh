@@ -175,7 +175,9 @@ cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int 
                                int Tkvp, bool all, cudaStream_t s);
 cudaError_t launch_marg_matrix_t(const int8_t* mc, __nv_bfloat16* mt, int BH, int Tq, int Tkv,
                                  int Tqp, bool all, cudaStream_t s);
-cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const MargArgs& a,
+// mapO: the output rows [BH][M][NN] bf16, box 64 x 128, 128-byte swizzle (TMA stores)
+cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapO,
+                             const MargArgs& a,
                              int BH, cudaStream_t s);
 
 cudaError_t launch_quant_fp8(const QuantArgs& a, int BH, cudaStream_t s);
@@ -189,6 +191,11 @@ cudaError_t launch_fused_pt(const CUtensorMap& mapQ, const CUtensorMap& mapK, co
                             const CUtensorMap& mapH, const CUtensorMap& mapZ, const FusedArgs& a, int D, int nsm,
                             cudaStream_t s);
 size_t fused_pt_smem_bytes(int D, int urec);
+// The split-union kernel: one tile per CTA, its steps alternating between two
+// softmax warpgroups (bf16 Q K^T and P V); one CTA per SM.
+cudaError_t launch_fused_sk(const CUtensorMap& mapQ, const CUtensorMap& mapK, const CUtensorMap& mapV,
+                            const CUtensorMap& mapH, const FusedArgs& a, int D, int nsm, cudaStream_t s);
+size_t fused_sk_smem_bytes(int D, int urec);
 cudaError_t launch_vquant_fp8(const __nv_bfloat16* V, const int64_t* sv, int H, int N, int T, int BH, int D,
                               unsigned int* vmax, uint8_t* V8T, cudaStream_t s);
 

@@ -11,9 +11,11 @@
 //   marg_matrix_kernel  M_c (int8) -> Mmarg (bf16 0/1, rows padded to T_kvp); all
 //                       ones for the variant whose linear branch covers every block
 //   marg_gemm_kernel    persistent, 128 x 256 output tiles, K step 64,
-//                       4-stage TMA ring, two TMEM accumulators; warp 0 loads,
-//                       warp 1 issues tcgen05.mma, warps 2-5 drain TMEM and
-//                       store bf16 while the next tile accumulates.
+//                       3-stage TMA ring, two TMEM accumulators; warp 0 loads,
+//                       warp 1 issues tcgen05.mma, warps 2-5 drain TMEM into a
+//                       swizzled bf16 staging tile that one thread stores with
+//                       TMA (whole 128-byte lines), while the next tile
+//                       accumulates.
 #include "kernels.cuh"
 
 namespace sla {
@@ -47,12 +49,16 @@ __global__ void marg_matrix_t_kernel(const int8_t* __restrict__ mc, __nv_bfloat1
 }
 
 namespace {
-constexpr int BM = 128, BN = 256, BK = 64, NST = 4;
+constexpr int BM = 128, BN = 256, BK = 64, NST = 3;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int B_BYTES = BK * BN * 2;   // 32 KB
 constexpr int STAGE = A_BYTES + B_BYTES;
-constexpr int OFF_BAR = NST * STAGE;
+constexpr int OFF_OUT = NST * STAGE;   // bf16 output tile: 4 chunks of [128 rows][64 columns]
+constexpr int OUT_BYTES = BM * BN * 2;
+constexpr int OFF_BAR = OFF_OUT + OUT_BYTES;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
+
+__device__ __forceinline__ void epi_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 }  // namespace
 
 // Persistent: CTA c takes tiles c, c + G, c + 2G, ... with the M tile index
@@ -61,6 +67,7 @@ constexpr int SMEM = OFF_BAR + 256 + 1024;
 // the main loop of the next.
 __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant__ CUtensorMap mapA,
                                                            const __grid_constant__ CUtensorMap mapB,
+                                                           const __grid_constant__ CUtensorMap mapO,
                                                            MargArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -154,39 +161,54 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
   } else {
     const int q4 = w & 3;
     const int row = 32 * q4 + ln;
+    const bool leader = tid == 64;  // issues the TMA stores of the output tile
+    uint8_t* sO = sm + OFF_OUT;
+    // Every epilogue warp runs every tile's two named barriers, also after a
+    // wait gave up (then it only skips the work), so none is left waiting.
+    bool ok = true;
     int lt = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++lt) {
       const int m0 = (t % Mt) * BM, n0 = ((t / Mt) % Nt) * BN, bh = t / (Mt * Nt);
       const int ab = lt & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (lt >> 1) & 1, a.err, DEV_TIMEOUT_MMA)))
-        break;
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (lt >> 1) & 1, a.err, DEV_TIMEOUT_MMA));
       tc_fence_after();
-      const int i = m0 + row;
-      const uint32_t taddr = tacc + 256 * ab + ((uint32_t)(32 * q4) << 16);
-      __nv_bfloat16* out = a.Hout + ((int64_t)bh * a.Tq + i) * a.NN;
+      // the previous tile's TMA stores have finished reading the staging tile
+      if (leader) bulk_wait_read_all();
+      epi_sync();
+      if (ok) {
+        const uint32_t taddr = tacc + 256 * ab + ((uint32_t)(32 * q4) << 16);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(taddr + c0, r);
-        tmem_ld_wait();
-        if (i < a.Tq) {
+        for (int c0 = 0; c0 < BN; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c0, r);
+          tmem_ld_wait();
+          // row `row` of chunk c0 / 64, 16-byte units (c0 % 64) / 8 .. + 3, 128-byte swizzle
+          uint8_t* chunk = sO + (c0 >> 6) * (BM * 128) + row * 128;
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
-            const int n = n0 + c0 + v * 8;
-            if (n < a.NN) {
-              uint4 q;
-              q.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-              q.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-              q.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-              q.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-              *reinterpret_cast<uint4*>(out + n) = q;
-            }
+            const int unit = ((c0 & 63) >> 3) + v;
+            uint4 q;
+            q.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+            q.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+            q.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+            q.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+            *reinterpret_cast<uint4*>(chunk + ((unit ^ (row & 7)) << 4)) = q;
           }
         }
+        // the accumulator has been read: the MMA warp may reuse it
+        tc_fence_before();
+        mbar_arrive(&acc_empty[ab]);
+        fence_proxy_async_smem();
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty[ab]);
+      epi_sync();
+      if (leader && ok) {
+#pragma unroll
+        for (int c = 0; c < BN / 64; ++c)
+          if (n0 + 64 * c < a.NN) tma_store_3d(&mapO, sO + c * (BM * 128), n0 + 64 * c, m0, bh);
+        bulk_commit_group();
+      }
     }
+    if (leader) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -212,8 +234,8 @@ cudaError_t launch_marg_matrix_t(const int8_t* mc, __nv_bfloat16* mt, int BH, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const MargArgs& a,
-                             int BH, cudaStream_t s) {
+cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapO,
+                             const MargArgs& a, int BH, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(marg_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM);
   if (e != cudaSuccess) return e;
@@ -223,7 +245,7 @@ cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, c
   const int ntiles = ((a.NN + BN - 1) / BN) * ((a.Tq + BM - 1) / BM) * BH;
   MargArgs b = a;
   b.BH = BH;
-  marg_gemm_kernel<<<ntiles < sms ? ntiles : sms, 192, SMEM, s>>>(mapA, mapB, b);
+  marg_gemm_kernel<<<ntiles < sms ? ntiles : sms, 192, SMEM, s>>>(mapA, mapB, mapO, b);
   return cudaGetLastError();
 }
 

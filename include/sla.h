@@ -282,11 +282,17 @@ sla_status_t sla_attention(const sla_params_t* p, const void* Q, const void* K, 
 /*
  * sla_attention with the activations in host memory: copies Q, K, V (host,
  * contiguous [B,H,N,d] bf16; page-locked memory makes the copies
- * asynchronous) into device staging buffers inside the workspace, runs
- * sla_attention and copies O back to O_host, all enqueued on `stream`.  The
- * parameters proj_w, proj_b, alpha, Wq, Wk stay device pointers.  The call
- * returns after enqueueing; O_host is valid once the stream has been
- * synchronised.  The params' strides must describe contiguous tensors.
+ * asynchronous) into device staging buffers inside the workspace, runs the
+ * forward and copies O back to O_host.  The (batch, head) problems are split
+ * into up to 6 chunks that are pipelined: chunk c + 1 is copied in while chunk
+ * c is computed on `stream` and chunk c - 1 is copied out, on two copy streams
+ * the library creates once per device (with their events; no device memory).
+ * Everything is ordered after the work already enqueued on `stream`, and
+ * `stream` waits for the last copy, so O_host is valid once `stream` has been
+ * synchronised.  The parameters proj_w, proj_b, alpha, Wq, Wk stay device
+ * pointers.  The params' strides must describe contiguous tensors.  Calls that
+ * overlap on one device must use different workspaces and may not run
+ * concurrently (the copy streams are shared).
  */
 sla_status_t sla_attention_host_workspace_size(const sla_params_t* p, size_t* bytes);
 sla_status_t sla_attention_host(const sla_params_t* p, const void* Q_host, const void* K_host,

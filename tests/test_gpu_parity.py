@@ -246,6 +246,25 @@ def test_lowbit_qk_and_fp8_pv_small_against_emulation(qk):
     _run(data, cfg)
 
 
+@pytest.mark.parametrize("N,kh,kl", [(2048, 0.1, 0.5), (4000, 0.05, 0.75), (640, 0.5, 0.2)])
+def test_mask_exact_ties_rank_the_lower_block_first(N, kh, kl):
+    # K built from 3 distinct 64-token blocks repeated: the pooled keys of the full
+    # blocks, and so the logits of a row, tie exactly (same bits in fp32 and fp64;
+    # a partial last block pools to a value of its own), and the mask must equal
+    # the oracle's order definition on every entry, ties included
+    g = torch.Generator().manual_seed(N)
+    d, T = 128, -(-N // 64)
+    Q = torch.randn(1, 2, N, d, generator=g).to(torch.bfloat16)
+    base = torch.randn(1, 2, 3, 64, d, generator=g)
+    K = base[:, :, torch.arange(T) % 3].reshape(1, 2, T * 64, d)[:, :, :N].to(torch.bfloat16).contiguous()
+    cfg = bnd.SlaConfig(k_h=kh, k_l=kl, combine="proj")
+    Qd, Kd = Q.cuda(), K.cuda()
+    mc, lut = bnd.sla_predict_mask(Qd, Kd, cfg)
+    torch.cuda.synchronize()
+    M_ref, logits, _ = O.predict_mask(_np(Q), _np(K), _oparams(cfg))
+    np.testing.assert_array_equal(mc.cpu().numpy().reshape(M_ref.shape), M_ref)
+
+
 def test_smooth_k_changes_nothing_graded():
     data = _small(1, 2, 2048, 128, seed=3)
     data["K"] = (data["K"].float() + 2.0).to(torch.bfloat16)
