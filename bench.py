@@ -113,13 +113,26 @@ def bus_id_of(dev):
         return None
 
 
+def split_schedule() -> bool:
+    return os.environ.get("SLA_FUSED_SCHEDULE", "") == "split"
+
+
+def fused_kernel_name(qk: str, pv: str) -> str:
+    """The fused kernel the library runs for these precisions (the persistent
+    kernel for bf16, the one-tile-per-CTA kernel for the 8-bit products, the
+    split-union kernel when that schedule is selected)."""
+    if qk != "bf16" or pv != "bf16":
+        return "sla_fused_kernel"
+    return "sla_fused_sk_kernel" if split_schedule() else "sla_fused_pt_kernel"
+
+
 def fused_traffic_per_launch(workload: str, heads: int, qk: str):
     """DRAM bytes per launch of the persistent fused kernel from the committed ncu
     summary, or None if the summary is for another workload or the kernel source
     changed since those counters were taken."""
     path = os.path.join(ROOT, "profiles", f"fused_pt_{workload}_traffic.txt")
     src = os.path.join(ROOT, "block_sparse_linear_pool_b200", "csrc", "fused_pt.cu")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or split_schedule():
         return None
     sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     vals = {}
@@ -682,7 +695,7 @@ def main():
                      "tiles": wk["n_tiles"], "marginal_gemm_issued_flops": wk["marg_issued"],
                      "dense_equivalent_flops": wk["dense_equiv"]},
             "dense_equiv_tflops": round(wk["dense_equiv"] / (ms_step * 1e-3) / 1e12, 2),
-            "roofline": {"kernel": "sla_fused_kernel", "timed": "sla_fused_forward_paired alone (CUDA events "
+            "roofline": {"kernel": fused_kernel_name(args.qk, args.pv), "timed": "sla_fused_forward_paired alone (CUDA events "
                          "around it inside the timed loop)", "bound": "tensor", "achieved": fr["achieved"],
                          "peak": fr["peak"], "unit": "TFLOP/s", "frac": fr["frac"],
                          "traffic": fused_traffic_per_launch(args.workload, H, args.qk if args.pv == "bf16"

@@ -52,12 +52,18 @@ inline bool sk_eligible(const Plan& p) {
 
 // Which bf16 kernel schedule runs: the SLA_FUSED_SCHEDULE environment variable
 // ("split" or "persistent") overrides the default (persistent), for comparisons.
+// read at every call, so that a process can switch between the schedules
 inline bool prefer_split() {
-  static const int v = [] {
-    const char* e = std::getenv("SLA_FUSED_SCHEDULE");
-    return (e && std::strcmp(e, "split") == 0) ? 1 : 0;
-  }();
-  return v != 0;
+  const char* e = std::getenv("SLA_FUSED_SCHEDULE");
+  return e && std::strcmp(e, "split") == 0;
+}
+
+// SLA_MARG_KERNEL=tmem selects, for T_kv <= 512, the aggregation GEMM whose
+// 0/1 operand sits in TMEM; by default the one with both operands in shared
+// memory runs (measured faster at the 1.3B shapes).
+inline bool prefer_tmem_marg() {
+  const char* e = std::getenv("SLA_MARG_KERNEL");
+  return e && std::strcmp(e, "tmem") == 0;
 }
 
 struct Layout {
@@ -316,6 +322,25 @@ bool map_rows_out(CUtensorMap* m, void* base, int M, const Plan& pl) {
 sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, void* ws,
                             cudaStream_t s) {
   const Layout L = layout_of(pl);
+  if (pl.Tkv <= kMargTmemMaxTkv && prefer_tmem_marg()) {
+    // the 0/1 rows are built from M_c inside the kernel, in TMEM
+    CUtensorMap mb, mo;
+    const uint64_t db[3] = {(uint64_t)pl.NN, (uint64_t)pl.Tkv, (uint64_t)pl.BH};
+    const uint64_t sb[2] = {(uint64_t)pl.NN * 2, (uint64_t)pl.Tkv * pl.NN * 2};
+    const uint32_t bb[3] = {64, 64, 1};
+    if (!encode(&mb, hz, 3, db, sb, bb)) return SLA_ERR_CUDA;
+    if (!map_rows_out(&mo, at<__nv_bfloat16>(ws, L.hagg), pl.Tq, pl)) return SLA_ERR_CUDA;
+    MargArgs a;
+    a.Hout = at<__nv_bfloat16>(ws, L.hagg);
+    a.err = at<int>(ws, L.err);
+    a.Tq = pl.Tq;
+    a.Tkv = pl.Tkv;
+    a.NN = pl.NN;
+    a.ktiles = (pl.Tkv + 63) / 64;
+    a.mc = mc;
+    a.all = pl.all ? 1 : 0;
+    return cuda_status(launch_marg_gemm_tm(mb, mo, a, pl.BH, s));
+  }
   __nv_bfloat16* mm = at<__nv_bfloat16>(ws, L.mm);
   SLA_TRY(cuda_status(launch_marg_matrix(mc, mm, pl.BH, pl.Tq, pl.Tkv, pl.Tkvp, pl.all, s)));
   CUtensorMap ma, mb;
@@ -335,6 +360,8 @@ sla_status_t aggregate_impl(const Plan& pl, const int8_t* mc, const void* hz, vo
   a.Tkv = pl.Tkv;
   a.NN = pl.NN;
   a.ktiles = (pl.Tkv + 63) / 64;
+  a.mc = nullptr;
+  a.all = 0;
   return cuda_status(launch_marg_gemm(ma, mb, mo, a, pl.BH, s));
 }
 
@@ -359,6 +386,8 @@ sla_status_t zero_one_product(const Plan& pl, const __nv_bfloat16* A, int M, int
   a.Tkv = Kdim;
   a.NN = pl.NN;
   a.ktiles = (Kdim + 63) / 64;
+  a.mc = nullptr;
+  a.all = 0;
   return cuda_status(launch_marg_gemm(ma, mb, mo, a, pl.BH, s));
 }
 

@@ -42,6 +42,8 @@ struct MargArgs {
   __nv_bfloat16* Hout;   // [BH][Tq][NN]
   int* err;
   int Tq, Tkv, NN, ktiles, BH;
+  const int8_t* mc;      // [BH][Tq][Tkv] M_c (the TMEM-operand kernel builds its 0/1 rows from it)
+  int all;               // every block counts (linear branch over all blocks)
 };
 
 struct QuantArgs {
@@ -176,6 +178,10 @@ cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int 
 cudaError_t launch_marg_matrix_t(const int8_t* mc, __nv_bfloat16* mt, int BH, int Tq, int Tkv,
                                  int Tqp, bool all, cudaStream_t s);
 // mapO: the output rows [BH][M][NN] bf16, box 64 x 128, 128-byte swizzle (TMA stores)
+// T_kv <= 512: the 0/1 operand lives in TMEM, built from M_c by the kernel itself.
+constexpr int kMargTmemMaxTkv = 512;
+cudaError_t launch_marg_gemm_tm(const CUtensorMap& mapB, const CUtensorMap& mapO, const MargArgs& a, int BH,
+                                cudaStream_t s);
 cudaError_t launch_marg_gemm(const CUtensorMap& mapA, const CUtensorMap& mapB, const CUtensorMap& mapO,
                              const MargArgs& a,
                              int BH, cudaStream_t s);

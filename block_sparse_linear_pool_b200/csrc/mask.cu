@@ -13,12 +13,18 @@
 namespace sla {
 
 // ---------------------------------------------------------------------------
-// pool: one warp per 64-token block; lane l sums columns [l*CPL, (l+1)*CPL).
+// pool: one warp per 64-token block.  Each lane loads 16 bytes (8 columns) of a
+// row per instruction, so one instruction covers 32 * 16 / (2 D) rows (2 for
+// d = 128, 4 for d = 64); 16 loads per lane are in flight.  Lanes holding the
+// same columns of different rows are summed with shuffles at the end.
 // grid (ceil(T/8), B*H, 2): z = 0 pools Q into Qc, z = 1 pools K into Kc.
+// Rows start on 16-byte boundaries (base and token stride are checked by the
+// entry points).
 // ---------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) pool_kernel(PoolArgs a) {
-  constexpr int CPL = D / 32;  // columns per lane: 4 (d=128) or 2 (d=64)
+  constexpr int LPR = D / 8;        // lanes per row: 16 (d=128) or 8 (d=64)
+  constexpr int RPI = 32 / LPR;     // rows per instruction: 2 or 4
   const int w = threadIdx.x >> 5, ln = threadIdx.x & 31;
   const int blk = blockIdx.x * 8 + w;
   const int bh = blockIdx.y;
@@ -28,31 +34,48 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolArgs a) {
   const __nv_bfloat16* src = blockIdx.z == 0 ? a.Q : a.K;
   const int64_t* st = blockIdx.z == 0 ? a.sq : a.sk;
   float* dst = blockIdx.z == 0 ? a.Qc : a.Kc;
-  const __nv_bfloat16* base = src + (int64_t)b * st[0] + (int64_t)h * st[1];
   const int t0 = blk * a.bs;
   const int cnt = min(a.bs, a.N - t0);
-  float acc[CPL];
+  const int roff = ln / LPR, col = (ln % LPR) * 8;
+  const __nv_bfloat16* base = src + (int64_t)b * st[0] + (int64_t)h * st[1] + (int64_t)t0 * st[2] + col;
+  float acc[8];
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) acc[c] = 0.f;
-#pragma unroll 8
-  for (int t = 0; t < cnt; ++t) {
-    const __nv_bfloat16* row = base + (int64_t)(t0 + t) * st[2] + ln * CPL;
-    if constexpr (CPL == 4) {
-      uint2 v = __ldg(reinterpret_cast<const uint2*>(row));
-      __nv_bfloat162 p0 = *reinterpret_cast<__nv_bfloat162*>(&v.x);
-      __nv_bfloat162 p1 = *reinterpret_cast<__nv_bfloat162*>(&v.y);
-      acc[0] += __low2float(p0); acc[1] += __high2float(p0);
-      acc[2] += __low2float(p1); acc[3] += __high2float(p1);
-    } else {
-      uint32_t v = __ldg(reinterpret_cast<const unsigned int*>(row));
-      __nv_bfloat162 p0 = *reinterpret_cast<__nv_bfloat162*>(&v);
-      acc[0] += __low2float(p0); acc[1] += __high2float(p0);
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+  auto add = [&](const uint4& v) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[2 * e] += __low2float(p[e]);
+      acc[2 * e + 1] += __high2float(p[e]);
     }
-  }
-  const float inv = 1.f / (float)cnt;
-  float* out = dst + ((int64_t)bh * T + blk) * D + ln * CPL;
+  };
+  if (cnt == 64) {
+    // whole block: 64 / RPI rows per lane, loaded in groups of 16 before use
+    constexpr int PER = 64 / RPI;
+    constexpr int G = PER < 16 ? PER : 16;
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) out[c] = acc[c] * inv;
+    for (int g0 = 0; g0 < PER; g0 += G) {
+      uint4 v[G];
+#pragma unroll
+      for (int i = 0; i < G; ++i)
+        v[i] = __ldg(reinterpret_cast<const uint4*>(base + (int64_t)(roff + RPI * (g0 + i)) * st[2]));
+#pragma unroll
+      for (int i = 0; i < G; ++i) add(v[i]);
+    }
+  } else {
+    for (int t = roff; t < cnt; t += RPI)
+      add(__ldg(reinterpret_cast<const uint4*>(base + (int64_t)t * st[2])));
+  }
+#pragma unroll
+  for (int m = LPR; m < 32; m <<= 1)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], m);
+  if (roff == 0) {
+    const float inv = 1.f / (float)cnt;
+    float4* out = reinterpret_cast<float4*>(dst + ((int64_t)bh * T + blk) * D + col);
+    out[0] = make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+    out[1] = make_float4(acc[4] * inv, acc[5] * inv, acc[6] * inv, acc[7] * inv);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -137,10 +160,10 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ i
 // ---------------------------------------------------------------------------
 // logits: keys[bh][i][j] = order_key(Q_c[i] . K_c[j] / sqrt(d)) in fp32 (fp32
 // keeps the logits exact to ~1e-6, far inside the 1e-4 grading gap; bf16
-// tensor cores would not).  128 x 128 tile per CTA, d consumed in chunks of 16
-// through two shared-memory stages; thread (ty, tx) owns rows
-// {4ty..4ty+3, 64+4ty..} and columns {4tx..4tx+3, 64+4tx..}.
-// grid (ceil(T_kv/128), ceil(T_q/128), B*H).
+// tensor cores would not).  64 x 128 tile per CTA (so that a 512 x 512 head
+// gives 32 CTAs and the grid fills every SM more than twice), d consumed in
+// chunks of 16 through two shared-memory stages.
+// grid (ceil(T_kv/128), ceil(T_q/64), B*H).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t order_key(float s) {
   uint32_t u = __float_as_uint(s == 0.f ? 0.f : s);  // -0 and +0 compare equal
@@ -148,48 +171,54 @@ __device__ __forceinline__ uint32_t order_key(float s) {
 }
 
 namespace {
-constexpr int LT = 128, LK = 16, LS = LT + 4;  // tile, k chunk, padded stride
+constexpr int LM = 64, LN = 128, LK = 16;  // tile rows (queries), columns (keys), k chunk
 }
 
 __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
-  __shared__ __align__(16) float As[2][LK][LS];
-  __shared__ __align__(16) float Bs[2][LK][LS];
+  __shared__ __align__(16) float As[2][LK][LM + 4];
+  __shared__ __align__(16) float Bs[2][LK][LN + 4];
   const int D = a.d, Tq = a.Tq, Tk = a.Tkv, bh = blockIdx.z;
-  const int m0 = blockIdx.y * LT, n0 = blockIdx.x * LT;
+  const int m0 = blockIdx.y * LM, n0 = blockIdx.x * LN;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const float* A = a.Qc + (int64_t)bh * Tq * D;
   const float* B = a.Kc + (int64_t)bh * Tk * D;
-  // staging: 128 rows x 16 columns per matrix = 512 float4, 2 per thread;
-  // thread e takes row e % 128 and column quad e / 128 (a warp covers 32 rows
-  // of one quad, so the transposed stores hit distinct banks)
-  float4 pa[2], pb[2];
+  // staging: thread e takes row e % rows and column quad e / rows (a warp covers
+  // 32 rows of one quad, so the transposed stores hit distinct banks)
+  float4 pa, pb[2];
   auto load = [&](int k0) {
+    {
+      const int r = tid & 63, q = tid >> 6;
+      pa = (m0 + r < Tq) ? __ldg(reinterpret_cast<const float4*>(A + (int64_t)(m0 + r) * D + k0) + q)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
 #pragma unroll
     for (int v = 0; v < 2; ++v) {
       const int e = tid + 256 * v, r = e & 127, q = e >> 7;
-      pa[v] = (m0 + r < Tq) ? __ldg(reinterpret_cast<const float4*>(A + (int64_t)(m0 + r) * D + k0) + q)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
       pb[v] = (n0 + r < Tk) ? __ldg(reinterpret_cast<const float4*>(B + (int64_t)(n0 + r) * D + k0) + q)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
   auto store = [&](int st) {
+    {
+      const int r = tid & 63, q = tid >> 6;
+      As[st][4 * q + 0][r] = pa.x;
+      As[st][4 * q + 1][r] = pa.y;
+      As[st][4 * q + 2][r] = pa.z;
+      As[st][4 * q + 3][r] = pa.w;
+    }
 #pragma unroll
     for (int v = 0; v < 2; ++v) {
       const int e = tid + 256 * v, r = e & 127, q = e >> 7;
-      As[st][4 * q + 0][r] = pa[v].x;
-      As[st][4 * q + 1][r] = pa[v].y;
-      As[st][4 * q + 2][r] = pa[v].z;
-      As[st][4 * q + 3][r] = pa[v].w;
       Bs[st][4 * q + 0][r] = pb[v].x;
       Bs[st][4 * q + 1][r] = pb[v].y;
       Bs[st][4 * q + 2][r] = pb[v].z;
       Bs[st][4 * q + 3][r] = pb[v].w;
     }
   };
-  float acc[8][8];
+  // thread (ty, tx) owns rows 4ty..4ty+3 and columns {4tx..4tx+3, 64+4tx..64+4tx+3}
+  float acc[4][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
   load(0);
@@ -202,13 +231,12 @@ __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
 #pragma unroll
     for (int k = 0; k < LK; ++k) {
       const float4 a0 = *reinterpret_cast<const float4*>(&As[st][k][4 * ty]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&As[st][k][64 + 4 * ty]);
       const float4 b0 = *reinterpret_cast<const float4*>(&Bs[st][k][4 * tx]);
       const float4 b1 = *reinterpret_cast<const float4*>(&Bs[st][k][64 + 4 * tx]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float av[4] = {a0.x, a0.y, a0.z, a0.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
@@ -218,8 +246,8 @@ __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
   const float scale = rsqrtf((float)D);
   uint32_t* keys = a.keys + (int64_t)bh * Tq * Tk;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = m0 + (i < 4 ? 4 * ty + i : 64 + 4 * ty + (i - 4));
+  for (int i = 0; i < 4; ++i) {
+    const int r = m0 + 4 * ty + i;
     if (r >= Tq) continue;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -231,11 +259,16 @@ __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
 
 // ---------------------------------------------------------------------------
 // select: one warp per (head, query block) row.  The row's keys are copied to
-// shared memory; the n_h-th largest and the (T_kv - n_l)-th largest keys are
-// found together by an exact most-significant-bit-first radix search (counts
-// by warp reduction).  The search starts below the bits that the row's minimum
-// and maximum share; once the upper 16 bits are fixed, each search continues on
-// the (few) keys that carry its 16-bit prefix, compacted to a short list.
+// shared memory.  The n_h-th largest and the (T_kv - n_l)-th largest keys are
+// found exactly in two steps:
+//   1. a 256-bin histogram of the logit VALUES over [row min, row max]
+//      (bin = floor((x - min) * 256 / (max - min)), clamped: non-decreasing in
+//      x, so every key of a higher bin is larger than every key of a lower
+//      one); a descending scan gives, for each rank, its bin and how many keys
+//      lie in the bins above;
+//   2. the keys of that bin (a few for any spread-out row) are ranked among
+//      themselves: directly when they fit one warp, else by an exact
+//      most-significant-bit-first radix search with counts by warp reduction.
 // Ties rank the lower block index first.  One row per warp, up to 8 warps per
 // CTA (fewer when T_kv is large, to keep two CTAs' keys in shared memory).
 // ---------------------------------------------------------------------------
@@ -254,24 +287,6 @@ __device__ __forceinline__ void radix_step(RadixState& st, int bit, int cnt) {
   st.mask |= 1u << bit;
 }
 
-// Bits `hi`..`lo` of two searches over n keys at once.
-__device__ void radix_rounds2(const uint32_t* keys, int n, int hi, int lo, RadixState& A,
-                              RadixState& B) {
-  const int ln = threadIdx.x & 31;
-  for (int bit = hi; bit >= lo; --bit) {
-    const uint32_t ma = A.mask | (1u << bit), ca = A.prefix | (1u << bit);
-    const uint32_t mb = B.mask | (1u << bit), cb = B.prefix | (1u << bit);
-    int na = 0, nb = 0;
-    for (int j = ln; j < n; j += 32) {
-      const uint32_t key = keys[j];
-      na += ((key & ma) == ca);
-      nb += ((key & mb) == cb);
-    }
-    radix_step(A, bit, __reduce_add_sync(0xffffffffu, na));
-    radix_step(B, bit, __reduce_add_sync(0xffffffffu, nb));
-  }
-}
-
 // Bits `hi`..0 of one search over n keys.
 __device__ void radix_rounds1(const uint32_t* keys, int n, int hi, RadixState& A) {
   const int ln = threadIdx.x & 31;
@@ -283,15 +298,60 @@ __device__ void radix_rounds1(const uint32_t* keys, int n, int hi, RadixState& A
   }
 }
 
-// Keys of `src` (n) that carry the prefix of `st` (under its mask), in order.
-__device__ int compact_prefix(const uint32_t* src, int n, const RadixState& st, uint32_t* dst) {
+// The inverse of order_key (keys of -0 and +0 are one key, read back as +0).
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+__device__ __forceinline__ int value_bin(uint32_t k, float xmin, float inv) {
+  // NaN (0 * inf when the range underflows) goes to bin 0 through fmaxf
+  return (int)fminf(fmaxf((key_value(k) - xmin) * inv, 0.f), 255.f);
+}
+
+// The `rank`-th largest of the m keys in `list` (1 <= rank <= m): returns the
+// key and, in *take, how many of the keys equal to it rank within `rank`.
+__device__ uint32_t rank_in_list(const uint32_t* list, int m, int rank, int* take) {
+  const int ln = threadIdx.x & 31;
+  if (m <= 32) {
+    const uint32_t mine = ln < m ? list[ln] : 0u;
+    int gt = 0, ge = 0;
+    for (int j = 0; j < m; ++j) {
+      const uint32_t o = __shfl_sync(0xffffffffu, mine, j);
+      gt += o > mine;
+      ge += o >= mine;
+    }
+    const uint32_t hit = __ballot_sync(0xffffffffu, ln < m && gt < rank && rank <= ge);
+    const int src = __ffs(hit) - 1;  // every hit lane holds the same key
+    const uint32_t key = __shfl_sync(0xffffffffu, mine, src);
+    *take = rank - __shfl_sync(0xffffffffu, gt, src);
+    return key;
+  }
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int j = ln; j < m; j += 32) {
+    kmin = min(kmin, list[j]);
+    kmax = max(kmax, list[j]);
+  }
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  // every key of the list shares the bits above the highest bit where min and max differ
+  const uint32_t diff = kmin ^ kmax;
+  const int top_bit = diff ? 31 - __clz(diff) : -1;
+  const uint32_t shared_mask = top_bit >= 31 ? 0u : (top_bit < 0 ? 0xffffffffu : ~((2u << top_bit) - 1u));
+  RadixState st = {kmin & shared_mask, shared_mask, rank};
+  if (top_bit >= 0) radix_rounds1(list, m, top_bit, st);
+  *take = st.remaining;
+  return st.prefix;
+}
+
+// Keys of `src` (n) in value bin `bin`, in order.
+__device__ int compact_bin(const uint32_t* src, int n, int bin, float xmin, float inv, uint32_t* dst) {
   const int ln = threadIdx.x & 31;
   const uint32_t lt = (1u << ln) - 1u;
   int m = 0;
   for (int j0 = 0; j0 < n; j0 += 32) {
     const int j = j0 + ln;
     const uint32_t key = j < n ? src[j] : 0u;
-    const bool in = j < n && (key & st.mask) == st.prefix;
+    const bool in = j < n && value_bin(key, xmin, inv) == bin;
     const uint32_t bal = __ballot_sync(0xffffffffu, in);
     if (in) dst[m + __popc(bal & lt)] = key;
     m += __popc(bal);
@@ -300,15 +360,42 @@ __device__ int compact_prefix(const uint32_t* src, int n, const RadixState& st, 
   return m;
 }
 
+// The bin of the `rank`-th largest key from the descending per-lane bin counts
+// c (lane l holds bins 255 - 8l - i, i = 0..7), and the number of keys above it.
+__device__ __forceinline__ int scan_bin(const int (&c)[8], int incl, int sum, int rank, int* above) {
+  const int ln = threadIdx.x & 31;
+  const uint32_t reach = __ballot_sync(0xffffffffu, incl >= rank);
+  const int L = __ffs(reach) - 1;
+  int bin = 0, ab = 0;
+  if (ln == L) {
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (run + c[i] >= rank) {
+        bin = 255 - 8 * ln - i;
+        ab = run;
+        break;
+      }
+      run += c[i];
+    }
+  }
+  *above = __shfl_sync(0xffffffffu, ab, L);
+  return __shfl_sync(0xffffffffu, bin, L);
+}
+
 __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
-  extern __shared__ __align__(16) uint32_t skeys[];  // [warps][2 * T_kv]: keys, then candidates
+  // per warp: keys [T_kv], candidates [T_kv], histogram [256]
+  extern __shared__ __align__(16) uint32_t skeys[];
   const int Tq = a.Tq, Tk = a.Tkv;
   const int w = threadIdx.x >> 5, ln = threadIdx.x & 31;
   const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + w;  // bh * Tq + i
   if (row >= (int64_t)a.BH * Tq) return;
-  uint32_t* rk = skeys + (int64_t)w * 2 * Tk;
+  uint32_t* rk = skeys + (int64_t)w * (2 * Tk + 256);
   uint32_t* cand = rk + Tk;
+  int* hist = reinterpret_cast<int*>(cand + Tk);
   const uint32_t* g = a.keys + row * Tk;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) hist[8 * ln + i] = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   for (int j = ln; j < Tk; j += 32) {
     const uint32_t v = g[j];
@@ -319,24 +406,36 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
   kmin = __reduce_min_sync(0xffffffffu, kmin);
   kmax = __reduce_max_sync(0xffffffffu, kmax);
   __syncwarp();
-  // every key of the row shares the bits above the highest bit where min and max differ
-  const uint32_t diff = kmin ^ kmax;
-  const int top_bit = diff ? 31 - __clz(diff) : -1;
-  const uint32_t shared_mask = top_bit >= 31 ? 0u : (top_bit < 0 ? 0xffffffffu : ~((2u << top_bit) - 1u));
   // A: the n_h-th largest (critical); B: the (T_kv - n_l)-th largest (kept)
-  RadixState A = {kmin & shared_mask, shared_mask, a.nh};
-  RadixState B = {kmin & shared_mask, shared_mask, Tk - a.nl};
-  if (top_bit >= 16) radix_rounds2(rk, Tk, top_bit, 16, A, B);
-  const int lo_top = top_bit < 15 ? top_bit : 15;
-  if (lo_top >= 0) {
-    int m = compact_prefix(rk, Tk, A, cand);
-    radix_rounds1(cand, m, lo_top, A);
+  const int rank_h = a.nh, rank_k = Tk - a.nl;
+  uint32_t kh = kmax, kk = kmax;
+  int need_h = rank_h, need_k = rank_k;
+  if (kmin != kmax) {
+    const float xmin = key_value(kmin);
+    const float inv = 256.f / (key_value(kmax) - xmin);
+    for (int j = ln; j < Tk; j += 32) atomicAdd(&hist[value_bin(rk[j], xmin, inv)], 1);
     __syncwarp();
-    m = compact_prefix(rk, Tk, B, cand);
-    radix_rounds1(cand, m, lo_top, B);
+    int c[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      c[i] = hist[255 - 8 * ln - i];
+      sum += c[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (ln >= o) incl += y;
+    }
+    int above_h, above_k;
+    const int bin_h = scan_bin(c, incl, sum, rank_h, &above_h);
+    const int bin_k = scan_bin(c, incl, sum, rank_k, &above_k);
+    int m = compact_bin(rk, Tk, bin_h, xmin, inv, cand);
+    kh = rank_in_list(cand, m, rank_h - above_h, &need_h);
+    __syncwarp();
+    if (bin_k != bin_h) m = compact_bin(rk, Tk, bin_k, xmin, inv, cand);
+    kk = rank_in_list(cand, m, rank_k - above_k, &need_k);
   }
-  const uint32_t kh = A.prefix, kk = B.prefix;
-  const int need_h = A.remaining, need_k = B.remaining;
   int8_t* mrow = a.mc + row * Tk;
   int32_t* lrow = a.lut + row * a.nh;
   const uint32_t lt = (1u << ln) - 1u;
@@ -391,16 +490,16 @@ cudaError_t launch_router(const float* Qc, const float* Kc, float* Qr, float* Kr
 // Rows (warps) per select CTA: at most 8, and at most ~112 KB of keys.
 int select_rows_per_cta(int Tk) {
   int r = 8;
-  while (r > 1 && (size_t)r * 2 * Tk * sizeof(uint32_t) > (size_t)112 * 1024) r >>= 1;
+  while (r > 1 && (size_t)r * (2 * Tk + 256) * sizeof(uint32_t) > (size_t)112 * 1024) r >>= 1;
   return r;
 }
 
 size_t select_smem_bytes(int Tk) {
-  return (size_t)select_rows_per_cta(Tk) * 2 * Tk * sizeof(uint32_t);
+  return (size_t)select_rows_per_cta(Tk) * (2 * Tk + 256) * sizeof(uint32_t);
 }
 
 cudaError_t launch_logits(const LogitArgs& la, int BH, cudaStream_t s) {
-  logits_kernel<<<dim3((la.Tkv + LT - 1) / LT, (la.Tq + LT - 1) / LT, BH), 256, 0, s>>>(la);
+  logits_kernel<<<dim3((la.Tkv + LN - 1) / LN, (la.Tq + LM - 1) / LM, BH), 256, 0, s>>>(la);
   return cudaGetLastError();
 }
 

@@ -194,6 +194,24 @@ def test_small_shapes(B, H, N, d, kh, kl, combine):
     _run(data, cfg, own_mask=True)
 
 
+# The library's alternative kernels, selected per call through the environment:
+# the aggregation GEMM with its 0/1 operand in TMEM and the split-union fused
+# schedule.
+@pytest.mark.parametrize("switch", [("SLA_MARG_KERNEL", "tmem"), ("SLA_FUSED_SCHEDULE", "split")])
+@pytest.mark.parametrize("B,H,N,d,kh,kl,combine,over_all", [
+    (1, 2, 1000, 64, 0.10, 0.50, "proj", False),     # ragged tail, T_kv = 16
+    (1, 3, 2049, 128, 0.05, 0.70, "alpha", False),   # odd T_q (33)
+    (1, 1, 3000, 128, 0.10, 0.40, "proj", True),     # linear branch over every block
+])
+def test_alternative_kernels(monkeypatch, switch, B, H, N, d, kh, kl, combine, over_all):
+    monkeypatch.setenv(*switch)
+    data = _small(B, H, N, d, seed=N + d + 3)
+    cfg = bnd.SlaConfig(k_h=kh, k_l=kl, combine=combine, linear_over_all=over_all)
+    if combine == "proj":
+        data["Wq"] = data["Wk"] = None
+    _run(data, cfg, own_mask=True)
+
+
 @pytest.mark.parametrize("B,H,N,d,kh,kl,combine,phi,over_all", [
     (1, 2, 1000, 64, 0.10, 0.50, "proj", "elu1", False),    # elu + 1 feature map
     (1, 2, 2049, 128, 0.05, 0.70, "alpha", "elu1", False),
@@ -330,10 +348,11 @@ def test_fp8_pv_wan14b_720p_sla2_full_size_sampled(wan14):
     _check_lowbit_exact(_run14(wan14, "bf16", "fp8_e4m3"))
 
 
-_XFAIL_LOWBIT = ("measured on the oracle's own emulation of the same quantisation at these sampled "
-                 "blocks: E4M3 Q K^T 7.4% max-abs, E4M3 Q K^T + P V 7.4%, INT8 Q K^T + E4M3 P V 6.6% "
-                 "against the stated 6%; E4M3 keeps 3 mantissa bits, so per-block (or per-row) scales "
-                 "and K smoothing leave a logit error of about 0.11 at logit std 3")
+_XFAIL_LOWBIT = ("measured at these sampled blocks against the unquantised oracle (kernel / the oracle's "
+                 "emulation of the same quantisation): E4M3 Q K^T 7.93% / 7.94% max-abs, E4M3 Q K^T + P V "
+                 "8.71% / 8.71%, INT8 Q K^T + E4M3 P V 5.99% / 6.03%, against the stated 6%; E4M3 keeps 3 "
+                 "mantissa bits, so per-block (or per-row) scales and K smoothing leave a logit error of "
+                 "about 0.11 at logit std 3, and the INT8 + E4M3 P V path sits on the bound")
 
 
 @pytest.mark.parametrize("qk,pv", [("fp8_e4m3", "bf16"), ("fp8_e4m3", "fp8_e4m3"), ("int8", "fp8_e4m3")])
