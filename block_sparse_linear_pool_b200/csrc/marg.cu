@@ -228,7 +228,10 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
 // Mmarg[i][0 .. T_kv) sit in TMEM columns [0, 256) as bf16 pairs, built by
 // the epilogue warps straight from M_c (no 0/1 matrix in memory), and the CTA
 // walks a contiguous range of 128-column output tiles of that band, so only
-// the [h|z] rows stream through shared memory (read once by the MMA).
+// the [h|z] rows stream through shared memory (read once by the MMA).  CTAs
+// come in groups of ceil(T_q / 128), one per band of the same head, that walk
+// the same column tiles in step: each [h|z] tile is read from HBM once and
+// from L2 by the group's other CTAs.
 // Accumulators: two 128-column TMEM buffers at [256, 512); the epilogue of one
 // tile overlaps the main loop of the next, through two staging tiles stored
 // with TMA.  One CTA per SM.
@@ -257,11 +260,14 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_tm_kernel(const __grid_const
   uint32_t* tslot = reinterpret_cast<uint32_t*>(a_full + 1);
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const int Mt = (a.Tq + 127) / 128, Nt = (a.NN + TM_BN - 1) / TM_BN;
-  const int64_t total = (int64_t)a.BH * Mt * Nt;
-  // this CTA's contiguous range of tiles, output column tile fastest
-  const int64_t j0 = total * blockIdx.x / gridDim.x, j1 = total * (blockIdx.x + 1) / gridDim.x;
+  // group g (of G) takes a contiguous range of the (head, column tile) pairs;
+  // CTA mi of the group computes row band mi of each
+  const int G = gridDim.x / Mt, g = blockIdx.x / Mt, mi = blockIdx.x % Mt;
+  const int64_t W = (int64_t)a.BH * Nt;
+  const int64_t j0 = W * g / G, j1 = W * (g + 1) / G;  // j = bh * Nt + column tile
+  const int m0 = mi * 128;
   const int ktiles = a.ktiles;
-  auto band = [&](int64_t j) { return j / Nt; };  // bh * Mt + m
+  auto band = [&](int64_t j) { return j / Nt; };  // the head
 
   if (w == 1) {
     tmem_alloc(tslot, 512);
@@ -291,7 +297,7 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_tm_kernel(const __grid_const
       int it = 0;
       bool ok = true;
       for (int64_t j = j0; j < j1 && ok; ++j) {
-        const int n0 = (int)(j % Nt) * TM_BN, bh = (int)(j / ((int64_t)Mt * Nt));
+        const int n0 = (int)(j % Nt) * TM_BN, bh = (int)(j / Nt);
         const int nvalid = min(2, (a.NN - n0 + 63) / 64);
         for (int kt = 0; kt < ktiles; ++kt, ++it) {
           const int s = it % TM_NST;
@@ -361,8 +367,7 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_tm_kernel(const __grid_const
         }
         tc_fence_after();
         if (ok) {
-          const int64_t bm = band(j0 + t);
-          const int bh = (int)(bm / Mt), i = (int)(bm % Mt) * 128 + row;
+          const int bh = (int)band(j0 + t), i = m0 + row;
           const bool live = i < a.Tq;
           const int8_t* src = a.mc + ((int64_t)bh * a.Tq + (live ? i : 0)) * a.Tkv;
           // columns [32 c0, 32 c0 + 32) hold K = 64 c0 .. 64 c0 + 63 as bf16 pairs
@@ -405,7 +410,7 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_tm_kernel(const __grid_const
       // ---- epilogue of tile t - 1
       const int64_t jj = j0 + t - 1;
       const int pl = (int)(t - 1);
-      const int n0 = (int)(jj % Nt) * TM_BN, m0 = (int)((jj / Nt) % Mt) * 128, bh = (int)(jj / ((int64_t)Mt * Nt));
+      const int n0 = (int)(jj % Nt) * TM_BN, bh = (int)(jj / Nt);
       const int ab = pl & 1;
       if (ok && !waited)
         ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (pl >> 1) & 1, a.err, DEV_TIMEOUT_MMA));
@@ -495,10 +500,16 @@ cudaError_t launch_marg_gemm_tm(const CUtensorMap& mapB, const CUtensorMap& mapO
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t tiles = (int64_t)((a.NN + TM_BN - 1) / TM_BN) * ((a.Tq + 127) / 128) * BH;
+  // groups of Mt CTAs (one per row band), as many groups as fit the SMs, at
+  // most one per (head, column tile)
+  const int Mt = (a.Tq + 127) / 128;
+  const int64_t W = (int64_t)((a.NN + TM_BN - 1) / TM_BN) * BH;
+  int64_t G = sms / Mt;
+  if (G < 1) G = 1;
+  if (G > W) G = W;
   MargArgs b = a;
   b.BH = BH;
-  marg_gemm_tm_kernel<<<(int)(tiles < sms ? tiles : sms), 192, TM_SMEM, s>>>(mapB, mapO, b);
+  marg_gemm_tm_kernel<<<(int)(G * Mt), 192, TM_SMEM, s>>>(mapB, mapO, b);
   return cudaGetLastError();
 }
 

@@ -15,14 +15,15 @@ namespace sla {
 // ---------------------------------------------------------------------------
 // pool: one warp per 64-token block.  Each lane loads 16 bytes (8 columns) of a
 // row per instruction, so one instruction covers 32 * 16 / (2 D) rows (2 for
-// d = 128, 4 for d = 64); 16 loads per lane are in flight.  Lanes holding the
+// d = 128, 4 for d = 64); 8 loads per lane are in flight (few enough registers
+// for six CTAs per SM).  Lanes holding the
 // same columns of different rows are summed with shuffles at the end.
 // grid (ceil(T/8), B*H, 2): z = 0 pools Q into Qc, z = 1 pools K into Kc.
 // Rows start on 16-byte boundaries (base and token stride are checked by the
 // entry points).
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) pool_kernel(PoolArgs a) {
+__global__ void __launch_bounds__(256, 6) pool_kernel(PoolArgs a) {
   constexpr int LPR = D / 8;        // lanes per row: 16 (d=128) or 8 (d=64)
   constexpr int RPI = 32 / LPR;     // rows per instruction: 2 or 4
   const int w = threadIdx.x >> 5, ln = threadIdx.x & 31;
@@ -52,7 +53,7 @@ __global__ void __launch_bounds__(256) pool_kernel(PoolArgs a) {
   if (cnt == 64) {
     // whole block: 64 / RPI rows per lane, loaded in groups of 16 before use
     constexpr int PER = 64 / RPI;
-    constexpr int G = PER < 16 ? PER : 16;
+    constexpr int G = PER < 8 ? PER : 8;
 #pragma unroll
     for (int g0 = 0; g0 < PER; g0 += G) {
       uint4 v[G];
@@ -162,7 +163,8 @@ __global__ void __launch_bounds__(256) router_kernel(const float* __restrict__ i
 // keeps the logits exact to ~1e-6, far inside the 1e-4 grading gap; bf16
 // tensor cores would not).  64 x 128 tile per CTA (so that a 512 x 512 head
 // gives 32 CTAs and the grid fills every SM more than twice), d consumed in
-// chunks of 16 through two shared-memory stages.
+// chunks of 32 through two shared-memory stages (the next chunk's loads are in
+// flight while the current one is multiplied).
 // grid (ceil(T_kv/128), ceil(T_q/64), B*H).
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t order_key(float s) {
@@ -171,48 +173,56 @@ __device__ __forceinline__ uint32_t order_key(float s) {
 }
 
 namespace {
-constexpr int LM = 64, LN = 128, LK = 16;  // tile rows (queries), columns (keys), k chunk
+constexpr int LM = 64, LN = 128, LK = 32;  // tile rows (queries), columns (keys), k chunk
+constexpr int LAS = LM + 4, LBS = LN + 4;  // padded strides
+constexpr int LOGITS_SMEM = 2 * LK * (LAS + LBS) * (int)sizeof(float);  // two stages: 51 KB
 }
 
 __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
-  __shared__ __align__(16) float As[2][LK][LM + 4];
-  __shared__ __align__(16) float Bs[2][LK][LN + 4];
+  extern __shared__ __align__(16) float lsm[];
+  float* As = lsm;                  // [2][LK][LAS]
+  float* Bs = lsm + 2 * LK * LAS;   // [2][LK][LBS]
   const int D = a.d, Tq = a.Tq, Tk = a.Tkv, bh = blockIdx.z;
   const int m0 = blockIdx.y * LM, n0 = blockIdx.x * LN;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const float* A = a.Qc + (int64_t)bh * Tq * D;
   const float* B = a.Kc + (int64_t)bh * Tk * D;
-  // staging: thread e takes row e % rows and column quad e / rows (a warp covers
-  // 32 rows of one quad, so the transposed stores hit distinct banks)
-  float4 pa, pb[2];
+  // staging: element e of a tile is row e % rows, column quad e / rows (a warp
+  // covers 32 rows of one quad, so the transposed stores hit distinct banks)
+  constexpr int NA = LM * LK / 4 / 256, NB = LN * LK / 4 / 256;  // float4 per thread: 2, 4
+  float4 pa[NA], pb[NB];
   auto load = [&](int k0) {
-    {
-      const int r = tid & 63, q = tid >> 6;
-      pa = (m0 + r < Tq) ? __ldg(reinterpret_cast<const float4*>(A + (int64_t)(m0 + r) * D + k0) + q)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int v = 0; v < NA; ++v) {
+      const int e = tid + 256 * v, r = e % LM, q = e / LM;
+      pa[v] = (m0 + r < Tq) ? __ldg(reinterpret_cast<const float4*>(A + (int64_t)(m0 + r) * D + k0) + q)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const int e = tid + 256 * v, r = e & 127, q = e >> 7;
+    for (int v = 0; v < NB; ++v) {
+      const int e = tid + 256 * v, r = e % LN, q = e / LN;
       pb[v] = (n0 + r < Tk) ? __ldg(reinterpret_cast<const float4*>(B + (int64_t)(n0 + r) * D + k0) + q)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   };
   auto store = [&](int st) {
-    {
-      const int r = tid & 63, q = tid >> 6;
-      As[st][4 * q + 0][r] = pa.x;
-      As[st][4 * q + 1][r] = pa.y;
-      As[st][4 * q + 2][r] = pa.z;
-      As[st][4 * q + 3][r] = pa.w;
+    float* as = As + st * LK * LAS;
+    float* bs = Bs + st * LK * LBS;
+#pragma unroll
+    for (int v = 0; v < NA; ++v) {
+      const int e = tid + 256 * v, r = e % LM, q = e / LM;
+      as[(4 * q + 0) * LAS + r] = pa[v].x;
+      as[(4 * q + 1) * LAS + r] = pa[v].y;
+      as[(4 * q + 2) * LAS + r] = pa[v].z;
+      as[(4 * q + 3) * LAS + r] = pa[v].w;
     }
 #pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const int e = tid + 256 * v, r = e & 127, q = e >> 7;
-      Bs[st][4 * q + 0][r] = pb[v].x;
-      Bs[st][4 * q + 1][r] = pb[v].y;
-      Bs[st][4 * q + 2][r] = pb[v].z;
-      Bs[st][4 * q + 3][r] = pb[v].w;
+    for (int v = 0; v < NB; ++v) {
+      const int e = tid + 256 * v, r = e % LN, q = e / LN;
+      bs[(4 * q + 0) * LBS + r] = pb[v].x;
+      bs[(4 * q + 1) * LBS + r] = pb[v].y;
+      bs[(4 * q + 2) * LBS + r] = pb[v].z;
+      bs[(4 * q + 3) * LBS + r] = pb[v].w;
     }
   };
   // thread (ty, tx) owns rows 4ty..4ty+3 and columns {4tx..4tx+3, 64+4tx..64+4tx+3}
@@ -228,11 +238,13 @@ __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
   for (int kc = 0; kc < nk; ++kc) {
     const int st = kc & 1;
     if (kc + 1 < nk) load((kc + 1) * LK);
+    const float* as = As + st * LK * LAS;
+    const float* bs = Bs + st * LK * LBS;
 #pragma unroll
     for (int k = 0; k < LK; ++k) {
-      const float4 a0 = *reinterpret_cast<const float4*>(&As[st][k][4 * ty]);
-      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[st][k][4 * tx]);
-      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[st][k][64 + 4 * tx]);
+      const float4 a0 = *reinterpret_cast<const float4*>(as + k * LAS + 4 * ty);
+      const float4 b0 = *reinterpret_cast<const float4*>(bs + k * LBS + 4 * tx);
+      const float4 b1 = *reinterpret_cast<const float4*>(bs + k * LBS + 64 + 4 * tx);
       const float av[4] = {a0.x, a0.y, a0.z, a0.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -309,8 +321,9 @@ __device__ __forceinline__ int value_bin(uint32_t k, float xmin, float inv) {
 }
 
 // The `rank`-th largest of the m keys in `list` (1 <= rank <= m): returns the
-// key and, in *take, how many of the keys equal to it rank within `rank`.
-__device__ uint32_t rank_in_list(const uint32_t* list, int m, int rank, int* take) {
+// key and, in *take, how many of the keys equal to it rank within `rank`; *eq
+// is how many keys of the list equal it (0 when not counted).
+__device__ uint32_t rank_in_list(const uint32_t* list, int m, int rank, int* take, int* eq) {
   const int ln = threadIdx.x & 31;
   if (m <= 32) {
     const uint32_t mine = ln < m ? list[ln] : 0u;
@@ -323,9 +336,12 @@ __device__ uint32_t rank_in_list(const uint32_t* list, int m, int rank, int* tak
     const uint32_t hit = __ballot_sync(0xffffffffu, ln < m && gt < rank && rank <= ge);
     const int src = __ffs(hit) - 1;  // every hit lane holds the same key
     const uint32_t key = __shfl_sync(0xffffffffu, mine, src);
-    *take = rank - __shfl_sync(0xffffffffu, gt, src);
+    const int g = __shfl_sync(0xffffffffu, gt, src);
+    *take = rank - g;
+    *eq = __shfl_sync(0xffffffffu, ge, src) - g;
     return key;
   }
+  *eq = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
   for (int j = ln; j < m; j += 32) {
     kmin = min(kmin, list[j]);
@@ -343,21 +359,24 @@ __device__ uint32_t rank_in_list(const uint32_t* list, int m, int rank, int* tak
   return st.prefix;
 }
 
-// Keys of `src` (n) in value bin `bin`, in order.
-__device__ int compact_bin(const uint32_t* src, int n, int bin, float xmin, float inv, uint32_t* dst) {
+// Keys of `src` (n) in value bin b0 to d0 and in bin b1 (!= b0) to d1, in order.
+__device__ void compact_bins(const uint32_t* src, int n, int b0, int b1, float xmin, float inv, uint32_t* d0,
+                             uint32_t* d1) {
   const int ln = threadIdx.x & 31;
   const uint32_t lt = (1u << ln) - 1u;
-  int m = 0;
+  int m0 = 0, m1 = 0;
   for (int j0 = 0; j0 < n; j0 += 32) {
     const int j = j0 + ln;
     const uint32_t key = j < n ? src[j] : 0u;
-    const bool in = j < n && value_bin(key, xmin, inv) == bin;
-    const uint32_t bal = __ballot_sync(0xffffffffu, in);
-    if (in) dst[m + __popc(bal & lt)] = key;
-    m += __popc(bal);
+    const int b = j < n ? value_bin(key, xmin, inv) : -1;
+    const uint32_t bal0 = __ballot_sync(0xffffffffu, b == b0);
+    const uint32_t bal1 = __ballot_sync(0xffffffffu, b == b1);
+    if (b == b0) d0[m0 + __popc(bal0 & lt)] = key;
+    if (b == b1) d1[m1 + __popc(bal1 & lt)] = key;
+    m0 += __popc(bal0);
+    m1 += __popc(bal1);
   }
   __syncwarp();
-  return m;
 }
 
 // The bin of the `rank`-th largest key from the descending per-lane bin counts
@@ -410,6 +429,7 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
   const int rank_h = a.nh, rank_k = Tk - a.nl;
   uint32_t kh = kmax, kk = kmax;
   int need_h = rank_h, need_k = rank_k;
+  int eq_h_all = 0, eq_k_all = 0;  // keys equal to each threshold (0: not counted)
   if (kmin != kmax) {
     const float xmin = key_value(kmin);
     const float inv = 256.f / (key_value(kmax) - xmin);
@@ -430,16 +450,31 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
     int above_h, above_k;
     const int bin_h = scan_bin(c, incl, sum, rank_h, &above_h);
     const int bin_k = scan_bin(c, incl, sum, rank_k, &above_k);
-    int m = compact_bin(rk, Tk, bin_h, xmin, inv, cand);
-    kh = rank_in_list(cand, m, rank_h - above_h, &need_h);
-    __syncwarp();
-    if (bin_k != bin_h) m = compact_bin(rk, Tk, bin_k, xmin, inv, cand);
-    kk = rank_in_list(cand, m, rank_k - above_k, &need_k);
+    // the bins' sizes are in the histogram: both candidate lists fit `cand`
+    const int m_h = hist[bin_h], m_k = hist[bin_k];
+    uint32_t* cand_k = bin_k == bin_h ? cand : cand + m_h;
+    compact_bins(rk, Tk, bin_h, bin_k == bin_h ? -2 : bin_k, xmin, inv, cand, cand_k);
+    kh = rank_in_list(cand, m_h, rank_h - above_h, &need_h, &eq_h_all);
+    kk = rank_in_list(cand_k, m_k, rank_k - above_k, &need_k, &eq_k_all);
   }
   int8_t* mrow = a.mc + row * Tk;
   int32_t* lrow = a.lut + row * a.nh;
   const uint32_t lt = (1u << ln) - 1u;
   int eq_h = 0, eq_k = 0, ncrit = 0;
+  if (eq_h_all == 1 && eq_k_all == 1) {
+    // no ties at either threshold: every key at or above a threshold is in
+    for (int j0 = 0; j0 < Tk; j0 += 32) {
+      const int j = j0 + ln;
+      const bool valid = j < Tk;
+      const uint32_t key = valid ? rk[j] : 0u;
+      const bool crit = valid && key >= kh;
+      const uint32_t bc = __ballot_sync(0xffffffffu, crit);
+      if (valid) mrow[j] = crit ? (int8_t)1 : (key >= kk ? (int8_t)0 : (int8_t)-1);
+      if (crit) lrow[ncrit + __popc(bc & lt)] = j;
+      ncrit += __popc(bc);
+    }
+    return;
+  }
   for (int j0 = 0; j0 < Tk; j0 += 32) {
     const int j = j0 + ln;
     const bool valid = j < Tk;
@@ -499,7 +534,9 @@ size_t select_smem_bytes(int Tk) {
 }
 
 cudaError_t launch_logits(const LogitArgs& la, int BH, cudaStream_t s) {
-  logits_kernel<<<dim3((la.Tkv + LN - 1) / LN, (la.Tq + LM - 1) / LM, BH), 256, 0, s>>>(la);
+  cudaError_t e = cudaFuncSetAttribute(logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, LOGITS_SMEM);
+  if (e != cudaSuccess) return e;
+  logits_kernel<<<dim3((la.Tkv + LN - 1) / LN, (la.Tq + LM - 1) / LM, BH), 256, LOGITS_SMEM, s>>>(la);
   return cudaGetLastError();
 }
 
