@@ -28,7 +28,9 @@
 //   warp 0      TMA producer: the tile's union record (bulk copy, two buffers),
 //               Q tile + Z rows, K and V of each entry, then H_a^T through the K
 //               ring and H_b^T through the V ring (one 64-column chunk per slot)
-//   warp 1      MMA issuer: S, P V, and the two linear-branch chains
+//   warp 1      MMA issuer (one thread, whose issue rate paces the loop: the
+//               shared-memory descriptors are formed once and advanced by
+//               constants): S, P V, and the two linear-branch chains
 //   warps 2-5   one query row per thread: online softmax with exp2 (lazy
 //               rescale of O only when the running max grows by more than 2^8),
 //               P over S in TMEM; then (training forward) the row's LSE and its
@@ -384,8 +386,14 @@ __global__ void __launch_bounds__(192, 2)
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
       const uint32_t id_pv = idesc_bf16(128, D, false, true);
       const uint32_t id_l = idesc_bf16(128, D, false, false);
-      const uint32_t q0 = smem_u32(sQ), k0 = smem_u32(sK), v0 = smem_u32(sV);
       const uint32_t tS = tbase + PT_COL_S, tO = tbase + PT_COL_O;
+      // Descriptors of ring slot 0 (and of Q); a byte offset o inside shared
+      // memory adds o >> 4 to the start-address field, which cannot carry out.
+      const uint64_t dQ = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK = sdesc_sw128(smem_u32(sK), 16, 1024);    // K tile or H_a chunk (K-major)
+      const uint64_t dVk = sdesc_sw128(smem_u32(sV), 16, 1024);   // H_b chunk (K-major)
+      const uint64_t dV = sdesc_sw128(smem_u32(sV), 8192, 1024);  // V tile (MN-major)
+      constexpr uint64_t SLOT = KT >> 4;
       uint32_t kuse = 0, vuse = 0, g = 0;  // ring uses, entries so far
       bool ok = true;
       int it = 0;
@@ -396,11 +404,10 @@ __global__ void __launch_bounds__(192, 2)
         if (first_of_tile && it > 0 && !mbar_wait(o_free, (it - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
         if (!mbar_wait(&v_full[vuse & 1], (vuse >> 1) & 1, a.err, DEV_TIMEOUT_TMA)) return false;
         tc_fence_after();
-        const uint32_t vt = v0 + (vuse & 1) * KT;
+        const uint64_t dv = dV + (vuse & 1) * SLOT;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ts(tO, tS + 64 * (ge & 1) + 8 * kk, sdesc_sw128(vt + kk * 2048, 8192, 1024), id_pv,
-                  (!first_of_tile || kk > 0) ? 1u : 0u);
+          umma_ts(tO, tS + 64 * (ge & 1) + 8 * kk, dv + kk * (2048 >> 4), id_pv, (!first_of_tile || kk > 0) ? 1u : 0u);
         umma_commit(&pv_done[ge & 1]);
         umma_commit(&v_empty[vuse & 1]);
         ++vuse;
@@ -417,13 +424,11 @@ __global__ void __launch_bounds__(192, 2)
           // score buffer ge & 1 still holds P_{ge-2}, whose P V this thread issued
           // earlier: tcgen05.mma ops of one thread run in issue order
           tc_fence_after();
-          const uint32_t kt = k0 + (kuse & 1) * KT;
+          const uint64_t dk = dK + (kuse & 1) * SLOT;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(q0 + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(kt + (kk / 4) * 8192 + (kk % 4) * 32, 16, 1024);
-            umma_ss(tS + 64 * (ge & 1), ad, bd, id_s, kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ss(tS + 64 * (ge & 1), dQ + ((kk / 4) * 16384 + (kk % 4) * 32) / 16,
+                    dk + ((kk / 4) * 8192 + (kk % 4) * 32) / 16, id_s, kk > 0 ? 1u : 0u);
           umma_commit(&s_full[ge & 1]);
           umma_commit(&k_empty[kuse & 1]);
           ++kuse;
@@ -438,14 +443,14 @@ __global__ void __launch_bounds__(192, 2)
           uint64_t* full = t == 0 ? k_full : v_full;
           uint64_t* empty = t == 0 ? k_empty : v_empty;
           uint32_t& use = t == 0 ? kuse : vuse;
-          const uint32_t base = t == 0 ? k0 : v0;
+          const uint64_t dbase = t == 0 ? dK : dVk;
           for (int c = 0; c < CH; ++c) {
             if (!mbar_wait(&full[use & 1], (use >> 1) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t ht = base + (use & 1) * KT;
+            const uint64_t dh = dbase + (use & 1) * SLOT;
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              umma_ts(tO, tS + t * (D / 2) + 8 * (4 * c + kk), sdesc_sw128(ht + kk * 32, 16, 1024), id_l, 1u);
+              umma_ts(tO, tS + t * (D / 2) + 8 * (4 * c + kk), dh + kk * (32 >> 4), id_l, 1u);
             umma_commit(&empty[use & 1]);
             ++use;
           }
