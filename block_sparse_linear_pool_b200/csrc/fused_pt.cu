@@ -175,14 +175,23 @@ __device__ __forceinline__ bool pt_softmax_entry(uint32_t tS, uint32_t tO, int n
         if (c + 32 >= nvalid) s1[c] = __float_as_uint(-INFINITY);
       }
     }
-    float t[32];
+    // row maximum with three-input max: 64 -> 22 -> 8 -> 3 -> 1
+    float t[22];
 #pragma unroll
-    for (int c = 0; c < 32; ++c) t[c] = fmaxf(__uint_as_float(s0[c]), __uint_as_float(s1[c]));
+    for (int i = 0; i < 21; ++i) {
+      const int e = 3 * i;  // values 0..31 from s0, 32..63 from s1
+      const float v0 = __uint_as_float(e < 32 ? s0[e] : s1[e - 32]);
+      const float v1 = __uint_as_float(e + 1 < 32 ? s0[e + 1] : s1[e + 1 - 32]);
+      const float v2 = __uint_as_float(e + 2 < 32 ? s0[e + 2] : s1[e + 2 - 32]);
+      t[i] = fmax3(v0, v1, v2);
+    }
+    t[21] = __uint_as_float(s1[31]);
 #pragma unroll
-    for (int st = 16; st >= 1; st >>= 1)
-#pragma unroll
-      for (int c = 0; c < st; ++c) t[c] = fmaxf(t[c], t[c + st]);
-    const float mx = t[0] * sl2;
+    for (int i = 0; i < 7; ++i) t[i] = fmax3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+    t[7] = t[21];
+    t[0] = fmax3(t[0], t[1], t[2]);
+    t[1] = fmax3(t[3], t[4], t[5]);
+    const float mx = fmax3(t[0], t[1], fmaxf(t[6], t[7])) * sl2;
     const bool first = (m == -INFINITY);
     grow = !first && (mx - m > PT_RESCALE_THRESHOLD);
     if (first) m = mx;  // O and l of this row are still exactly 0
@@ -190,24 +199,27 @@ __device__ __forceinline__ bool pt_softmax_entry(uint32_t tS, uint32_t tO, int n
       fsc = pt_ex2(m - mx);
       m = mx;
     }
-    const float nm = -m;
-    float u[32];
+    // p = 2^(s sl2 - m): the scaling in pairs (one instruction, two roundings
+    // identical to fmaf), the sum in pairs
+    const uint64_t sc2 = f2_pack(sl2, sl2), nm2 = f2_pack(-m, -m);
+    uint64_t u2[16];
 #pragma unroll
     for (int c = 0; c < 16; ++c) {
-      const float p0 = pt_ex2(fmaf(__uint_as_float(s0[2 * c]), sl2, nm));
-      const float p1 = pt_ex2(fmaf(__uint_as_float(s0[2 * c + 1]), sl2, nm));
-      const float p2 = pt_ex2(fmaf(__uint_as_float(s1[2 * c]), sl2, nm));
-      const float p3 = pt_ex2(fmaf(__uint_as_float(s1[2 * c + 1]), sl2, nm));
-      u[c] = p0 + p1;
-      u[16 + c] = p2 + p3;
+      float x0, x1, x2, x3;
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1])), sc2, nm2), x0, x1);
+      f2_unpack(f2_fma(f2_pack(__uint_as_float(s1[2 * c]), __uint_as_float(s1[2 * c + 1])), sc2, nm2), x2, x3);
+      const float p0 = pt_ex2(x0), p1 = pt_ex2(x1), p2 = pt_ex2(x2), p3 = pt_ex2(x3);
       pk[c] = pack_bf16x2(p0, p1);
       pk[16 + c] = pack_bf16x2(p2, p3);
+      u2[c] = f2_add(f2_pack(p0, p1), f2_pack(p2, p3));
     }
 #pragma unroll
-    for (int st = 16; st >= 1; st >>= 1)
+    for (int st = 8; st >= 1; st >>= 1)
 #pragma unroll
-      for (int c = 0; c < st; ++c) u[c] += u[c + st];
-    l = l * fsc + u[0];
+      for (int c = 0; c < st; ++c) u2[c] = f2_add(u2[c], u2[c + st]);
+    float ul, uh;
+    f2_unpack(u2[0], ul, uh);
+    l = l * fsc + (ul + uh);
   }
   tmem_st32(tS, pk);
   if (__any_sync(0xffffffffu, grow)) {
