@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(BwdRowsArgs a) {
       for (int c = ln; c < D; c += 32) g[c] = 0.f;
       if (ln == 0) {
         gden[r] = 0.f;
-        a.ld2[(int64_t)bh * a.Tq * 64 + n0 + r] = make_float2(INFINITY, 0.f);  // P = 0 there
+        a.ld2[(int64_t)bh * a.Tq * 64 + n0 + r] = make_float2(-INFINITY, 0.f);  // P = 0 there
       }
       continue;
     }
@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(256) bwd_rows_kernel(BwdRowsArgs a) {
       da += __shfl_xor_sync(0xffffffffu, da, o);
     }
     if (ln == 0) {
-      a.ld2[(int64_t)bh * a.Tq * 64 + n] = make_float2(a.lse[(int64_t)bh * a.N + n] * LOG2E, dd);
+      a.ld2[(int64_t)bh * a.Tq * 64 + n] = make_float2(-a.lse[(int64_t)bh * a.N + n] * LOG2E, -dd);
       gden[r] = -cl * dol / den[r];
     }
     dalpha_part += da;

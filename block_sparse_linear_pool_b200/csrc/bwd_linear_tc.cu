@@ -240,8 +240,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     const float gden = valid ? -cl * dol / den : 0.f;
     sgden[r] = gden;
-    if (valid) a.ld2[(int64_t)bh * a.Tq * 64 + n] = make_float2(a.lse[(int64_t)bh * a.N + n] * LOG2E_T, dd);
-    else if (t == 0 || has1) a.ld2[(int64_t)bh * a.Tq * 64 + n] = make_float2(INFINITY, 0.f);
+    if (valid) a.ld2[(int64_t)bh * a.Tq * 64 + n] = make_float2(-a.lse[(int64_t)bh * a.N + n] * LOG2E_T, -dd);
+    else if (t == 0 || has1) a.ld2[(int64_t)bh * a.Tq * 64 + n] = make_float2(-INFINITY, 0.f);
     if (a.combine == 1 && a.dalpha) {
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) da += __shfl_xor_sync(0xffffffffu, da, o);

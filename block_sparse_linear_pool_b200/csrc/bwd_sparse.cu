@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&sp_full[x], 1);
-      mbar_init(&ds_ready[x], 256);
+      mbar_init(&ds_ready[x], 8);
     }
     mbar_init(dq_done, 1);
     fence_barrier_init();
@@ -271,12 +271,13 @@ __global__ void __launch_bounds__(320, 1)
         const int x = k & 1, sk = k % NK;
         if (!mbar_wait(&ds_ready[x], (k >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
         tc_fence_after();
-        const uint32_t kt = smem_u32(sK + sk * L::T64);
+        // descriptors advanced by constants: a byte offset o adds o >> 4
+        const uint64_t dk = sdesc_sw128(smem_u32(sK), 8192, 1024) + (uint64_t)(sk * L::T64 >> 4);
         // keys 16 kk .. 16 kk + 15: packed at columns 32 (kk / 2) + 8 (kk % 2)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_ts(tbase + COL_DQ, tbase + 128 * x + 32 * (kk / 2) + 8 * (kk % 2),
-                  sdesc_sw128(kt + kk * 2048, 8192, 1024), id_q, (k > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tbase + COL_DQ, tbase + 128 * x + 32 * (kk / 2) + 8 * (kk % 2), dk + kk * (2048 >> 4), id_q,
+                  (k > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&k_empty[sk]);
         return true;
       };
@@ -287,14 +288,14 @@ __global__ void __launch_bounds__(320, 1)
         tc_fence_after();
         // S and dP into buffer x; its previous contents (entry k - 2) were consumed
         // by the dQ MMA issued earlier by this thread (in-order execution)
-        const uint32_t kt = smem_u32(sK + sk * L::T64), vt = smem_u32(sV + sv * L::T64);
+        const uint64_t dq0 = sdesc_sw128(q0, 16, 1024), do0 = sdesc_sw128(o0, 16, 1024);
+        const uint64_t dkt = sdesc_sw128(smem_u32(sK), 16, 1024) + (uint64_t)(sk * L::T64 >> 4);
+        const uint64_t dvt = sdesc_sw128(smem_u32(sV), 16, 1024) + (uint64_t)(sv * L::T64 >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32, offk = (kk / 4) * 8192 + (kk % 4) * 32;
-          umma_ss(tbase + 128 * x, sdesc_sw128(q0 + off, 16, 1024), sdesc_sw128(kt + offk, 16, 1024), id_s,
-                  kk > 0 ? 1u : 0u);
-          umma_ss(tbase + 128 * x + 64, sdesc_sw128(o0 + off, 16, 1024), sdesc_sw128(vt + offk, 16, 1024),
-                  id_s, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4, offk = ((kk / 4) * 8192 + (kk % 4) * 32) >> 4;
+          umma_ss(tbase + 128 * x, dq0 + off, dkt + offk, id_s, kk > 0 ? 1u : 0u);
+          umma_ss(tbase + 128 * x + 64, do0 + off, dvt + offk, id_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sp_full[x]);
         umma_commit(&v_empty[sv]);
@@ -314,11 +315,13 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
     const int n = 64 * (half == 0 ? ia : ibl) + (r & 63);
     const bool valid = (n < a.N) && (half == 0 || has_b);
-    // (lse log2 e, D) of this row; P = 0 on rows that do not exist
-    const float2 ld = valid ? a.ld2[(int64_t)bh * a.Tq * 64 + n] : make_float2(INFINITY, 0.f);
-    const float lse2 = ld.x, Dr = ld.y;
+    // (-lse log2 e, -D) of this row; P = 0 on rows that do not exist
+    const float2 ld = valid ? a.ld2[(int64_t)bh * a.Tq * 64 + n] : make_float2(-INFINITY, 0.f);
     const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
     const float sl2 = a.scale_log2;
+    // paired constants: P = 2^(s sl2 - lse2), dS = P (cs dP - D)
+    const uint64_t sc2 = f2_pack(sl2, sl2), nl2 = f2_pack(ld.x, ld.x), cs2 = f2_pack(cs, cs),
+                   nd2 = f2_pack(ld.y, ld.y);
     bool ok = true;
     for (int k = 0; k < U; ++k) {
       const int x = k & 1;
@@ -335,17 +338,20 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld32(ts + 32 * hs, s0);
         tmem_ld32(ts + 64 + 32 * hs, d0);
         tmem_ld_wait();
-        const int nvalid = a.N - 64 * (int)uidx[k] - 32 * hs;
+        const int nvalid = a.N - 64 * (int)uidx[k] - 32 * hs;  // warp-uniform
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          float ds[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 2 * c + e;
-            const float pr = col < nvalid ? ex2b(fmaf(__uint_as_float(s0[col]), sl2, -lse2)) : 0.f;
-            ds[e] = pr * (cs * __uint_as_float(d0[col]) - Dr);
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1])), sc2, nl2), x0, x1);
+          float p0 = ex2b(x0), p1 = ex2b(x1);
+          if (nvalid < 32) {  // columns past N (the last key block) have P = 0
+            p0 = 2 * c < nvalid ? p0 : 0.f;
+            p1 = 2 * c + 1 < nvalid ? p1 : 0.f;
           }
-          pk[c] = pack_bf16x2(ds[0], ds[1]);
+          const uint64_t g = f2_fma(f2_pack(__uint_as_float(d0[2 * c]), __uint_as_float(d0[2 * c + 1])), cs2, nd2);
+          float d0s, d1s;
+          f2_unpack(f2_mul(f2_pack(p0, p1), g), d0s, d1s);
+          pk[c] = pack_bf16x2(d0s, d1s);
         }
       } else {
 #pragma unroll
@@ -356,7 +362,8 @@ __global__ void __launch_bounds__(320, 1)
       tmem_st16(ts + 32 * hs, pk);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&ds_ready[x]);
+      __syncwarp();
+      if (ln == 0) mbar_arrive(&ds_ready[x]);  // one arrival per warp
     }
     if (ok && U >= 1) ok = __all_sync(0xffffffffu, mbar_wait(dq_done, 0, a.err, DEV_TIMEOUT_MMA));
     if (ok) {
@@ -472,7 +479,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&q_full[x], 1);
       mbar_init(&q_empty[x], 1);
       mbar_init(&sp_full[x], 1);
-      mbar_init(&ds_ready[x], 256);
+      mbar_init(&ds_ready[x], 8);
     }
     mbar_init(kv_done, 1);
     fence_barrier_init();
@@ -559,15 +566,16 @@ __global__ void __launch_bounds__(320, 1)
         const int x = e & 1;
         if (!mbar_wait(&ds_ready[x], (e >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
         tc_fence_after();
-        const uint32_t qt = smem_u32(sQ + x * L::T64), ot = smem_u32(sdO + x * L::T64);
+        // descriptors advanced by constants: a byte offset o adds o >> 4
+        const uint64_t dqt = sdesc_sw128(smem_u32(sQ), 8192, 1024) + (uint64_t)(x * L::T64 >> 4);
+        const uint64_t dot = sdesc_sw128(smem_u32(sdO), 8192, 1024) + (uint64_t)(x * L::T64 >> 4);
         // query rows 16 kk .. 16 kk + 15: packed at columns 32 (kk / 2) + 8 (kk % 2)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint32_t ca = 32 * (kk / 2) + 8 * (kk % 2);
-          umma_ts(tbase + COL_DV, tbase + 128 * x + ca, sdesc_sw128(ot + kk * 2048, 8192, 1024), id_o,
+          umma_ts(tbase + COL_DV, tbase + 128 * x + ca, dot + kk * (2048 >> 4), id_o, (e > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(tbase + COL_DK, tbase + 128 * x + 64 + ca, dqt + kk * (2048 >> 4), id_o,
                   (e > 0 || kk > 0) ? 1u : 0u);
-          umma_ts(tbase + COL_DK, tbase + 128 * x + 64 + ca, sdesc_sw128(qt + kk * 2048, 8192, 1024),
-                  id_o, (e > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&q_empty[x]);
         return true;
@@ -579,14 +587,14 @@ __global__ void __launch_bounds__(320, 1)
         // S^T = K Q_e^T and dP^T = V dO_e^T (M = 128 key rows, N = 64 query rows) into
         // buffer x; its previous contents (entry e - 2) were consumed by MMAs issued
         // earlier by this thread, which execute in order
-        const uint32_t qt = smem_u32(sQ + x * L::T64), ot = smem_u32(sdO + x * L::T64);
+        const uint64_t dk0 = sdesc_sw128(k0, 16, 1024), dv0 = sdesc_sw128(v0, 16, 1024);
+        const uint64_t dqt = sdesc_sw128(smem_u32(sQ), 16, 1024) + (uint64_t)(x * L::T64 >> 4);
+        const uint64_t dot = sdesc_sw128(smem_u32(sdO), 16, 1024) + (uint64_t)(x * L::T64 >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off2 = (kk / 4) * 16384 + (kk % 4) * 32, off1 = (kk / 4) * 8192 + (kk % 4) * 32;
-          umma_ss(tbase + 128 * x, sdesc_sw128(k0 + off2, 16, 1024), sdesc_sw128(qt + off1, 16, 1024), id_s,
-                  kk > 0 ? 1u : 0u);
-          umma_ss(tbase + 128 * x + 64, sdesc_sw128(v0 + off2, 16, 1024), sdesc_sw128(ot + off1, 16, 1024),
-                  id_s, kk > 0 ? 1u : 0u);
+          const uint32_t off2 = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4, off1 = ((kk / 4) * 8192 + (kk % 4) * 32) >> 4;
+          umma_ss(tbase + 128 * x, dk0 + off2, dqt + off1, id_s, kk > 0 ? 1u : 0u);
+          umma_ss(tbase + 128 * x + 64, dv0 + off2, dot + off1, id_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sp_full[x]);
         if (e >= 1 && !issue_grads(e - 1)) { ok = false; break; }
@@ -623,20 +631,23 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld32(ts + 32 * hs, s0);
         tmem_ld32(ts + 64 + 32 * hs, d0);
         tmem_ld_wait();
-        const float2* ldv = sLD + x * 64 + 32 * hs;  // (lse log2 e, D) of this thread's 32 query rows
+        // (-lse log2 e, -D) of this thread's 32 query rows
+        const float4* ldv = reinterpret_cast<const float4*>(sLD + x * 64 + 32 * hs);
+        const uint64_t sc2 = f2_pack(sl2, sl2), cs2 = f2_pack(cs, cs);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          float pv[2], ds[2];
-#pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const int col = 2 * c + e2;
-            const float2 l2 = ldv[col];
-            const float pr = ex2b(fmaf(__uint_as_float(s0[col]), sl2, -l2.x));
-            pv[e2] = pr;
-            ds[e2] = pr * (cs * __uint_as_float(d0[col]) - l2.y);
-          }
-          pp[c] = pack_bf16x2(pv[0], pv[1]);
-          pd[c] = pack_bf16x2(ds[0], ds[1]);
+          const float4 l4 = ldv[c];  // rows 2c and 2c + 1
+          float p0, p1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1])), sc2,
+                           f2_pack(l4.x, l4.z)), p0, p1);
+          p0 = ex2b(p0);
+          p1 = ex2b(p1);
+          const uint64_t g = f2_fma(f2_pack(__uint_as_float(d0[2 * c]), __uint_as_float(d0[2 * c + 1])), cs2,
+                                    f2_pack(l4.y, l4.w));
+          float d0s, d1s;
+          f2_unpack(f2_mul(f2_pack(p0, p1), g), d0s, d1s);
+          pp[c] = pack_bf16x2(p0, p1);
+          pd[c] = pack_bf16x2(d0s, d1s);
         }
       } else {
 #pragma unroll
@@ -648,7 +659,8 @@ __global__ void __launch_bounds__(320, 1)
       tmem_st16(ts + 64 + 32 * hs, pd);
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&ds_ready[x]);
+      __syncwarp();
+      if (ln == 0) mbar_arrive(&ds_ready[x]);  // one arrival per warp
     }
     if (ok && U >= 1) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, a.err, DEV_TIMEOUT_MMA));
     if (ok) {

@@ -93,7 +93,7 @@ struct BwdRowsArgs {
   const __nv_bfloat16* hagg;  // [BH][Tq][NN] forward's [H'_i^T | Z_i]
   const float* alpha;       // [BH] (SLA2) or nullptr
   const float* lse;         // [BH][N] from the forward
-  float2* ld2;              // [BH][T_q * 64] out: (lse * log2 e, D = dO^s . o^s); (+inf, 0) past N
+  float2* ld2;              // [BH][T_q * 64] out: (-lse * log2 e, -D), D = dO^s . o^s; (-inf, 0) past N
   float* dq_lin;            // [BH][N][d] out
   __nv_bfloat16* dhz;       // [BH][Tq][NN] out: [dH'_i^T | dZ_i]
   float* dalpha;            // [BH] accumulated (SLA2) or nullptr
@@ -118,7 +118,7 @@ struct BwdSparseArgs {
   const int32_t* lut;       // [BH][Tq][nh]
   const int32_t* rptr;      // [BH][Tkv + 1] reverse lists: query blocks with j critical
   const int32_t* rows;      // [BH][Tq * nh]
-  const float2* ld2;        // [BH][T_q * 64] (lse * log2 e, D) per query row, padded rows (+inf, 0)
+  const float2* ld2;        // [BH][T_q * 64] (-lse * log2 e, -D) per query row, padded rows (-inf, 0)
   const float* alpha;       // [BH] (SLA2) or nullptr
   const float* q_lin;       // [BH][N][d] dq (linear part), or dk (linear) for the key kernel
   const float* v_lin;       // [BH][N][d] dv (linear part) for the key kernel
