@@ -424,16 +424,24 @@ __global__ void __launch_bounds__(192, 2)
             if (c + 32 >= nvalid) s1[c] = __float_as_uint(-INFINITY);
           }
         }
-        float t[32];
+        // row maximum with three-input max: 64 -> 22 -> 8 -> 3 -> 1
+        float t[22];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) t[c] = fmaxf(__uint_as_float(s0[c]), __uint_as_float(s1[c]));
+        for (int i = 0; i < 21; ++i) {
+          const int e = 3 * i;  // values 0..31 from s0, 32..63 from s1
+          t[i] = fmax3(__uint_as_float(e < 32 ? s0[e] : s1[e - 32]),
+                       __uint_as_float(e + 1 < 32 ? s0[e + 1] : s1[e + 1 - 32]),
+                       __uint_as_float(e + 2 < 32 ? s0[e + 2] : s1[e + 2 - 32]));
+        }
+        t[21] = __uint_as_float(s1[31]);
 #pragma unroll
-        for (int st = 16; st >= 1; st >>= 1)
-#pragma unroll
-          for (int c = 0; c < st; ++c) t[c] = fmaxf(t[c], t[c + st]);
+        for (int i = 0; i < 7; ++i) t[i] = fmax3(t[3 * i], t[3 * i + 1], t[3 * i + 2]);
+        t[7] = t[21];
+        t[0] = fmax3(t[0], t[1], t[2]);
+        t[1] = fmax3(t[3], t[4], t[5]);
         // 8-bit scores carry the two block scales: s = (q^ . k^) s_Q s_K
         const float sc = FP8 ? sl2 * sq_half * usk[k] : sl2;
-        const float mx = t[0] * sc;
+        const float mx = fmax3(t[0], t[1], fmaxf(t[6], t[7])) * sc;
         // lazy rescale: keep the running max unless it grows by more than 2^8.
         // FP8 P V: the running max is kept in whole log2 units (the row max
         // rounded up), so every rescale is an exact power of two and the final
@@ -466,16 +474,16 @@ __global__ void __launch_bounds__(192, 2)
             m = mt;
           }
         }
-        const float nm = -m;
-        float u[32];
+        // p = 2^(s sc - m): scaling in pairs (each rounded as fmaf), sums in pairs
+        const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(-m, -m);
+        uint64_t u2[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2(fmaf(__uint_as_float(s0[2 * c]), sc, nm));
-          const float p1 = ex2(fmaf(__uint_as_float(s0[2 * c + 1]), sc, nm));
-          const float p2 = ex2(fmaf(__uint_as_float(s1[2 * c]), sc, nm));
-          const float p3 = ex2(fmaf(__uint_as_float(s1[2 * c + 1]), sc, nm));
-          u[c] = p0 + p1;
-          u[16 + c] = p2 + p3;
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s0[2 * c]), __uint_as_float(s0[2 * c + 1])), sc2, nm2), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(s1[2 * c]), __uint_as_float(s1[2 * c + 1])), sc2, nm2), x2, x3);
+          const float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
+          u2[c] = f2_add(f2_pack(p0, p1), f2_pack(p2, p3));
           if (PV8) {  // E4M3(448 p), four tokens per 32-bit column
             const __nv_fp8x2_storage_t a01 =
                 __nv_cvt_float2_to_fp8x2(make_float2(448.f * p0, 448.f * p1), __NV_SATFINITE, __NV_E4M3);
@@ -490,10 +498,12 @@ __global__ void __launch_bounds__(192, 2)
         }
 
 #pragma unroll
-        for (int st = 16; st >= 1; st >>= 1)
+        for (int st = 8; st >= 1; st >>= 1)
 #pragma unroll
-          for (int c = 0; c < st; ++c) u[c] += u[c + st];
-        l += u[0];
+          for (int c = 0; c < st; ++c) u2[c] = f2_add(u2[c], u2[c + st]);
+        float ul, uh;
+        f2_unpack(u2[0], ul, uh);
+        l += ul + uh;
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) pk[c] = 0u;
