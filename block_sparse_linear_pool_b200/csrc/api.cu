@@ -289,7 +289,7 @@ sla_status_t predict_mask_impl(const Plan& pl, const sla_params_t* p, const void
 }
 
 sla_status_t precompute_impl(const Plan& pl, const sla_params_t* p, const void* K, const void* V,
-                             const float* proj_w, void* hz, void* ws, cudaStream_t s) {
+                             const float* proj_w, void* hz, void* ws, cudaStream_t s, int ctas_per_sm = 2) {
   CUtensorMap mk, mv, mo;
   if (!map_bhnd(&mk, K, pl, p->stride_k, 64) || !map_bhnd(&mv, V, pl, p->stride_v, 64))
     return SLA_ERR_CUDA;
@@ -308,7 +308,7 @@ sla_status_t precompute_impl(const Plan& pl, const sla_params_t* p, const void* 
   a.Tkv = pl.Tkv;
   a.nitems = pl.BH * pl.Tkv;
   a.phi = pl.phi;
-  return cuda_status(launch_kv_prep(mk, mv, mo, a, pl.d, s));
+  return cuda_status(launch_kv_prep(mk, mv, mo, a, pl.d, s, ctas_per_sm));
 }
 
 // [BH][M][NN] bf16 rows as TMA store tiles of 64 columns x 128 rows (128-byte swizzle)
@@ -538,6 +538,37 @@ bool contiguous(const sla_params_t* p) {
   return true;
 }
 
+// A second stream per device (no device memory), created once, for the part of
+// the one-call forward that does not depend on the mask: the linear statistics
+// (kv_prep) run beside mask prediction and the pairing of query blocks.
+#ifndef SLA_OVERLAP_KV_CTAS_PER_SM
+#define SLA_OVERLAP_KV_CTAS_PER_SM 1
+#endif
+struct SidePipe {
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  bool ok = false;
+};
+std::mutex& side_mutex() {
+  static std::mutex m;
+  return m;
+}
+// The caller holds side_mutex().
+SidePipe* side_pipe() {
+  static SidePipe pipes[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  SidePipe& sp = pipes[dev];
+  if (!sp.ok) {
+    if (cudaStreamCreateWithFlags(&sp.side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&sp.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&sp.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    sp.ok = true;
+  }
+  return &sp;
+}
+
 sla_status_t attention_impl(const Plan& pl, const sla_params_t* p, const void* Q, const void* K,
                             const void* V, const float* proj_w, const float* proj_b,
                             const float* alpha, const float* Wq, const float* Wk, void* O,
@@ -547,10 +578,38 @@ sla_status_t attention_impl(const Plan& pl, const sla_params_t* p, const void* Q
   int32_t* lut = at<int32_t>(ws, L.lut);
   void* hz = at<void>(ws, L.hz);
   const bool alpha_mode = p->combine == SLA_COMBINE_ALPHA;
-  SLA_TRY(predict_mask_impl(pl, p, Q, K, alpha_mode ? Wq : nullptr, alpha_mode ? Wk : nullptr, mc,
-                            lut, ws, s));
-  SLA_TRY(precompute_impl(pl, p, K, V, alpha_mode ? nullptr : proj_w, hz, ws, s));
-  return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, ws, s);
+  const float* wq = alpha_mode ? Wq : nullptr;
+  const float* wk = alpha_mode ? Wk : nullptr;
+  const float* pw = alpha_mode ? nullptr : proj_w;
+  // Under stream capture the side stream would join the caller's graph until
+  // the capture ends: there everything runs in order on `s`.
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return SLA_ERR_CUDA;
+  if (cap != cudaStreamCaptureStatusNone) {
+    SLA_TRY(predict_mask_impl(pl, p, Q, K, wq, wk, mc, lut, ws, s));
+    SLA_TRY(precompute_impl(pl, p, K, V, pw, hz, ws, s));
+    return forward_impl(pl, p, Q, K, V, mc, lut, hz, proj_b, alpha, O, ws, s);
+  }
+  sla_status_t st_kv = SLA_OK, st = SLA_OK;
+  {
+    std::lock_guard<std::mutex> lock(side_mutex());
+    SidePipe* sp = side_pipe();
+    if (!sp) return SLA_ERR_CUDA;
+    // fork: the side stream starts after everything already on `s`
+    if (cudaEventRecord(sp->fork, s) != cudaSuccess || cudaStreamWaitEvent(sp->side, sp->fork, 0) != cudaSuccess)
+      return SLA_ERR_CUDA;
+    // kv_prep on fewer CTAs per SM, so that the mask kernels find room beside it
+    st_kv = precompute_impl(pl, p, K, V, pw, hz, ws, sp->side, SLA_OVERLAP_KV_CTAS_PER_SM);
+    // join (recorded whatever happened, so `s` never waits on a stale event)
+    const bool joined = cudaEventRecord(sp->join, sp->side) == cudaSuccess;
+    st = predict_mask_impl(pl, p, Q, K, wq, wk, mc, lut, ws, s);
+    if (st == SLA_OK) st = pairing_impl(pl, lut, ws, s);
+    if (!joined || cudaStreamWaitEvent(s, sp->join, 0) != cudaSuccess) return SLA_ERR_CUDA;
+  }
+  SLA_TRY(st_kv);
+  SLA_TRY(st);
+  SLA_TRY(aggregate_impl(pl, mc, hz, ws, s));
+  return fused_impl(pl, p, Q, K, V, lut, proj_b, alpha, O, ws, s, nullptr, nullptr, /*pair=*/false);
 }
 
 // ---------------------------------------------------------------------------

@@ -171,7 +171,7 @@ cudaError_t launch_select(const SelectArgs& a, int BH, cudaStream_t s);
 
 // mapO: hz viewed as (a: d, b: d, j: T_kv, bh) tiles of 64 x d for TMA stores.
 cudaError_t launch_kv_prep(const CUtensorMap& mapK, const CUtensorMap& mapV, const CUtensorMap& mapO,
-                           const KvPrepArgs& a, int D, cudaStream_t s);
+                           const KvPrepArgs& a, int D, cudaStream_t s, int ctas_per_sm = 2);
 
 cudaError_t launch_marg_matrix(const int8_t* mc, __nv_bfloat16* mm, int BH, int Tq, int Tkv,
                                int Tkvp, bool all, cudaStream_t s);

@@ -320,7 +320,8 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
 
 template <int D>
 static cudaError_t launch_kv_prep_t(const CUtensorMap& mapK, const CUtensorMap& mapV,
-                                    const CUtensorMap& mapO, const KvPrepArgs& a, cudaStream_t s) {
+                                    const CUtensorMap& mapO, const KvPrepArgs& a, cudaStream_t s,
+                                    int ctas_per_sm) {
   using L = KvSmem<D>;
   cudaError_t e = cudaFuncSetAttribute(kv_prep_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::ALLOC);
@@ -328,15 +329,15 @@ static cudaError_t launch_kv_prep_t(const CUtensorMap& mapK, const CUtensorMap& 
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = min(a.nitems, 2 * sms);
+  const int grid = min(a.nitems, (ctas_per_sm == 1 ? 1 : 2) * sms);
   kv_prep_kernel<D><<<grid, 128, L::ALLOC, s>>>(mapK, mapV, mapO, a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_kv_prep(const CUtensorMap& mapK, const CUtensorMap& mapV, const CUtensorMap& mapO,
-                           const KvPrepArgs& a, int D, cudaStream_t s) {
-  return D == 128 ? launch_kv_prep_t<128>(mapK, mapV, mapO, a, s)
-                  : launch_kv_prep_t<64>(mapK, mapV, mapO, a, s);
+                           const KvPrepArgs& a, int D, cudaStream_t s, int ctas_per_sm) {
+  return D == 128 ? launch_kv_prep_t<128>(mapK, mapV, mapO, a, s, ctas_per_sm)
+                  : launch_kv_prep_t<64>(mapK, mapV, mapO, a, s, ctas_per_sm);
 }
 
 }  // namespace sla

@@ -271,7 +271,14 @@ sla_status_t sla_workspace_pairs(const sla_params_t* p, size_t* offset, size_t* 
  * The whole forward in one call: sla_predict_mask, sla_precompute_linear and
  * sla_forward, with mc, lut and hz kept in the workspace
  * (sla_attention_workspace_size bytes).  proj_w / proj_b are used by the SLA
- * combine, Wq / Wk / alpha by SLA2 (Wq, Wk may be NULL).
+ * combine, Wq / Wk / alpha by SLA2 (Wq, Wk may be NULL).  The linear
+ * statistics (sla_precompute_linear) run on a second stream that the library
+ * creates once per device (with two events; no device memory), beside mask
+ * prediction and the pairing of query blocks on `stream`; everything is
+ * ordered after the work already on `stream`, and `stream` waits for the
+ * second stream before the aggregation, so the call behaves as if all of it
+ * ran on `stream`.  Calls from several host threads serialise their enqueueing
+ * on that stream.  Under stream capture everything runs on `stream` in order.
  */
 sla_status_t sla_attention_workspace_size(const sla_params_t* p, size_t* bytes);
 sla_status_t sla_attention(const sla_params_t* p, const void* Q, const void* K, const void* V,

@@ -407,6 +407,39 @@ def test_split_entry_points_and_host_buffers_match_forward():
     assert bnd.sla_get_device_status(ws)[0] == 0 and bnd.sla_get_device_status(wsh)[0] == 0
 
 
+def test_one_call_forward_on_streams_and_in_a_cuda_graph():
+    # sla_attention forks the linear statistics onto the library's second stream
+    # and joins it back: the output must not depend on the caller's stream, on
+    # work already queued there, or on running the call inside a captured graph
+    # (where it falls back to one stream).
+    data = _small(1, 3, 2500, 128, seed=17)
+    cfg = bnd.SlaConfig(k_h=0.08, k_l=0.5, combine="proj")
+    dev = "cuda"
+    Q, K, V = (data[k].to(dev) for k in ("Q", "K", "V"))
+    pw, pb = data["proj_w"].to(dev), data["proj_b"].to(dev)
+    ref = bnd.sla_attention(Q, K, V, cfg, proj_w=pw, proj_b=pb)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    O = torch.empty_like(Q)
+    p = bnd.make_params(Q, cfg, K, V, O)
+    ws = bnd.new_workspace(bnd.sla_attention_workspace_size(p), dev)
+    with torch.cuda.stream(s):
+        Q2 = Q * 1  # produced on s just before the call: the side stream must wait for it
+        for _ in range(3):
+            bnd.sla_attention(Q2, K, V, cfg, proj_w=pw, proj_b=pb, out=O, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(O, ref)
+    g = torch.cuda.CUDAGraph()
+    O.zero_()
+    with torch.cuda.graph(g):
+        bnd.sla_attention(Q, K, V, cfg, proj_w=pw, proj_b=pb, out=O, workspace=ws)
+    O.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(O, ref)
+    assert bnd.sla_get_device_status(ws)[0] == 0
+
+
 def test_strided_views_are_honoured():
     # Q, K, V as views of one [B, N, 3, H, d] buffer (strides != contiguous)
     B, H, N, d = 1, 2, 1500, 128
