@@ -11,11 +11,11 @@
 //   marg_matrix_kernel  M_c (int8) -> Mmarg (bf16 0/1, rows padded to T_kvp); all
 //                       ones for the variant whose linear branch covers every block
 //   marg_gemm_kernel    persistent, 128 x 256 output tiles, K step 64,
-//                       3-stage TMA ring, two TMEM accumulators; warp 0 loads,
+//                       4-stage TMA ring, two TMEM accumulators; warp 0 loads,
 //                       warp 1 issues tcgen05.mma, warps 2-5 drain TMEM into a
-//                       swizzled bf16 staging tile that one thread stores with
-//                       TMA (whole 128-byte lines), while the next tile
-//                       accumulates.
+//                       swizzled bf16 staging tile (128 columns at a time)
+//                       that one thread stores with TMA (whole 128-byte
+//                       lines), while the next tile accumulates.
 #include "kernels.cuh"
 
 namespace sla {
@@ -49,12 +49,15 @@ __global__ void marg_matrix_t_kernel(const int8_t* __restrict__ mc, __nv_bfloat1
 }
 
 namespace {
-constexpr int BM = 128, BN = 256, BK = 64, NST = 3;
+// Four 48 KB stages (192 KB of loads in flight per SM: the [h|z] tiles come
+// partly from HBM, and fewer bytes in flight left the tensor pipe waiting) and
+// a 32 KB staging tile that takes the 256 output columns in two halves.
+constexpr int BM = 128, BN = 256, BK = 64, NST = 4;
 constexpr int A_BYTES = BM * BK * 2;   // 16 KB
 constexpr int B_BYTES = BK * BN * 2;   // 32 KB
 constexpr int STAGE = A_BYTES + B_BYTES;
-constexpr int OFF_OUT = NST * STAGE;   // bf16 output tile: 4 chunks of [128 rows][64 columns]
-constexpr int OUT_BYTES = BM * BN * 2;
+constexpr int OFF_OUT = NST * STAGE;   // bf16 staging: 2 chunks of [128 rows][64 columns]
+constexpr int OUT_BYTES = BM * 128 * 2;
 constexpr int OFF_BAR = OFF_OUT + OUT_BYTES;
 constexpr int SMEM = OFF_BAR + 256 + 1024;
 
@@ -172,40 +175,46 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
       const int ab = lt & 1;
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[ab], (lt >> 1) & 1, a.err, DEV_TIMEOUT_MMA));
       tc_fence_after();
-      // the previous tile's TMA stores have finished reading the staging tile
-      if (leader) bulk_wait_read_all();
-      epi_sync();
-      if (ok) {
-        const uint32_t taddr = tacc + 256 * ab + ((uint32_t)(32 * q4) << 16);
+      const uint32_t taddr = tacc + 256 * ab + ((uint32_t)(32 * q4) << 16);
+      for (int hf = 0; hf < 2; ++hf) {
+        // the previous TMA stores have finished reading the staging tile
+        if (leader) bulk_wait_read_all();
+        epi_sync();
+        if (ok) {
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(taddr + c0, r);
-          tmem_ld_wait();
-          // row `row` of chunk c0 / 64, 16-byte units (c0 % 64) / 8 .. + 3, 128-byte swizzle
-          uint8_t* chunk = sO + (c0 >> 6) * (BM * 128) + row * 128;
+          for (int c0 = 128 * hf; c0 < 128 * hf + 128; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(taddr + c0, r);
+            tmem_ld_wait();
+            // row `row` of staging chunk (c0 / 64) % 2, 16-byte units (c0 % 64) / 8 .. + 3, 128-byte swizzle
+            uint8_t* chunk = sO + ((c0 >> 6) & 1) * (BM * 128) + row * 128;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int unit = ((c0 & 63) >> 3) + v;
-            uint4 q;
-            q.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
-            q.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
-            q.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
-            q.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
-            *reinterpret_cast<uint4*>(chunk + ((unit ^ (row & 7)) << 4)) = q;
+            for (int v = 0; v < 4; ++v) {
+              const int unit = ((c0 & 63) >> 3) + v;
+              uint4 q;
+              q.x = pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1]));
+              q.y = pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3]));
+              q.z = pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5]));
+              q.w = pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7]));
+              *reinterpret_cast<uint4*>(chunk + ((unit ^ (row & 7)) << 4)) = q;
+            }
           }
+          if (hf == 1) {
+            // the accumulator has been read: the MMA warp may reuse it
+            tc_fence_before();
+            mbar_arrive(&acc_empty[ab]);
+          }
+          fence_proxy_async_smem();
         }
-        // the accumulator has been read: the MMA warp may reuse it
-        tc_fence_before();
-        mbar_arrive(&acc_empty[ab]);
-        fence_proxy_async_smem();
-      }
-      epi_sync();
-      if (leader && ok) {
+        epi_sync();
+        if (leader && ok) {
 #pragma unroll
-        for (int c = 0; c < BN / 64; ++c)
-          if (n0 + 64 * c < a.NN) tma_store_3d(&mapO, sO + c * (BM * 128), n0 + 64 * c, m0, bh);
-        bulk_commit_group();
+          for (int c = 0; c < 2; ++c) {
+            const int col = n0 + 128 * hf + 64 * c;
+            if (col < a.NN) tma_store_3d(&mapO, sO + c * (BM * 128), col, m0, bh);
+          }
+          bulk_commit_group();
+        }
       }
     }
     if (leader) bulk_wait_all();
@@ -237,7 +246,7 @@ __global__ void __launch_bounds__(192, 1) marg_gemm_kernel(const __grid_constant
 // with TMA.  One CTA per SM.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr int TM_BN = 128, TM_BK = 64, TM_NST = 6;
+constexpr int TM_BN = 128, TM_BK = 64, TM_NST = 10;  // 160 KB of [h|z] loads in flight
 constexpr int TM_STAGE = TM_BK * TM_BN * 2;        // 16 KB: [2 chunks][64 K rows][128 B]
 constexpr int TM_OFF_OUT = TM_NST * TM_STAGE;      // staging: 2 x [2 chunks][128 rows][128 B]
 constexpr int TM_OUT = 128 * TM_BN * 2;            // 32 KB
