@@ -225,12 +225,13 @@ __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
       bs[(4 * q + 3) * LBS + r] = pb[v].w;
     }
   };
-  // thread (ty, tx) owns rows 4ty..4ty+3 and columns {4tx..4tx+3, 64+4tx..64+4tx+3}
-  float acc[4][8];
+  // thread (ty, tx) owns rows 4ty..4ty+3 and columns {4tx..4tx+3, 64+4tx..64+4tx+3},
+  // accumulated in column pairs with the paired fp32 FMA (each half rounded as fmaf)
+  uint64_t acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
   load(0);
   store(0);
   __syncthreads();
@@ -246,11 +247,13 @@ __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
       const float4 b0 = *reinterpret_cast<const float4*>(bs + k * LBS + 4 * tx);
       const float4 b1 = *reinterpret_cast<const float4*>(bs + k * LBS + 64 + 4 * tx);
       const float av[4] = {a0.x, a0.y, a0.z, a0.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      const uint64_t bp[4] = {f2_pack(b0.x, b0.y), f2_pack(b0.z, b0.w), f2_pack(b1.x, b1.y), f2_pack(b1.z, b1.w)};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int i = 0; i < 4; ++i) {
+        const uint64_t ap = f2_pack(av[i], av[i]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) acc[i][j] = f2_fma(ap, bp[j], acc[i][j]);
+      }
     }
     if (kc + 1 < nk) store(st ^ 1);
     __syncthreads();
@@ -262,9 +265,15 @@ __global__ void __launch_bounds__(256) logits_kernel(LogitArgs a) {
     const int r = m0 + 4 * ty + i;
     if (r >= Tq) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int c = n0 + (j < 4 ? 4 * tx + j : 64 + 4 * tx + (j - 4));
-      if (c < Tk) keys[(int64_t)r * Tk + c] = order_key(acc[i][j] * scale);
+    for (int jj = 0; jj < 4; ++jj) {
+      float v[2];
+      f2_unpack(acc[i][jj], v[0], v[1]);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j = 2 * jj + h;
+        const int c = n0 + (j < 4 ? 4 * tx + j : 64 + 4 * tx + (j - 4));
+        if (c < Tk) keys[(int64_t)r * Tk + c] = order_key(v[h] * scale);
+      }
     }
   }
 }
