@@ -147,18 +147,23 @@ __global__ void __launch_bounds__(192, 1)
     const float cl = a.combine == 1 ? 1.f - a.alpha[bh] : 1.f;
     const __nv_bfloat16* qrow = a.Q + (int64_t)b * a.sq[0] + (int64_t)h * a.sq[1] + (int64_t)n * a.sq[2];
     bool ok = __all_sync(0xffffffffu, mbar_wait(h_full, 0, err, DEV_TIMEOUT_TMA));
-    // ---- phase 1: phi(q) (bf16) into sF, den = phi(q) . Z_t + eps
+    // ---- phase 1: phi(q) (bf16) into sF, den = phi(q) . Z_t + eps.  The row is
+    // loaded once, all 16 loads in flight, and kept in registers.
+    uint4 qv[TD / 8];
+#pragma unroll
+    for (int c = 0; c < TD / 8; ++c)
+      qv[c] = valid ? __ldg(reinterpret_cast<const uint4*>(qrow) + c) : make_uint4(0u, 0u, 0u, 0u);
     float m = -INFINITY, s = 0.f;
     if (valid && a.phi == 0) {
-      for (int c = 0; c < TD; c += 8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(qrow + c);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int c = 0; c < TD / 8; ++c) {
+        const uint32_t u[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) m = fmaxf(m, bfv(u[e / 2], e & 1));
       }
-      for (int c = 0; c < TD; c += 8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(qrow + c);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int c = 0; c < TD / 8; ++c) {
+        const uint32_t u[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) s += exp2f((bfv(u[e / 2], e & 1) - m) * LOG2E_T);
       }
@@ -170,10 +175,11 @@ __global__ void __launch_bounds__(192, 1)
     float den = a.eps;
     if (ok) {
       const __nv_bfloat16* z = sZ + t * TD;
+#pragma unroll
       for (int c = 0; c < TD; c += 8) {
         uint32_t o4[4] = {0u, 0u, 0u, 0u};
         if (valid) {
-          const uint4 v = *reinterpret_cast<const uint4*>(qrow + c);
+          const uint4 v = qv[c / 8];
           const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -201,6 +207,16 @@ __global__ void __launch_bounds__(192, 1)
       const float inv_den = 1.f / den;
 #pragma unroll 1
       for (int c0 = 0; c0 < TD; c0 += 32) {
+        // this chunk's dO and o^s loads go out before the TMEM load, all in flight
+        uint4 dq4[4];
+        float4 os4[8];
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+          dq4[v4] = valid ? __ldg(reinterpret_cast<const uint4*>(drow + c0) + v4) : make_uint4(0u, 0u, 0u, 0u);
+          os4[2 * v4] = valid ? __ldg(reinterpret_cast<const float4*>(osrow + c0) + 2 * v4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          os4[2 * v4 + 1] = valid ? __ldg(reinterpret_cast<const float4*>(osrow + c0) + 2 * v4 + 1)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
         uint32_t nv[32];
         tmem_ld32(tl + TD * t + c0, nv);
         tmem_ld_wait();
@@ -208,18 +224,14 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
         for (int c8 = 0; c8 < 32; c8 += 8) {
           float dov[8], osv[8];
-          if (valid) {
-            const uint4 v = *reinterpret_cast<const uint4*>(drow + c0 + c8);
+          {
+            const uint4 v = dq4[c8 / 8];
             const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 8; ++e) dov[e] = bfv(u[e / 2], e & 1);
-            const float4 o0 = *reinterpret_cast<const float4*>(osrow + c0 + c8);
-            const float4 o1 = *reinterpret_cast<const float4*>(osrow + c0 + c8 + 4);
+            const float4 o0 = os4[c8 / 4], o1 = os4[c8 / 4 + 1];
             osv[0] = o0.x; osv[1] = o0.y; osv[2] = o0.z; osv[3] = o0.w;
             osv[4] = o1.x; osv[5] = o1.y; osv[6] = o1.z; osv[7] = o1.w;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) dov[e] = osv[e] = 0.f;
           }
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -520,6 +532,7 @@ __global__ void __launch_bounds__(192, 1)
     // W~ as bf16 into sW (row o = r), the K-major B operand of G3 / MN-major B of G2
     if (proj) {
       const float* wr = a.proj_w + (int64_t)r * TD;
+#pragma unroll 4
       for (int c = 0; c < TD; c += 8) {
         const float4 x0 = *reinterpret_cast<const float4*>(wr + c);
         const float4 x1 = *reinterpret_cast<const float4*>(wr + c + 4);
@@ -530,18 +543,21 @@ __global__ void __launch_bounds__(192, 1)
     }
     bool ok = __all_sync(0xffffffffu, mbar_wait(in_full, 0, err, DEV_TIMEOUT_TMA));
     // ---- phi(K) in place (bf16); rows that do not exist get 0
-    const __nv_bfloat16* krow = a.K + (int64_t)b * a.sk[0] + (int64_t)h * a.sk[1] + (int64_t)n * a.sk[2];
     float m = -INFINITY, s = 0.f;
-    if (valid && a.phi == 0) {
-      for (int c = 0; c < TD; c += 8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(krow + c);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    if (ok && valid && a.phi == 0) {  // from the K tile in shared memory (loaded by TMA)
+      uint4 kv[TD / 8];
+#pragma unroll
+      for (int c = 0; c < TD / 8; ++c)
+        kv[c] = *reinterpret_cast<const uint4*>(sF + (c / 8) * TILE + sw128_offset(r, (c % 8) * 16));
+#pragma unroll
+      for (int c = 0; c < TD / 8; ++c) {
+        const uint32_t u[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) m = fmaxf(m, bfv(u[e / 2], e & 1));
       }
-      for (int c = 0; c < TD; c += 8) {
-        const uint4 v = *reinterpret_cast<const uint4*>(krow + c);
-        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int c = 0; c < TD / 8; ++c) {
+        const uint32_t u[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) s += exp2f((bfv(u[e / 2], e & 1) - m) * LOG2E_T);
       }
