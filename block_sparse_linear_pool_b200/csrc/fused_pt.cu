@@ -28,14 +28,18 @@
 //   warp 0      TMA producer: the tile's union record (bulk copy, two buffers),
 //               Q tile + Z rows, K and V of each entry, then H_a^T through the K
 //               ring and H_b^T through the V ring (one 64-column chunk per slot)
-//   warp 1      MMA issuer (one thread, whose issue rate paces the loop: the
-//               shared-memory descriptors are formed once and advanced by
-//               constants): S, P V, and the two linear-branch chains
+//   warp 1      MMA issuer (one thread; the shared-memory descriptors are
+//               formed once and advanced by constants): S, P V, and the two
+//               linear-branch chains.  S_{k+1} is issued as soon as P_{k-1} V
+//               is, so that it runs beside the softmax of entry k: the two
+//               score buffers are what keeps the tensor pipe fed within a CTA.
 //   warps 2-5   one query row per thread: online softmax with exp2 (lazy
-//               rescale of O only when the running max grows by more than 2^8),
-//               P over S in TMEM; then (training forward) the row's LSE and its
-//               sparse-branch output o^s from O before the linear term joins it,
-//               phi~(q), P', and the epilogue
+//               rescale of O only when the running max grows by more than 2^8;
+//               the scaling and the row sum in paired fp32 instructions, the
+//               row maximum with three-input max), P over S in TMEM; then
+//               (training forward) the row's LSE and its sparse-branch output
+//               o^s from O before the linear term joins it, phi~(q), P', and
+//               the epilogue
 //
 // TMEM: S_0 in columns [0, 64), S_1 in [64, 128) (P', after the loop, over
 // [0, d)), O in [128, 128 + d).
