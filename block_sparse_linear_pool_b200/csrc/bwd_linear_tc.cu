@@ -322,13 +322,18 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) dst[(int64_t)(c0 + e) * TD + aa] = __float2bfloat16(__uint_as_float(hv[e]));
         }
-        // dZ_t[a] = sum_{rows of block tt} gden_r phi(q_r)[a]
-        float dz = 0.f;
-        for (int rr = 64 * tt; rr < 64 * tt + 64; ++rr) {
+        // dZ_t[a] = sum_{rows of block tt} gden_r phi(q_r)[a], in eight partial sums
+        float dzp[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) dzp[q] = 0.f;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          const int rr = 64 * tt + k;
           const __nv_bfloat16* fp = reinterpret_cast<const __nv_bfloat16*>(
               sF + (aa / 64) * TILE + sw128_offset(rr, (aa % 64) * 2));
-          dz = fmaf(sgden[rr], __bfloat162float(*fp), dz);
+          dzp[k & 7] = fmaf(sgden[rr], __bfloat162float(*fp), dzp[k & 7]);
         }
+        const float dz = ((dzp[0] + dzp[1]) + (dzp[2] + dzp[3])) + ((dzp[4] + dzp[5]) + (dzp[6] + dzp[7]));
         dst[TD * TD + aa] = __float2bfloat16(dz);
       }
     }

@@ -178,10 +178,15 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
         }
       }
       constexpr float LOG2E = 1.4426950408889634f;
+      auto ex2 = [](float v) {
+        float y;
+        asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(v));
+        return y;
+      };
       float inv;
       if (a.phi == 1) {  // elu(x) + 1
 #pragma unroll
-        for (int e = 0; e < NE; ++e) x[e] = x[e] > 0.f ? x[e] + 1.f : exp2f(x[e] * LOG2E);
+        for (int e = 0; e < NE; ++e) x[e] = x[e] > 0.f ? x[e] + 1.f : ex2(x[e] * LOG2E);
         inv = (t < cnt) ? 1.f : 0.f;
       } else {           // softmax over d
         float m = x[0];
@@ -191,7 +196,7 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
         float sum = 0.f;
 #pragma unroll
         for (int e = 0; e < NE; ++e) {
-          x[e] = exp2f((x[e] - m) * LOG2E);
+          x[e] = ex2((x[e] - m) * LOG2E);
           sum += x[e];
         }
         sum += __shfl_xor_sync(0xffffffffu, sum, 1);
@@ -257,15 +262,19 @@ __global__ void __launch_bounds__(128) kv_prep_kernel(const __grid_constant__ CU
         ++n_issued;
       }
     }
-    // z_j = column sums of phi(K_j) (the bf16 values the MMA consumes)
+    // z_j = column sums of phi(K_j) (the bf16 values the MMA consumes): eight
+    // partial sums, so that the 64 shared-memory loads are not one dependent chain
     float z = 0.f;
     if (tid < D) {
       const int chunk = tid / 64, byte = (tid % 64) * 2;
-      for (int t = 0; t < 64; ++t) {
-        const __nv_bfloat16 v =
-            *reinterpret_cast<const __nv_bfloat16*>(sK + chunk * 8192 + sw128_offset(t, byte));
-        z += __bfloat162float(v);
-      }
+      float zp[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) zp[q] = 0.f;
+#pragma unroll
+      for (int t = 0; t < 64; ++t)
+        zp[t & 7] += __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16*>(sK + chunk * 8192 + sw128_offset(t, byte)));
+      z = ((zp[0] + zp[1]) + (zp[2] + zp[3])) + ((zp[4] + zp[5]) + (zp[6] + zp[7]));
     }
     {
       const bool ok = mbar_wait(mma_bar, mma_phase & 1, a.err, DEV_TIMEOUT_MMA);
