@@ -103,14 +103,14 @@ cudaError_t launch_rlut(const int8_t* mc, int32_t* rcnt, int32_t* rptr, int32_t*
 // [128x, 128x + 64) (dS over its first 32 columns) and dP at [128x + 64,
 // 128x + 128); dQ at [256, 256 + d).  S, dP of entry k+1 are computed while the
 // row threads turn entry k into dS.  Shared: Q and dO tiles (128 rows), a
-// 3-slot K ring (K_k serves S_k and, later, dQ += dS_k K_k) and a 2-slot V ring.
+// 4-slot K ring (K_k serves S_k and, later, dQ += dS_k K_k) and a 3-slot V ring.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DqSmem {
   static constexpr int CH = D / 64;
   static constexpr int T128 = 128 * D * 2;
   static constexpr int T64 = 64 * D * 2;
-  static constexpr int NK = 3, NV = 2;
+  static constexpr int NK = 4, NV = 3;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_DO = OFF_Q + T128;
   static constexpr int OFF_K = OFF_DO + T128;
@@ -140,15 +140,15 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sK = sm + L::OFF_K;
   uint8_t* sV = sm + L::OFF_V;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
-  uint64_t* in_full = bars + 0;    // Q and dO
-  uint64_t* k_full = bars + 1;     // [NK]
-  uint64_t* k_empty = bars + 4;    // [NK]
-  uint64_t* v_full = bars + 7;     // [NV]
-  uint64_t* v_empty = bars + 9;    // [NV]
-  uint64_t* sp_full = bars + 11;   // [2] S and dP of buffer x
-  uint64_t* ds_ready = bars + 13;  // [2] dS written by all row threads
-  uint64_t* dq_done = bars + 15;   // the last dQ MMA completed
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* in_full = bars + 0;          // Q and dO
+  uint64_t* k_full = bars + 1;           // [NK]
+  uint64_t* k_empty = k_full + NK;       // [NK]
+  uint64_t* v_full = k_empty + NK;       // [NV]
+  uint64_t* v_empty = v_full + NV;       // [NV]
+  uint64_t* sp_full = v_empty + NV;      // [2] S and dP of buffer x
+  uint64_t* ds_ready = sp_full + 2;      // [2] dS written by all row threads
+  uint64_t* dq_done = ds_ready + 2;      // the last dQ MMA completed
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(dq_done + 1);
   int* s_count = reinterpret_cast<int*>(tslot + 1);
   const int Tkvr = (a.Tkv + 15) & ~15;
   uint8_t* fa = sm + L::OFF_U;
@@ -407,8 +407,11 @@ __global__ void __launch_bounds__(320, 1)
 // S^T at [128x, 128x + 64) (P^T over its first 32 columns) and dP^T at
 // [128x + 64, 128x + 128) (dS^T over its first 32), dV [256, 256 + d),
 // dK [384, 384 + d).  S^T, dP^T of entry e+1 are computed while the key-row
-// threads work on entry e.  Shared: K pair and V pair (128 rows), a 2-slot
-// ring of (Q_i, dO_i, the 64 (lse log2 e, D) pairs of block i).
+// threads work on entry e.  Shared: K pair and V pair (128 rows), a 4-slot
+// ring of (Q_i, dO_i, the 64 (lse log2 e, D) pairs of block i).  A slot is
+// freed only when the dV / dK MMAs of its entry complete, one entry after its
+// S^T; with two slots the load of entry e + 2 could start only then, and the
+// tensor pipe waited out a whole load every entry.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DkvSmem {
@@ -417,10 +420,11 @@ struct DkvSmem {
   static constexpr int T64 = 64 * D * 2;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + T128;
-  static constexpr int OFF_Q = OFF_V + T128;        // [2] slots
-  static constexpr int OFF_DO = OFF_Q + 2 * T64;    // [2]
-  static constexpr int OFF_LD = OFF_DO + 2 * T64;   // [2][64] float2
-  static constexpr int OFF_BAR = OFF_LD + 2 * 64 * 8;
+  static constexpr int NQ = 4;                      // ring slots
+  static constexpr int OFF_Q = OFF_V + T128;        // [NQ] slots
+  static constexpr int OFF_DO = OFF_Q + NQ * T64;   // [NQ]
+  static constexpr int OFF_LD = OFF_DO + NQ * T64;  // [NQ][64] float2
+  static constexpr int OFF_BAR = OFF_LD + NQ * 64 * 8;
   static constexpr int OFF_U = OFF_BAR + 256;
   // at least 120 KB so that a second CTA (which would wait for the 512 TMEM
   // columns) is never placed on the same SM
@@ -446,13 +450,14 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sdO = sm + L::OFF_DO;
   float2* sLD = reinterpret_cast<float2*>(sm + L::OFF_LD);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::OFF_BAR);
+  constexpr int NQ = L::NQ;
   uint64_t* kv_full = bars + 0;
-  uint64_t* q_full = bars + 1;    // [2] ring slots
-  uint64_t* q_empty = bars + 3;   // [2]
-  uint64_t* sp_full = bars + 5;   // [2] score buffers
-  uint64_t* ds_ready = bars + 7;  // [2]
-  uint64_t* kv_done = bars + 9;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 10);
+  uint64_t* q_full = bars + 1;             // [NQ] ring slots
+  uint64_t* q_empty = q_full + NQ;         // [NQ]
+  uint64_t* sp_full = q_empty + NQ;        // [2] score buffers
+  uint64_t* ds_ready = sp_full + 2;        // [2]
+  uint64_t* kv_done = ds_ready + 2;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(kv_done + 1);
   int* s_count = reinterpret_cast<int*>(tslot + 1);
   const int Tqr = (a.Tq + 15) & ~15;
   uint8_t* fa = sm + L::OFF_U;
@@ -475,9 +480,11 @@ __global__ void __launch_bounds__(320, 1)
   }
   if (tid == 0) {
     mbar_init(kv_full, 1);
-    for (int x = 0; x < 2; ++x) {
+    for (int x = 0; x < NQ; ++x) {
       mbar_init(&q_full[x], 1);
       mbar_init(&q_empty[x], 1);
+    }
+    for (int x = 0; x < 2; ++x) {
       mbar_init(&sp_full[x], 1);
       mbar_init(&ds_ready[x], 8);
     }
@@ -541,18 +548,18 @@ __global__ void __launch_bounds__(320, 1)
       }
       bool ok = true;
       for (int e = 0; e < U && ok; ++e) {
-        const int i = uidx[e], x = e & 1;
-        if (e >= 2 && !mbar_wait(&q_empty[x], ((e - 2) >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
+        const int i = uidx[e], sq = e % NQ;
+        if (e >= NQ && !mbar_wait(&q_empty[sq], ((e / NQ) - 1) & 1, a.err, DEV_TIMEOUT_SYNC)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&q_full[x], 2 * L::T64 + 64 * 8);
+        mbar_arrive_expect_tx(&q_full[sq], 2 * L::T64 + 64 * 8);
 #pragma unroll
         for (int c = 0; c < L::CH; ++c) {
-          tma_load_4d(sQ + x * L::T64 + c * 8192, &mapQ1, &q_full[x], c * 64, 64 * i, h, b);
-          tma_load_4d(sdO + x * L::T64 + c * 8192, &mapdO1, &q_full[x], c * 64, 64 * i, h, b);
+          tma_load_4d(sQ + sq * L::T64 + c * 8192, &mapQ1, &q_full[sq], c * 64, 64 * i, h, b);
+          tma_load_4d(sdO + sq * L::T64 + c * 8192, &mapdO1, &q_full[sq], c * 64, 64 * i, h, b);
         }
-        bulk_load(sLD + x * 64, a.ld2 + (int64_t)bh * a.Tq * 64 + 64 * i, 64 * 8, &q_full[x]);
+        bulk_load(sLD + sq * 64, a.ld2 + (int64_t)bh * a.Tq * 64 + 64 * i, 64 * 8, &q_full[sq]);
       }
     }
   } else if (w == 1) {
@@ -563,12 +570,12 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = mbar_wait(kv_full, 0, a.err, DEV_TIMEOUT_TMA);
       // dV += P^T dO_e and dK += dS^T Q_e (P^T, dS^T bf16 pairs from TMEM buffer e & 1)
       auto issue_grads = [&](int e) -> bool {
-        const int x = e & 1;
+        const int x = e & 1, sq = e % NQ;
         if (!mbar_wait(&ds_ready[x], (e >> 1) & 1, a.err, DEV_TIMEOUT_SYNC)) return false;
         tc_fence_after();
         // descriptors advanced by constants: a byte offset o adds o >> 4
-        const uint64_t dqt = sdesc_sw128(smem_u32(sQ), 8192, 1024) + (uint64_t)(x * L::T64 >> 4);
-        const uint64_t dot = sdesc_sw128(smem_u32(sdO), 8192, 1024) + (uint64_t)(x * L::T64 >> 4);
+        const uint64_t dqt = sdesc_sw128(smem_u32(sQ), 8192, 1024) + (uint64_t)(sq * L::T64 >> 4);
+        const uint64_t dot = sdesc_sw128(smem_u32(sdO), 8192, 1024) + (uint64_t)(sq * L::T64 >> 4);
         // query rows 16 kk .. 16 kk + 15: packed at columns 32 (kk / 2) + 8 (kk % 2)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
@@ -577,19 +584,19 @@ __global__ void __launch_bounds__(320, 1)
           umma_ts(tbase + COL_DK, tbase + 128 * x + 64 + ca, dqt + kk * (2048 >> 4), id_o,
                   (e > 0 || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&q_empty[x]);
+        umma_commit(&q_empty[sq]);
         return true;
       };
       for (int e = 0; e < U && ok; ++e) {
-        const int x = e & 1;
-        if (!mbar_wait(&q_full[x], (e >> 1) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
+        const int x = e & 1, sq = e % NQ;
+        if (!mbar_wait(&q_full[sq], (e / NQ) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
         tc_fence_after();
         // S^T = K Q_e^T and dP^T = V dO_e^T (M = 128 key rows, N = 64 query rows) into
         // buffer x; its previous contents (entry e - 2) were consumed by MMAs issued
         // earlier by this thread, which execute in order
         const uint64_t dk0 = sdesc_sw128(k0, 16, 1024), dv0 = sdesc_sw128(v0, 16, 1024);
-        const uint64_t dqt = sdesc_sw128(smem_u32(sQ), 16, 1024) + (uint64_t)(x * L::T64 >> 4);
-        const uint64_t dot = sdesc_sw128(smem_u32(sdO), 16, 1024) + (uint64_t)(x * L::T64 >> 4);
+        const uint64_t dqt = sdesc_sw128(smem_u32(sQ), 16, 1024) + (uint64_t)(sq * L::T64 >> 4);
+        const uint64_t dot = sdesc_sw128(smem_u32(sdO), 16, 1024) + (uint64_t)(sq * L::T64 >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off2 = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4, off1 = ((kk / 4) * 8192 + (kk % 4) * 32) >> 4;
@@ -632,7 +639,7 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld32(ts + 64 + 32 * hs, d0);
         tmem_ld_wait();
         // (-lse log2 e, -D) of this thread's 32 query rows
-        const float4* ldv = reinterpret_cast<const float4*>(sLD + x * 64 + 32 * hs);
+        const float4* ldv = reinterpret_cast<const float4*>(sLD + (e % NQ) * 64 + 32 * hs);
         const uint64_t sc2 = f2_pack(sl2, sl2), cs2 = f2_pack(cs, cs);
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
