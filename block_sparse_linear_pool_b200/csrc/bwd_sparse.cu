@@ -188,6 +188,20 @@ __global__ void __launch_bounds__(320, 1)
   }
   for (int j = tid; j < 2 * Tkvr; j += blockDim.x) fa[j] = 0;
   __syncthreads();
+  if (tid == 0) {  // the Q and dO tiles do not depend on the union: load them while it is built
+    tma_prefetch_desc(&mapQ);
+    tma_prefetch_desc(&mapdO);
+    tma_prefetch_desc(&mapK);
+    tma_prefetch_desc(&mapV);
+    mbar_arrive_expect_tx(in_full, 2 * L::T128);
+#pragma unroll
+    for (int c = 0; c < L::CH; ++c) {
+      tma_load_4d(sQ + c * 16384, &mapQ, in_full, c * 64, 64 * ia, h, b);
+      tma_load_4d(sQ + c * 16384 + 8192, &mapQ, in_full, c * 64, 64 * ibl, h, b);
+      tma_load_4d(sdO + c * 16384, &mapdO, in_full, c * 64, 64 * ia, h, b);
+      tma_load_4d(sdO + c * 16384 + 8192, &mapdO, in_full, c * 64, 64 * ibl, h, b);
+    }
+  }
   {
     const int32_t* la = a.lut + ((int64_t)bh * a.Tq + ia) * a.nh;
     const int32_t* lb = a.lut + ((int64_t)bh * a.Tq + ibl) * a.nh;
@@ -227,18 +241,6 @@ __global__ void __launch_bounds__(320, 1)
 
   if (w == 0) {
     if (ln == 0) {
-      tma_prefetch_desc(&mapQ);
-      tma_prefetch_desc(&mapdO);
-      tma_prefetch_desc(&mapK);
-      tma_prefetch_desc(&mapV);
-      mbar_arrive_expect_tx(in_full, 2 * L::T128);
-#pragma unroll
-      for (int c = 0; c < L::CH; ++c) {
-        tma_load_4d(sQ + c * 16384, &mapQ, in_full, c * 64, 64 * ia, h, b);
-        tma_load_4d(sQ + c * 16384 + 8192, &mapQ, in_full, c * 64, 64 * ibl, h, b);
-        tma_load_4d(sdO + c * 16384, &mapdO, in_full, c * 64, 64 * ia, h, b);
-        tma_load_4d(sdO + c * 16384 + 8192, &mapdO, in_full, c * 64, 64 * ibl, h, b);
-      }
       bool ok = true;
       for (int k = 0; k < U && ok; ++k) {
         const int j = uidx[k], sk = k % NK, sv = k % NV;
@@ -322,9 +324,15 @@ __global__ void __launch_bounds__(320, 1)
     // paired constants: P = 2^(s sl2 - lse2), dS = P (cs dP - D)
     const uint64_t sc2 = f2_pack(sl2, sl2), nl2 = f2_pack(ld.x, ld.x), cs2 = f2_pack(cs, cs),
                    nd2 = f2_pack(ld.y, ld.y);
+    // this thread's half of the row's fp32 linear part, added in the epilogue
+    const float* lin = a.q_lin + ((int64_t)bh * a.N + n) * D + (D / 2) * hs;
     bool ok = true;
     for (int k = 0; k < U; ++k) {
       const int x = k & 1;
+      if (valid && k == (U > 3 ? U - 3 : 0)) {  // into L2 a few entries ahead of the epilogue
+#pragma unroll
+        for (int c = 0; c < D / 2; c += 32) prefetch_l2(lin + c);
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&sp_full[x], (k >> 1) & 1, a.err, DEV_TIMEOUT_MMA))) {
         ok = false;
         break;
@@ -368,13 +376,18 @@ __global__ void __launch_bounds__(320, 1)
     if (ok && U >= 1) ok = __all_sync(0xffffffffu, mbar_wait(dq_done, 0, a.err, DEV_TIMEOUT_MMA));
     if (ok) {
       tc_fence_after();
-      __nv_bfloat16* orow = a.out0 + (int64_t)b * a.s0[0] + (int64_t)h * a.s0[1] + (int64_t)n * a.s0[2];
-      const float* lin = a.q_lin + ((int64_t)bh * a.N + n) * D;
-#pragma unroll 1
-      for (int c0 = (D / 2) * hs; c0 < (D / 2) * (hs + 1); c0 += 32) {  // this thread's half of the row
+      __nv_bfloat16* orow = a.out0 + (int64_t)b * a.s0[0] + (int64_t)h * a.s0[1] + (int64_t)n * a.s0[2] +
+                            (D / 2) * hs;
+      // all of this thread's linear part in flight before the first TMEM read
+      float4 lv[D / 8];
+#pragma unroll
+      for (int q = 0; q < D / 8; ++q)
+        lv[q] = valid ? __ldg(reinterpret_cast<const float4*>(lin) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c0 = 0; c0 < D / 2; c0 += 32) {  // this thread's half of the row
         uint32_t v[32];
         if (U >= 1) {
-          tmem_ld32(tl + COL_DQ + c0, v);
+          tmem_ld32(tl + COL_DQ + (D / 2) * hs + c0, v);
           tmem_ld_wait();
         } else {
 #pragma unroll
@@ -383,12 +396,13 @@ __global__ void __launch_bounds__(320, 1)
         if (valid) {
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
-            float y[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = __uint_as_float(v[8 * q8 + e]) * a.scale + lin[c0 + 8 * q8 + e];
+            const float4 l0 = lv[c0 / 4 + 2 * q8], l1 = lv[c0 / 4 + 2 * q8 + 1];
+            const float* vf = reinterpret_cast<const float*>(v + 8 * q8);
             *reinterpret_cast<uint4*>(orow + c0 + 8 * q8) =
-                make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                           pack_bf16x2(y[6], y[7]));
+                make_uint4(pack_bf16x2(vf[0] * a.scale + l0.x, vf[1] * a.scale + l0.y),
+                           pack_bf16x2(vf[2] * a.scale + l0.z, vf[3] * a.scale + l0.w),
+                           pack_bf16x2(vf[4] * a.scale + l1.x, vf[5] * a.scale + l1.y),
+                           pack_bf16x2(vf[6] * a.scale + l1.z, vf[7] * a.scale + l1.w));
           }
         }
       }
@@ -493,6 +507,20 @@ __global__ void __launch_bounds__(320, 1)
   }
   for (int i = tid; i < 2 * Tqr; i += blockDim.x) fa[i] = 0;
   __syncthreads();
+  if (tid == 0) {  // the K and V pair does not depend on the union: load it while it is built
+    tma_prefetch_desc(&mapK2);
+    tma_prefetch_desc(&mapV2);
+    tma_prefetch_desc(&mapQ1);
+    tma_prefetch_desc(&mapdO1);
+    mbar_arrive_expect_tx(kv_full, 2 * L::T128);
+#pragma unroll
+    for (int c = 0; c < L::CH; ++c) {
+      tma_load_4d(sK + c * 16384, &mapK2, kv_full, c * 64, 64 * ja, h, b);
+      tma_load_4d(sK + c * 16384 + 8192, &mapK2, kv_full, c * 64, 64 * jbl, h, b);
+      tma_load_4d(sV + c * 16384, &mapV2, kv_full, c * 64, 64 * ja, h, b);
+      tma_load_4d(sV + c * 16384 + 8192, &mapV2, kv_full, c * 64, 64 * jbl, h, b);
+    }
+  }
   {
     const int32_t* rp = a.rptr + (int64_t)bh * (a.Tkv + 1);
     const int32_t* rl = a.rows + (int64_t)bh * a.Tq * a.nh;
@@ -534,18 +562,6 @@ __global__ void __launch_bounds__(320, 1)
 
   if (w == 0) {
     if (ln == 0) {
-      tma_prefetch_desc(&mapK2);
-      tma_prefetch_desc(&mapV2);
-      tma_prefetch_desc(&mapQ1);
-      tma_prefetch_desc(&mapdO1);
-      mbar_arrive_expect_tx(kv_full, 2 * L::T128);
-#pragma unroll
-      for (int c = 0; c < L::CH; ++c) {
-        tma_load_4d(sK + c * 16384, &mapK2, kv_full, c * 64, 64 * ja, h, b);
-        tma_load_4d(sK + c * 16384 + 8192, &mapK2, kv_full, c * 64, 64 * jbl, h, b);
-        tma_load_4d(sV + c * 16384, &mapV2, kv_full, c * 64, 64 * ja, h, b);
-        tma_load_4d(sV + c * 16384 + 8192, &mapV2, kv_full, c * 64, 64 * jbl, h, b);
-      }
       bool ok = true;
       for (int e = 0; e < U && ok; ++e) {
         const int i = uidx[e], sq = e % NQ;
@@ -622,9 +638,19 @@ __global__ void __launch_bounds__(320, 1)
     const bool valid = (n < a.N) && (half == 0 || has_b);
     const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
     const float sl2 = a.scale_log2;
+    // this thread's halves of the key row's fp32 linear parts (dK, dV), added in the epilogue
+    const float* lin_k = a.q_lin + ((int64_t)bh * a.N + n) * D + (D / 2) * hs;
+    const float* lin_v = a.v_lin + ((int64_t)bh * a.N + n) * D + (D / 2) * hs;
     bool ok = true;
     for (int e = 0; e < U; ++e) {
       const int x = e & 1;
+      if (valid && e == (U > 3 ? U - 3 : 0)) {  // into L2 a few entries ahead of the epilogue
+#pragma unroll
+        for (int c = 0; c < D / 2; c += 32) {
+          prefetch_l2(lin_k + c);
+          prefetch_l2(lin_v + c);
+        }
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&sp_full[x], (e >> 1) & 1, a.err, DEV_TIMEOUT_MMA))) {
         ok = false;
         break;
@@ -672,15 +698,21 @@ __global__ void __launch_bounds__(320, 1)
     if (ok && U >= 1) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, a.err, DEV_TIMEOUT_MMA));
     if (ok) {
       tc_fence_after();
+#pragma unroll 1
       for (int which = 0; which < 2; ++which) {
         __nv_bfloat16* base = which == 0 ? a.out0 : a.out1;
         const int64_t* st = which == 0 ? a.s0 : a.s1;
-        const float* lin = (which == 0 ? a.q_lin : a.v_lin) + ((int64_t)bh * a.N + n) * D;
+        const float* lin = which == 0 ? lin_k : lin_v;
         const float f = which == 0 ? a.scale : cs;  // dK = acc / sqrt(d); dV = c_s acc
-        __nv_bfloat16* orow = base + (int64_t)b * st[0] + (int64_t)h * st[1] + (int64_t)n * st[2];
-        const uint32_t col = which == 0 ? COL_DK : COL_DV;
-#pragma unroll 1
-        for (int c0 = (D / 2) * hs; c0 < (D / 2) * (hs + 1); c0 += 32) {  // this thread's half
+        __nv_bfloat16* orow = base + (int64_t)b * st[0] + (int64_t)h * st[1] + (int64_t)n * st[2] + (D / 2) * hs;
+        const uint32_t col = (which == 0 ? COL_DK : COL_DV) + (D / 2) * hs;
+        // all of this half row's linear part in flight before the first TMEM read
+        float4 lv[D / 8];
+#pragma unroll
+        for (int q = 0; q < D / 8; ++q)
+          lv[q] = valid ? __ldg(reinterpret_cast<const float4*>(lin) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int c0 = 0; c0 < D / 2; c0 += 32) {
           uint32_t v[32];
           if (U >= 1) {
             tmem_ld32(tl + col + c0, v);
@@ -692,12 +724,13 @@ __global__ void __launch_bounds__(320, 1)
           if (valid) {
 #pragma unroll
             for (int q8 = 0; q8 < 4; ++q8) {
-              float y[8];
-#pragma unroll
-              for (int e8 = 0; e8 < 8; ++e8) y[e8] = __uint_as_float(v[8 * q8 + e8]) * f + lin[c0 + 8 * q8 + e8];
+              const float4 l0 = lv[c0 / 4 + 2 * q8], l1 = lv[c0 / 4 + 2 * q8 + 1];
+              const float* vf = reinterpret_cast<const float*>(v + 8 * q8);
               *reinterpret_cast<uint4*>(orow + c0 + 8 * q8) =
-                  make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
-                             pack_bf16x2(y[6], y[7]));
+                  make_uint4(pack_bf16x2(vf[0] * f + l0.x, vf[1] * f + l0.y),
+                             pack_bf16x2(vf[2] * f + l0.z, vf[3] * f + l0.w),
+                             pack_bf16x2(vf[4] * f + l1.x, vf[5] * f + l1.y),
+                             pack_bf16x2(vf[6] * f + l1.z, vf[7] * f + l1.w));
             }
           }
         }
