@@ -101,8 +101,12 @@ cudaError_t launch_rlut(const int8_t* mc, int32_t* rcnt, int32_t* rptr, int32_t*
 // ---------------------------------------------------------------------------
 // dQ.  TMEM (512 columns, one CTA per SM): two score buffers x = 0, 1 with S at
 // [128x, 128x + 64) (dS over its first 32 columns) and dP at [128x + 64,
-// 128x + 128); dQ at [256, 256 + d).  S, dP of entry k+1 are computed while the
-// row threads turn entry k into dS.  Shared: Q and dO tiles (128 rows), a
+// 128x + 128); dQ at [256, 256 + d); the CTA's Q and dO rows (bf16 pairs) at
+// [384, 384 + d/2) and [448, 448 + d/2).  S, dP of entry k+1 are computed while
+// the row threads turn entry k into dS.  S = Q K^T and dP = dO V^T take Q and
+// dO from TMEM and only the 64-key tile from shared memory; an M = 128, N = 64
+// MMA costs about the same either way (some 65 cycles per K = 16 step), and
+// this form measured about 1% faster than both operands in shared memory.  Shared: Q and dO tiles (128 rows), a
 // 4-slot K ring (K_k serves S_k and, later, dQ += dS_k K_k) and a 3-slot V ring.
 // ---------------------------------------------------------------------------
 template <int D>
@@ -131,7 +135,7 @@ __global__ void __launch_bounds__(320, 1)
                   BwdSparseArgs a) {
   using L = DqSmem<D>;
   constexpr int NK = L::NK, NV = L::NV;
-  constexpr uint32_t COL_DQ = 256;
+  constexpr uint32_t COL_DQ = 256, COL_Q = 384, COL_DO = 448;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~uintptr_t(1023));
@@ -148,7 +152,8 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* sp_full = v_empty + NV;      // [2] S and dP of buffer x
   uint64_t* ds_ready = sp_full + 2;      // [2] dS written by all row threads
   uint64_t* dq_done = ds_ready + 2;      // the last dQ MMA completed
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(dq_done + 1);
+  uint64_t* qt_ready = dq_done + 1;      // Q and dO copied into TMEM by the row threads
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(qt_ready + 1);
   int* s_count = reinterpret_cast<int*>(tslot + 1);
   const int Tkvr = (a.Tkv + 15) & ~15;
   uint8_t* fa = sm + L::OFF_U;
@@ -184,6 +189,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&ds_ready[x], 8);
     }
     mbar_init(dq_done, 1);
+    mbar_init(qt_ready, 8);
     fence_barrier_init();
   }
   for (int j = tid; j < 2 * Tkvr; j += blockDim.x) fa[j] = 0;
@@ -266,8 +272,7 @@ __global__ void __launch_bounds__(320, 1)
     if (ln == 0) {
       const uint32_t id_s = idesc_bf16(128, 64, false, false);
       const uint32_t id_q = idesc_bf16(128, D, false, true);
-      const uint32_t q0 = smem_u32(sQ), o0 = smem_u32(sdO);
-      bool ok = mbar_wait(in_full, 0, a.err, DEV_TIMEOUT_TMA);
+      bool ok = mbar_wait(qt_ready, 0, a.err, DEV_TIMEOUT_SYNC);
       // dQ += dS_k K_k: dS (bf16 pairs) from TMEM buffer k & 1, K as the MN-major B operand
       auto issue_dq = [&](int k) -> bool {
         const int x = k & 1, sk = k % NK;
@@ -289,15 +294,15 @@ __global__ void __launch_bounds__(320, 1)
         if (!mbar_wait(&v_full[sv], (k / NV) & 1, a.err, DEV_TIMEOUT_TMA)) { ok = false; break; }
         tc_fence_after();
         // S and dP into buffer x; its previous contents (entry k - 2) were consumed
-        // by the dQ MMA issued earlier by this thread (in-order execution)
-        const uint64_t dq0 = sdesc_sw128(q0, 16, 1024), do0 = sdesc_sw128(o0, 16, 1024);
+        // by the dQ MMA issued earlier by this thread (in-order execution).  Q and dO
+        // from TMEM: d = 16 kk .. 16 kk + 15 at columns 8 kk .. 8 kk + 7.
         const uint64_t dkt = sdesc_sw128(smem_u32(sK), 16, 1024) + (uint64_t)(sk * L::T64 >> 4);
         const uint64_t dvt = sdesc_sw128(smem_u32(sV), 16, 1024) + (uint64_t)(sv * L::T64 >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = ((kk / 4) * 16384 + (kk % 4) * 32) >> 4, offk = ((kk / 4) * 8192 + (kk % 4) * 32) >> 4;
-          umma_ss(tbase + 128 * x, dq0 + off, dkt + offk, id_s, kk > 0 ? 1u : 0u);
-          umma_ss(tbase + 128 * x + 64, do0 + off, dvt + offk, id_s, kk > 0 ? 1u : 0u);
+          const uint32_t offk = ((kk / 4) * 8192 + (kk % 4) * 32) >> 4;
+          umma_ts(tbase + 128 * x, tbase + COL_Q + 8 * kk, dkt + offk, id_s, kk > 0 ? 1u : 0u);
+          umma_ts(tbase + 128 * x + 64, tbase + COL_DO + 8 * kk, dvt + offk, id_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&sp_full[x]);
         umma_commit(&v_empty[sv]);
@@ -326,8 +331,36 @@ __global__ void __launch_bounds__(320, 1)
                    nd2 = f2_pack(ld.y, ld.y);
     // this thread's half of the row's fp32 linear part, added in the epilogue
     const float* lin = a.q_lin + ((int64_t)bh * a.N + n) * D + (D / 2) * hs;
-    bool ok = true;
-    for (int k = 0; k < U; ++k) {
+    // this thread's half of the row's Q and dO (d = (D/2) hs ..) from the swizzled
+    // tiles into TMEM as bf16 pairs, the A operands of the S and dP MMAs
+    bool ok = __all_sync(0xffffffffu, mbar_wait(in_full, 0, a.err, DEV_TIMEOUT_TMA));
+    if (ok) {
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint8_t* src = which == 0 ? sQ : sdO;
+        uint32_t qv[D / 4];
+#pragma unroll
+        for (int u = 0; u < D / 16; ++u) {  // 16-byte units: 8 bf16 = 4 columns each
+          const int d0 = (D / 2) * hs + 8 * u;
+          const uint4 t = *reinterpret_cast<const uint4*>(src + (d0 / 64) * 16384 + sw128_offset(r, (d0 % 64) * 2));
+          qv[4 * u] = t.x;
+          qv[4 * u + 1] = t.y;
+          qv[4 * u + 2] = t.z;
+          qv[4 * u + 3] = t.w;
+        }
+        const uint32_t col = (which == 0 ? COL_Q : COL_DO) + (D / 4) * hs;
+        if constexpr (D == 128) {
+          tmem_st32(tl + col, qv);
+        } else {
+          tmem_st16(tl + col, qv);
+        }
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (ok && ln == 0) mbar_arrive(qt_ready);
+    for (int k = 0; k < U && ok; ++k) {
       const int x = k & 1;
       if (valid && k == (U > 3 ? U - 3 : 0)) {  // into L2 a few entries ahead of the epilogue
 #pragma unroll
