@@ -146,9 +146,17 @@ __global__ void __launch_bounds__(192, 1)
     const float cs = a.combine == 1 ? a.alpha[bh] : 1.f;
     const float cl = a.combine == 1 ? 1.f - a.alpha[bh] : 1.f;
     const __nv_bfloat16* qrow = a.Q + (int64_t)b * a.sq[0] + (int64_t)h * a.sq[1] + (int64_t)n * a.sq[2];
-    bool ok = __all_sync(0xffffffffu, mbar_wait(h_full, 0, err, DEV_TIMEOUT_TMA));
+    const __nv_bfloat16* drow = a.dO + (int64_t)b * a.so[0] + (int64_t)h * a.so[1] + (int64_t)n * a.so[2];
+    const float* osrow = a.os + ((int64_t)bh * a.N + n) * TD;
+    if (valid) {  // phase 2's rows into L2 while phase 1 runs
+#pragma unroll
+      for (int c = 0; c < TD; c += 64) prefetch_l2(drow + c);
+#pragma unroll
+      for (int c = 0; c < TD; c += 32) prefetch_l2(osrow + c);
+    }
     // ---- phase 1: phi(q) (bf16) into sF, den = phi(q) . Z_t + eps.  The row is
-    // loaded once, all 16 loads in flight, and kept in registers.
+    // loaded once, all 16 loads in flight, and kept in registers; the H' and Z
+    // tiles are waited for only where den needs Z.
     uint4 qv[TD / 8];
 #pragma unroll
     for (int c = 0; c < TD / 8; ++c)
@@ -173,6 +181,7 @@ __global__ void __launch_bounds__(192, 1)
       return a.phi == 1 ? (x > 0.f ? x + 1.f : exp2f(x * LOG2E_T)) : exp2f((x - m) * LOG2E_T) * inv_s;
     };
     float den = a.eps;
+    bool ok = __all_sync(0xffffffffu, mbar_wait(h_full, 0, err, DEV_TIMEOUT_TMA));
     if (ok) {
       const __nv_bfloat16* z = sZ + t * TD;
 #pragma unroll
@@ -202,8 +211,6 @@ __global__ void __launch_bounds__(192, 1)
     float dd = 0.f, dol = 0.f, da = 0.f;
     if (ok) {
       tc_fence_after();
-      const __nv_bfloat16* drow = a.dO + (int64_t)b * a.so[0] + (int64_t)h * a.so[1] + (int64_t)n * a.so[2];
-      const float* osrow = a.os + ((int64_t)bh * a.N + n) * TD;
       const float inv_den = 1.f / den;
 #pragma unroll 1
       for (int c0 = 0; c0 < TD; c0 += 32) {
