@@ -4,7 +4,7 @@
 // the three products run as tcgen05.mma:
 //   G1  NUM_t  = phi(Q) H'_t           M = 128 rows, N = d, K = d   (t = 0, 1)
 //   G2  dphi_t = gp H'_t^T             M = 128 rows, N = d, K = d
-//   G3  dH'_t  = phi(Q_t)^T gp_t       M = d, N = d, K = 64 rows of block t
+//   G3  dH'_t^T = gp_t^T phi(Q_t)      M = d, N = d, K = 64 rows of block t
 // G1 and G2 are computed for all 128 rows against both blocks' H' (each row
 // keeps the half of its own block), so every per-row scalar (den, o'_r . dO_r,
 // D_r) stays with the thread that owns the row.  H'_t arrives by TMA as the
@@ -14,8 +14,9 @@
 //   warp 0      TMA: both blocks' H' tiles and Z rows
 //   warp 1      tcgen05.mma issuer
 //   warps 2-5   one row each: phi(q) -> shared (bf16, swizzled), den; then o',
-//               D, gp -> shared, gden; then dq (linear part); finally one column
-//               a of dH'_t each (G3's lanes are a) and dZ_t[a]
+//               D, gp -> shared, gden; then dq (linear part); finally one row
+//               o of dH'_t^T each (G3's lanes are o; the output is [o][a]) and
+//               dZ_t[a] for a = its row
 // TMEM (512 columns, one CTA per SM): G1 and then G2 at [0, 2d), G3 at [2d, 4d).
 #include "kernels.cuh"
 
@@ -36,6 +37,11 @@ constexpr float LOG2E_T = 1.4426950408889634f;
 
 __device__ __forceinline__ float bfv(uint32_t packed, int hi) {
   return __uint_as_float(hi ? (packed & 0xffff0000u) : (packed << 16));
+}
+__device__ __forceinline__ float ex2a(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 }  // namespace
 
@@ -126,12 +132,13 @@ __global__ void __launch_bounds__(192, 1)
             umma_ss(tbase + TD * t, sdesc_sw128(g0 + (kk / 4) * TILE + (kk % 4) * 32, 16, 1024),
                     sdesc_sw128(h0 + t * TILE + kk * 2048, 2 * TILE, 1024), id_km, kk > 0 ? 1u : 0u);
         umma_commit(dphi_full);
-        // G3: dH'_t[a][o] = sum_{r in block t} F[r][a] GP[r][o]  (A: M = a contiguous; B: N = o contiguous)
+        // G3, transposed: dH'_t^T[o][a] = sum_{r in block t} GP[r][o] F[r][a]  (A: M = o contiguous;
+        // B: N = a contiguous), so that a TMEM lane holds one row o of the [o][a] output
         for (int t = 0; t < 2; ++t)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_ss(tbase + 2 * TD + TD * t, sdesc_sw128(f0 + t * 8192 + kk * 2048, TILE, 1024),
-                    sdesc_sw128(g0 + t * 8192 + kk * 2048, TILE, 1024), id_mm, kk > 0 ? 1u : 0u);
+            umma_ss(tbase + 2 * TD + TD * t, sdesc_sw128(g0 + t * 8192 + kk * 2048, TILE, 1024),
+                    sdesc_sw128(f0 + t * 8192 + kk * 2048, TILE, 1024), id_mm, kk > 0 ? 1u : 0u);
         umma_commit(dh_full);
       }
     }
@@ -161,29 +168,43 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
     for (int c = 0; c < TD / 8; ++c)
       qv[c] = valid ? __ldg(reinterpret_cast<const uint4*>(qrow) + c) : make_uint4(0u, 0u, 0u, 0u);
+    // softmax phi: the row maximum in four partial maxima, then 2^((x - m) log2 e)
+    // once per element, kept in sphi until it is normalised below, with the row
+    // sum in four partial sums
+    float* myphi = sphi + r * (TD + 1);
     float m = -INFINITY, s = 0.f;
     if (valid && a.phi == 0) {
+      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c = 0; c < TD / 8; ++c) {
         const uint32_t u[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, bfv(u[e / 2], e & 1));
+        for (int e = 0; e < 4; ++e) mp[e] = fmax3(mp[e], bfv(u[e], 0), bfv(u[e], 1));
       }
+      m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+      float sp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < TD / 8; ++c) {
         const uint32_t u[4] = {qv[c].x, qv[c].y, qv[c].z, qv[c].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s += exp2f((bfv(u[e / 2], e & 1) - m) * LOG2E_T);
+        for (int e = 0; e < 4; ++e) {
+          const float e0 = ex2a((bfv(u[e], 0) - m) * LOG2E_T), e1 = ex2a((bfv(u[e], 1) - m) * LOG2E_T);
+          myphi[8 * c + 2 * e] = e0;
+          myphi[8 * c + 2 * e + 1] = e1;
+          sp[e] += e0 + e1;
+        }
       }
+      s = (sp[0] + sp[1]) + (sp[2] + sp[3]);
     }
     const float inv_s = (a.phi == 0 && s > 0.f) ? 1.f / s : 1.f;
-    auto phi_of = [&](float x) {
-      return a.phi == 1 ? (x > 0.f ? x + 1.f : exp2f(x * LOG2E_T)) : exp2f((x - m) * LOG2E_T) * inv_s;
+    auto phi_at = [&](int col, float x) {
+      return a.phi == 1 ? (x > 0.f ? x + 1.f : ex2a(x * LOG2E_T)) : myphi[col] * inv_s;
     };
     float den = a.eps;
     bool ok = __all_sync(0xffffffffu, mbar_wait(h_full, 0, err, DEV_TIMEOUT_TMA));
     if (ok) {
       const __nv_bfloat16* z = sZ + t * TD;
+      float dp[4] = {0.f, 0.f, 0.f, 0.f};  // den in four partial sums
 #pragma unroll
       for (int c = 0; c < TD; c += 8) {
         uint32_t o4[4] = {0u, 0u, 0u, 0u};
@@ -192,17 +213,18 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t u[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float f0 = phi_of(bfv(u[e], 0)), f1 = phi_of(bfv(u[e], 1));
-            sphi[r * (TD + 1) + c + 2 * e] = f0;
-            sphi[r * (TD + 1) + c + 2 * e + 1] = f1;
+            const float f0 = phi_at(c + 2 * e, bfv(u[e], 0)), f1 = phi_at(c + 2 * e + 1, bfv(u[e], 1));
+            myphi[c + 2 * e] = f0;
+            myphi[c + 2 * e + 1] = f1;
             o4[e] = pack_bf16x2(f0, f1);
-            den = fmaf(bfv(o4[e], 0), __bfloat162float(z[c + 2 * e]),
-                       fmaf(bfv(o4[e], 1), __bfloat162float(z[c + 2 * e + 1]), den));
+            dp[e] = fmaf(bfv(o4[e], 0), __bfloat162float(z[c + 2 * e]),
+                         fmaf(bfv(o4[e], 1), __bfloat162float(z[c + 2 * e + 1]), dp[e]));
           }
         }
         *reinterpret_cast<uint4*>(sF + (c / 64) * TILE + sw128_offset(r, (c % 64) * 2)) =
             make_uint4(o4[0], o4[1], o4[2], o4[3]);
       }
+      den += (dp[0] + dp[1]) + (dp[2] + dp[3]);
     }
     fence_proxy_async_smem();
     mbar_arrive(fq_ready);
@@ -275,6 +297,7 @@ __global__ void __launch_bounds__(192, 1)
       const __nv_bfloat16* z = sZ + t * TD;
       float dot = 0.f;
       if (a.phi == 0) {
+        float dq4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums
 #pragma unroll 1
         for (int c0 = 0; c0 < TD; c0 += 32) {
           uint32_t dv[32];
@@ -283,10 +306,11 @@ __global__ void __launch_bounds__(192, 1)
           if (valid) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              dot = fmaf(sphi[r * (TD + 1) + c0 + e], __uint_as_float(dv[e]) + gden * __bfloat162float(z[c0 + e]),
-                         dot);
+              dq4[e & 3] = fmaf(myphi[c0 + e], __uint_as_float(dv[e]) + gden * __bfloat162float(z[c0 + e]),
+                                dq4[e & 3]);
           }
         }
+        dot = (dq4[0] + dq4[1]) + (dq4[2] + dq4[3]);
       }
       float* out = a.dq_lin + ((int64_t)bh * a.N + n) * TD;
 #pragma unroll 1
@@ -300,7 +324,7 @@ __global__ void __launch_bounds__(192, 1)
             float y[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float f = sphi[r * (TD + 1) + c0 + e4 + e];
+              const float f = myphi[c0 + e4 + e];
               const float dphi = __uint_as_float(dv[e4 + e]) + gden * __bfloat162float(z[c0 + e4 + e]);
               // elu + 1: d phi / dx = 1 where x > 0 (phi > 1), else e^x = phi
               y[e] = a.phi == 1 ? dphi * (f > 1.f ? 1.f : f) : f * (dphi - dot);
@@ -310,8 +334,9 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
     }
-    // ---- phase 4: thread r owns column a = r of dH'_t (G3's lanes) and dZ_t[a];
-    // the waits on fq_ready / gp_ready order the other rows' phi(q) and gden writes
+    // ---- phase 4: thread r owns row o = r of dH'_t^T (G3's lanes: the [o][a] row
+    // of the output, 16-byte stores) and dZ_t[a = r]; the waits on fq_ready /
+    // gp_ready order the other rows' phi(q) and gden writes
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(dh_full, 0, err, DEV_TIMEOUT_MMA) &&
                                              mbar_wait(fq_ready, 0, err, DEV_TIMEOUT_SYNC) &&
                                              mbar_wait(gp_ready, 0, err, DEV_TIMEOUT_SYNC));
@@ -326,8 +351,14 @@ __global__ void __launch_bounds__(192, 1)
           uint32_t hv[32];
           tmem_ld32(tl + 2 * TD + TD * tt + c0, hv);
           tmem_ld_wait();
+          uint4* d4 = reinterpret_cast<uint4*>(dst + (int64_t)aa * TD + c0);  // row o = aa, a = c0 ..
 #pragma unroll
-          for (int e = 0; e < 32; ++e) dst[(int64_t)(c0 + e) * TD + aa] = __float2bfloat16(__uint_as_float(hv[e]));
+          for (int v4 = 0; v4 < 4; ++v4)
+            d4[v4] = make_uint4(
+                pack_bf16x2(__uint_as_float(hv[8 * v4]), __uint_as_float(hv[8 * v4 + 1])),
+                pack_bf16x2(__uint_as_float(hv[8 * v4 + 2]), __uint_as_float(hv[8 * v4 + 3])),
+                pack_bf16x2(__uint_as_float(hv[8 * v4 + 4]), __uint_as_float(hv[8 * v4 + 5])),
+                pack_bf16x2(__uint_as_float(hv[8 * v4 + 6]), __uint_as_float(hv[8 * v4 + 7])));
         }
         // dZ_t[a] = sum_{rows of block tt} gden_r phi(q_r)[a], in eight partial sums
         float dzp[8];
@@ -561,22 +592,28 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
       for (int c = 0; c < TD / 8; ++c)
         kv[c] = *reinterpret_cast<const uint4*>(sF + (c / 8) * TILE + sw128_offset(r, (c % 8) * 16));
+      // the row maximum and sum in four partial maxima / sums each
+      float mp[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c = 0; c < TD / 8; ++c) {
         const uint32_t u[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, bfv(u[e / 2], e & 1));
+        for (int e = 0; e < 4; ++e) mp[e] = fmax3(mp[e], bfv(u[e], 0), bfv(u[e], 1));
       }
+      m = fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3]));
+      float sp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < TD / 8; ++c) {
         const uint32_t u[4] = {kv[c].x, kv[c].y, kv[c].z, kv[c].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s += exp2f((bfv(u[e / 2], e & 1) - m) * LOG2E_T);
+        for (int e = 0; e < 4; ++e)
+          sp[e] += ex2a((bfv(u[e], 0) - m) * LOG2E_T) + ex2a((bfv(u[e], 1) - m) * LOG2E_T);
       }
+      s = (sp[0] + sp[1]) + (sp[2] + sp[3]);
     }
     const float inv_s = (a.phi == 0 && s > 0.f) ? 1.f / s : 1.f;
     auto phi_of = [&](float x) {
-      return a.phi == 1 ? (x > 0.f ? x + 1.f : exp2f(x * LOG2E_T)) : exp2f((x - m) * LOG2E_T) * inv_s;
+      return a.phi == 1 ? (x > 0.f ? x + 1.f : ex2a(x * LOG2E_T)) : ex2a((x - m) * LOG2E_T) * inv_s;
     };
     // phi(K) in place in sF (bf16, the MMA operand) and in fp32 in TMEM columns
     // [3d, 4d) of this row's lane, for the phi backward at the end
@@ -684,6 +721,7 @@ __global__ void __launch_bounds__(192, 1)
       const __nv_bfloat16* z = sZ + t * TD;
       float dot = 0.f;
       if (a.phi == 0) {
+        float dq4[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums
 #pragma unroll 1
         for (int c0 = 0; c0 < TD; c0 += 32) {
           uint32_t dv[32], fv[32];
@@ -693,9 +731,11 @@ __global__ void __launch_bounds__(192, 1)
           if (valid) {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              dot = fmaf(__uint_as_float(fv[e]), __uint_as_float(dv[e]) + __bfloat162float(z[c0 + e]), dot);
+              dq4[e & 3] = fmaf(__uint_as_float(fv[e]), __uint_as_float(dv[e]) + __bfloat162float(z[c0 + e]),
+                                dq4[e & 3]);
           }
         }
+        dot = (dq4[0] + dq4[1]) + (dq4[2] + dq4[3]);
       }
       float* out = a.dk_lin + ((int64_t)bh * a.N + n) * TD;
 #pragma unroll 1
