@@ -470,12 +470,13 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* sW = sm + K_OFF_W;
   const __nv_bfloat16* sZ = reinterpret_cast<const __nv_bfloat16*>(sm + K_OFF_Z);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + K_OFF_BAR);
-  uint64_t* in_full = bars + 0;
+  uint64_t* in_full = bars + 0;   // dh' tiles, Z rows, V pair
   uint64_t* fk_ready = bars + 1;
   uint64_t* g1_full = bars + 2;
   uint64_t* u_ready = bars + 3;
   uint64_t* g2_full = bars + 4;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 5);
+  uint64_t* k_full = bars + 5;    // K pair: phi(K) starts while the rest is loading
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + 6);
 
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const int p = blockIdx.x, bh = blockIdx.y;
@@ -494,6 +495,7 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(g1_full, 1);
     mbar_init(u_ready, 128);
     mbar_init(g2_full, 1);
+    mbar_init(k_full, 1);
     fence_barrier_init();
   }
   tc_fence_before();
@@ -507,7 +509,10 @@ __global__ void __launch_bounds__(192, 1)
       tma_prefetch_desc(&mapZ);
       tma_prefetch_desc(&mapK2);
       tma_prefetch_desc(&mapV2);
-      mbar_arrive_expect_tx(in_full, 2 * (2 * TILE + TD * 2) + 4 * TILE);
+      mbar_arrive_expect_tx(k_full, 2 * TILE);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) tma_load_4d(sF + c * TILE, &mapK2, k_full, c * 64, 128 * p, h, b);
+      mbar_arrive_expect_tx(in_full, 2 * (2 * TILE + TD * 2) + 2 * TILE);
       for (int t = 0; t < 2; ++t) {
         const int j = (t == 1 && has1) ? j1 : j0;  // a missing second block reuses the first
 #pragma unroll
@@ -517,10 +522,7 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tma_load_4d(sF + c * TILE, &mapK2, in_full, c * 64, 128 * p, h, b);
-        tma_load_4d(sV + c * TILE, &mapV2, in_full, c * 64, 128 * p, h, b);
-      }
+      for (int c = 0; c < 2; ++c) tma_load_4d(sV + c * TILE, &mapV2, in_full, c * 64, 128 * p, h, b);
     }
   } else if (w == 1) {
     if (ln == 0) {
@@ -528,7 +530,7 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t id_km = idesc_bf16(128, TD, false, true);
       const uint32_t g0 = smem_u32(sG), f0 = smem_u32(sF), v0 = smem_u32(sV), u0 = smem_u32(sU),
                      w0 = smem_u32(sW);
-      bool ok = mbar_wait(fk_ready, 0, err, DEV_TIMEOUT_SYNC);
+      bool ok = mbar_wait(in_full, 0, err, DEV_TIMEOUT_TMA) && mbar_wait(fk_ready, 0, err, DEV_TIMEOUT_SYNC);
       if (ok) {
         tc_fence_after();
         // G1: U_t[r][o] = sum_a F[r][a] dh'_t[a][o]
@@ -573,18 +575,20 @@ __global__ void __launch_bounds__(192, 1)
     const bool valid = (t == 0 || has1) && n < a.N;
     const uint32_t tl = tbase + ((uint32_t)(32 * q4) << 16);
     // W~ as bf16 into sW (row o = r), the K-major B operand of G3 / MN-major B of G2
-    if (proj) {
-      const float* wr = a.proj_w + (int64_t)r * TD;
-#pragma unroll 4
+    if (proj) {  // the whole row's loads in flight at once
+      const float4* wr4 = reinterpret_cast<const float4*>(a.proj_w + (int64_t)r * TD);
+      float4 x[TD / 4];
+#pragma unroll
+      for (int c = 0; c < TD / 4; ++c) x[c] = __ldg(wr4 + c);
+#pragma unroll
       for (int c = 0; c < TD; c += 8) {
-        const float4 x0 = *reinterpret_cast<const float4*>(wr + c);
-        const float4 x1 = *reinterpret_cast<const float4*>(wr + c + 4);
+        const float4 x0 = x[c / 4], x1 = x[c / 4 + 1];
         *reinterpret_cast<uint4*>(sW + (c / 64) * TILE + sw128_offset(r, (c % 64) * 2)) =
             make_uint4(pack_bf16x2(x0.x, x0.y), pack_bf16x2(x0.z, x0.w), pack_bf16x2(x1.x, x1.y),
                        pack_bf16x2(x1.z, x1.w));
       }
     }
-    bool ok = __all_sync(0xffffffffu, mbar_wait(in_full, 0, err, DEV_TIMEOUT_TMA));
+    bool ok = __all_sync(0xffffffffu, mbar_wait(k_full, 0, err, DEV_TIMEOUT_TMA));
     // ---- phi(K) in place (bf16); rows that do not exist get 0
     float m = -INFINITY, s = 0.f;
     if (ok && valid && a.phi == 0) {  // from the K tile in shared memory (loaded by TMA)
@@ -699,7 +703,8 @@ __global__ void __launch_bounds__(192, 1)
     mbar_arrive(u_ready);
     // ---- dv (SLA) and dk = phi backward of dphi_t + dz_t.  tcgen05.ld is a
     // warp-wide instruction: every lane runs it, only valid rows store.
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(g2_full, 0, err, DEV_TIMEOUT_MMA));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(g2_full, 0, err, DEV_TIMEOUT_MMA) &&
+                                             mbar_wait(in_full, 0, err, DEV_TIMEOUT_TMA));  // Z rows
     if (ok) {
       tc_fence_after();
       if (proj) {
